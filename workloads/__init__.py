@@ -1,0 +1,142 @@
+"""Seeded synthetic inputs for the trellis-coded quantized linear layer.
+
+This module is shared by the CUDA path's tests/benchmark and by the CPU oracle.
+It holds no arithmetic of the method: it only names the layer shapes and draws
+the random arrays the method consumes as inputs (packed code words, +-1 sign
+vectors, the HYB lookup table, activations).
+
+Workloads (synthetic stand-ins for the Llama-2/3-shaped layers the QTIP
+OpenReview discussion times and evaluates; no weights or datasets are used):
+
+  tiny      m=n=256,            k=2, L=16, V=1, 1MAD,  alpha=1,    batch 1
+  attn4096  m=n=4096,           k=2, L=16, V=1, 3INST, alpha=0.02, batch 1
+  mlp_up    m=11008, n=4096,    k=3, L=16, V=2, HYB Q=9,  alpha=1, batch 1/4/8
+  mlp_down  m=4096,  n=11008,   k=3, L=16, V=2, HYB Q=9,  alpha=1, batch 1/4/8
+  large     m=28672, n=8192,    k=4, L=16, V=1, 1MAD,  alpha=0.01, batch 1/4/16
+  halftcq   m=14336, n=4096, rows [0,7168) k=2 and [7168,14336) k=3,
+            L=16, V=1, 3INST, alpha=1, batch 64/256
+
+Distributions: code words are uniform uint32, signs uniform +-1 (int8), the
+HYB table holds 2^Q x V standard normals rounded to fp16 (numpy's float16
+cast), activations x ~ N(0,1) cast to fp16.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import numpy as np
+
+CODE_1MAD = 0
+CODE_3INST = 1
+CODE_HYB = 2
+CODE_NAMES = {CODE_1MAD: "1MAD", CODE_3INST: "3INST", CODE_HYB: "HYB"}
+
+T_BLOCK = 256  # columns per independent trellis block (fixed by the format)
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerSpec:
+    name: str
+    m: int
+    n: int
+    k: int                      # bits per weight (uniform layers)
+    L: int
+    V: int
+    code: int
+    alpha: float
+    seed: int
+    Q: int = 0                  # HYB table index bits
+    m_top: Optional[int] = None  # half-TCQ: rows [0, m_top) at k_top, rest at k_bot
+    k_top: Optional[int] = None
+    k_bot: Optional[int] = None
+    batches: Sequence[int] = (1,)
+
+    @property
+    def mixed(self) -> bool:
+        return self.m_top is not None
+
+    def row_parts(self):
+        """[(row0, rows, k)] in stream order."""
+        if self.mixed:
+            return [(0, self.m_top, self.k_top), (self.m_top, self.m - self.m_top, self.k_bot)]
+        return [(0, self.m, self.k)]
+
+    @property
+    def n_words(self) -> int:
+        return sum(rows * self.n * k for _, rows, k in self.row_parts()) // 32
+
+    @property
+    def stream_bytes(self) -> int:
+        return self.n_words * 4
+
+    @property
+    def bits_per_weight(self) -> float:
+        return self.n_words * 32 / (self.m * self.n)
+
+
+WORKLOADS = {
+    "tiny": LayerSpec("tiny", 256, 256, 2, 16, 1, CODE_1MAD, 1.0, seed=0, batches=(1,)),
+    "attn4096": LayerSpec("attn4096", 4096, 4096, 2, 16, 1, CODE_3INST, 0.02, seed=1, batches=(1,)),
+    "mlp_up": LayerSpec("mlp_up", 11008, 4096, 3, 16, 2, CODE_HYB, 1.0, seed=2, Q=9, batches=(1, 4, 8)),
+    "mlp_down": LayerSpec("mlp_down", 4096, 11008, 3, 16, 2, CODE_HYB, 1.0, seed=2, Q=9, batches=(1, 4, 8)),
+    "large": LayerSpec("large", 28672, 8192, 4, 16, 1, CODE_1MAD, 0.01, seed=3, batches=(1, 4, 16)),
+    "halftcq": LayerSpec("halftcq", 14336, 4096, 0, 16, 1, CODE_3INST, 1.0, seed=4,
+                         m_top=7168, k_top=2, k_bot=3, batches=(64, 256)),
+}
+
+# The up and down projections of the MLP pair draw from one seeded stream
+# (up first), so that the two layers of the pair are distinct.
+_STREAM_ORDER = {"mlp_down": 1}
+
+
+@dataclasses.dataclass
+class LayerInputs:
+    spec: LayerSpec
+    codes: np.ndarray       # uint32 [n_words], canonical stream order
+    s_in: np.ndarray        # int8 [n], +-1
+    s_out: np.ndarray       # int8 [m], +-1
+    lut: Optional[np.ndarray]  # float16 [2^Q, V] for HYB, else None
+
+
+def _rng(seed, instance, stream=0):
+    if instance == 0 and stream == 0:
+        return np.random.default_rng(seed)
+    return np.random.default_rng([seed, stream, instance])
+
+
+def hyb_table(Q: int, V: int, seed: int) -> np.ndarray:
+    """2^Q x V standard-normal entries rounded to fp16 (numpy's float16 cast)."""
+    return np.random.default_rng(seed).standard_normal((1 << Q, V)).astype(np.float16)
+
+
+def make_layer(spec: LayerSpec, instance: int = 0) -> LayerInputs:
+    """Draw the layer's code stream, signs and table.
+
+    instance 0 is the canonical draw for the workload's seed; other instances
+    are independent layers of the same shape (used to rotate through more
+    bytes than the L2 cache holds when timing).
+    """
+    stream = _STREAM_ORDER.get(spec.name, 0)
+    rng = _rng(spec.seed, instance, stream)
+    codes = rng.integers(0, 2**32, size=spec.n_words, dtype=np.uint32)
+    s_in = (2 * rng.integers(0, 2, size=spec.n) - 1).astype(np.int8)
+    s_out = (2 * rng.integers(0, 2, size=spec.m) - 1).astype(np.int8)
+    lut = None
+    if spec.code == CODE_HYB:
+        lut = hyb_table(spec.Q, spec.V, spec.seed + 1000 * instance)
+    return LayerInputs(spec, codes, s_in, s_out, lut)
+
+
+def make_x(spec: LayerSpec, batch: int, instance: int = 0) -> np.ndarray:
+    """Activations x ~ N(0,1) in fp16, shape [batch, n]."""
+    rng = np.random.default_rng([spec.seed, 77, batch, instance])
+    return rng.standard_normal((batch, spec.n)).astype(np.float16)
+
+
+def random_layer(m: int, n: int, k: int, L: int, V: int, code: int, seed: int,
+                 alpha: float = 1.0, Q: int = 9, m_top=None, k_top=None, k_bot=None) -> LayerInputs:
+    """A small seeded layer of any supported shape (tests of ragged/edge shapes)."""
+    spec = LayerSpec(f"rand_{m}x{n}_k{k}", m, n, k if m_top is None else 0, L, V, code, alpha,
+                     seed, Q=Q if code == CODE_HYB else 0, m_top=m_top, k_top=k_top, k_bot=k_bot)
+    return make_layer(spec)
