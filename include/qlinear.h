@@ -1,0 +1,173 @@
+/*
+ * qlinear.h -- C ABI of the trellis-coded quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes
+ *
+ *     y = alpha * diag(s_out) * H_m^T * W_hat * H_n * diag(s_in) * x
+ *
+ * where H_d = I_{d/B} (x) H_B is the normalised Walsh-Hadamard transform on
+ * consecutive blocks of B entries (B = the largest power of two dividing d),
+ * s_in / s_out are random +-1 sign vectors and alpha is a per-layer scale.
+ * This is incoherence processing with a randomized Hadamard transform as on
+ * the QuIP# page (Fig. 2) and in the QTIP OpenReview discussion ("Incoherence
+ * Processing (W2)").  W_hat (m x n) is never stored: it is decoded on the fly
+ * from a bitshift-trellis bit stream (QTIP discussion, "Figure 2 (Q4)" and
+ * "Ablations and fast inference (W1 and W2)") through one of three codes
+ * (QTIP discussion, "Inference speed analysis (W2)" and the comment on HYB
+ * cost, "Bit Accounting (Q2)"):
+ *
+ *   QL_CODE_1MAD   x = A*s + B mod 2^32; value = fp16(C1 * (sum of the 4 bytes of x - 510))
+ *   QL_CODE_3INST  x = A*s + B mod 2^32; m = (x & MASK) ^ XOR;
+ *                  value = fp16(float16(m & 0xffff) + float16(m >> 16))
+ *   QL_CODE_HYB    x = A*s + B mod 2^32; entry = lut[x >> (32 - Q)] (V fp16 values);
+ *                  bit 15 of x negates the entry's first value
+ *
+ * with the constants (A, B per code; C1 = 443 * 2^-16; MASK = 0x9CFF8FFF,
+ * XOR = 0x20003000) fixed by this library's format.  Values are rounded to
+ * fp16 exactly once.
+ *
+ * Stream format (the pages print only the bit string of the Figure 2 example;
+ * this is the library's reading):
+ *   - packed_codes is a uint32 array read as one bit string, most significant
+ *     bit of each word first.
+ *   - Every row is cut into blocks of T = 256 columns; block j of row r is an
+ *     independent trellis of S = 256*k bits starting at bit r*n*k + j*S.
+ *   - Step t of a block carries bits [t*kV, (t+1)*kV); its L-bit state is the
+ *     window of the block's bits ending at bit (t+1)*kV, read cyclically
+ *     (tail-biting), and yields the V values of columns 256*j + t*V + e.
+ *   - A half-TCQ layer (Q-Palette's mixed-bitwidth layer) stores rows
+ *     [0, m_top) at k_top bits per weight first, then rows [m_top, m) at
+ *     k_bot bits per weight.
+ *
+ * Conventions for every entry point:
+ *   - Return value: QL_OK (0) or a negative QL_E_* code; qlinear_strerror()
+ *     names it.  Argument errors are detected on the host before any work.
+ *   - Device pointers are CUDA global-memory pointers of the device that was
+ *     current when the handle was created; "stream" is a cudaStream_t (NULL =
+ *     the legacy default stream).  forward/decode/eval_code are asynchronous
+ *     with respect to the host and ordered on that stream.
+ *   - A handle may be used from one host thread at a time; calls on one
+ *     handle must be ordered (one stream, or streams ordered by events),
+ *     because they share the handle's scratch buffers.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QL_OK 0
+#define QL_E_ARG (-1)          /* invalid argument (null pointer, bad size, bad value)   */
+#define QL_E_UNSUPPORTED (-2)  /* valid for the format but not implemented by this build */
+#define QL_E_CUDA (-3)         /* a CUDA runtime call failed                              */
+#define QL_E_OOM (-4)          /* device allocation failed                                */
+#define QL_E_TIMEOUT (-5)      /* a bounded device-side wait gave up                      */
+#define QL_E_DEVICE (-6)       /* a device-side check failed (see qlinear_get_status)     */
+
+#define QL_CODE_1MAD 0
+#define QL_CODE_3INST 1
+#define QL_CODE_HYB 2
+
+#define QL_F32 0
+#define QL_F16 1
+
+typedef struct qlinear_s* qlinear_t;
+
+/* The code that maps a trellis state to V values.
+ *   kind: QL_CODE_1MAD or QL_CODE_3INST (V must be 1), or QL_CODE_HYB (V = 1 or 2).
+ *   Q:    HYB only, table index bits, 1..9 (the discussion uses Q = 9; "you can
+ *         go down to Q~6").
+ *   lut:  HYB only, device pointer to 2^Q x V fp16 values, row-major
+ *         (entry i = lut[i*V .. i*V+V-1]).  Copied by create. */
+typedef struct {
+    int kind;
+    int Q;
+    const void* lut;
+} ql_code_t;
+
+/* Facts about a handle (qlinear_info). */
+typedef struct {
+    int m, n, L, V, code, Q;
+    int k_top, k_bot, m_top;   /* uniform layers: k_top = k_bot = k, m_top = m */
+    int B_n, B_m;              /* Hadamard block sizes                           */
+    size_t stream_bytes;       /* packed code words: m*n*k/8 (mixed: per part)   */
+    size_t sign_bytes;         /* bit-packed signs: (n + m) bits, word-padded    */
+    size_t lut_bytes;          /* HYB table: 2^Q * V * 2 bytes                   */
+    size_t scratch_bytes;      /* device scratch currently held by the handle    */
+} ql_info_t;
+
+/* Create a uniform-bitrate layer.
+ *   m, n:         output and input sizes; n % 256 == 0, m % 16 == 0, and the
+ *                 Hadamard block sizes B(n), B(m) must not exceed 32768.
+ *   k:            bits per weight, 1..4.   L: state bits, k*V <= L <= 16.
+ *   V:            values per trellis step (1 or 2, see ql_code_t).
+ *   packed_codes: device pointer, n_words = m*n*k/32 uint32 in the stream format above.
+ *   s_in, s_out:  device pointers, int8 +-1, n and m entries (any other value -> QL_E_ARG).
+ *   alpha:        finite scale.
+ * The handle copies codes (re-laid out for the kernels), signs (bit-packed)
+ * and the HYB table into library-owned device memory; the caller may free its
+ * buffers when create returns.  Synchronises the device before returning.
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED, QL_E_OOM, QL_E_CUDA. */
+int qlinear_create(qlinear_t* out, int m, int n, int k, int L, int V, ql_code_t code,
+                   const uint32_t* packed_codes, size_t n_words,
+                   const int8_t* s_in, const int8_t* s_out, float alpha);
+
+/* Create a half-TCQ layer (Q-Palette page: two TCQ quantizers of different
+ * bitwidth in one layer): rows [0, m_top) at k_top bits, rows [m_top, m) at
+ * k_bot bits.  m_top % 16 == 0, 0 < m_top < m.  n_words = (m_top*k_top +
+ * (m - m_top)*k_bot) * n / 32.  Otherwise as qlinear_create. */
+int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int k_bot,
+                         int L, int V, ql_code_t code,
+                         const uint32_t* packed_codes, size_t n_words,
+                         const int8_t* s_in, const int8_t* s_out, float alpha);
+
+/* y = W x for a batch of inputs.
+ *   x: device pointer, fp16 [batch][n] row-major.
+ *   y: device pointer, [batch][m] row-major, fp32 (y_dtype = QL_F32) or fp16 (QL_F16).
+ *   batch >= 0 (0 is a no-op).  batch <= 8 runs the fused decode-GEMV kernels;
+ *   larger batches run the decode-to-shared-memory tcgen05 GEMM.
+ * The first call with a batch larger than any before it allocates scratch;
+ * make such a call before capturing forward into a CUDA graph.
+ * Errors: QL_E_ARG, QL_E_OOM, QL_E_CUDA (launch failure). */
+int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream);
+
+/* As qlinear_forward, with x and y in host memory: copies x to the device,
+ * runs forward and copies y back, all on `stream`, and waits for the stream
+ * before returning (y is ready on return).  Pinned host memory makes the
+ * copies asynchronous DMA transfers; pageable memory also works. */
+int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype,
+                         void* stream);
+
+/* Write W_hat as fp16 [m][n] row-major to the device pointer w_hat (the code
+ * values before alpha, signs and Hadamard transforms).  For testing. */
+int qlinear_decode(qlinear_t h, void* w_hat, void* stream);
+
+/* Evaluate a code on `count` states (device pointer, uint32, each < 2^L) and
+ * write fp16 [count][V] to the device pointer out.  For testing the codes
+ * exhaustively. */
+int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int count, void* out,
+                      void* stream);
+
+/* Read the handle's device status word (synchronises the device).  Returns
+ * QL_OK, or QL_E_DEVICE / QL_E_TIMEOUT if a kernel recorded a failed check or
+ * an expired bounded wait since the last call; reading clears the word. */
+int qlinear_get_status(qlinear_t h);
+
+/* Fill *info. */
+int qlinear_info(qlinear_t h, ql_info_t* info);
+
+/* Free the handle and its device memory (synchronises the device). */
+int qlinear_destroy(qlinear_t h);
+
+/* Name of a status code (static string). */
+const char* qlinear_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

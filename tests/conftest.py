@@ -10,4 +10,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a) and the built library")
-    config.addinivalue_line("markers", "slow: full-size workloads")
+
+
+def pytest_sessionstart(session):
+    # Build libqlinear.so in-tree if it is missing or older than its sources
+    # (nvcc cross-compiles without a GPU).
+    from trellis_coded_matmul_b200 import build
+    build.build()

@@ -1,0 +1,86 @@
+"""The C ABI without a GPU: the library builds for sm_100a, loads, exports every
+function include/qlinear.h declares, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def tcm():
+    from trellis_coded_matmul_b200 import build
+    build.build()
+    import trellis_coded_matmul_b200 as tcm
+    return tcm
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "qlinear.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlinear_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = _declared()
+    for n in ("qlinear_create", "qlinear_create_mixed", "qlinear_forward", "qlinear_decode",
+              "qlinear_eval_code", "qlinear_get_status", "qlinear_destroy", "qlinear_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(tcm):
+    lib = ctypes.CDLL(tcm.lib_path())
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) <= set(tcm.ABI_SYMBOLS) | {n for n in _declared() if n not in tcm.ABI_SYMBOLS}
+    assert sorted(tcm.ABI_SYMBOLS) == _declared()
+
+
+def test_strerror(tcm):
+    assert tcm.qlinear_strerror(0) == "ok"
+    assert tcm.qlinear_strerror(tcm.QL_E_ARG) == "invalid argument"
+    assert tcm.qlinear_strerror(12345) == "unknown status"
+
+
+def _create(lib, tcm, m=256, n=256, k=2, L=16, V=1, kind=0, Q=0, n_words=None, alpha=1.0, out=True):
+    h = ctypes.c_void_p()
+    code = tcm.ql_code_t(kind, Q, None)
+    nw = m * n * k // 32 if n_words is None else n_words
+    return lib.qlinear_create(ctypes.byref(h) if out else None, m, n, k, L, V, code, None, nw, None, None, alpha)
+
+
+def test_create_rejects_bad_arguments_on_the_host(tcm):
+    lib = tcm.raw_library()
+    assert _create(lib, tcm, out=False) == tcm.QL_E_ARG
+    assert _create(lib, tcm, m=0) == tcm.QL_E_ARG
+    assert _create(lib, tcm, n=100) == tcm.QL_E_UNSUPPORTED          # n not a multiple of 256
+    assert _create(lib, tcm, m=40) == tcm.QL_E_UNSUPPORTED           # m not a multiple of 16
+    assert _create(lib, tcm, k=5) == tcm.QL_E_UNSUPPORTED
+    assert _create(lib, tcm, L=17) == tcm.QL_E_UNSUPPORTED
+    assert _create(lib, tcm, L=1, k=2) == tcm.QL_E_UNSUPPORTED       # L < kV
+    assert _create(lib, tcm, V=2, kind=tcm.QL_CODE_1MAD) == tcm.QL_E_UNSUPPORTED
+    assert _create(lib, tcm, kind=7) == tcm.QL_E_ARG
+    assert _create(lib, tcm, n_words=7) == tcm.QL_E_ARG
+    assert _create(lib, tcm, alpha=float("nan")) == tcm.QL_E_ARG
+    assert _create(lib, tcm, m=65536 * 2, n=256) == tcm.QL_E_UNSUPPORTED  # Hadamard block > 32768
+    # well-formed sizes but host (non-device) pointers
+    assert _create(lib, tcm) == tcm.QL_E_ARG
+
+
+def test_other_entry_points_reject_null_handles(tcm):
+    lib = tcm.raw_library()
+    assert lib.qlinear_forward(None, None, 1, None, 0, None) == tcm.QL_E_ARG
+    assert lib.qlinear_forward_host(None, None, 1, None, 0, None) == tcm.QL_E_ARG
+    assert lib.qlinear_decode(None, None, None) == tcm.QL_E_ARG
+    assert lib.qlinear_get_status(None) == tcm.QL_E_ARG
+    assert lib.qlinear_destroy(None) == tcm.QL_E_ARG
+    assert lib.qlinear_info(None, None) == tcm.QL_E_ARG
+    code = tcm.ql_code_t(0, 0, None)
+    assert lib.qlinear_eval_code(code, 17, 1, None, 4, None, None) == tcm.QL_E_ARG
+    assert lib.qlinear_eval_code(tcm.ql_code_t(1, 0, None), 16, 2, None, 4, None, None) == tcm.QL_E_UNSUPPORTED
+    mixed = lib.qlinear_create_mixed
+    h = ctypes.c_void_p()
+    assert mixed(ctypes.byref(h), 64, 256, 64, 2, 3, 16, 1, code, None, 0, None, None, 1.0) == tcm.QL_E_ARG

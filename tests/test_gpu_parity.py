@@ -1,0 +1,199 @@
+"""CUDA path against the float64 oracle, element by element, through the C ABI.
+
+Decoded weights (qlinear_decode, qlinear_eval_code) must be bit-exact with the
+oracle's fp16 rounding; layer outputs must satisfy
+max|y - y_ref| <= tol * max|y_ref| with tol = 2e-3 for batch <= 8 (fp32
+accumulation) and 5e-3 for the tensor-core path."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only hosts
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import trellis_coded_matmul_b200 as tcm  # noqa: E402
+import workloads as wl  # noqa: E402
+from oracle import codes as ocodes, fp16 as ofp16, qlinear as oq  # noqa: E402
+from gpu_util import TOL_GEMV, TOL_TC, make_handle, rel_err, sample_rows  # noqa: E402
+
+L16 = 1 << 16
+
+
+def _bits(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- codes
+@pytest.mark.parametrize("kind,fn", [(wl.CODE_1MAD, ocodes.one_mad), (wl.CODE_3INST, ocodes.three_inst)],
+                         ids=["1MAD", "3INST"])
+def test_eval_code_every_state_bit_exact(kind, fn):
+    states = torch.arange(L16, dtype=torch.int32, device="cuda")
+    got = tcm.qlinear_eval_code(kind, 16, 1, states)
+    torch.cuda.synchronize()
+    ref = ofp16.encode(fn(np.arange(L16)))
+    assert np.array_equal(_bits(got)[:, 0], ref)
+
+
+@pytest.mark.parametrize("V,Q", [(2, 9), (1, 9), (2, 6), (1, 4)])
+def test_eval_code_hyb_every_state_bit_exact(V, Q):
+    lut_np = wl.hyb_table(Q, V, 2)
+    lut = torch.from_numpy(lut_np.copy()).cuda()
+    states = torch.arange(L16, dtype=torch.int32, device="cuda")
+    got = tcm.qlinear_eval_code(wl.CODE_HYB, 16, V, states, Q=Q, lut=lut)
+    torch.cuda.synchronize()
+    ref = ofp16.encode(ocodes.hyb(np.arange(L16), lut_np))
+    assert np.array_equal(_bits(got), ref)
+
+
+def test_eval_code_odd_count_and_small_L():
+    states = torch.arange(0, 1001, dtype=torch.int32, device="cuda")
+    got = tcm.qlinear_eval_code(wl.CODE_3INST, 10, 1, states)
+    ref = ofp16.encode(ocodes.three_inst(np.arange(1001) & 1023))
+    assert np.array_equal(_bits(got)[:, 0], ref)
+
+
+# ---------------------------------------------------------------- decode
+SMALL = [
+    # m, n, k, L, V, code, extra
+    (256, 256, 2, 16, 1, wl.CODE_1MAD, {}),
+    (48, 768, 3, 16, 1, wl.CODE_3INST, {}),
+    (32, 512, 4, 16, 1, wl.CODE_1MAD, {}),
+    (16, 256, 1, 16, 1, wl.CODE_3INST, {}),
+    (64, 512, 3, 16, 2, wl.CODE_HYB, {"Q": 9}),
+    (32, 256, 1, 16, 2, wl.CODE_HYB, {"Q": 6}),
+    (32, 1024, 2, 16, 1, wl.CODE_HYB, {"Q": 5}),
+    (32, 512, 4, 16, 2, wl.CODE_HYB, {"Q": 9}),
+    (16, 256, 2, 2, 1, wl.CODE_1MAD, {}),         # L = kV: plain VQ
+    (16, 256, 2, 7, 1, wl.CODE_3INST, {}),        # short state
+    (16, 256, 3, 6, 2, wl.CODE_HYB, {"Q": 9}),    # L = kV with V = 2
+]
+
+
+def _small_layer(m, n, k, L, V, code, extra, seed=0):
+    return wl.random_layer(m, n, k, L, V, code, seed=1000 + m + n + k * 7 + L, alpha=0.5, **extra)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}_k{c[2]}_L{c[3]}_V{c[4]}_c{c[5]}")
+def test_decode_small_bit_exact(case):
+    li = _small_layer(*case)
+    h = make_handle(li)
+    w = tcm.qlinear_decode(h)
+    torch.cuda.synchronize()
+    ref = oq.Layer.from_inputs(li).decode_bits(np.arange(li.spec.m))
+    assert np.array_equal(_bits(w), ref)
+
+
+def test_decode_mixed_bit_exact():
+    li = wl.random_layer(64, 512, 0, 16, 1, wl.CODE_3INST, 5, m_top=32, k_top=2, k_bot=3)
+    h = make_handle(li)
+    w = tcm.qlinear_decode(h)
+    ref = oq.Layer.from_inputs(li).decode_bits(np.arange(64))
+    assert np.array_equal(_bits(w), ref)
+
+
+# ---------------------------------------------------------------- forward
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}_k{c[2]}_L{c[3]}_V{c[4]}_c{c[5]}")
+@pytest.mark.parametrize("batch", [1, 3, 8])
+def test_forward_small(case, batch):
+    li = _small_layer(*case)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=3)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_GEMV
+
+
+@pytest.mark.parametrize("batch", [9, 16, 33])
+def test_forward_larger_batches(batch):
+    li = _small_layer(*SMALL[1])
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=4)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_TC
+
+
+def test_forward_fp16_output_and_zero_batch():
+    li = _small_layer(*SMALL[0])
+    h = make_handle(li)
+    x = wl.make_x(li.spec, 2, instance=5)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda(), out_dtype=torch.float16)
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert y.dtype == torch.float16
+    assert rel_err(y.float().cpu().numpy(), y_ref) <= TOL_GEMV + 2.0 ** -11
+    empty = torch.empty((0, li.spec.n), dtype=torch.float16, device="cuda")
+    assert tcm.qlinear_forward(h, empty).shape == (0, li.spec.m)
+
+
+def test_forward_host_buffers():
+    li = _small_layer(*SMALL[4])
+    h = make_handle(li)
+    x = torch.from_numpy(wl.make_x(li.spec, 4, instance=6)).pin_memory()
+    y = tcm.qlinear_forward_host(h, x)
+    assert not y.is_cuda
+    y_ref = oq.Layer.from_inputs(li).forward(x.numpy())
+    assert rel_err(y.numpy(), y_ref) <= TOL_GEMV
+
+
+def test_forward_mixed_small():
+    li = wl.random_layer(64, 512, 0, 16, 1, wl.CODE_3INST, 5, m_top=32, k_top=2, k_bot=3)
+    h = make_handle(li)
+    for batch in (1, 8, 20):
+        x = wl.make_x(li.spec, batch, instance=7)
+        y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+        tol = TOL_GEMV if batch <= 8 else TOL_TC
+        assert rel_err(y.cpu().numpy(), oq.Layer.from_inputs(li).forward(x)) <= tol
+
+
+def test_bad_signs_are_rejected():
+    li = _small_layer(*SMALL[0])
+    li.s_in[5] = 0
+    with pytest.raises(tcm.QLinearError) as e:
+        make_handle(li)
+    assert e.value.status == tcm.QL_E_ARG
+
+
+def test_info_reports_the_bit_accounting():
+    li = wl.make_layer(wl.WORKLOADS["mlp_up"])
+    h = make_handle(li)
+    info = tcm.qlinear_info(h)
+    sp = li.spec
+    assert info["stream_bytes"] == sp.m * sp.n * sp.k // 8
+    assert info["sign_bytes"] * 8 >= sp.m + sp.n and info["sign_bytes"] * 8 < sp.m + sp.n + 64
+    assert info["lut_bytes"] == 2048
+    assert (info["B_n"], info["B_m"]) == (4096, 256)
+
+
+# ---------------------------------------------------------------- full-size workloads
+FULL = [("tiny", 1), ("attn4096", 1), ("mlp_up", 8), ("mlp_down", 4), ("large", 4), ("large", 16),
+        ("halftcq", 64), ("halftcq", 256)]
+
+
+@pytest.mark.parametrize("name", ["tiny", "attn4096", "mlp_up", "mlp_down", "large", "halftcq"])
+def test_full_decode_sampled_rows_bit_exact(name):
+    sp = wl.WORKLOADS[name]
+    li = wl.make_layer(sp)
+    h = make_handle(li)
+    w = tcm.qlinear_decode(h)
+    rng = np.random.default_rng(42)
+    rows = np.unique(np.concatenate([[0, sp.m - 1], rng.integers(0, sp.m, 10),
+                                     [sp.m_top - 1, sp.m_top] if sp.mixed else []])).astype(np.int64)
+    ref = oq.Layer.from_inputs(li).decode_bits(rows)
+    got = _bits(w[torch.from_numpy(rows).cuda()])
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name,batch", FULL, ids=lambda v: str(v))
+def test_full_forward_sampled_outputs(name, batch):
+    sp = wl.WORKLOADS[name]
+    li = wl.make_layer(sp)
+    h = make_handle(li)
+    x = wl.make_x(sp, batch)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda()).cpu().numpy()
+    layer = oq.Layer.from_inputs(li)
+    rows = sample_rows(sp.m, layer.B_m, 1 if layer.B_m >= 4096 else 3, seed=batch)
+    y_ref = layer.forward_rows(x, rows)
+    tol = TOL_GEMV if batch <= 8 else TOL_TC
+    assert rel_err(y[:, rows], y_ref) <= tol

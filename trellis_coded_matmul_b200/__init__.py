@@ -1,0 +1,232 @@
+"""Python binding of libqlinear.so (include/qlinear.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module turns
+torch tensors into pointers and status codes into exceptions.  It has no
+fallback: if libqlinear.so is missing the import fails, and every call needs
+CUDA tensors on the device the handle was created on.
+
+    import trellis_coded_matmul_b200 as tcm
+    h = tcm.qlinear_create(m, n, k, L, V, tcm.QL_CODE_3INST, codes, s_in, s_out, alpha)
+    y = tcm.qlinear_forward(h, x)            # x: cuda fp16 [batch, n] -> y fp32 [batch, m]
+    tcm.qlinear_destroy(h)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m trellis_coded_matmul_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+QL_OK = 0
+QL_E_ARG = -1
+QL_E_UNSUPPORTED = -2
+QL_E_CUDA = -3
+QL_E_OOM = -4
+QL_E_TIMEOUT = -5
+QL_E_DEVICE = -6
+QL_CODE_1MAD = 0
+QL_CODE_3INST = 1
+QL_CODE_HYB = 2
+QL_F32 = 0
+QL_F16 = 1
+
+# Every function include/qlinear.h declares (checked by the CPU tests).
+ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_forward", "qlinear_forward_host",
+               "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
+               "qlinear_destroy", "qlinear_strerror")
+
+
+class ql_code_t(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("Q", ctypes.c_int), ("lut", ctypes.c_void_p)]
+
+
+class ql_info_t(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int) for f in ("m", "n", "L", "V", "code", "Q", "k_top", "k_bot", "m_top", "B_n", "B_m")] + \
+               [(f, ctypes.c_size_t) for f in ("stream_bytes", "sign_bytes", "lut_bytes", "scratch_bytes")]
+
+
+_vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+_lib.qlinear_create.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, ql_code_t, _vp, _sz, _vp, _vp, _f]
+_lib.qlinear_create_mixed.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _i, _i, ql_code_t, _vp, _sz, _vp,
+                                      _vp, _f]
+_lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
+_lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
+_lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
+_lib.qlinear_eval_code.argtypes = [ql_code_t, _i, _i, _vp, _i, _vp, _vp]
+_lib.qlinear_get_status.argtypes = [_vp]
+_lib.qlinear_info.argtypes = [_vp, ctypes.POINTER(ql_info_t)]
+_lib.qlinear_destroy.argtypes = [_vp]
+_lib.qlinear_strerror.argtypes = [_i]
+_lib.qlinear_strerror.restype = ctypes.c_char_p
+for _name in ABI_SYMBOLS:
+    if _name != "qlinear_strerror":
+        getattr(_lib, _name).restype = _i
+
+
+class QLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {qlinear_strerror(status)} ({status})")
+        self.status = status
+
+
+def qlinear_strerror(status: int) -> str:
+    return _lib.qlinear_strerror(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != QL_OK:
+        raise QLinearError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _cuda(t, name, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} must have dtype {dtype}")
+    return t
+
+
+class QLinearHandle:
+    """Owns a qlinear_t; destroyed explicitly or when garbage-collected."""
+
+    def __init__(self, ptr: int, m: int, n: int):
+        self.ptr = ptr
+        self.m = m
+        self.n = n
+
+    def __del__(self):
+        if getattr(self, "ptr", None):
+            try:
+                _lib.qlinear_destroy(self.ptr)
+            except Exception:
+                pass
+            self.ptr = None
+
+
+def _code(kind: int, Q: int = 0, lut=None) -> ql_code_t:
+    if lut is not None:
+        import torch
+        _cuda(lut, "lut", torch.float16)
+    return ql_code_t(kind, Q, _ptr(lut))
+
+
+def qlinear_create(m, n, k, L, V, kind, codes, s_in, s_out, alpha, Q=0, lut=None) -> QLinearHandle:
+    """codes: CUDA uint32/int32 [m*n*k/32]; s_in, s_out: CUDA int8 +-1; lut: CUDA fp16 [2^Q, V] (HYB)."""
+    import torch
+    _cuda(codes, "codes", (torch.int32, torch.uint32))
+    _cuda(s_in, "s_in", torch.int8)
+    _cuda(s_out, "s_out", torch.int8)
+    out = _vp()
+    _check(_lib.qlinear_create(ctypes.byref(out), m, n, k, L, V, _code(kind, Q, lut), _ptr(codes), codes.numel(),
+                               _ptr(s_in), _ptr(s_out), float(alpha)), "qlinear_create")
+    return QLinearHandle(out.value, m, n)
+
+
+def qlinear_create_mixed(m, n, m_top, k_top, k_bot, L, V, kind, codes, s_in, s_out, alpha, Q=0,
+                         lut=None) -> QLinearHandle:
+    import torch
+    _cuda(codes, "codes", (torch.int32, torch.uint32))
+    _cuda(s_in, "s_in", torch.int8)
+    _cuda(s_out, "s_out", torch.int8)
+    out = _vp()
+    _check(_lib.qlinear_create_mixed(ctypes.byref(out), m, n, m_top, k_top, k_bot, L, V, _code(kind, Q, lut),
+                                     _ptr(codes), codes.numel(), _ptr(s_in), _ptr(s_out), float(alpha)),
+           "qlinear_create_mixed")
+    return QLinearHandle(out.value, m, n)
+
+
+def qlinear_forward(h: QLinearHandle, x, y=None, out_dtype=None, stream=None):
+    """x: CUDA fp16 [batch, n] -> y [batch, m] (fp32 unless out_dtype/y says fp16)."""
+    import torch
+    _cuda(x, "x", torch.float16)
+    batch = x.shape[0] if x.dim() == 2 else 0
+    if x.dim() != 2 or x.shape[1] != h.n:
+        raise ValueError("x must be [batch, n]")
+    if y is None:
+        y = torch.empty((batch, h.m), dtype=out_dtype or torch.float32, device=x.device)
+    _cuda(y, "y", (torch.float32, torch.float16))
+    if tuple(y.shape) != (batch, h.m):
+        raise ValueError("y must be [batch, m]")
+    ydt = QL_F16 if y.dtype == torch.float16 else QL_F32
+    _check(_lib.qlinear_forward(h.ptr, _ptr(x), batch, _ptr(y), ydt, _stream(stream)), "qlinear_forward")
+    return y
+
+
+def qlinear_forward_host(h: QLinearHandle, x, y=None, out_dtype=None, stream=None):
+    """x: CPU fp16 [batch, n] (pinned for asynchronous copies) -> y CPU [batch, m]; returns when y is ready."""
+    import torch
+    if x.is_cuda or x.dtype != torch.float16 or not x.is_contiguous() or x.dim() != 2 or x.shape[1] != h.n:
+        raise ValueError("x must be a contiguous CPU fp16 tensor [batch, n]")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, h.m), dtype=out_dtype or torch.float32, pin_memory=x.is_pinned())
+    if y.is_cuda or tuple(y.shape) != (batch, h.m) or y.dtype not in (torch.float32, torch.float16):
+        raise ValueError("y must be a CPU fp32/fp16 tensor [batch, m]")
+    ydt = QL_F16 if y.dtype == torch.float16 else QL_F32
+    _check(_lib.qlinear_forward_host(h.ptr, _ptr(x), batch, _ptr(y), ydt, _stream(stream)), "qlinear_forward_host")
+    return y
+
+
+def qlinear_decode(h: QLinearHandle, w_hat=None, stream=None):
+    """W_hat as CUDA fp16 [m, n] (code values before alpha, signs and transforms)."""
+    import torch
+    if w_hat is None:
+        w_hat = torch.empty((h.m, h.n), dtype=torch.float16, device="cuda")
+    _cuda(w_hat, "w_hat", torch.float16)
+    _check(_lib.qlinear_decode(h.ptr, _ptr(w_hat), _stream(stream)), "qlinear_decode")
+    return w_hat
+
+
+def qlinear_eval_code(kind, L, V, states, Q=0, lut=None, out=None, stream=None):
+    """states: CUDA uint32/int32 [count] -> fp16 [count, V]."""
+    import torch
+    _cuda(states, "states", (torch.int32, torch.uint32))
+    if out is None:
+        out = torch.empty((states.numel(), V), dtype=torch.float16, device=states.device)
+    _check(_lib.qlinear_eval_code(_code(kind, Q, lut), L, V, _ptr(states), states.numel(), _ptr(out),
+                                  _stream(stream)), "qlinear_eval_code")
+    return out
+
+
+def qlinear_get_status(h: QLinearHandle) -> int:
+    return _lib.qlinear_get_status(h.ptr)
+
+
+def qlinear_info(h: QLinearHandle) -> dict:
+    info = ql_info_t()
+    _check(_lib.qlinear_info(h.ptr, ctypes.byref(info)), "qlinear_info")
+    return {f: getattr(info, f) for f, _ in ql_info_t._fields_}
+
+
+def qlinear_destroy(h: QLinearHandle) -> None:
+    if h.ptr:
+        _check(_lib.qlinear_destroy(h.ptr), "qlinear_destroy")
+        h.ptr = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def raw_library():
+    """The ctypes handle of libqlinear.so (for tests that call the ABI directly)."""
+    return _lib

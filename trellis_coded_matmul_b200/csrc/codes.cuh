@@ -1,0 +1,113 @@
+// codes.cuh -- device-side trellis window extraction and the three codes.
+//
+// The codes (QTIP OpenReview discussion: "Inference speed analysis (W2)", the
+// comment on HYB cost, "HYB Uniqueness (Q2)", "Bit Accounting (Q2)"):
+//   1MAD : x = A*s + B; value = fp16(C1 * (byte0 + byte1 + byte2 + byte3 - 510))
+//   3INST: x = A*s + B; m = (x & MASK) ^ XOR; value = fp16(half(m.lo) + half(m.hi))
+//   HYB  : x = A*s + B; entry = lut[x >> (32 - Q)]; bit 15 of x negates value 0
+// Every value is rounded to fp16 exactly once:
+//   * 1MAD: the byte sum is produced directly as the fp16 bit pattern of
+//     1536 + d (one dp4a whose accumulator is 0x6400 + 512 - 510; the
+//     pattern 0x6400 + t is the half 1024 + t for 0 <= t < 1024), then one
+//     half-precision FMA computes (1536 + d)*C1 - 1536*C1 = d*C1 with a single
+//     rounding.  C1 = 443 * 2^-16 has 9 significant bits, so C1 and 1536*C1
+//     are exact halves.
+//   * 3INST: the two halves are finite normal halves; one fp16 add rounds once.
+//   * HYB: no arithmetic on values, only a sign-bit xor.
+// The constants are part of the stream format; they were chosen by a seeded
+// search against the statistical properties the discussion states for the
+// codes (approximately N(0,1) at L = 16, successors of a state decorrelated).
+#pragma once
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace qlk {
+
+constexpr int kCode1MAD = 0;
+constexpr int kCode3INST = 1;
+constexpr int kCodeHYB = 2;
+
+constexpr uint32_t kA1MAD = 0x61616D4Bu, kB1MAD = 0xE29B5692u;
+constexpr uint32_t kA3INST = 0x6C9FB67Bu, kB3INST = 0xA1E8CAB9u;
+constexpr uint32_t kMask3INST = 0x9CFF8FFFu, kXor3INST = 0x20003000u;
+constexpr uint32_t kAHYB = 0xBB6071B9u, kBHYB = 0x989D49ADu;
+
+// 3INST masks applied after regrouping two states' low halves (resp. high
+// halves) into one register: the low-half mask/xor in both halves, and the
+// high-half mask/xor in both halves.
+constexpr uint32_t kMask3Lo2 = (kMask3INST & 0xFFFFu) * 0x10001u;
+constexpr uint32_t kXor3Lo2 = (kXor3INST & 0xFFFFu) * 0x10001u;
+constexpr uint32_t kMask3Hi2 = (kMask3INST >> 16) * 0x10001u;
+constexpr uint32_t kXor3Hi2 = (kXor3INST >> 16) * 0x10001u;
+
+// 1MAD constants as half2 bit patterns: C1 = 443*2^-16 = 0x1EEC, -1536*C1 = -10.3828125 = 0xC931.
+constexpr uint32_t kC1x2 = 0x1EEC1EECu;
+constexpr uint32_t kNegBiasC1x2 = 0xC931C931u;
+constexpr uint32_t kDp4aAcc = 0x6600u - 510u;
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Two V=1 states -> their two fp16 values packed (state a in the low half).
+template <int CODE>
+__device__ __forceinline__ uint32_t code_pair(uint32_t sa, uint32_t sb, const uint32_t* lut_lane, int qshift);
+
+template <>
+__device__ __forceinline__ uint32_t code_pair<kCode1MAD>(uint32_t sa, uint32_t sb, const uint32_t*, int) {
+    uint32_t xa = kA1MAD * sa + kB1MAD;
+    uint32_t xb = kA1MAD * sb + kB1MAD;
+    uint32_t ra = __dp4a(xa, 0x01010101u, kDp4aAcc);
+    uint32_t rb = __dp4a(xb, 0x01010101u, kDp4aAcc);
+    return hfma2_u32(__byte_perm(ra, rb, 0x5410), kC1x2, kNegBiasC1x2);
+}
+
+template <>
+__device__ __forceinline__ uint32_t code_pair<kCode3INST>(uint32_t sa, uint32_t sb, const uint32_t*, int) {
+    uint32_t xa = kA3INST * sa + kB3INST;
+    uint32_t xb = kA3INST * sb + kB3INST;
+    uint32_t lo = (__byte_perm(xa, xb, 0x5410) & kMask3Lo2) ^ kXor3Lo2;
+    uint32_t hi = (__byte_perm(xa, xb, 0x7632) & kMask3Hi2) ^ kXor3Hi2;
+    return hadd2_u32(lo, hi);
+}
+
+// HYB with V = 1: table words hold the fp16 value in their low half.  The
+// table is replicated per lane in shared memory: entry i of lane l is word
+// i*32 + l, so 32 lanes with arbitrary indices never share a bank.
+template <>
+__device__ __forceinline__ uint32_t code_pair<kCodeHYB>(uint32_t sa, uint32_t sb, const uint32_t* lut_lane, int qshift) {
+    uint32_t xa = kAHYB * sa + kBHYB;
+    uint32_t xb = kAHYB * sb + kBHYB;
+    uint32_t ea = lut_lane[(xa >> qshift) * 32u] ^ (xa & 0x8000u);
+    uint32_t eb = lut_lane[(xb >> qshift) * 32u] ^ (xb & 0x8000u);
+    return __byte_perm(ea, eb, 0x5410);
+}
+
+// HYB with V = 2: one state -> one table word (value 0 low, value 1 high).
+__device__ __forceinline__ uint32_t code_hyb_v2(uint32_t s, const uint32_t* lut_lane, int qshift) {
+    uint32_t x = kAHYB * s + kBHYB;
+    return lut_lane[(x >> qshift) * 32u] ^ (x & 0x8000u);
+}
+
+// 16-bit window of a thread-row's bit string ending at bit `end` (compile-time
+// after unrolling).  cw[0] holds the 32 bits before the thread's own range,
+// cw[1..] its own words, most significant bit first.  The L-bit state is the
+// low L bits of this window (callers mask with (1 << L) - 1).
+template <int NW>
+__device__ __forceinline__ uint32_t window16(const uint32_t (&cw)[NW], int end) {
+    const int start = end - 16;
+    const int a = start >> 5;
+    const int o = start & 31;
+    if (o <= 16) return cw[a] >> (16 - o);
+    return __funnelshift_r(cw[a + 1], cw[a], 48 - o);
+}
+
+}  // namespace qlk

@@ -1,0 +1,386 @@
+// gemv.cu -- fused trellis decode + matrix-vector product for batch <= 8, and
+// the decode / eval_code test kernels built on the same device functions.
+//
+// Decode follows the QTIP discussion: the bitshift trellis makes every state
+// a window of the stored bits, so a lane can decode any run of steps on its
+// own ("the bitshift trellis also enables parallel decoding"), and the codes
+// are computed in INT32 ALU (1MAD, 3INST) or with a small table in banked
+// shared memory (HYB).  Decoded weights stay in registers: they are the A
+// operand of m16n8k16 half-precision MMAs whose B operand is x' (batch padded
+// to 8 columns) and whose fp32 accumulators hold 16 rows x 8 batch columns.
+//
+// Work split: the m x n matrix is a grid of units (16 rows x 256 columns).
+// Units are numbered row-tile-major; every warp of the grid takes one
+// contiguous, equally sized range of units, accumulates while the row tile is
+// unchanged and adds its partial sums into z with atomics when it moves on.
+// The k-slot order inside an MMA is free (both operands use it): lane c
+// feeds its own 4 consecutive columns per MMA, so every lane walks a
+// contiguous run of trellis steps and the matching x' values are one 8-byte
+// load (see the fragment layout in rht.cu).
+#include <cuda_fp16.h>
+
+#include "codes.cuh"
+#include "internal.h"
+#include "layout.cuh"
+
+namespace qlk {
+
+struct DecodeArgs {
+    const uint32_t* words;  // part's words, kernel layout
+    int rt;                 // row tiles in the part
+    int nb;                 // blocks per row
+    uint32_t lmask;         // (1 << L) - 1
+    int qshift;             // HYB: 32 - Q
+    const uint32_t* lut;    // HYB: 2^Q words in global memory
+    int lut_entries;
+};
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const uint32_t* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint2 ldg_stream_v2(const uint32_t* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
+// Load lane's two thread-rows of one unit into w[h][0 .. 2K-1].
+template <int K>
+__device__ __forceinline__ void load_unit(uint32_t (&w)[2][2 * K], const uint32_t* unit_base, int lane) {
+    using UL = UnitLayout<K>;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int q = 0; q < UL::NV; ++q) {
+            const uint32_t* p = unit_base + ((h * UL::NV + q) * 32 + lane) * UL::VW;
+            if (UL::VW == 4) {
+                const uint4 v = ldg_stream_v4(p);
+                w[h][q * 4 + 0] = v.x;
+                w[h][q * 4 + 1] = v.y;
+                w[h][q * 4 + 2] = v.z;
+                w[h][q * 4 + 3] = v.w;
+            } else {
+                const uint2 v = ldg_stream_v2(p);
+                w[h][q * 2 + 0] = v.x;
+                w[h][q * 2 + 1] = v.y;
+            }
+        }
+    }
+}
+
+// Fill the per-lane replicated HYB table in shared memory.
+__device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lut, int entries) {
+    for (int i = threadIdx.x; i < entries * 32; i += blockDim.x) smem[i] = lut[i >> 5];
+}
+
+// The four A-operand registers of MMA number u (0..15) of a unit:
+//   a[0] = row g,     columns 4u, 4u+1 of the lane's run    a[2] = row g,     columns 4u+2, 4u+3
+//   a[1] = row g + 8, columns 4u, 4u+1                       a[3] = row g + 8, columns 4u+2, 4u+3
+// cw[h] holds the 32 bits before the lane's run of thread-row h, then its 2K words.
+template <int CODE, int K, int V>
+__device__ __forceinline__ void decode_mma_operand(uint32_t (&a)[4], const uint32_t (&cw)[2][2 * K + 1], int u,
+                                                   uint32_t lmask, const uint32_t* lut_lane, int qshift) {
+    constexpr int kV = K * V;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (V == 1) {
+            const uint32_t s0 = window16(cw[h], 32 + (4 * u + 1) * kV) & lmask;
+            const uint32_t s1 = window16(cw[h], 32 + (4 * u + 2) * kV) & lmask;
+            const uint32_t s2 = window16(cw[h], 32 + (4 * u + 3) * kV) & lmask;
+            const uint32_t s3 = window16(cw[h], 32 + (4 * u + 4) * kV) & lmask;
+            a[h] = code_pair<CODE>(s0, s1, lut_lane, qshift);
+            a[2 + h] = code_pair<CODE>(s2, s3, lut_lane, qshift);
+        } else {
+            const uint32_t s0 = window16(cw[h], 32 + (2 * u + 1) * kV) & lmask;
+            const uint32_t s1 = window16(cw[h], 32 + (2 * u + 2) * kV) & lmask;
+            a[h] = code_hyb_v2(s0, lut_lane, qshift);
+            a[2 + h] = code_hyb_v2(s1, lut_lane, qshift);
+        }
+    }
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+struct GemvArgs {
+    DecodeArgs dec;
+    const uint2* xf;  // x' fragment layout
+    int batch;        // 1..8
+    float* z;         // [batch][m]
+    int m;
+    int row0;         // first layer row of the part
+};
+
+template <int CODE, int K, int V>
+__global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
+    extern __shared__ uint32_t lut_smem[];
+    using UL = UnitLayout<K>;
+    const int lane = threadIdx.x & 31;
+    if (CODE == kCodeHYB) {
+        fill_lut_smem(lut_smem, p.dec.lut, p.dec.lut_entries);
+        __syncthreads();
+    }
+    const uint32_t* lut_lane = lut_smem + lane;
+    const int wpb = blockDim.x >> 5;
+    const long long nwarps = (long long)gridDim.x * wpb;
+    const long long gw = (long long)blockIdx.x * wpb + (threadIdx.x >> 5);
+    const int nb = p.dec.nb;
+    const long long U = (long long)p.dec.rt * nb;
+    const long long u0 = U * gw / nwarps, u1 = U * (gw + 1) / nwarps;
+    if (u0 >= u1) return;
+
+    const int g = lane >> 2, c = lane & 3;
+    const int src_lane = (lane & ~3) | ((c + 3) & 3);
+    const int batch = p.batch;
+
+    uint32_t nxt[2][2 * K];
+    load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int R = (int)(u0 / nb), j = (int)(u0 % nb);
+    int curR = R;
+
+    auto flush = [&](int tile) {
+        const int row = p.row0 + tile * kRowTile + g;
+        const int b0 = 2 * c, b1 = 2 * c + 1;
+        if (b0 < batch) {
+            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
+            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
+        }
+        if (b1 < batch) {
+            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
+            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
+        }
+    };
+
+    for (long long unit = u0; unit < u1; ++unit) {
+        uint32_t cw[2][2 * K + 1];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int w = 0; w < 2 * K; ++w) cw[h][w + 1] = nxt[h][w];
+        if (unit + 1 < u1) load_unit<K>(nxt, p.dec.words + (unit + 1) * UL::UW, lane);
+        if (R != curR) {
+            flush(curR);
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            curR = R;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
+
+        const uint2* xb = p.xf + (size_t)j * 16 * batch * 4 + g * 4 + c;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            uint32_t a[4];
+            decode_mma_operand<CODE, K, V>(a, cw, u, p.dec.lmask, lut_lane, p.dec.qshift);
+            uint2 bv = make_uint2(0u, 0u);
+            if (g < batch) bv = __ldg(xb + (size_t)u * batch * 4);
+            mma_16816(acc, a, bv.x, bv.y);
+        }
+        if (++j == nb) {
+            j = 0;
+            ++R;
+        }
+    }
+    flush(curR);
+}
+
+// ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
+template <int CODE, int K, int V>
+__global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
+    extern __shared__ uint32_t lut_smem[];
+    using UL = UnitLayout<K>;
+    const int lane = threadIdx.x & 31;
+    if (CODE == kCodeHYB) {
+        fill_lut_smem(lut_smem, p.lut, p.lut_entries);
+        __syncthreads();
+    }
+    const uint32_t* lut_lane = lut_smem + lane;
+    const int g = lane >> 2, c = lane & 3;
+    const int src_lane = (lane & ~3) | ((c + 3) & 3);
+    const long long U = (long long)p.rt * p.nb;
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); unit < U;
+         unit += nwarps) {
+        uint32_t w[2][2 * K];
+        load_unit<K>(w, p.words + unit * UL::UW, lane);
+        uint32_t cw[2][2 * K + 1];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = w[h][i];
+            cw[h][0] = __shfl_sync(0xffffffffu, w[h][2 * K - 1], src_lane);
+        }
+        const int R = (int)(unit / p.nb), j = (int)(unit % p.nb);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            uint32_t a[4];
+            decode_mma_operand<CODE, K, V>(a, cw, u, p.lmask, lut_lane, p.qshift);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const size_t row = (size_t)row0 + R * kRowTile + 8 * h + g;
+                uint2* dst = (uint2*)(w_hat + row * n + (size_t)j * kT + 64 * c + 4 * u);
+                *dst = make_uint2(a[h], a[2 + h]);
+            }
+        }
+    }
+}
+
+// ---- qlinear_eval_code ----
+template <int CODE, int V>
+__global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count, uint32_t lmask, int qshift,
+                                 const uint32_t* __restrict__ lut, int lut_entries, __half* __restrict__ out) {
+    extern __shared__ uint32_t lut_smem[];
+    const int lane = threadIdx.x & 31;
+    if (CODE == kCodeHYB) {
+        fill_lut_smem(lut_smem, lut, lut_entries);
+        __syncthreads();
+    }
+    const uint32_t* lut_lane = lut_smem + lane;
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (V == 2) {
+        if (t < count) ((uint32_t*)out)[t] = code_hyb_v2(states[t] & lmask, lut_lane, qshift);
+    } else {
+        const int i0 = 2 * t;
+        if (i0 >= count) return;
+        const uint32_t s0 = states[i0] & lmask;
+        const uint32_t s1 = (i0 + 1 < count) ? (states[i0 + 1] & lmask) : s0;
+        const uint32_t pr = code_pair<CODE>(s0, s1, lut_lane, qshift);
+        const unsigned short* hv = (const unsigned short*)&pr;
+        ((unsigned short*)out)[i0] = hv[0];
+        if (i0 + 1 < count) ((unsigned short*)out)[i0 + 1] = hv[1];
+    }
+}
+
+// ---- dispatch ----
+template <template <int, int, int> class F, typename... Args>
+static cudaError_t dispatch(int code, int k, int V, Args&&... args) {
+    if (code == kCode1MAD && V == 1) {
+        switch (k) {
+            case 1: return F<kCode1MAD, 1, 1>::run(args...);
+            case 2: return F<kCode1MAD, 2, 1>::run(args...);
+            case 3: return F<kCode1MAD, 3, 1>::run(args...);
+            case 4: return F<kCode1MAD, 4, 1>::run(args...);
+        }
+    } else if (code == kCode3INST && V == 1) {
+        switch (k) {
+            case 1: return F<kCode3INST, 1, 1>::run(args...);
+            case 2: return F<kCode3INST, 2, 1>::run(args...);
+            case 3: return F<kCode3INST, 3, 1>::run(args...);
+            case 4: return F<kCode3INST, 4, 1>::run(args...);
+        }
+    } else if (code == kCodeHYB && V == 1) {
+        switch (k) {
+            case 1: return F<kCodeHYB, 1, 1>::run(args...);
+            case 2: return F<kCodeHYB, 2, 1>::run(args...);
+            case 3: return F<kCodeHYB, 3, 1>::run(args...);
+            case 4: return F<kCodeHYB, 4, 1>::run(args...);
+        }
+    } else if (code == kCodeHYB && V == 2) {
+        switch (k) {
+            case 1: return F<kCodeHYB, 1, 2>::run(args...);
+            case 2: return F<kCodeHYB, 2, 2>::run(args...);
+            case 3: return F<kCodeHYB, 3, 2>::run(args...);
+            case 4: return F<kCodeHYB, 4, 2>::run(args...);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+static DecodeArgs make_decode_args(const Layer& L, const Part& part) {
+    DecodeArgs d;
+    d.words = L.words + part.word_off;
+    d.rt = part.rows / kRowTile;
+    d.nb = L.n / kT;
+    d.lmask = (1u << L.L) - 1u;
+    d.qshift = 32 - L.Q;
+    d.lut = L.lut;
+    d.lut_entries = (L.code == kCodeHYB) ? (1 << L.Q) : 0;
+    return d;
+}
+
+template <int CODE, int K, int V>
+struct GemvLaunch {
+    static cudaError_t run(const GemvArgs& a, int grid, cudaStream_t st) {
+        const size_t smem = (size_t)a.dec.lut_entries * 32 * 4;
+        auto kern = gemv_kernel<CODE, K, V>;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<grid, 256, smem, st>>>(a);
+        return cudaGetLastError();
+    }
+};
+
+cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, int batch, float* z,
+                        cudaStream_t st) {
+    GemvArgs a;
+    a.dec = make_decode_args(L, part);
+    a.xf = (const uint2*)xp_frag;
+    a.batch = batch;
+    a.z = z;
+    a.m = L.m;
+    a.row0 = part.row0;
+    const long long units = (long long)a.dec.rt * a.dec.nb;
+    long long grid = (long long)L.num_sms * 2;
+    const long long need = (units + 7) / 8;  // at least one unit per warp
+    if (grid > need) grid = need;
+    if (grid < 1) grid = 1;
+    return dispatch<GemvLaunch>(L.code, part.k, L.V, a, (int)grid, st);
+}
+
+template <int CODE, int K, int V>
+struct DecodeLaunch {
+    static cudaError_t run(const DecodeArgs& d, __half* w, int n, int row0, int grid, cudaStream_t st) {
+        const size_t smem = (size_t)d.lut_entries * 32 * 4;
+        auto kern = decode_kernel<CODE, K, V>;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<grid, 256, smem, st>>>(d, w, n, row0);
+        return cudaGetLastError();
+    }
+};
+
+cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st) {
+    DecodeArgs d = make_decode_args(L, part);
+    const long long units = (long long)d.rt * d.nb;
+    long long grid = (units + 7) / 8;
+    if (grid > (long long)L.num_sms * 8) grid = (long long)L.num_sms * 8;
+    return dispatch<DecodeLaunch>(L.code, part.k, L.V, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
+}
+
+template <int CODE, int K, int V>
+struct EvalLaunch {
+    static cudaError_t run(const uint32_t* states, int count, uint32_t lmask, int qshift, const uint32_t* lut,
+                           int entries, __half* out, cudaStream_t st) {
+        if (K != 1) return cudaErrorInvalidValue;  // k is irrelevant to the code; one instance suffices
+        const size_t smem = (size_t)entries * 32 * 4;
+        auto kern = eval_code_kernel<CODE, V>;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        const int items = V == 2 ? count : (count + 1) / 2;
+        kern<<<(items + 255) / 256, 256, smem, st>>>(states, count, lmask, qshift, lut, entries, out);
+        return cudaGetLastError();
+    }
+};
+
+cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words, const uint32_t* states,
+                             int count, void* out, cudaStream_t st) {
+    const uint32_t lmask = (1u << L) - 1u;
+    const int entries = code == kCodeHYB ? (1 << Q) : 0;
+    return dispatch<EvalLaunch>(code, 1, V, states, count, lmask, 32 - Q, lut_words, entries, (__half*)out, st);
+}
+
+}  // namespace qlk

@@ -1,0 +1,72 @@
+// internal.h -- the handle and the kernel launchers shared by the library's .cu files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qlinear.h"
+
+namespace qlk {
+
+constexpr int kT = 256;            // columns per trellis block
+constexpr int kRowTile = 16;       // rows per decode tile (the m16n8k16 M dimension)
+constexpr int kMaxHadamard = 32768;
+
+// Device status word bits (qlinear_get_status).
+constexpr int kStatusBadSign = 1;
+constexpr int kStatusTimeout = 2;
+constexpr int kStatusBounds = 4;
+
+// One run of rows sharing a bitrate.  Its code words are stored re-laid out
+// for the decode kernels (see layout.cuh) starting at word `word_off` of the
+// handle's word buffer.
+struct Part {
+    int row0;
+    int rows;
+    int k;
+    size_t word_off;
+    size_t n_words;
+};
+
+struct Layer {
+    int device;
+    int m, n, L, V, code, Q;
+    float alpha;
+    int B_n, B_m;
+    int nparts;
+    Part parts[2];
+    uint32_t* words;      // all parts, kernel layout
+    uint32_t* sin_bits;   // bit i set <=> s_in[i] == -1
+    uint32_t* sout_bits;
+    uint32_t* lut;        // HYB: 2^Q words (V = 2: value 0 low half, value 1 high; V = 1: low half)
+    int* status;          // device status word
+    // scratch, grown on demand
+    void* xp;             // transformed input x' (fp16)
+    size_t xp_bytes;
+    float* z;             // W_hat x' before the output transform, fp32 [batch][m]
+    size_t z_bytes;
+    void* host_stage;     // device staging for qlinear_forward_host (x then y)
+    size_t host_stage_bytes;
+    int num_sms;
+};
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_relayout(const uint32_t* src, uint32_t* dst, const Part& part, int n, cudaStream_t st);
+cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* status, cudaStream_t st);
+cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
+
+// x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
+cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
+// x (fp16 [batch][n]) -> x' fp16 [batch][n] row-major.
+cudaError_t launch_rht_in_rowmajor(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
+// z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16.
+cudaError_t launch_rht_out(const Layer& L, const float* z, int batch, void* y, int y_dtype, cudaStream_t st);
+
+// z[b][row0 + r] += sum_c W_hat[row0 + r][c] x'[b][c] for the part's rows; batch <= 8.
+cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, int batch, float* z,
+                        cudaStream_t st);
+cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
+cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words,
+                             const uint32_t* states, int count, void* out, cudaStream_t st);
+
+}  // namespace qlk

@@ -1,0 +1,367 @@
+// qlinear_abi.cu -- the C ABI declared in include/qlinear.h (host side).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+using namespace qlk;
+
+struct qlinear_s {
+    Layer L;
+};
+
+namespace {
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            ok = false;
+            return;
+        }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+int is_device_pointer(const void* p) {
+    if (!p) return 0;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+int pow2_block(int d) { return d & -d; }
+
+template <typename T>
+int dev_alloc(T** p, size_t bytes) {
+    *p = nullptr;
+    if (bytes == 0) return QL_OK;
+    if (cudaMalloc((void**)p, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return QL_E_OOM;
+    }
+    return QL_OK;
+}
+
+void free_layer(Layer& L) {
+    cudaFree(L.words);
+    cudaFree(L.sin_bits);
+    cudaFree(L.sout_bits);
+    cudaFree(L.lut);
+    cudaFree(L.status);
+    cudaFree(L.xp);
+    cudaFree(L.z);
+    cudaFree(L.host_stage);
+    std::memset(&L, 0, sizeof(L));
+}
+
+int check_code(const ql_code_t& code, int V) {
+    if (code.kind == QL_CODE_1MAD || code.kind == QL_CODE_3INST) return V == 1 ? QL_OK : QL_E_UNSUPPORTED;
+    if (code.kind != QL_CODE_HYB) return QL_E_ARG;
+    if (V != 1 && V != 2) return QL_E_ARG;
+    if (code.Q < 1 || code.Q > 9) return QL_E_UNSUPPORTED;
+    if (!is_device_pointer(code.lut)) return QL_E_ARG;
+    return QL_OK;
+}
+
+// Shared by both create calls. parts: [(rows, k)].
+int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k, int L,
+                  int V, ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
+                  const int8_t* s_out, float alpha) {
+    if (!out) return QL_E_ARG;
+    *out = nullptr;
+    if (m <= 0 || n <= 0 || !std::isfinite(alpha)) return QL_E_ARG;
+    if (V != 1 && V != 2) return QL_E_ARG;
+    if (n % kT != 0 || m % kRowTile != 0) return QL_E_UNSUPPORTED;
+    if (pow2_block(n) > kMaxHadamard || pow2_block(m) > kMaxHadamard) return QL_E_UNSUPPORTED;
+    size_t expect_words = 0;
+    for (int i = 0; i < nparts; ++i) {
+        const int k = part_k[i];
+        if (k < 1 || k > 4) return QL_E_UNSUPPORTED;
+        if (L < k * V || L > 16) return QL_E_UNSUPPORTED;
+        if (part_rows[i] <= 0 || part_rows[i] % kRowTile != 0) return QL_E_ARG;
+        expect_words += (size_t)part_rows[i] * n * k / 32;
+    }
+    if (n_words != expect_words) return QL_E_ARG;
+    int rc = check_code(code, V);
+    if (rc != QL_OK) return rc;
+    if (!is_device_pointer(packed_codes) || !is_device_pointer(s_in) || !is_device_pointer(s_out))
+        return QL_E_ARG;
+
+    qlinear_s* h = new (std::nothrow) qlinear_s;
+    if (!h) return QL_E_OOM;
+    std::memset(&h->L, 0, sizeof(Layer));
+    Layer& Ly = h->L;
+    cudaGetDevice(&Ly.device);
+    cudaDeviceGetAttribute(&Ly.num_sms, cudaDevAttrMultiProcessorCount, Ly.device);
+    Ly.m = m;
+    Ly.n = n;
+    Ly.L = L;
+    Ly.V = V;
+    Ly.code = code.kind;
+    Ly.Q = code.kind == QL_CODE_HYB ? code.Q : 0;
+    Ly.alpha = alpha;
+    Ly.B_n = pow2_block(n);
+    Ly.B_m = pow2_block(m);
+    Ly.nparts = nparts;
+    size_t off = 0;
+    int row0 = 0;
+    for (int i = 0; i < nparts; ++i) {
+        Ly.parts[i].row0 = row0;
+        Ly.parts[i].rows = part_rows[i];
+        Ly.parts[i].k = part_k[i];
+        Ly.parts[i].word_off = off;
+        Ly.parts[i].n_words = (size_t)part_rows[i] * n * part_k[i] / 32;
+        off += Ly.parts[i].n_words;
+        row0 += part_rows[i];
+    }
+
+    rc = dev_alloc(&Ly.words, n_words * 4);
+    if (rc == QL_OK) rc = dev_alloc(&Ly.sin_bits, (size_t)((n + 31) / 32) * 4);
+    if (rc == QL_OK) rc = dev_alloc(&Ly.sout_bits, (size_t)((m + 31) / 32) * 4);
+    if (rc == QL_OK) rc = dev_alloc(&Ly.status, sizeof(int));
+    if (rc == QL_OK && Ly.code == QL_CODE_HYB) rc = dev_alloc(&Ly.lut, ((size_t)1 << Ly.Q) * 4);
+    if (rc != QL_OK) {
+        free_layer(Ly);
+        delete h;
+        return rc;
+    }
+    cudaStream_t st = 0;
+    cudaError_t e = cudaMemsetAsync(Ly.status, 0, sizeof(int), st);
+    for (int i = 0; i < nparts && e == cudaSuccess; ++i)
+        e = launch_relayout(packed_codes + Ly.parts[i].word_off, Ly.words, Ly.parts[i], n, st);
+    if (e == cudaSuccess) e = launch_pack_signs(s_in, n, Ly.sin_bits, Ly.status, st);
+    if (e == cudaSuccess) e = launch_pack_signs(s_out, m, Ly.sout_bits, Ly.status, st);
+    if (e == cudaSuccess && Ly.code == QL_CODE_HYB) e = launch_copy_lut(code.lut, Ly.Q, V, Ly.lut, st);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    int status = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(&status, Ly.status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        free_layer(Ly);
+        delete h;
+        return QL_E_CUDA;
+    }
+    if (status & kStatusBadSign) {
+        free_layer(Ly);
+        delete h;
+        return QL_E_ARG;
+    }
+    *out = h;
+    return QL_OK;
+}
+
+// Grow a scratch buffer to at least `bytes`.
+int ensure(void** buf, size_t* have, size_t bytes) {
+    if (*have >= bytes) return QL_OK;
+    if (*buf) cudaFree(*buf);
+    *buf = nullptr;
+    *have = 0;
+    if (cudaMalloc(buf, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        *buf = nullptr;
+        return QL_E_OOM;
+    }
+    *have = bytes;
+    return QL_OK;
+}
+
+int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
+    const int chunk = batch < 8 ? batch : 8;
+    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)chunk * L.n * 2);
+    if (rc == QL_OK) rc = ensure((void**)&L.z, &L.z_bytes, (size_t)chunk * L.m * 4);
+    if (rc != QL_OK) return rc;
+    const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
+    for (int b0 = 0; b0 < batch; b0 += 8) {
+        const int nb = batch - b0 < 8 ? batch - b0 : 8;
+        const void* xb = (const char*)x + (size_t)b0 * L.n * 2;
+        void* yb = (char*)y + (size_t)b0 * L.m * ysz;
+        cudaError_t e = launch_rht_in_frag(L, xb, nb, L.xp, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(L.z, 0, (size_t)nb * L.m * 4, st);
+        for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) e = launch_gemv(L, L.parts[i], L.xp, nb, L.z, st);
+        if (e == cudaSuccess) e = launch_rht_out(L, L.z, nb, yb, y_dtype, st);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return QL_E_CUDA;
+        }
+    }
+    return QL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlinear_create(qlinear_t* out, int m, int n, int k, int L, int V, ql_code_t code, const uint32_t* packed_codes,
+                   size_t n_words, const int8_t* s_in, const int8_t* s_out, float alpha) {
+    const int rows[1] = {m};
+    const int ks[1] = {k};
+    return create_common(out, m, n, 1, rows, ks, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+}
+
+int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int k_bot, int L, int V,
+                         ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
+                         const int8_t* s_out, float alpha) {
+    if (!out) return QL_E_ARG;
+    *out = nullptr;
+    if (m_top <= 0 || m_top >= m) return QL_E_ARG;
+    const int rows[2] = {m_top, m - m_top};
+    const int ks[2] = {k_top, k_bot};
+    return create_common(out, m, n, 2, rows, ks, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+}
+
+int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream) {
+    if (!h || batch < 0 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
+    if (batch == 0) return QL_OK;
+    if (!x || !y) return QL_E_ARG;
+    DeviceGuard g(h->L.device);
+    if (!g.ok) return QL_E_CUDA;
+    return forward_device(h->L, x, batch, y, y_dtype, (cudaStream_t)stream);
+}
+
+int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype, void* stream) {
+    if (!h || batch < 0 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
+    if (batch == 0) return QL_OK;
+    if (!x_host || !y_host) return QL_E_ARG;
+    Layer& L = h->L;
+    DeviceGuard g(L.device);
+    if (!g.ok) return QL_E_CUDA;
+    const size_t xbytes = (size_t)batch * L.n * 2;
+    const size_t ybytes = (size_t)batch * L.m * (y_dtype == QL_F16 ? 2 : 4);
+    const size_t xoff = (ybytes + 255) / 256 * 256;
+    int rc = ensure(&L.host_stage, &L.host_stage_bytes, xoff + xbytes);
+    if (rc != QL_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* stage = (char*)L.host_stage;
+    if (cudaMemcpyAsync(stage + xoff, x_host, xbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    rc = forward_device(L, stage + xoff, batch, stage, y_dtype, st);
+    if (rc != QL_OK) return rc;
+    if (cudaMemcpyAsync(y_host, stage, ybytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    return QL_OK;
+}
+
+int qlinear_decode(qlinear_t h, void* w_hat, void* stream) {
+    if (!h || !w_hat) return QL_E_ARG;
+    DeviceGuard g(h->L.device);
+    if (!g.ok) return QL_E_CUDA;
+    for (int i = 0; i < h->L.nparts; ++i) {
+        if (launch_decode(h->L, h->L.parts[i], w_hat, (cudaStream_t)stream) != cudaSuccess) {
+            cudaGetLastError();
+            return QL_E_CUDA;
+        }
+    }
+    return QL_OK;
+}
+
+int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int count, void* out, void* stream) {
+    if (count < 0 || L < 1 || L > 16) return QL_E_ARG;
+    int rc = check_code(code, V);
+    if (rc != QL_OK) return rc;
+    if (count == 0) return QL_OK;
+    if (!states || !out) return QL_E_ARG;
+    uint32_t* lut_words = nullptr;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (code.kind == QL_CODE_HYB) {
+        if (cudaMallocAsync((void**)&lut_words, ((size_t)1 << code.Q) * 4, st) != cudaSuccess) {
+            cudaGetLastError();
+            return QL_E_OOM;
+        }
+        if (launch_copy_lut(code.lut, code.Q, V, lut_words, st) != cudaSuccess) {
+            cudaGetLastError();
+            cudaFreeAsync(lut_words, st);
+            return QL_E_CUDA;
+        }
+    }
+    cudaError_t e = launch_eval_code(code.kind, L, V, code.Q, lut_words, states, count, out, st);
+    if (lut_words) cudaFreeAsync(lut_words, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    return QL_OK;
+}
+
+int qlinear_get_status(qlinear_t h) {
+    if (!h) return QL_E_ARG;
+    DeviceGuard g(h->L.device);
+    int status = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(&status, h->L.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(h->L.status, 0, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    if (status & kStatusTimeout) return QL_E_TIMEOUT;
+    if (status) return QL_E_DEVICE;
+    return QL_OK;
+}
+
+int qlinear_info(qlinear_t h, ql_info_t* info) {
+    if (!h || !info) return QL_E_ARG;
+    const Layer& L = h->L;
+    std::memset(info, 0, sizeof(*info));
+    info->m = L.m;
+    info->n = L.n;
+    info->L = L.L;
+    info->V = L.V;
+    info->code = L.code;
+    info->Q = L.Q;
+    info->k_top = L.parts[0].k;
+    info->k_bot = L.parts[L.nparts - 1].k;
+    info->m_top = L.parts[0].rows;
+    info->B_n = L.B_n;
+    info->B_m = L.B_m;
+    size_t words = 0;
+    for (int i = 0; i < L.nparts; ++i) words += L.parts[i].n_words;
+    info->stream_bytes = words * 4;
+    info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
+    info->lut_bytes = L.code == QL_CODE_HYB ? ((size_t)1 << L.Q) * L.V * 2 : 0;
+    info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
+    return QL_OK;
+}
+
+int qlinear_destroy(qlinear_t h) {
+    if (!h) return QL_E_ARG;
+    {
+        DeviceGuard g(h->L.device);
+        cudaDeviceSynchronize();
+        free_layer(h->L);
+    }
+    delete h;
+    return QL_OK;
+}
+
+const char* qlinear_strerror(int status) {
+    switch (status) {
+        case QL_OK: return "ok";
+        case QL_E_ARG: return "invalid argument";
+        case QL_E_UNSUPPORTED: return "unsupported configuration";
+        case QL_E_CUDA: return "CUDA runtime error";
+        case QL_E_OOM: return "device allocation failed";
+        case QL_E_TIMEOUT: return "bounded device wait expired";
+        case QL_E_DEVICE: return "device-side check failed";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"
