@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Throughput of the trellis-coded quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--batch B]
+
+A step is one forward y = W x of the layer (input random-sign Hadamard
+transform, fused trellis decode + contraction, output transform) over one
+batch of synthetic inputs.  The default workload is the 2-bit 4096 x 4096
+3INST layer at batch 1.  Steps rotate through enough independent layer
+instances that their code words (4 MiB each) exceed the 126 MB L2 four times
+over, so every step streams its weights from HBM; the rotation is replayed
+from a CUDA graph.  One JSON line goes to stdout (rank 0).
+
+N > 1: one process per GPU (torchrun, NCCL process group for the barrier and
+the max-over-ranks timing only); each rank runs its own independent layer
+instances (weak scaling, no collective on the data path).
+
+--impl reference runs the float64 CPU oracle as the reference arm on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "quantized-linear tokens/s and compressed-weight HBM GB/s (% of B200 peak)"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50000)
+    p.add_argument("--warmup", type=int, default=500)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="attn4096", choices=sorted(wl.WORKLOADS))
+    p.add_argument("--batch", type=int, default=None)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    a = p.parse_args()
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def config_dict(sp, batch, n_inst, extra=None):
+    d = {"workload": f"{sp.name}: m={sp.m} n={sp.n} bits/weight={sp.bits_per_weight:g} L={sp.L} V={sp.V} "
+                     f"code={wl.CODE_NAMES[sp.code]}" + (f" Q={sp.Q}" if sp.Q else ""),
+         "global_batch": batch, "seq_len": 1, "parallelism": "independent layer instances per GPU",
+         "l2": f"inputs larger than L2: rotating {n_inst} layer instances "
+               f"({n_inst * sp.stream_bytes / 2**20:.0f} MiB of code words)"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        time.sleep(0.12)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle arms
+def _oracle_chunked(sp, batch, blocks_per_step, steps, deadline=None):
+    """Run the oracle forward in steps of `blocks_per_step` 256-column blocks of
+    W_hat (row-major order): the first step of every forward also applies the
+    input transform, the step that completes z the output transform.
+    Returns (seconds, blocks processed)."""
+    from oracle import hadamard, qlinear
+    layer = qlinear.Layer.from_inputs(wl.make_layer(sp))
+    x = wl.make_x(sp, batch)
+    nb = sp.n // 256
+    total = sp.m * nb
+    z = np.zeros((batch, sp.m))
+    xp = None
+    pos = 0
+    done = 0
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        if pos == 0:
+            xp = layer.input_transform(x)
+            z[:] = 0.0
+        left = blocks_per_step
+        while left > 0:
+            r, j0 = divmod(pos, nb)
+            j1 = min(nb, j0 + left)
+            W = layer.decode_rows([r], np.arange(j0, j1))
+            z[:, r] += xp[:, j0 * 256:j1 * 256] @ W[0]
+            left -= j1 - j0
+            pos += j1 - j0
+            done += j1 - j0
+            if pos == total:
+                y = layer.alpha * layer.s_out * hadamard.apply_blockwise(z, layer.B_m)
+                assert np.all(np.isfinite(y))
+                pos = 0
+                break
+        if deadline is not None and time.perf_counter() - t0 > deadline:
+            break
+    return time.perf_counter() - t0, done
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(sp, batch, budget_s=15.0):
+    nb = sp.n // 256
+    secs, blocks = _oracle_chunked(sp, batch, 16 * nb, steps=10**9, deadline=budget_s)
+    fwd = blocks / (sp.m * nb)
+    return {"value": batch * fwd / secs, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{blocks // nb} of {sp.m} rows of W_hat ({fwd:.3f} forwards) of {sp.name} at batch {batch}: "
+                      f"float64 trellis walk, code evaluation, dense Hadamard blocks, matrix product; "
+                      f"{secs:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sp = wl.WORKLOADS[args.workload]
+    batch = args.batch or sp.batches[0]
+    # calibrate: blocks per step so that warmup + steps fit in about two minutes
+    nb = sp.n // 256
+    t_row, _ = _oracle_chunked(sp, batch, nb, 1)
+    per_block = t_row / nb
+    budget = 120.0
+    bps = int(max(1, min(sp.m * nb, budget / max(1, args.steps + args.warmup) / per_block)))
+    _oracle_chunked(sp, batch, bps, args.warmup)
+    secs, done = _oracle_chunked(sp, batch, bps, args.steps)
+    value = batch * (done / (sp.m * nb)) / secs
+    rows = bps / nb
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(sp, batch, 1, {"step": f"{bps} blocks of 256 columns of W_hat per step "
+                                                         f"(1/{sp.m * nb / bps:g} of a forward)"}),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": f"{done} blocks of 256 columns of W_hat in {args.steps} steps of {bps}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ CUDA arm
+def _source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "trellis_coded_matmul_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_key, launch_units):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel_key)
+    if not d or d.get("source_hash") != _source_hash():
+        return None
+    return d["dram_bytes"] * launch_units / d["units"]
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 with torch.distributed.run")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import trellis_coded_matmul_b200 as tcm
+
+    def make_handle(li):
+        sp_ = li.spec
+        codes = torch.from_numpy(li.codes.view(np.int32).copy()).cuda()
+        s_in = torch.from_numpy(li.s_in.copy()).cuda()
+        s_out = torch.from_numpy(li.s_out.copy()).cuda()
+        lut = torch.from_numpy(li.lut.copy()).cuda() if li.lut is not None else None
+        if sp_.mixed:
+            return tcm.qlinear_create_mixed(sp_.m, sp_.n, sp_.m_top, sp_.k_top, sp_.k_bot, sp_.L, sp_.V, sp_.code,
+                                            codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
+        return tcm.qlinear_create(sp_.m, sp_.n, sp_.k, sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha,
+                                  Q=sp_.Q, lut=lut)
+
+    sp = wl.WORKLOADS[args.workload]
+    batch = args.batch or sp.batches[0]
+    n_inst = int(min(512, max(1, math.ceil(4 * L2_BYTES / sp.stream_bytes))))
+    handles = [make_handle(wl.make_layer(sp, instance=1 + rank * 4096 + i)) for i in range(n_inst)]
+    xs = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).cuda() for i in range(n_inst)]
+    ys = [torch.empty((batch, sp.m), dtype=torch.float32, device="cuda") for _ in range(n_inst)]
+    stream = torch.cuda.Stream()
+
+    def run_steps(count, start=0):
+        for s in range(start, start + count):
+            i = s % n_inst
+            tcm.qlinear_forward(handles[i], xs[i], ys[i])
+
+    def capture(count):
+        if count == 0:
+            return None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run_steps(count)
+        return g
+
+    with torch.cuda.stream(stream):
+        run_steps(n_inst)  # allocate per-handle scratch before capture
+    torch.cuda.synchronize()
+    g_full, g_tail, g_warm = capture(n_inst), capture(args.steps % n_inst), capture(args.warmup % n_inst)
+
+    def replay(steps, full, tail_graph):
+        for _ in range(steps // n_inst):
+            full.replay()
+        if steps % n_inst:
+            tail_graph.replay()
+
+    def timed(fn):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            fn()
+            end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return start.elapsed_time(end) * 1e-3
+
+    clocks = ClockSampler(local)
+    with torch.cuda.stream(stream):
+        replay(args.warmup, g_full, g_warm)
+    secs = timed(lambda: replay(args.steps, g_full, g_tail))
+    clk = clocks.stop()
+
+    # The decode-GEMV kernel's own duration: the same steps again, from a graph
+    # whose forwards carry CUDA events around that kernel (events between
+    # programmatically dependent launches serialise them, so this pass is
+    # separate from the throughput measurement above).
+    for h in handles:
+        tcm.qlinear_profile_enable(h, 1)
+    prof_steps = min(args.steps, 4 * n_inst)
+    g_prof = capture(n_inst)
+    g_prof_tail = capture(prof_steps % n_inst)
+    with torch.cuda.stream(stream):
+        g_prof.replay()
+    prof_secs = timed(lambda: replay(prof_steps, g_prof, g_prof_tail))
+    kern_ms, kern_n = 0.0, 0
+    for h in handles:
+        ms, n = tcm.qlinear_profile_read(h)
+        kern_ms += ms
+        kern_n += n
+        tcm.qlinear_profile_enable(h, 0)
+    kern_s = kern_ms * 1e-3 / max(1, kern_n)
+    if world > 1:
+        t = torch.tensor([secs, kern_s], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        secs, kern_s = float(t[0]), float(t[1])
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        x_h = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).pin_memory() for i in range(4)]
+        y_h = [torch.empty((batch, sp.m), dtype=torch.float32).pin_memory() for _ in range(4)]
+        e2e_steps = min(args.steps, 2000)
+        with torch.cuda.stream(stream):
+            for s in range(8):
+                tcm.qlinear_forward_host(handles[s % n_inst], x_h[s % 4], y_h[s % 4], stream=stream)
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        es.record(stream)
+        for s in range(e2e_steps):
+            tcm.qlinear_forward_host(handles[s % n_inst], x_h[s % 4], y_h[s % 4], stream=stream)
+        ee.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = es.elapsed_time(ee) * 1e-3
+        if world > 1:
+            t = torch.tensor([e2e_s], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = float(t[0])
+        e2e = {"value": world * e2e_steps * batch / e2e_s, "unit": "tokens/s",
+               "h2d_bytes_per_step": batch * sp.n * 2, "d2h_bytes_per_step": batch * sp.m * 4,
+               "steps": e2e_steps}
+
+    line = None
+    if rank == 0:
+        pk, pk_kind = peaks()
+        alg_bytes = sp.stream_bytes + batch * sp.n * 2 + batch * sp.m * 4
+        achieved = alg_bytes / kern_s / 1e9
+        value = world * args.steps * batch / secs
+        launches_per_step = 2 + len(sp.row_parts())
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+                "config": config_dict(sp, batch, n_inst),
+                "hbm_gbs_step": sp.stream_bytes * args.steps * world / secs / 1e9,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": achieved / pk["hbm_gbs"], "traffic": _traffic("gemv_" + sp.name, 1),
+                             "kernel": "gemv_kernel (fused trellis decode + m16n8k16 MMA)",
+                             "kernel_us": kern_s * 1e6, "peak_kind": pk_kind,
+                             "alg_bytes_per_launch": alg_bytes,
+                             "timing": f"CUDA events around the kernel in a replay of {prof_steps} steps "
+                                       f"({prof_secs / prof_steps * 1e6:.2f} us/step with the events)"},
+                "gpu_launches": launches_per_step * args.steps,
+                "clocks": clk, "e2e": e2e}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(sp, batch)
+        print(json.dumps(line), flush=True)
+    for h in handles:
+        tcm.qlinear_destroy(h)
+    del g_full, g_tail, g_warm, g_prof, g_prof_tail
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", "29517", __file__] + sys.argv[1:]
+        return subprocess.call(cmd)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

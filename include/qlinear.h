@@ -160,6 +160,21 @@ int qlinear_get_status(qlinear_t h);
 /* Fill *info. */
 int qlinear_info(qlinear_t h, ql_info_t* info);
 
+/* Profiling: record a pair of CUDA events around the dominant kernel launch(es)
+ * of every forward (the decode-GEMV, or the tensor-core GEMM) on the
+ * forward's own stream.  Pairs go to a ring of `capacity` slots owned by the
+ * handle (pair i of the ring is reused by launch i + capacity); capacity 0
+ * stops recording and frees the events.  Recording works inside CUDA graph
+ * capture: the captured graph re-records the same slots on every replay.
+ * Errors: QL_E_ARG (capacity < 0 or > 65536), QL_E_CUDA. */
+int qlinear_profile_enable(qlinear_t h, int capacity);
+
+/* Synchronise the device and report the summed elapsed time of the recorded
+ * slots (each slot counted once, with its most recent record) and how many
+ * slots hold a record.  Slots keep their records; graph replays overwrite
+ * them in place. */
+int qlinear_profile_read(qlinear_t h, double* total_ms, int* slots);
+
 /* Free the handle and its device memory (synchronises the device). */
 int qlinear_destroy(qlinear_t h);
 

@@ -53,12 +53,13 @@ class Layer:
         return hadamard.block_size(self.m)
 
     # ---- decode -----------------------------------------------------------
-    def decode_rows(self, rows) -> np.ndarray:
-        """W_hat rows as float64 (fp16-exact values), [len(rows), n]."""
+    def decode_rows(self, rows, blocks=None) -> np.ndarray:
+        """W_hat rows as float64 (fp16-exact values), [len(rows), n]; with
+        `blocks`, only those 256-column blocks, [len(rows), len(blocks)*T]."""
         rows = np.asarray(rows, dtype=np.int64)
-        states = trellis.block_states(self.words, rows, self.n, self.parts, self.L, self.V)
+        states = trellis.block_states(self.words, rows, self.n, self.parts, self.L, self.V, blocks)
         vals = codes.evaluate(self.code, states, self.V, self.lut)  # [r, nb, steps, V]
-        return vals.reshape(len(rows), self.n)
+        return vals.reshape(len(rows), -1)
 
     def decode_bits(self, rows) -> np.ndarray:
         """W_hat rows as fp16 bit patterns, uint16 [len(rows), n]."""

@@ -66,16 +66,17 @@ def walk_tailbiting(chunks: np.ndarray, prefix: np.ndarray, L: int, kV: int) -> 
     return states
 
 
-def block_states(words: np.ndarray, rows: np.ndarray, n: int, parts, L: int, V: int) -> np.ndarray:
-    """States of every step of every block of the given rows.
+def block_states(words: np.ndarray, rows: np.ndarray, n: int, parts, L: int, V: int, blocks=None) -> np.ndarray:
+    """States of every step of the given blocks (default: all) of the given rows.
 
-    Returns int [len(rows), n/T, T/V].  Each row's k is taken from `parts`
-    (half-TCQ layers carry two k values).
+    Returns int [len(rows), len(blocks), T/V].  Each row's k is taken from
+    `parts` (half-TCQ layers carry two k values).
     """
     T = bitstream.T
     rows = np.asarray(rows, dtype=np.int64)
     base, kk = bitstream.row_base_bits(rows, n, parts)
-    nb = n // T
+    blocks = np.arange(n // T) if blocks is None else np.asarray(blocks, dtype=np.int64)
+    nb = len(blocks)
     steps = T // V
     out = np.empty((len(rows), nb, steps), dtype=np.int64)
     for k in np.unique(kk):
@@ -85,7 +86,7 @@ def block_states(words: np.ndarray, rows: np.ndarray, n: int, parts, L: int, V: 
         S = T * k
         assert L >= kV, "a state must hold at least one step's bits"
         # bit offset of every block start: [rows_sel, nb]
-        bstart = base[sel][:, None] + np.arange(nb)[None, :] * S
+        bstart = base[sel][:, None] + blocks[None, :] * S
         bstart = bstart.reshape(-1)
         chunks = np.stack([bitstream.field(words, bstart + t * kV, kV) for t in range(steps)], axis=1)
         prefix = bitstream.field(words, bstart + S - (L - kV), L - kV) if L > kV else np.zeros_like(bstart)

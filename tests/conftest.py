@@ -1,7 +1,6 @@
+import importlib.util
 import os
 import sys
-
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
@@ -14,6 +13,10 @@ def pytest_configure(config):
 
 def pytest_sessionstart(session):
     # Build libqlinear.so in-tree if it is missing or older than its sources
-    # (nvcc cross-compiles without a GPU).
-    from trellis_coded_matmul_b200 import build
-    build.build()
+    # (nvcc cross-compiles without a GPU).  The build script is loaded by path
+    # so that a stale library is never imported before it is rebuilt.
+    path = os.path.join(ROOT, "trellis_coded_matmul_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_tcm_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()

@@ -197,3 +197,33 @@ def test_full_forward_sampled_outputs(name, batch):
     y_ref = layer.forward_rows(x, rows)
     tol = TOL_GEMV if batch <= 8 else TOL_TC
     assert rel_err(y[:, rows], y_ref) <= tol
+
+
+def test_forward_in_cuda_graph_with_profiling():
+    """forward is capturable in a CUDA graph after a first (allocating) call,
+    replays give the oracle's result, and the profiling slots record the
+    main kernel on every replay."""
+    li = _small_layer(*SMALL[1])
+    h = make_handle(li)
+    tcm.qlinear_profile_enable(h, 4)
+    xs = [torch.from_numpy(wl.make_x(li.spec, 2, instance=10 + i)).cuda() for i in range(3)]
+    ys = [torch.zeros((2, li.spec.m), device="cuda") for _ in range(3)]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        tcm.qlinear_forward(h, xs[0], ys[0])
+    torch.cuda.synchronize()
+    for y in ys:
+        y.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for x, y in zip(xs, ys):
+            tcm.qlinear_forward(h, x, y)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    ref = oq.Layer.from_inputs(li)
+    for x, y in zip(xs, ys):
+        assert rel_err(y.cpu().numpy(), ref.forward(x.cpu().numpy())) <= TOL_GEMV
+    ms, slots = tcm.qlinear_profile_read(h)
+    assert slots == 4 and ms > 0
+    tcm.qlinear_profile_enable(h, 0)

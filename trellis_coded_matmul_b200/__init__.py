@@ -37,7 +37,7 @@ QL_F16 = 1
 # Every function include/qlinear.h declares (checked by the CPU tests).
 ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
-               "qlinear_destroy", "qlinear_strerror")
+               "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read")
 
 
 class ql_code_t(ctypes.Structure):
@@ -61,6 +61,8 @@ _lib.qlinear_get_status.argtypes = [_vp]
 _lib.qlinear_info.argtypes = [_vp, ctypes.POINTER(ql_info_t)]
 _lib.qlinear_destroy.argtypes = [_vp]
 _lib.qlinear_strerror.argtypes = [_i]
+_lib.qlinear_profile_enable.argtypes = [_vp, _i]
+_lib.qlinear_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]
 _lib.qlinear_strerror.restype = ctypes.c_char_p
 for _name in ABI_SYMBOLS:
     if _name != "qlinear_strerror":
@@ -221,6 +223,17 @@ def qlinear_destroy(h: QLinearHandle) -> None:
     if h.ptr:
         _check(_lib.qlinear_destroy(h.ptr), "qlinear_destroy")
         h.ptr = None
+
+
+def qlinear_profile_enable(h: QLinearHandle, capacity: int) -> None:
+    _check(_lib.qlinear_profile_enable(h.ptr, capacity), "qlinear_profile_enable")
+
+
+def qlinear_profile_read(h: QLinearHandle):
+    """(summed milliseconds of the recorded main-kernel launches, number of recorded slots)."""
+    ms, n = ctypes.c_double(), ctypes.c_int()
+    _check(_lib.qlinear_profile_read(h.ptr, ctypes.byref(ms), ctypes.byref(n)), "qlinear_profile_read")
+    return ms.value, n.value
 
 
 def lib_path() -> str:

@@ -17,6 +17,10 @@
 // The constants are part of the stream format; they were chosen by a seeded
 // search against the statistical properties the discussion states for the
 // codes (approximately N(0,1) at L = 16, successors of a state decorrelated).
+//
+// Instruction balance on sm_100a: IMAD, IDP4A/IDP2A and the packed-half
+// HADD2/HFMA2 issue to one pipe, LOP3/PRMT/SHF to another, each at half the
+// issue rate; the decode below splits its work between the two.
 #pragma once
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -57,57 +61,95 @@ __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c
     return d;
 }
 
+// Low / high 16 bits of r through the dot-product unit (the FMA pipe), so
+// that the extraction does not compete with the LOP3/PRMT/SHF work.
+// (Inline PTX keeps the compiler from rewriting the dot product with a
+// constant operand into shifts and masks on the other pipe.)
+__device__ __forceinline__ uint32_t half_lo(uint32_t r) {
+    uint32_t d;
+    asm volatile("dp2a.lo.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(r), "r"(0x0001u), "r"(0u));
+    return d;
+}
+__device__ __forceinline__ uint32_t half_hi(uint32_t r) {
+    uint32_t d;
+    asm volatile("dp2a.lo.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(r), "r"(0x0100u), "r"(0u));
+    return d;
+}
+
 // Two V=1 states -> their two fp16 values packed (state a in the low half).
 template <int CODE>
 __device__ __forceinline__ uint32_t code_pair(uint32_t sa, uint32_t sb, const uint32_t* lut_lane, int qshift);
 
 template <>
 __device__ __forceinline__ uint32_t code_pair<kCode1MAD>(uint32_t sa, uint32_t sb, const uint32_t*, int) {
-    uint32_t xa = kA1MAD * sa + kB1MAD;
-    uint32_t xb = kA1MAD * sb + kB1MAD;
-    uint32_t ra = __dp4a(xa, 0x01010101u, kDp4aAcc);
-    uint32_t rb = __dp4a(xb, 0x01010101u, kDp4aAcc);
+    const uint32_t xa = kA1MAD * sa + kB1MAD;
+    const uint32_t xb = kA1MAD * sb + kB1MAD;
+    const uint32_t ra = __dp4a(xa, 0x01010101u, kDp4aAcc);
+    const uint32_t rb = __dp4a(xb, 0x01010101u, kDp4aAcc);
     return hfma2_u32(__byte_perm(ra, rb, 0x5410), kC1x2, kNegBiasC1x2);
 }
 
 template <>
 __device__ __forceinline__ uint32_t code_pair<kCode3INST>(uint32_t sa, uint32_t sb, const uint32_t*, int) {
-    uint32_t xa = kA3INST * sa + kB3INST;
-    uint32_t xb = kA3INST * sb + kB3INST;
-    uint32_t lo = (__byte_perm(xa, xb, 0x5410) & kMask3Lo2) ^ kXor3Lo2;
-    uint32_t hi = (__byte_perm(xa, xb, 0x7632) & kMask3Hi2) ^ kXor3Hi2;
+    const uint32_t xa = kA3INST * sa + kB3INST;
+    const uint32_t xb = kA3INST * sb + kB3INST;
+    const uint32_t lo = (__byte_perm(xa, xb, 0x5410) & kMask3Lo2) ^ kXor3Lo2;
+    const uint32_t hi = (__byte_perm(xa, xb, 0x7632) & kMask3Hi2) ^ kXor3Hi2;
     return hadd2_u32(lo, hi);
 }
 
-// HYB with V = 1: table words hold the fp16 value in their low half.  The
-// table is replicated per lane in shared memory: entry i of lane l is word
-// i*32 + l, so 32 lanes with arbitrary indices never share a bank.
+// HYB: the table is replicated per lane in shared memory: entry i of lane l
+// is word i*32 + l, so 32 lanes with arbitrary indices never share a bank.
+__device__ __forceinline__ uint32_t hyb_word(uint32_t x, const uint32_t* lut_lane, int qshift) {
+    return lut_lane[(x >> qshift) * 32u] ^ (x & 0x8000u);
+}
+
+// HYB with V = 1: table words hold the fp16 value in their low half.
 template <>
 __device__ __forceinline__ uint32_t code_pair<kCodeHYB>(uint32_t sa, uint32_t sb, const uint32_t* lut_lane, int qshift) {
-    uint32_t xa = kAHYB * sa + kBHYB;
-    uint32_t xb = kAHYB * sb + kBHYB;
-    uint32_t ea = lut_lane[(xa >> qshift) * 32u] ^ (xa & 0x8000u);
-    uint32_t eb = lut_lane[(xb >> qshift) * 32u] ^ (xb & 0x8000u);
+    const uint32_t ea = hyb_word(kAHYB * sa + kBHYB, lut_lane, qshift);
+    const uint32_t eb = hyb_word(kAHYB * sb + kBHYB, lut_lane, qshift);
     return __byte_perm(ea, eb, 0x5410);
 }
 
 // HYB with V = 2: one state -> one table word (value 0 low, value 1 high).
 __device__ __forceinline__ uint32_t code_hyb_v2(uint32_t s, const uint32_t* lut_lane, int qshift) {
-    uint32_t x = kAHYB * s + kBHYB;
-    return lut_lane[(x >> qshift) * 32u] ^ (x & 0x8000u);
+    return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
 }
 
-// 16-bit window of a thread-row's bit string ending at bit `end` (compile-time
-// after unrolling).  cw[0] holds the 32 bits before the thread's own range,
-// cw[1..] its own words, most significant bit first.  The L-bit state is the
-// low L bits of this window (callers mask with (1 << L) - 1).
+// Bits [a, a + 32) of a thread-row's bit string (most significant bit first):
+// cw[0] holds the 32 bits before the thread's own range, cw[1..] its words.
+// `a` is a compile-time constant after unrolling.
 template <int NW>
-__device__ __forceinline__ uint32_t window16(const uint32_t (&cw)[NW], int end) {
-    const int start = end - 16;
-    const int a = start >> 5;
-    const int o = start & 31;
-    if (o <= 16) return cw[a] >> (16 - o);
-    return __funnelshift_r(cw[a + 1], cw[a], 48 - o);
+__device__ __forceinline__ uint32_t bits32(const uint32_t (&cw)[NW], int a) {
+    const int w = a >> 5, o = a & 31;
+    if (o == 0) return cw[w];
+    return __funnelshift_l(cw[w + 1], cw[w], o);
+}
+
+// Trellis states of one thread-row: state t is the L-bit window ending at
+// bit 32 + (t+1)*kV of the thread-row string (the low L bits of the 16-bit
+// window, see the tail-biting rule in include/qlinear.h).
+//
+// When 16 is a multiple of kV, the windows of steps t and t + 16/kV are the
+// two halves of one 32-bit funnel shift: one SHF serves two states.
+template <int kV, bool L16, int NW>
+__device__ __forceinline__ void state_pair(const uint32_t (&cw)[NW], int t, uint32_t lmask, uint32_t& s_t,
+                                           uint32_t& s_t2) {
+    const uint32_t r = bits32(cw, 32 + (t + 1) * kV - 16);
+    if (L16) {
+        s_t = half_hi(r);
+        s_t2 = half_lo(r);
+    } else {
+        s_t = (r >> 16) & lmask;
+        s_t2 = r & lmask;
+    }
+}
+
+template <int kV, bool L16, int NW>
+__device__ __forceinline__ uint32_t state_one(const uint32_t (&cw)[NW], int t, uint32_t lmask) {
+    const uint32_t r = bits32(cw, 32 + (t + 1) * kV - 32);
+    return L16 ? half_lo(r) : (r & lmask);
 }
 
 }  // namespace qlk

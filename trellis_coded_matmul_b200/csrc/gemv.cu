@@ -76,29 +76,73 @@ __device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lu
     for (int i = threadIdx.x; i < entries * 32; i += blockDim.x) smem[i] = lut[i >> 5];
 }
 
-// The four A-operand registers of MMA number u (0..15) of a unit:
-//   a[0] = row g,     columns 4u, 4u+1 of the lane's run    a[2] = row g,     columns 4u+2, 4u+3
-//   a[1] = row g + 8, columns 4u, 4u+1                       a[3] = row g + 8, columns 4u+2, 4u+3
-// cw[h] holds the 32 bits before the lane's run of thread-row h, then its 2K words.
-template <int CODE, int K, int V>
-__device__ __forceinline__ void decode_mma_operand(uint32_t (&a)[4], const uint32_t (&cw)[2][2 * K + 1], int u,
-                                                   uint32_t lmask, const uint32_t* lut_lane, int qshift) {
-    constexpr int kV = K * V;
+// A operands of the 16 m16n8k16 MMAs of one unit.  MMA u takes, for each
+// thread-row h (row g for h = 0, row g + 8 for h = 1), the lane's columns
+// 4u .. 4u+3 of its run, i.e. steps 4u .. 4u+3 (V = 1) or 2u, 2u+1 (V = 2):
+//   a[0] = row g, columns 4u, 4u+1      a[2] = row g, columns 4u+2, 4u+3
+//   a[1] = row g+8, columns 4u, 4u+1    a[3] = row g+8, columns 4u+2, 4u+3
+// Paired extraction (16 % kV == 0): steps t and t + 16/kV share one funnel
+// shift, which pairs MMA u with MMA u + MP (MP = 16/kV/steps-per-MMA).
+template <int CODE, int K, int V, bool L16>
+struct UnitDecoder {
+    static constexpr int kV = K * V;
+    static constexpr int SPM = 4 / V;                  // steps per MMA per thread-row
+    static constexpr bool kPair = (16 % kV) == 0;
+    static constexpr int P = kPair ? 16 / kV : 1;      // step distance of paired windows
+    static constexpr int MP = kPair ? P / SPM : 1;     // MMA distance of paired MMAs
+    static constexpr int NW = 2 * K + 1;
+
+    // states of steps [t0, t0 + SPM) into s[0..SPM) and, when paired, of
+    // [t0 + P, t0 + P + SPM) into s2[0..SPM)
+    static __device__ __forceinline__ void states(const uint32_t (&cw)[NW], int t0, uint32_t lmask,
+                                                  uint32_t (&s)[SPM], uint32_t (&s2)[SPM]) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (V == 1) {
-            const uint32_t s0 = window16(cw[h], 32 + (4 * u + 1) * kV) & lmask;
-            const uint32_t s1 = window16(cw[h], 32 + (4 * u + 2) * kV) & lmask;
-            const uint32_t s2 = window16(cw[h], 32 + (4 * u + 3) * kV) & lmask;
-            const uint32_t s3 = window16(cw[h], 32 + (4 * u + 4) * kV) & lmask;
-            a[h] = code_pair<CODE>(s0, s1, lut_lane, qshift);
-            a[2 + h] = code_pair<CODE>(s2, s3, lut_lane, qshift);
-        } else {
-            const uint32_t s0 = window16(cw[h], 32 + (2 * u + 1) * kV) & lmask;
-            const uint32_t s1 = window16(cw[h], 32 + (2 * u + 2) * kV) & lmask;
-            a[h] = code_hyb_v2(s0, lut_lane, qshift);
-            a[2 + h] = code_hyb_v2(s1, lut_lane, qshift);
+        for (int q = 0; q < SPM; ++q) {
+            if (kPair)
+                state_pair<kV, L16>(cw, t0 + q, lmask, s[q], s2[q]);
+            else
+                s[q] = state_one<kV, L16>(cw, t0 + q, lmask);
         }
+    }
+
+    static __device__ __forceinline__ void codes(const uint32_t (&s)[SPM], uint32_t& lo, uint32_t& hi,
+                                                 const uint32_t* lut_lane, int qshift) {
+        if (V == 1) {
+            lo = code_pair<CODE>(s[0], s[1], lut_lane, qshift);
+            hi = code_pair<CODE>(s[2], s[3], lut_lane, qshift);
+        } else {
+            lo = code_hyb_v2(s[0], lut_lane, qshift);
+            hi = code_hyb_v2(s[SPM - 1], lut_lane, qshift);
+        }
+    }
+
+    // Operands of MMA u (and, when paired, of MMA u + MP into a2).
+    static __device__ __forceinline__ void operands(const uint32_t (&cw)[2][NW], int u, uint32_t lmask,
+                                                    const uint32_t* lut_lane, int qshift, uint32_t (&a)[4],
+                                                    uint32_t (&a2)[4]) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t s[SPM], s2[SPM];
+            states(cw[h], u * SPM, lmask, s, s2);
+            codes(s, a[h], a[2 + h], lut_lane, qshift);
+            if (kPair) codes(s2, a2[h], a2[2 + h], lut_lane, qshift);
+        }
+    }
+};
+
+// Calls f(u, a) for u = 0..15 with the A operands of MMA u, in the order
+// that lets paired extraction share its funnel shifts.
+template <int CODE, int K, int V, bool L16, typename F>
+__device__ __forceinline__ void for_each_mma(const uint32_t (&cw)[2][2 * K + 1], uint32_t lmask,
+                                             const uint32_t* lut_lane, int qshift, F&& f) {
+    using D = UnitDecoder<CODE, K, V, L16>;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        if (D::kPair && ((u / D::MP) & 1)) continue;  // produced together with MMA u - MP
+        uint32_t a[4], a2[4];
+        D::operands(cw, u, lmask, lut_lane, qshift, a, a2);
+        f(u, a);
+        if (D::kPair) f(u + D::MP, a2);
     }
 }
 
@@ -119,8 +163,12 @@ struct GemvArgs {
     int row0;         // first layer row of the part
 };
 
-template <int CODE, int K, int V>
-__global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
+// One CTA per SM.  CTA b takes units [U*b/G, U*(b+1)/G) of the part (G CTAs)
+// and splits them evenly over its warps; the launcher sizes the CTA so that
+// every warp gets the same whole number of units (to within one), which keeps
+// every SM and every warp equally loaded.
+template <int CODE, int K, int V, bool L16>
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p) {
     extern __shared__ uint32_t lut_smem[];
     using UL = UnitLayout<K>;
     const int lane = threadIdx.x & 31;
@@ -129,13 +177,16 @@ __global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
         __syncthreads();
     }
     const uint32_t* lut_lane = lut_smem + lane;
-    const int wpb = blockDim.x >> 5;
-    const long long nwarps = (long long)gridDim.x * wpb;
-    const long long gw = (long long)blockIdx.x * wpb + (threadIdx.x >> 5);
     const int nb = p.dec.nb;
     const long long U = (long long)p.dec.rt * nb;
-    const long long u0 = U * gw / nwarps, u1 = U * (gw + 1) / nwarps;
-    if (u0 >= u1) return;
+    const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
+    const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
+    const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
+    if (u0 >= u1) {
+        grid_dependency_wait();
+        grid_launch_dependents();
+        return;
+    }
 
     const int g = lane >> 2, c = lane & 3;
     const int src_lane = (lane & ~3) | ((c + 3) & 3);
@@ -143,6 +194,11 @@ __global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
 
     uint32_t nxt[2][2 * K];
     load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
+    // Programmatic dependent launch: the code words (and the HYB table) are
+    // written once at create time, so they are fetched before waiting for the
+    // kernel that produces x' (and, before it, the consumer of the previous z).
+    grid_dependency_wait();
+    grid_launch_dependents();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int R = (int)(u0 / nb), j = (int)(u0 % nb);
     int curR = R;
@@ -176,14 +232,11 @@ __global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
         for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
 
         const uint2* xb = p.xf + (size_t)j * 16 * batch * 4 + g * 4 + c;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            uint32_t a[4];
-            decode_mma_operand<CODE, K, V>(a, cw, u, p.dec.lmask, lut_lane, p.dec.qshift);
+        for_each_mma<CODE, K, V, L16>(cw, p.dec.lmask, lut_lane, p.dec.qshift, [&](int u, const uint32_t(&a)[4]) {
             uint2 bv = make_uint2(0u, 0u);
             if (g < batch) bv = __ldg(xb + (size_t)u * batch * 4);
             mma_16816(acc, a, bv.x, bv.y);
-        }
+        });
         if (++j == nb) {
             j = 0;
             ++R;
@@ -193,7 +246,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(GemvArgs p) {
 }
 
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
-template <int CODE, int K, int V>
+template <int CODE, int K, int V, bool L16>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
     extern __shared__ uint32_t lut_smem[];
     using UL = UnitLayout<K>;
@@ -219,17 +272,14 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __res
             cw[h][0] = __shfl_sync(0xffffffffu, w[h][2 * K - 1], src_lane);
         }
         const int R = (int)(unit / p.nb), j = (int)(unit % p.nb);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            uint32_t a[4];
-            decode_mma_operand<CODE, K, V>(a, cw, u, p.lmask, lut_lane, p.qshift);
+        for_each_mma<CODE, K, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const size_t row = (size_t)row0 + R * kRowTile + 8 * h + g;
                 uint2* dst = (uint2*)(w_hat + row * n + (size_t)j * kT + 64 * c + 4 * u);
                 *dst = make_uint2(a[h], a[2 + h]);
             }
-        }
+        });
     }
 }
 
@@ -260,35 +310,43 @@ __global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count,
 }
 
 // ---- dispatch ----
-template <template <int, int, int> class F, typename... Args>
-static cudaError_t dispatch(int code, int k, int V, Args&&... args) {
+template <template <int, int, int, bool> class F, bool L16, typename... Args>
+static cudaError_t dispatch_l(int code, int k, int V, Args&&... args);
+
+template <template <int, int, int, bool> class F, typename... Args>
+static cudaError_t dispatch(int code, int k, int V, bool l16, Args&&... args) {
+    return l16 ? dispatch_l<F, true>(code, k, V, args...) : dispatch_l<F, false>(code, k, V, args...);
+}
+
+template <template <int, int, int, bool> class F, bool L16, typename... Args>
+static cudaError_t dispatch_l(int code, int k, int V, Args&&... args) {
     if (code == kCode1MAD && V == 1) {
         switch (k) {
-            case 1: return F<kCode1MAD, 1, 1>::run(args...);
-            case 2: return F<kCode1MAD, 2, 1>::run(args...);
-            case 3: return F<kCode1MAD, 3, 1>::run(args...);
-            case 4: return F<kCode1MAD, 4, 1>::run(args...);
+            case 1: return F<kCode1MAD, 1, 1, L16>::run(args...);
+            case 2: return F<kCode1MAD, 2, 1, L16>::run(args...);
+            case 3: return F<kCode1MAD, 3, 1, L16>::run(args...);
+            case 4: return F<kCode1MAD, 4, 1, L16>::run(args...);
         }
     } else if (code == kCode3INST && V == 1) {
         switch (k) {
-            case 1: return F<kCode3INST, 1, 1>::run(args...);
-            case 2: return F<kCode3INST, 2, 1>::run(args...);
-            case 3: return F<kCode3INST, 3, 1>::run(args...);
-            case 4: return F<kCode3INST, 4, 1>::run(args...);
+            case 1: return F<kCode3INST, 1, 1, L16>::run(args...);
+            case 2: return F<kCode3INST, 2, 1, L16>::run(args...);
+            case 3: return F<kCode3INST, 3, 1, L16>::run(args...);
+            case 4: return F<kCode3INST, 4, 1, L16>::run(args...);
         }
     } else if (code == kCodeHYB && V == 1) {
         switch (k) {
-            case 1: return F<kCodeHYB, 1, 1>::run(args...);
-            case 2: return F<kCodeHYB, 2, 1>::run(args...);
-            case 3: return F<kCodeHYB, 3, 1>::run(args...);
-            case 4: return F<kCodeHYB, 4, 1>::run(args...);
+            case 1: return F<kCodeHYB, 1, 1, L16>::run(args...);
+            case 2: return F<kCodeHYB, 2, 1, L16>::run(args...);
+            case 3: return F<kCodeHYB, 3, 1, L16>::run(args...);
+            case 4: return F<kCodeHYB, 4, 1, L16>::run(args...);
         }
     } else if (code == kCodeHYB && V == 2) {
         switch (k) {
-            case 1: return F<kCodeHYB, 1, 2>::run(args...);
-            case 2: return F<kCodeHYB, 2, 2>::run(args...);
-            case 3: return F<kCodeHYB, 3, 2>::run(args...);
-            case 4: return F<kCodeHYB, 4, 2>::run(args...);
+            case 1: return F<kCodeHYB, 1, 2, L16>::run(args...);
+            case 2: return F<kCodeHYB, 2, 2, L16>::run(args...);
+            case 3: return F<kCodeHYB, 3, 2, L16>::run(args...);
+            case 4: return F<kCodeHYB, 4, 2, L16>::run(args...);
         }
     }
     return cudaErrorInvalidValue;
@@ -306,17 +364,18 @@ static DecodeArgs make_decode_args(const Layer& L, const Part& part) {
     return d;
 }
 
-template <int CODE, int K, int V>
+template <int CODE, int K, int V, bool L16>
 struct GemvLaunch {
-    static cudaError_t run(const GemvArgs& a, int grid, cudaStream_t st) {
+    static cudaError_t run(const GemvArgs& a, int grid, int threads, cudaStream_t st) {
         const size_t smem = (size_t)a.dec.lut_entries * 32 * 4;
-        auto kern = gemv_kernel<CODE, K, V>;
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        auto kern = gemv_kernel<CODE, K, V, L16>;
+        static bool attr_set = false;
+        if (smem > 48 * 1024 && !attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
             if (e != cudaSuccess) return e;
+            attr_set = true;
         }
-        kern<<<grid, 256, smem, st>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a);
     }
 };
 
@@ -330,21 +389,23 @@ cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, i
     a.m = L.m;
     a.row0 = part.row0;
     const long long units = (long long)a.dec.rt * a.dec.nb;
-    long long grid = (long long)L.num_sms * 2;
-    const long long need = (units + 7) / 8;  // at least one unit per warp
-    if (grid > need) grid = need;
-    if (grid < 1) grid = 1;
-    return dispatch<GemvLaunch>(L.code, part.k, L.V, a, (int)grid, st);
+    long long grid = units < L.num_sms ? units : L.num_sms;
+    const long long per_cta = (units + grid - 1) / grid;
+    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
+    const int warps = (int)((per_cta + per_warp - 1) / per_warp);
+    return dispatch<GemvLaunch>(L.code, part.k, L.V, L.L == 16, a, (int)grid, warps * 32, st);
 }
 
-template <int CODE, int K, int V>
+template <int CODE, int K, int V, bool L16>
 struct DecodeLaunch {
     static cudaError_t run(const DecodeArgs& d, __half* w, int n, int row0, int grid, cudaStream_t st) {
         const size_t smem = (size_t)d.lut_entries * 32 * 4;
-        auto kern = decode_kernel<CODE, K, V>;
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        auto kern = decode_kernel<CODE, K, V, L16>;
+        static bool attr_set = false;
+        if (smem > 48 * 1024 && !attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
             if (e != cudaSuccess) return e;
+            attr_set = true;
         }
         kern<<<grid, 256, smem, st>>>(d, w, n, row0);
         return cudaGetLastError();
@@ -356,19 +417,21 @@ cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStr
     const long long units = (long long)d.rt * d.nb;
     long long grid = (units + 7) / 8;
     if (grid > (long long)L.num_sms * 8) grid = (long long)L.num_sms * 8;
-    return dispatch<DecodeLaunch>(L.code, part.k, L.V, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
+    return dispatch<DecodeLaunch>(L.code, part.k, L.V, L.L == 16, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
 }
 
-template <int CODE, int K, int V>
+template <int CODE, int K, int V, bool L16>
 struct EvalLaunch {
     static cudaError_t run(const uint32_t* states, int count, uint32_t lmask, int qshift, const uint32_t* lut,
                            int entries, __half* out, cudaStream_t st) {
-        if (K != 1) return cudaErrorInvalidValue;  // k is irrelevant to the code; one instance suffices
+        if (K != 1 || !L16) return cudaErrorInvalidValue;  // one instance suffices: the code ignores k and L
         const size_t smem = (size_t)entries * 32 * 4;
         auto kern = eval_code_kernel<CODE, V>;
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static bool attr_set = false;
+        if (smem > 48 * 1024 && !attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
             if (e != cudaSuccess) return e;
+            attr_set = true;
         }
         const int items = V == 2 ? count : (count + 1) / 2;
         kern<<<(items + 255) / 256, 256, smem, st>>>(states, count, lmask, qshift, lut, entries, out);
@@ -380,7 +443,7 @@ cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_
                              int count, void* out, cudaStream_t st) {
     const uint32_t lmask = (1u << L) - 1u;
     const int entries = code == kCodeHYB ? (1 << Q) : 0;
-    return dispatch<EvalLaunch>(code, 1, V, states, count, lmask, 32 - Q, lut_words, entries, (__half*)out, st);
+    return dispatch<EvalLaunch>(code, 1, V, true, states, count, lmask, 32 - Q, lut_words, entries, (__half*)out, st);
 }
 
 }  // namespace qlk

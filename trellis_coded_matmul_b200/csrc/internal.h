@@ -12,6 +12,8 @@ constexpr int kT = 256;            // columns per trellis block
 constexpr int kRowTile = 16;       // rows per decode tile (the m16n8k16 M dimension)
 constexpr int kMaxHadamard = 32768;
 
+constexpr int kGemvMaxWarps = 24;  // decode-GEMV: warps of its one CTA per SM (<= 85 registers/thread)
+
 // Device status word bits (qlinear_get_status).
 constexpr int kStatusBadSign = 1;
 constexpr int kStatusTimeout = 2;
@@ -43,12 +45,42 @@ struct Layer {
     // scratch, grown on demand
     void* xp;             // transformed input x' (fp16)
     size_t xp_bytes;
-    float* z;             // W_hat x' before the output transform, fp32 [batch][m]
+    float* z;             // W_hat x' before the output transform, fp32 [batch][m]; all-zero between forwards
     size_t z_bytes;
+    int z_dirty;          // z may hold partial sums (a forward failed part-way)
     void* host_stage;     // device staging for qlinear_forward_host (x then y)
     size_t host_stage_bytes;
     int num_sms;
+    // profiling ring (qlinear_profile_enable)
+    cudaEvent_t* prof_ev;  // 2 * prof_cap events
+    int prof_cap;
+    int prof_next;
+    int prof_count;
 };
+
+// Programmatic dependent launch (PDL): the kernel may start while the
+// previous kernel on the stream is still running; it must call
+// grid_dependency_wait() before touching anything that kernel (or any earlier
+// work on the stream) writes, and calls grid_launch_dependents() to let the
+// next kernel start early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_relayout(const uint32_t* src, uint32_t* dst, const Part& part, int n, cudaStream_t st);
@@ -59,8 +91,8 @@ cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cu
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
 // x (fp16 [batch][n]) -> x' fp16 [batch][n] row-major.
 cudaError_t launch_rht_in_rowmajor(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
-// z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16.
-cudaError_t launch_rht_out(const Layer& L, const float* z, int batch, void* y, int y_dtype, cudaStream_t st);
+// z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
+cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st);
 
 // z[b][row0 + r] += sum_c W_hat[row0 + r][c] x'[b][c] for the part's rows; batch <= 8.
 cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, int batch, float* z,

@@ -56,7 +56,15 @@ int dev_alloc(T** p, size_t bytes) {
     return QL_OK;
 }
 
+void free_profiling(Layer& L) {
+    for (int i = 0; i < 2 * L.prof_cap; ++i) cudaEventDestroy(L.prof_ev[i]);
+    delete[] L.prof_ev;
+    L.prof_ev = nullptr;
+    L.prof_cap = L.prof_next = L.prof_count = 0;
+}
+
 void free_layer(Layer& L) {
+    free_profiling(L);
     cudaFree(L.words);
     cudaFree(L.sin_bits);
     cudaFree(L.sout_bits);
@@ -164,6 +172,16 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     return QL_OK;
 }
 
+// Record an event on st; inside stream capture it becomes an event-record
+// node of the graph (so every replay re-records it) instead of a capture-
+// internal dependency marker.
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return e;
+    return cudaEventRecordWithFlags(ev, st, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0);
+}
+
 // Grow a scratch buffer to at least `bytes`.
 int ensure(void** buf, size_t* have, size_t bytes) {
     if (*have >= bytes) return QL_OK;
@@ -179,22 +197,40 @@ int ensure(void** buf, size_t* have, size_t bytes) {
     return QL_OK;
 }
 
+// The z accumulator is all-zero between forwards: it is zeroed when
+// allocated, and the output-transform kernel re-zeroes what it consumed.
 int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
     const int chunk = batch < 8 ? batch : 8;
     int rc = ensure(&L.xp, &L.xp_bytes, (size_t)chunk * L.n * 2);
-    if (rc == QL_OK) rc = ensure((void**)&L.z, &L.z_bytes, (size_t)chunk * L.m * 4);
     if (rc != QL_OK) return rc;
+    const size_t zb = (size_t)chunk * L.m * 4;
+    if (L.z_bytes < zb || L.z_dirty) {
+        rc = ensure((void**)&L.z, &L.z_bytes, zb);
+        if (rc != QL_OK) return rc;
+        if (cudaMemsetAsync(L.z, 0, L.z_bytes, st) != cudaSuccess) {
+            cudaGetLastError();
+            return QL_E_CUDA;
+        }
+        L.z_dirty = 0;
+    }
     const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
     for (int b0 = 0; b0 < batch; b0 += 8) {
         const int nb = batch - b0 < 8 ? batch - b0 : 8;
         const void* xb = (const char*)x + (size_t)b0 * L.n * 2;
         void* yb = (char*)y + (size_t)b0 * L.m * ysz;
         cudaError_t e = launch_rht_in_frag(L, xb, nb, L.xp, st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(L.z, 0, (size_t)nb * L.m * 4, st);
+        const int slot = L.prof_cap ? L.prof_next : -1;
+        if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
         for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) e = launch_gemv(L, L.parts[i], L.xp, nb, L.z, st);
+        if (e == cudaSuccess && slot >= 0) {
+            e = record_event(L.prof_ev[2 * slot + 1], st);
+            L.prof_next = (L.prof_next + 1) % L.prof_cap;
+            if (L.prof_count < L.prof_cap) ++L.prof_count;
+        }
         if (e == cudaSuccess) e = launch_rht_out(L, L.z, nb, yb, y_dtype, st);
         if (e != cudaSuccess) {
             cudaGetLastError();
+            L.z_dirty = 1;  // a partial forward may have left sums in z
             return QL_E_CUDA;
         }
     }
@@ -337,6 +373,51 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
     info->lut_bytes = L.code == QL_CODE_HYB ? ((size_t)1 << L.Q) * L.V * 2 : 0;
     info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
+    return QL_OK;
+}
+
+int qlinear_profile_enable(qlinear_t h, int capacity) {
+    if (!h || capacity < 0 || capacity > 65536) return QL_E_ARG;
+    Layer& L = h->L;
+    DeviceGuard g(L.device);
+    if (!g.ok) return QL_E_CUDA;
+    cudaDeviceSynchronize();
+    free_profiling(L);
+    if (capacity == 0) return QL_OK;
+    L.prof_ev = new (std::nothrow) cudaEvent_t[2 * (size_t)capacity];
+    if (!L.prof_ev) return QL_E_OOM;
+    for (int i = 0; i < 2 * capacity; ++i) {
+        if (cudaEventCreate(&L.prof_ev[i]) != cudaSuccess) {
+            cudaGetLastError();
+            L.prof_cap = i / 2;
+            for (int j = 2 * L.prof_cap; j < i; ++j) cudaEventDestroy(L.prof_ev[j]);
+            free_profiling(L);
+            return QL_E_CUDA;
+        }
+    }
+    L.prof_cap = capacity;
+    return QL_OK;
+}
+
+int qlinear_profile_read(qlinear_t h, double* total_ms, int* slots) {
+    if (!h || !total_ms || !slots) return QL_E_ARG;
+    Layer& L = h->L;
+    DeviceGuard g(L.device);
+    if (!g.ok || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    double sum = 0.0;
+    for (int i = 0; i < L.prof_count; ++i) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, L.prof_ev[2 * i], L.prof_ev[2 * i + 1]) != cudaSuccess) {
+            cudaGetLastError();
+            return QL_E_CUDA;
+        }
+        sum += ms;
+    }
+    *total_ms = sum;
+    *slots = L.prof_count;
     return QL_OK;
 }
 

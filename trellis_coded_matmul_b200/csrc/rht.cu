@@ -5,10 +5,21 @@
 //   input:  x' = H_n diag(s_in) x      (per block of B_n consecutive entries)
 //   output: y  = alpha diag(s_out) H_m z
 //
-// H_B is the normalised Sylvester matrix; the in-place butterfly
-// (a, b) -> (a + b, a - b) over strides 1, 2, 4, ... produces it in natural
-// order, and the 1/sqrt(B) normalisation is applied once at the end.  One CTA
-// transforms one Hadamard block of one batch row in shared memory (fp32).
+// H_B is the normalised Sylvester matrix.  The fast transform applies the
+// butterfly (a, b) -> (a + b, a - b) for every stride 1, 2, ..., B/2 (the
+// strides commute).  A group of T = B/E threads owns one block, E consecutive
+// entries per thread:
+//   * strides 1 .. E/2 inside a thread's registers,
+//   * strides E .. 16E by warp shuffles (lane bit j <-> stride E*2^j),
+//   * the remaining strides (blocks of more than 32E entries) through shared
+//     memory, four strides per pass (a thread takes 16 entries base + q*h),
+//     with one word of padding per 16 so the passes are free of bank
+//     conflicts.
+// The 1/sqrt(B) normalisation is applied once, at the end, in fp32.  A CTA
+// holds several groups when blocks are small.  Both kernels are launched as
+// programmatic dependents: they wait for the previous kernel before touching
+// their inputs.  The output kernel also re-zeroes the z entries it consumed,
+// so the accumulation buffer is ready for the next forward without a memset.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -16,65 +27,196 @@
 namespace qlk {
 
 __device__ __forceinline__ bool sign_neg(const uint32_t* bits, int i) { return (bits[i >> 5] >> (i & 31)) & 1u; }
+__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
 
-__device__ __forceinline__ void fwht_smem(float* buf, int B) {
-    for (int hs = 1; hs < B; hs <<= 1) {
-        for (int t = threadIdx.x; t < (B >> 1); t += blockDim.x) {
-            const int i0 = ((t / hs) * 2 * hs) + (t % hs);
-            const int i1 = i0 + hs;
-            const float a = buf[i0], b = buf[i1];
-            buf[i0] = a + b;
-            buf[i1] = a - b;
+template <int LOGR>
+__device__ __forceinline__ void fwht_pass(float* buf, int B, int h, int tid, int nthreads) {
+    constexpr int R = 1 << LOGR;
+    const int groups = B >> LOGR;
+    for (int gi = tid; gi < groups; gi += nthreads) {
+        const int base = (gi / h) * (h << LOGR) + (gi % h);
+        float v[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) v[q] = buf[pad16(base + q * h)];
+#pragma unroll
+        for (int s = 0; s < LOGR; ++s) {
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+                if (!(q & (1 << s))) {
+                    const float a = v[q], b = v[q | (1 << s)];
+                    v[q] = a + b;
+                    v[q | (1 << s)] = a - b;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < R; ++q) buf[pad16(base + q * h)] = v[q];
+    }
+}
+
+// Strides E.. of the remaining FWHT through shared memory (padded layout) by
+// the `nthreads` threads of the group, starting at stride h0; ends with a
+// CTA barrier after every pass.
+__device__ __forceinline__ void fwht_smem_passes(float* buf, int B, int h0, int tid, int nthreads) {
+    int h = h0;
+    while (h < B) {
+        const int rem = 31 - __clz(B / h);  // log2(B / h)
+        if (rem >= 4) {
+            fwht_pass<4>(buf, B, h, tid, nthreads);
+            h <<= 4;
+        } else if (rem == 3) {
+            fwht_pass<3>(buf, B, h, tid, nthreads);
+            h <<= 3;
+        } else if (rem == 2) {
+            fwht_pass<2>(buf, B, h, tid, nthreads);
+            h <<= 2;
+        } else {
+            fwht_pass<1>(buf, B, h, tid, nthreads);
+            h <<= 1;
         }
         __syncthreads();
+    }
+}
+
+// Full FWHT of a group's block: v holds the thread's E consecutive entries
+// (thread tid of T owns entries [tid*E, tid*E + E)); on return v holds the
+// same positions of the transformed block.  `buf` is the group's shared
+// memory (B + B/16 floats), used only when T > 32.  Every thread of the CTA
+// must call this with the same B (it contains CTA barriers when T > 32).
+template <int E>
+__device__ __forceinline__ void fwht_block(float (&v)[E], int B, int tid, int T, float* buf) {
+#pragma unroll
+    for (int s = 1; s < E; s <<= 1) {
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            if (!(q & s)) {
+                const float a = v[q], b = v[q | s];
+                v[q] = a + b;
+                v[q | s] = a - b;
+            }
+        }
+    }
+    const int lanes = T < 32 ? T : 32;
+    const int lane = threadIdx.x & 31;
+    for (int j = 1; j < lanes; j <<= 1) {
+        const bool upper = lane & j;
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[q], j);
+            v[q] = upper ? (o - v[q]) : (v[q] + o);
+        }
+    }
+    if (T > 32) {
+#pragma unroll
+        for (int q = 0; q < E; ++q) buf[pad16(tid * E + q)] = v[q];
+        __syncthreads();
+        fwht_smem_passes(buf, B, 32 * E, tid, T);
+#pragma unroll
+        for (int q = 0; q < E; ++q) v[q] = buf[pad16(tid * E + q)];
     }
 }
 
 // Fragment layout of x' for the decode-GEMV: the 8-byte group
 //   frag[((j*16 + u) * batch + b) * 4 + c] = x'[b][256 j + 64 c + 4 u + 0..3]
 // is what lane (g = b, c) needs as its B operand for the u-th m16n8k16 MMA of
-// block j (see gemv.cu).
-__device__ __forceinline__ size_t frag_index(int col, int b, int batch) {
+// block j (see gemv.cu).  Returns the index of the first of the four halves.
+__device__ __forceinline__ size_t frag_index4(int col, int b, int batch) {
     const int j = col >> 8, within = col & 255;
     const int c = within >> 6, r = within & 63;
-    const int u = r >> 2, e = r & 3;
-    return ((((size_t)j * 16 + u) * batch + b) * 4 + c) * 4 + e;
+    const int u = r >> 2;
+    return ((((size_t)j * 16 + u) * batch + b) * 4 + c) * 4;
 }
 
-template <bool FRAG>
-__global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, int B,
+struct RhtGeometry {
+    int B;        // Hadamard block size
+    int per_row;  // Hadamard blocks per batch row (d / B)
+    int total;    // batch * per_row
+    int groups;   // Hadamard blocks per CTA
+    int tpg;      // threads per group (B / E)
+};
+
+// E = 16 entries per thread (32 for B = 32768, to stay within 1024 threads).
+static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
+    RhtGeometry g;
+    g.B = B;
+    g.per_row = d / B;
+    g.total = batch * g.per_row;
+    g.tpg = B / E < 1 ? 1 : B / E;
+    g.groups = g.tpg >= 256 ? 1 : 256 / g.tpg;
+    if (g.groups > g.total) g.groups = g.total;
+    return g;
+}
+
+// FRAG: write x' in the decode-GEMV fragment layout (else row-major [batch][n]).
+template <bool FRAG, int E>
+__global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, RhtGeometry geo,
                               const uint32_t* __restrict__ sin_bits, __half* __restrict__ out) {
-    extern __shared__ float buf[];
-    const int blk = blockIdx.x, b = blockIdx.y;
-    const __half* xb = x + (size_t)b * n + (size_t)blk * B;
-    for (int i = threadIdx.x; i < B; i += blockDim.x) {
-        float v = __half2float(xb[i]);
-        buf[i] = sign_neg(sin_bits, blk * B + i) ? -v : v;
+    extern __shared__ float smem[];
+    grid_dependency_wait();
+    const int B = geo.B;
+    const int grp = threadIdx.x / geo.tpg, tid = threadIdx.x % geo.tpg;
+    const int item = blockIdx.x * geo.groups + grp;
+    const bool active = item < geo.total;
+    float* buf = smem + (size_t)grp * (B + B / 16);
+    const int b = active ? item / geo.per_row : 0;
+    const int col = (active ? (item % geo.per_row) * B : 0) + tid * E;
+    float v[E];
+    if (active) {
+        const __half* xs = x + (size_t)b * n + col;
+        const uint32_t sw = sin_bits[col >> 5] >> (col & 31);  // E <= 32 consecutive sign bits
+#pragma unroll
+        for (int q = 0; q < E; q += 8) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(xs + q);
+            const __half* hv = reinterpret_cast<const __half*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float f = __half2float(hv[e]);
+                v[q + e] = ((sw >> (q + e)) & 1u) ? -f : f;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < E; ++q) v[q] = 0.f;
     }
-    __syncthreads();
-    fwht_smem(buf, B);
+    fwht_block<E>(v, B, tid, geo.tpg, buf);
+    grid_launch_dependents();
+    if (!active) return;
     const float scale = rsqrtf((float)B);
-    for (int i = threadIdx.x; i < B; i += blockDim.x) {
-        const int col = blk * B + i;
-        const __half v = __float2half_rn(buf[i] * scale);
+#pragma unroll
+    for (int q = 0; q < E; q += 4) {
+        const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
+        const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
         if (FRAG)
-            out[frag_index(col, b, batch)] = v;
+            *reinterpret_cast<uint2*>(out + frag_index4(col + q, b, batch)) = w;
         else
-            out[(size_t)b * n + col] = v;
+            *reinterpret_cast<uint2*>(out + (size_t)b * n + col + q) = w;
     }
+}
+
+template <bool FRAG, int E>
+static cudaError_t launch_rht_in_e(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
+    const RhtGeometry geo = rht_geometry(L.n, L.B_n, batch, E);
+    const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
+    auto kern = rht_in_kernel<FRAG, E>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (kMaxHadamard + kMaxHadamard / 16) * 4);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int grid = (geo.total + geo.groups - 1) / geo.groups;
+    return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, (const __half*)x, batch, L.n, geo,
+                      (const uint32_t*)L.sin_bits, (__half*)xp);
 }
 
 template <bool FRAG>
 static cudaError_t launch_rht_in(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    const int B = L.B_n;
-    const size_t smem = (size_t)B * sizeof(float);
-    auto kern = rht_in_kernel<FRAG>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(L.n / B, batch);
-    const int threads = B >= 1024 ? 1024 : (B >= 64 ? B : 64);
-    kern<<<grid, threads, smem, st>>>((const __half*)x, batch, L.n, B, L.sin_bits, (__half*)xp);
-    return cudaGetLastError();
+    return L.B_n > 16384 ? launch_rht_in_e<FRAG, 32>(L, x, batch, xp, st)
+                         : launch_rht_in_e<FRAG, 16>(L, x, batch, xp, st);
 }
 
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
@@ -85,37 +227,81 @@ cudaError_t launch_rht_in_rowmajor(const Layer& L, const void* x, int batch, voi
     return launch_rht_in<false>(L, x, batch, xp, st);
 }
 
-template <bool F16>
-__global__ void rht_out_kernel(const float* __restrict__ z, int batch, int m, int B,
+// Entries per thread of the output transform: B_m may be as small as 16.
+template <bool F16, int E>
+__global__ void rht_out_kernel(float* __restrict__ z, int batch, int m, RhtGeometry geo,
                                const uint32_t* __restrict__ sout_bits, float alpha, void* __restrict__ y) {
-    extern __shared__ float buf[];
-    const int blk = blockIdx.x, b = blockIdx.y;
-    const float* zb = z + (size_t)b * m + (size_t)blk * B;
-    for (int i = threadIdx.x; i < B; i += blockDim.x) buf[i] = zb[i];
-    __syncthreads();
-    fwht_smem(buf, B);
+    extern __shared__ float smem[];
+    grid_dependency_wait();
+    const int B = geo.B;
+    const int grp = threadIdx.x / geo.tpg, tid = threadIdx.x % geo.tpg;
+    const int item = blockIdx.x * geo.groups + grp;
+    const bool active = item < geo.total;
+    float* buf = smem + (size_t)grp * (B + B / 16);
+    const int b = active ? item / geo.per_row : 0;
+    const int row = (active ? (item % geo.per_row) * B : 0) + tid * E;
+    float v[E];
+    if (active) {
+        float* zs = z + (size_t)b * m + row;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(zs + q);
+            v[q] = t.x;
+            v[q + 1] = t.y;
+            v[q + 2] = t.z;
+            v[q + 3] = t.w;
+            *reinterpret_cast<float4*>(zs + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < E; ++q) v[q] = 0.f;
+    }
+    fwht_block<E>(v, B, tid, geo.tpg, buf);
+    grid_launch_dependents();
+    if (!active) return;
     const float scale = alpha * rsqrtf((float)B);
-    for (int i = threadIdx.x; i < B; i += blockDim.x) {
-        const int row = blk * B + i;
-        float v = buf[i] * scale;
-        if (sign_neg(sout_bits, row)) v = -v;
-        if (F16)
-            ((__half*)y)[(size_t)b * m + row] = __float2half_rn(v);
-        else
-            ((float*)y)[(size_t)b * m + row] = v;
+    const uint32_t sw = sout_bits[row >> 5] >> (row & 31);
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = ((sw >> q) & 1u) ? -v[q] * scale : v[q] * scale;
+    if (F16) {
+        __half* ys = (__half*)y + (size_t)b * m + row;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) {
+            const __half2 lo = __floats2half2_rn(v[q], v[q + 1]);
+            const __half2 hi = __floats2half2_rn(v[q + 2], v[q + 3]);
+            uint2 w;
+            w.x = *reinterpret_cast<const uint32_t*>(&lo);
+            w.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(ys + q) = w;
+        }
+    } else {
+        float* ys = (float*)y + (size_t)b * m + row;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) *reinterpret_cast<float4*>(ys + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
     }
 }
 
-cudaError_t launch_rht_out(const Layer& L, const float* z, int batch, void* y, int y_dtype, cudaStream_t st) {
-    const int B = L.B_m;
-    const size_t smem = (size_t)B * sizeof(float);
-    auto kern = (y_dtype == QL_F16) ? rht_out_kernel<true> : rht_out_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(L.m / B, batch);
-    const int threads = B >= 1024 ? 1024 : (B >= 64 ? B : 64);
-    kern<<<grid, threads, smem, st>>>(z, batch, L.m, B, L.sout_bits, L.alpha, y);
-    return cudaGetLastError();
+template <bool F16, int E>
+static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y, cudaStream_t st) {
+    const RhtGeometry geo = rht_geometry(L.m, L.B_m, batch, E);
+    const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
+    auto kern = rht_out_kernel<F16, E>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (kMaxHadamard + kMaxHadamard / 16) * 4);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int grid = (geo.total + geo.groups - 1) / geo.groups;
+    return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, z, batch, L.m, geo,
+                      (const uint32_t*)L.sout_bits, L.alpha, y);
+}
+
+cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st) {
+    const bool f16 = y_dtype == QL_F16;
+    if (L.B_m > 16384) return f16 ? launch_rht_out_e<true, 32>(L, z, batch, y, st) : launch_rht_out_e<false, 32>(L, z, batch, y, st);
+    return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
 }
 
 }  // namespace qlk
