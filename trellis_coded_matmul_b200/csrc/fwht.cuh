@@ -1,0 +1,122 @@
+// fwht.cuh -- fast Walsh-Hadamard transform building blocks (device code).
+//
+// H_B is the normalised Sylvester matrix; the fast transform applies the
+// butterfly (a, b) -> (a + b, a - b) for every stride 1, 2, ..., B/2 (the
+// strides commute).  A group of T = B/E threads owns one block, E consecutive
+// entries per thread: strides below E in registers, strides E .. 16E by warp
+// shuffles, longer strides through padded shared memory four at a time.
+#pragma once
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace qlk {
+
+__device__ __forceinline__ bool sign_neg(const uint32_t* bits, int i) { return (bits[i >> 5] >> (i & 31)) & 1u; }
+__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
+
+template <int LOGR>
+__device__ __forceinline__ void fwht_pass(float* buf, int B, int h, int tid, int nthreads) {
+    constexpr int R = 1 << LOGR;
+    const int groups = B >> LOGR;
+    for (int gi = tid; gi < groups; gi += nthreads) {
+        const int base = (gi / h) * (h << LOGR) + (gi % h);
+        float v[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) v[q] = buf[pad16(base + q * h)];
+#pragma unroll
+        for (int s = 0; s < LOGR; ++s) {
+#pragma unroll
+            for (int q = 0; q < R; ++q) {
+                if (!(q & (1 << s))) {
+                    const float a = v[q], b = v[q | (1 << s)];
+                    v[q] = a + b;
+                    v[q | (1 << s)] = a - b;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < R; ++q) buf[pad16(base + q * h)] = v[q];
+    }
+}
+
+// Strides E.. of the remaining FWHT through shared memory (padded layout) by
+// the `nthreads` threads of the group, starting at stride h0; ends with a
+// CTA barrier after every pass.
+// Threads with active == false touch no memory but take part in every barrier.
+__device__ __forceinline__ void fwht_smem_passes(float* buf, int B, int h0, int tid, int nthreads, bool active) {
+    int h = h0;
+    while (h < B) {
+        const int rem = 31 - __clz(B / h);  // log2(B / h)
+        if (rem >= 4) {
+            if (active) fwht_pass<4>(buf, B, h, tid, nthreads);
+            h <<= 4;
+        } else if (rem == 3) {
+            if (active) fwht_pass<3>(buf, B, h, tid, nthreads);
+            h <<= 3;
+        } else if (rem == 2) {
+            if (active) fwht_pass<2>(buf, B, h, tid, nthreads);
+            h <<= 2;
+        } else {
+            if (active) fwht_pass<1>(buf, B, h, tid, nthreads);
+            h <<= 1;
+        }
+        __syncthreads();
+    }
+}
+
+// Full FWHT of a group's block: v holds the thread's E consecutive entries
+// (thread tid of T owns entries [tid*E, tid*E + E)); on return v holds the
+// same positions of the transformed block.  `buf` is the group's shared
+// memory (B + B/16 floats), used only when T > 32.  Every thread of the CTA
+// must call this with the same B (it contains CTA barriers when T > 32);
+// threads with use_smem == false (spare threads outside any group) skip the
+// shared-memory traffic but keep the barriers.
+template <int E>
+__device__ __forceinline__ void fwht_block(float (&v)[E], int B, int tid, int T, float* buf, bool use_smem = true) {
+#pragma unroll
+    for (int s = 1; s < E; s <<= 1) {
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            if (!(q & s)) {
+                const float a = v[q], b = v[q | s];
+                v[q] = a + b;
+                v[q | s] = a - b;
+            }
+        }
+    }
+    const int lanes = T < 32 ? T : 32;
+    const int lane = threadIdx.x & 31;
+    for (int j = 1; j < lanes; j <<= 1) {
+        const bool upper = lane & j;
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[q], j);
+            v[q] = upper ? (o - v[q]) : (v[q] + o);
+        }
+    }
+    if (T > 32) {
+        if (use_smem) {
+#pragma unroll
+            for (int q = 0; q < E; ++q) buf[pad16(tid * E + q)] = v[q];
+        }
+        __syncthreads();
+        fwht_smem_passes(buf, B, 32 * E, tid, T, use_smem);
+        if (use_smem) {
+#pragma unroll
+            for (int q = 0; q < E; ++q) v[q] = buf[pad16(tid * E + q)];
+        }
+    }
+}
+
+// Fragment layout of x' for the decode-GEMV: the 8-byte group
+//   frag[((j*16 + u) * batch + b) * 4 + c] = x'[b][256 j + 64 c + 4 u + 0..3]
+// is what lane (g = b, c) needs as its B operand for the u-th m16n8k16 MMA of
+// block j (see gemv.cu).  Returns the index of the first of the four halves.
+__device__ __forceinline__ size_t frag_index4(int col, int b, int batch) {
+    const int j = col >> 8, within = col & 255;
+    const int c = within >> 6, r = within & 63;
+    const int u = r >> 2;
+    return ((((size_t)j * 16 + u) * batch + b) * 4 + c) * 4;
+}
+
+}  // namespace qlk

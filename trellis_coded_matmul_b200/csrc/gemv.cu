@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 
 #include "codes.cuh"
+#include "fwht.cuh"
 #include "internal.h"
 #include "layout.cuh"
 
@@ -156,21 +157,78 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 
 struct GemvArgs {
     DecodeArgs dec;
-    const uint2* xf;  // x' fragment layout
+    const uint2* xf;  // x' fragment layout in global memory (when x' is not computed in-kernel)
     int batch;        // 1..8
-    float* z;         // [batch][m]
+    float* z;         // [batch][m], all-zero on entry (the output transform re-zeroes it)
     int m;
     int row0;         // first layer row of the part
+    // input transform in-kernel (XSMEM): x' = H_n diag(s_in) x into shared memory
+    const __half* x;  // [batch][n]
+    const uint32_t* sin_bits;
+    int n, B_n;
+    int groups_in;    // thread groups (B_n/16 threads each) of the in-kernel input transform
 };
 
-// One CTA per SM.  CTA b takes units [U*b/G, U*(b+1)/G) of the part (G CTAs)
+// x' = H_n diag(s_in) x for every column and batch row, fp16, into the
+// fragment layout in shared memory.  Groups of B_n/16 threads take one
+// (batch row, Hadamard block) at a time; all threads run the same rounds.
+__device__ __forceinline__ void input_transform_smem(const GemvArgs& p, __half* xs, float* fw) {
+    const int B = p.B_n, T = B / 16;
+    const int G = p.groups_in;  // groups with their own FWHT scratch; spare threads only join barriers
+    const int grp = threadIdx.x / T, tid = threadIdx.x % T;
+    const int per_row = p.n / B, total = p.batch * per_row;
+    const float scale = rsqrtf((float)B);
+    for (int r0 = 0; r0 < total; r0 += G) {
+        const int item = r0 + grp;
+        const bool active = grp < G && item < total;
+        const int b = active ? item / per_row : 0;
+        const int col = (active ? (item % per_row) * B : 0) + tid * 16;
+        float v[16];
+        if (active) {
+            const __half* src = p.x + (size_t)b * p.n + col;
+            const uint32_t sw = p.sin_bits[col >> 5] >> (col & 31);
+#pragma unroll
+            for (int q = 0; q < 16; q += 8) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(src + q);
+                const __half* hv = reinterpret_cast<const __half*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float f = __half2float(hv[e]);
+                    v[q + e] = ((sw >> (q + e)) & 1u) ? -f : f;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = 0.f;
+        }
+        fwht_block<16>(v, B, tid, T, fw + (size_t)(grp < G ? grp : 0) * (B + B / 16), grp < G);
+        if (active) {
+#pragma unroll
+            for (int q = 0; q < 16; q += 4) {
+                const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
+                const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
+                uint2 w;
+                w.x = *reinterpret_cast<const uint32_t*>(&lo);
+                w.y = *reinterpret_cast<const uint32_t*>(&hi);
+                *reinterpret_cast<uint2*>(xs + frag_index4(col + q, b, p.batch)) = w;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// One CTA per SM.  CTA i takes units [U*i/G, U*(i+1)/G) of the part (G CTAs)
 // and splits them evenly over its warps; the launcher sizes the CTA so that
 // every warp gets the same whole number of units (to within one), which keeps
-// every SM and every warp equally loaded.
-template <int CODE, int K, int V, bool L16>
-__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p) {
-    extern __shared__ uint32_t lut_smem[];
+// every SM and every warp equally loaded.  Every thread runs every phase (no
+// early exit), since the in-kernel transforms use CTA barriers.
+template <int CODE, int K, int V, bool L16, bool XSMEM>
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p, GemvSmem sm) {
+    extern __shared__ uint32_t smem[];
     using UL = UnitLayout<K>;
+    uint32_t* lut_smem = smem;
+    __half* xs = reinterpret_cast<__half*>(smem + sm.lut_words);
+    float* fw = reinterpret_cast<float*>(smem + sm.lut_words + sm.xs_words);
     const int lane = threadIdx.x & 31;
     if (CODE == kCodeHYB) {
         fill_lut_smem(lut_smem, p.dec.lut, p.dec.lut_entries);
@@ -182,27 +240,23 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p)
     const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
     const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
     const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
-    if (u0 >= u1) {
-        grid_dependency_wait();
-        grid_launch_dependents();
-        return;
-    }
 
     const int g = lane >> 2, c = lane & 3;
     const int src_lane = (lane & ~3) | ((c + 3) & 3);
     const int batch = p.batch;
 
     uint32_t nxt[2][2 * K];
-    load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
+    if (u0 < u1) load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
     // Programmatic dependent launch: the code words (and the HYB table) are
     // written once at create time, so they are fetched before waiting for the
-    // kernel that produces x' (and, before it, the consumer of the previous z).
+    // previous kernel (the producer of x or x', the consumer of the last z).
     grid_dependency_wait();
+    if (XSMEM) input_transform_smem(p, xs, fw);
     grid_launch_dependents();
+
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int R = (int)(u0 / nb), j = (int)(u0 % nb);
     int curR = R;
-
     auto flush = [&](int tile) {
         const int row = p.row0 + tile * kRowTile + g;
         const int b0 = 2 * c, b1 = 2 * c + 1;
@@ -221,7 +275,7 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int w = 0; w < 2 * K; ++w) cw[h][w + 1] = nxt[h][w];
+            for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = nxt[h][i];
         if (unit + 1 < u1) load_unit<K>(nxt, p.dec.words + (unit + 1) * UL::UW, lane);
         if (R != curR) {
             flush(curR);
@@ -231,10 +285,15 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p)
 #pragma unroll
         for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
 
-        const uint2* xb = p.xf + (size_t)j * 16 * batch * 4 + g * 4 + c;
+        const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
         for_each_mma<CODE, K, V, L16>(cw, p.dec.lmask, lut_lane, p.dec.qshift, [&](int u, const uint32_t(&a)[4]) {
             uint2 bv = make_uint2(0u, 0u);
-            if (g < batch) bv = __ldg(xb + (size_t)u * batch * 4);
+            if (g < batch) {
+                if (XSMEM)
+                    bv = reinterpret_cast<const uint2*>(xs)[xoff + (size_t)u * batch * 4];
+                else
+                    bv = __ldg(p.xf + xoff + (size_t)u * batch * 4);
+            }
             mma_16816(acc, a, bv.x, bv.y);
         });
         if (++j == nb) {
@@ -242,7 +301,7 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p)
             ++R;
         }
     }
-    flush(curR);
+    if (u0 < u1) flush(curR);
 }
 
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
@@ -366,21 +425,76 @@ static DecodeArgs make_decode_args(const Layer& L, const Part& part) {
 
 template <int CODE, int K, int V, bool L16>
 struct GemvLaunch {
-    static cudaError_t run(const GemvArgs& a, int grid, int threads, cudaStream_t st) {
-        const size_t smem = (size_t)a.dec.lut_entries * 32 * 4;
-        auto kern = gemv_kernel<CODE, K, V, L16>;
+    static cudaError_t run(const GemvArgs& a, const GemvSmem& sm, bool xsmem, int grid, int threads,
+                           cudaStream_t st) {
+        const size_t smem = (size_t)(sm.lut_words + sm.xs_words + sm.fw_words) * 4;
+        if (xsmem) {
+            if (!L16) return cudaErrorInvalidValue;
+            auto kern = gemv_kernel<CODE, K, V, true, true>;
+            static bool attr_set = false;
+            if (!attr_set) {
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
+                if (e != cudaSuccess) return e;
+                attr_set = true;
+            }
+            return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
+        }
+        auto kern = gemv_kernel<CODE, K, V, L16, false>;
         static bool attr_set = false;
-        if (smem > 48 * 1024 && !attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
+        if (!attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
             if (e != cudaSuccess) return e;
             attr_set = true;
         }
-        return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a);
+        return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
     }
 };
 
-cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, int batch, float* z,
-                        cudaStream_t st) {
+// CTA shape: one CTA per SM, warps sized so every warp gets the same whole
+// number of units.  The input transform runs in-kernel (each CTA computes
+// x' into its shared memory while its first code words are in flight) when
+// x is small; otherwise a separate kernel writes x' to global memory.
+GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
+    GemvPlan pl;
+    const long long nb = L.n / kT;
+    const long long units = (long long)(part.rows / kRowTile) * nb;
+    pl.grid = (int)(units < L.num_sms ? units : L.num_sms);
+    const long long per_cta = (units + pl.grid - 1) / pl.grid;
+    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
+    int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
+    const int lut_words = L.code == kCodeHYB ? (32 << L.Q) : 0;
+    const int budget = kGemvMaxSmem / 4 - lut_words;
+    const int t_in = L.B_n / 16;
+    const int xs_words = batch * L.n / 2;
+    pl.xsmem = L.L == 16 && L.nparts == 1 && (long long)batch * L.n <= kFuseInElems &&
+               t_in <= kGemvMaxWarps * 32;
+    int fw = 0;
+    pl.groups_in = 0;
+    if (pl.xsmem) {
+        if (threads < t_in) threads = t_in;
+        // thread groups of B_n/16 threads; a group of more than a warp needs
+        // its own FWHT scratch (B_n + B_n/16 floats)
+        int g = threads / t_in;
+        const int work = batch * (L.n / L.B_n);
+        if (g > work) g = work;
+        if (g < 1) g = 1;
+        if (t_in > 32) {
+            const int per = L.B_n + L.B_n / 16;
+            while (g > 1 && xs_words + g * per > budget) --g;
+            fw = g * per;
+        }
+        pl.groups_in = g;
+        if (xs_words + fw > budget) pl.xsmem = false, fw = 0, pl.groups_in = 0;
+    }
+    pl.threads = threads;
+    pl.sm.lut_words = lut_words;
+    pl.sm.xs_words = pl.xsmem ? xs_words : 0;
+    pl.sm.fw_words = fw;
+    return pl;
+}
+
+cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
+                        int batch, float* z, cudaStream_t st) {
     GemvArgs a;
     a.dec = make_decode_args(L, part);
     a.xf = (const uint2*)xp_frag;
@@ -388,12 +502,12 @@ cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, i
     a.z = z;
     a.m = L.m;
     a.row0 = part.row0;
-    const long long units = (long long)a.dec.rt * a.dec.nb;
-    long long grid = units < L.num_sms ? units : L.num_sms;
-    const long long per_cta = (units + grid - 1) / grid;
-    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
-    const int warps = (int)((per_cta + per_warp - 1) / per_warp);
-    return dispatch<GemvLaunch>(L.code, part.k, L.V, L.L == 16, a, (int)grid, warps * 32, st);
+    a.x = (const __half*)x;
+    a.sin_bits = L.sin_bits;
+    a.n = L.n;
+    a.B_n = L.B_n;
+    a.groups_in = pl.groups_in;
+    return dispatch<GemvLaunch>(L.code, part.k, L.V, L.L == 16, a, pl.sm, pl.xsmem, pl.grid, pl.threads, st);
 }
 
 template <int CODE, int K, int V, bool L16>

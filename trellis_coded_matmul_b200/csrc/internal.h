@@ -12,7 +12,12 @@ constexpr int kT = 256;            // columns per trellis block
 constexpr int kRowTile = 16;       // rows per decode tile (the m16n8k16 M dimension)
 constexpr int kMaxHadamard = 32768;
 
-constexpr int kGemvMaxWarps = 24;  // decode-GEMV: warps of its one CTA per SM (<= 85 registers/thread)
+constexpr int kGemvMaxWarps = 24;        // decode-GEMV: warps of its one CTA per SM (<= 85 registers/thread)
+constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
+constexpr int kFuseInElems = 16384;  // batch * n up to which the GEMV computes x' itself
+constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
+constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
+constexpr int kTcMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA
 
 // Device status word bits (qlinear_get_status).
 constexpr int kStatusBadSign = 1;
@@ -89,15 +94,33 @@ cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cu
 
 // x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
-// x (fp16 [batch][n]) -> x' fp16 [batch][n] row-major.
-cudaError_t launch_rht_in_rowmajor(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
+// x (fp16 [batch][n]) -> x' as tensor-core operand tiles: [n/64][npad][128 B],
+// the 16-byte chunk c of row b at chunk c ^ (b % 8) (rows >= batch untouched).
+cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st);
 // z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st);
 
-// z[b][row0 + r] += sum_c W_hat[row0 + r][c] x'[b][c] for the part's rows; batch <= 8.
-cudaError_t launch_gemv(const Layer& L, const Part& part, const void* xp_frag, int batch, float* z,
-                        cudaStream_t st);
+// How one decode-GEMV launch is shaped: grid and CTA size, its shared memory
+// (32-bit words: replicated HYB table, x' fragments, FWHT scratch), and
+// whether the input transform runs inside it (xsmem).
+struct GemvSmem {
+    int lut_words, xs_words, fw_words;
+};
+struct GemvPlan {
+    int grid, threads;
+    bool xsmem;
+    int groups_in;
+    GemvSmem sm;
+};
+GemvPlan plan_gemv(const Layer& L, const Part& part, int batch);
+// z[b][row0 + r] += sum_c W_hat[row0 + r][c] x'[b][c] for the part's rows, batch <= 8;
+// with pl.xsmem x' is computed from x in-kernel, else read from xp_frag.
+cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
+                        int batch, float* z, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
+// z[b][row] = W_hat x' for all parts, x' in tensor-core tiles with npad (multiple
+// of 16, <= 256) rows, b < batch; one 128-row tile per CTA.
+cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st);
 cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words,
                              const uint32_t* states, int count, void* out, cudaStream_t st);
 

@@ -198,30 +198,68 @@ int ensure(void** buf, size_t* have, size_t bytes) {
 }
 
 // The z accumulator is all-zero between forwards: it is zeroed when
-// allocated, and the output-transform kernel re-zeroes what it consumed.
-int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
-    const int chunk = batch < 8 ? batch : 8;
-    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)chunk * L.n * 2);
+// allocated, and the output-transform kernel re-zeroes what it consumed (the
+// tensor-core GEMM overwrites z, which keeps the same invariant).
+int prepare_z(Layer& L, size_t bytes, cudaStream_t st) {
+    if (L.z_bytes >= bytes && !L.z_dirty) return QL_OK;
+    int rc = ensure((void**)&L.z, &L.z_bytes, bytes);
     if (rc != QL_OK) return rc;
-    const size_t zb = (size_t)chunk * L.m * 4;
-    if (L.z_bytes < zb || L.z_dirty) {
-        rc = ensure((void**)&L.z, &L.z_bytes, zb);
-        if (rc != QL_OK) return rc;
-        if (cudaMemsetAsync(L.z, 0, L.z_bytes, st) != cudaSuccess) {
-            cudaGetLastError();
-            return QL_E_CUDA;
-        }
-        L.z_dirty = 0;
+    if (cudaMemsetAsync(L.z, 0, L.z_bytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
     }
+    L.z_dirty = 0;
+    return QL_OK;
+}
+
+// batch <= 8: decode-GEMV (input transform in-kernel for small x, else a
+// separate kernel), then the output transform.
+int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
+    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)batch * L.n * 2);
+    if (rc == QL_OK) rc = prepare_z(L, (size_t)batch * L.m * 4, st);
+    if (rc != QL_OK) return rc;
+    // One plan for all parts (a half-TCQ layer never fuses the input transform).
+    const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
+    cudaError_t e = cudaSuccess;
+    if (!pl.xsmem) e = launch_rht_in_frag(L, x, batch, L.xp, st);
+    const int slot = L.prof_cap ? L.prof_next : -1;
+    if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
+    for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) {
+        const GemvPlan pi = i == 0 ? pl : plan_gemv(L, L.parts[i], batch);
+        e = launch_gemv(L, L.parts[i], pi, x, L.xp, batch, L.z, st);
+    }
+    if (e == cudaSuccess && slot >= 0) {
+        e = record_event(L.prof_ev[2 * slot + 1], st);
+        L.prof_next = (L.prof_next + 1) % L.prof_cap;
+        if (L.prof_count < L.prof_cap) ++L.prof_count;
+    }
+    if (e == cudaSuccess) e = launch_rht_out(L, L.z, batch, y, y_dtype, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        L.z_dirty = 1;  // a partial forward may have left sums in z
+        return QL_E_CUDA;
+    }
+    return QL_OK;
+}
+
+// batch > 8: input transform into tensor-core operand tiles, tcgen05 GEMM,
+// output transform; batches above 256 run in passes of 256.
+int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
+    const int chunk = batch < kTcMaxN ? batch : kTcMaxN;
+    const int npad_max = (chunk + 15) / 16 * 16;
+    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)npad_max * L.n * 2);
+    if (rc == QL_OK) rc = prepare_z(L, (size_t)chunk * L.m * 4, st);
+    if (rc != QL_OK) return rc;
     const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
-    for (int b0 = 0; b0 < batch; b0 += 8) {
-        const int nb = batch - b0 < 8 ? batch - b0 : 8;
+    for (int b0 = 0; b0 < batch; b0 += kTcMaxN) {
+        const int nb = batch - b0 < kTcMaxN ? batch - b0 : kTcMaxN;
+        const int npad = (nb + 15) / 16 * 16;
         const void* xb = (const char*)x + (size_t)b0 * L.n * 2;
         void* yb = (char*)y + (size_t)b0 * L.m * ysz;
-        cudaError_t e = launch_rht_in_frag(L, xb, nb, L.xp, st);
+        cudaError_t e = launch_rht_in_umma(L, xb, nb, npad, L.xp, st);
         const int slot = L.prof_cap ? L.prof_next : -1;
         if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-        for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) e = launch_gemv(L, L.parts[i], L.xp, nb, L.z, st);
+        if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, L.z, st);
         if (e == cudaSuccess && slot >= 0) {
             e = record_event(L.prof_ev[2 * slot + 1], st);
             L.prof_next = (L.prof_next + 1) % L.prof_cap;
@@ -230,11 +268,15 @@ int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cud
         if (e == cudaSuccess) e = launch_rht_out(L, L.z, nb, yb, y_dtype, st);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            L.z_dirty = 1;  // a partial forward may have left sums in z
+            L.z_dirty = 1;
             return QL_E_CUDA;
         }
     }
     return QL_OK;
+}
+
+int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
+    return batch <= kGemvMaxBatch ? forward_gemv(L, x, batch, y, y_dtype, st) : forward_tc(L, x, batch, y, y_dtype, st);
 }
 
 }  // namespace

@@ -22,110 +22,10 @@
 // so the accumulation buffer is ready for the next forward without a memset.
 #include <cuda_fp16.h>
 
+#include "fwht.cuh"
 #include "internal.h"
 
 namespace qlk {
-
-__device__ __forceinline__ bool sign_neg(const uint32_t* bits, int i) { return (bits[i >> 5] >> (i & 31)) & 1u; }
-__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
-
-template <int LOGR>
-__device__ __forceinline__ void fwht_pass(float* buf, int B, int h, int tid, int nthreads) {
-    constexpr int R = 1 << LOGR;
-    const int groups = B >> LOGR;
-    for (int gi = tid; gi < groups; gi += nthreads) {
-        const int base = (gi / h) * (h << LOGR) + (gi % h);
-        float v[R];
-#pragma unroll
-        for (int q = 0; q < R; ++q) v[q] = buf[pad16(base + q * h)];
-#pragma unroll
-        for (int s = 0; s < LOGR; ++s) {
-#pragma unroll
-            for (int q = 0; q < R; ++q) {
-                if (!(q & (1 << s))) {
-                    const float a = v[q], b = v[q | (1 << s)];
-                    v[q] = a + b;
-                    v[q | (1 << s)] = a - b;
-                }
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < R; ++q) buf[pad16(base + q * h)] = v[q];
-    }
-}
-
-// Strides E.. of the remaining FWHT through shared memory (padded layout) by
-// the `nthreads` threads of the group, starting at stride h0; ends with a
-// CTA barrier after every pass.
-__device__ __forceinline__ void fwht_smem_passes(float* buf, int B, int h0, int tid, int nthreads) {
-    int h = h0;
-    while (h < B) {
-        const int rem = 31 - __clz(B / h);  // log2(B / h)
-        if (rem >= 4) {
-            fwht_pass<4>(buf, B, h, tid, nthreads);
-            h <<= 4;
-        } else if (rem == 3) {
-            fwht_pass<3>(buf, B, h, tid, nthreads);
-            h <<= 3;
-        } else if (rem == 2) {
-            fwht_pass<2>(buf, B, h, tid, nthreads);
-            h <<= 2;
-        } else {
-            fwht_pass<1>(buf, B, h, tid, nthreads);
-            h <<= 1;
-        }
-        __syncthreads();
-    }
-}
-
-// Full FWHT of a group's block: v holds the thread's E consecutive entries
-// (thread tid of T owns entries [tid*E, tid*E + E)); on return v holds the
-// same positions of the transformed block.  `buf` is the group's shared
-// memory (B + B/16 floats), used only when T > 32.  Every thread of the CTA
-// must call this with the same B (it contains CTA barriers when T > 32).
-template <int E>
-__device__ __forceinline__ void fwht_block(float (&v)[E], int B, int tid, int T, float* buf) {
-#pragma unroll
-    for (int s = 1; s < E; s <<= 1) {
-#pragma unroll
-        for (int q = 0; q < E; ++q) {
-            if (!(q & s)) {
-                const float a = v[q], b = v[q | s];
-                v[q] = a + b;
-                v[q | s] = a - b;
-            }
-        }
-    }
-    const int lanes = T < 32 ? T : 32;
-    const int lane = threadIdx.x & 31;
-    for (int j = 1; j < lanes; j <<= 1) {
-        const bool upper = lane & j;
-#pragma unroll
-        for (int q = 0; q < E; ++q) {
-            const float o = __shfl_xor_sync(0xffffffffu, v[q], j);
-            v[q] = upper ? (o - v[q]) : (v[q] + o);
-        }
-    }
-    if (T > 32) {
-#pragma unroll
-        for (int q = 0; q < E; ++q) buf[pad16(tid * E + q)] = v[q];
-        __syncthreads();
-        fwht_smem_passes(buf, B, 32 * E, tid, T);
-#pragma unroll
-        for (int q = 0; q < E; ++q) v[q] = buf[pad16(tid * E + q)];
-    }
-}
-
-// Fragment layout of x' for the decode-GEMV: the 8-byte group
-//   frag[((j*16 + u) * batch + b) * 4 + c] = x'[b][256 j + 64 c + 4 u + 0..3]
-// is what lane (g = b, c) needs as its B operand for the u-th m16n8k16 MMA of
-// block j (see gemv.cu).  Returns the index of the first of the four halves.
-__device__ __forceinline__ size_t frag_index4(int col, int b, int batch) {
-    const int j = col >> 8, within = col & 255;
-    const int c = within >> 6, r = within & 63;
-    const int u = r >> 2;
-    return ((((size_t)j * 16 + u) * batch + b) * 4 + c) * 4;
-}
 
 struct RhtGeometry {
     int B;        // Hadamard block size
@@ -147,10 +47,20 @@ static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
     return g;
 }
 
-// FRAG: write x' in the decode-GEMV fragment layout (else row-major [batch][n]).
-template <bool FRAG, int E>
+// Output layouts of x': the decode-GEMV fragment layout, row-major [batch][n],
+// or the tensor-core operand tiles (64-column K stages of npad rows of 128
+// bytes, 16-byte chunk c of row b stored at chunk c ^ (b % 8)).
+enum { kXpFrag = 0, kXpRowMajor = 1, kXpUmma = 2 };
+
+__device__ __forceinline__ size_t umma_tile_index4(int col, int b, int npad) {
+    const int s = col >> 6, kin = col & 63;
+    const int chunk = (kin >> 3) ^ (b & 7);
+    return (((size_t)s * npad + b) * 128 + chunk * 16 + (kin & 7) * 2) / 2;  // in halves
+}
+
+template <int MODE, int E>
 __global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, RhtGeometry geo,
-                              const uint32_t* __restrict__ sin_bits, __half* __restrict__ out) {
+                              const uint32_t* __restrict__ sin_bits, __half* __restrict__ out, int npad) {
     extern __shared__ float smem[];
     grid_dependency_wait();
     const int B = geo.B;
@@ -189,18 +99,20 @@ __global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, Rh
         uint2 w;
         w.x = *reinterpret_cast<const uint32_t*>(&lo);
         w.y = *reinterpret_cast<const uint32_t*>(&hi);
-        if (FRAG)
+        if (MODE == kXpFrag)
             *reinterpret_cast<uint2*>(out + frag_index4(col + q, b, batch)) = w;
+        else if (MODE == kXpUmma)
+            *reinterpret_cast<uint2*>(out + umma_tile_index4(col + q, b, npad)) = w;
         else
             *reinterpret_cast<uint2*>(out + (size_t)b * n + col + q) = w;
     }
 }
 
-template <bool FRAG, int E>
-static cudaError_t launch_rht_in_e(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
+template <int MODE, int E>
+static cudaError_t launch_rht_in_e(const Layer& L, const void* x, int batch, void* xp, int npad, cudaStream_t st) {
     const RhtGeometry geo = rht_geometry(L.n, L.B_n, batch, E);
     const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
-    auto kern = rht_in_kernel<FRAG, E>;
+    auto kern = rht_in_kernel<MODE, E>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -210,21 +122,21 @@ static cudaError_t launch_rht_in_e(const Layer& L, const void* x, int batch, voi
     }
     const int grid = (geo.total + geo.groups - 1) / geo.groups;
     return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, (const __half*)x, batch, L.n, geo,
-                      (const uint32_t*)L.sin_bits, (__half*)xp);
+                      (const uint32_t*)L.sin_bits, (__half*)xp, npad);
 }
 
-template <bool FRAG>
-static cudaError_t launch_rht_in(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    return L.B_n > 16384 ? launch_rht_in_e<FRAG, 32>(L, x, batch, xp, st)
-                         : launch_rht_in_e<FRAG, 16>(L, x, batch, xp, st);
+template <int MODE>
+static cudaError_t launch_rht_in(const Layer& L, const void* x, int batch, void* xp, int npad, cudaStream_t st) {
+    return L.B_n > 16384 ? launch_rht_in_e<MODE, 32>(L, x, batch, xp, npad, st)
+                         : launch_rht_in_e<MODE, 16>(L, x, batch, xp, npad, st);
 }
 
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    return launch_rht_in<true>(L, x, batch, xp, st);
+    return launch_rht_in<kXpFrag>(L, x, batch, xp, 0, st);
 }
 
-cudaError_t launch_rht_in_rowmajor(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    return launch_rht_in<false>(L, x, batch, xp, st);
+cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st) {
+    return launch_rht_in<kXpUmma>(L, x, batch, xt, npad, st);
 }
 
 // Entries per thread of the output transform: B_m may be as small as 16.
