@@ -98,6 +98,7 @@ typedef struct {
     size_t sign_bytes;         /* bit-packed signs: (n + m) bits, word-padded    */
     size_t lut_bytes;          /* HYB table: 2^Q * V * 2 bytes                   */
     size_t scratch_bytes;      /* device scratch currently held by the handle    */
+    int last_launches;         /* kernels launched by the most recent forward    */
 } ql_info_t;
 
 /* Create a uniform-bitrate layer.

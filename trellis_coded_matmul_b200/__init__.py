@@ -46,7 +46,8 @@ class ql_code_t(ctypes.Structure):
 
 class ql_info_t(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int) for f in ("m", "n", "L", "V", "code", "Q", "k_top", "k_bot", "m_top", "B_n", "B_m")] + \
-               [(f, ctypes.c_size_t) for f in ("stream_bytes", "sign_bytes", "lut_bytes", "scratch_bytes")]
+               [(f, ctypes.c_size_t) for f in ("stream_bytes", "sign_bytes", "lut_bytes", "scratch_bytes")] + \
+               [("last_launches", ctypes.c_int)]
 
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float

@@ -53,6 +53,7 @@ struct Layer {
     float* z;             // W_hat x' before the output transform, fp32 [batch][m]; all-zero between forwards
     size_t z_bytes;
     int z_dirty;          // z may hold partial sums (a forward failed part-way)
+    int last_launches;    // kernels launched by the most recent forward
     void* host_stage;     // device staging for qlinear_forward_host (x then y)
     size_t host_stage_bytes;
     int num_sms;

@@ -221,6 +221,7 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
     // One plan for all parts (a half-TCQ layer never fuses the input transform).
     const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
     cudaError_t e = cudaSuccess;
+    L.last_launches = L.nparts + 1 + (pl.xsmem ? 0 : 1);
     if (!pl.xsmem) e = launch_rht_in_frag(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
@@ -251,6 +252,7 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
     if (rc == QL_OK) rc = prepare_z(L, (size_t)chunk * L.m * 4, st);
     if (rc != QL_OK) return rc;
     const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
+    L.last_launches = 3 * ((batch + kTcMaxN - 1) / kTcMaxN);
     for (int b0 = 0; b0 < batch; b0 += kTcMaxN) {
         const int nb = batch - b0 < kTcMaxN ? batch - b0 : kTcMaxN;
         const int npad = (nb + 15) / 16 * 16;
@@ -415,6 +417,7 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
     info->lut_bytes = L.code == QL_CODE_HYB ? ((size_t)1 << L.Q) * L.V * 2 : 0;
     info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
+    info->last_launches = L.last_launches;
     return QL_OK;
 }
 
@@ -488,3 +491,4 @@ const char* qlinear_strerror(int status) {
 }
 
 }  // extern "C"
+
