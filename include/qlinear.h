@@ -67,6 +67,7 @@ extern "C" {
 #define QL_E_OOM (-4)          /* device allocation failed                                */
 #define QL_E_TIMEOUT (-5)      /* a bounded device-side wait gave up                      */
 #define QL_E_DEVICE (-6)       /* a device-side check failed (see qlinear_get_status)     */
+#define QL_E_SCRATCH (-7)      /* sizes exceed the fixed scratch of qlinear_forward_noalloc */
 
 #define QL_CODE_1MAD 0
 #define QL_CODE_3INST 1
@@ -142,6 +143,27 @@ int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype,
  * copies asynchronous DMA transfers; pageable memory also works. */
 int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype,
                          void* stream);
+
+/* As qlinear_forward for batch <= 8, without allocating or freeing any
+ * memory.  None of the pages has a counterpart: this serves callers that
+ * cannot let a library allocate while they run (cudaMalloc/cudaFree may
+ * synchronise the whole device and stall a serving process's other streams;
+ * runtimes that pre-carve all free HBM into their own pools leave no room).
+ *   Scratch: x' and the fp32 accumulator z live in one fixed array of
+ *   QL_NOALLOC_SCRATCH_BYTES in the library's static device memory, per
+ *   device: round_up(batch*n*2, 256) + batch*m*4 bytes must fit, else
+ *   QL_E_SCRATCH (before any device work).  Every call clears its part of z
+ *   on `stream` first.
+ *   Sharing: all handles on a device share the array, so calls that overlap
+ *   in time (different streams or host threads) race and give wrong y; calls
+ *   in order on one stream are safe.
+ *   Set-up: a device's first call looks up the array's address
+ *   (cudaGetSymbolAddress), which may load the library's device code; make
+ *   that first call before any stream capture.
+ *   Profiling slots (qlinear_profile_enable) are not recorded by this call.
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED (batch > 8), QL_E_SCRATCH, QL_E_CUDA. */
+#define QL_NOALLOC_SCRATCH_BYTES (2 * 1024 * 1024)
+int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream);
 
 /* Write W_hat as fp16 [m][n] row-major to the device pointer w_hat (the code
  * values before alpha, signs and Hadamard transforms).  For testing. */

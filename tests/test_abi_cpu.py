@@ -84,3 +84,12 @@ def test_other_entry_points_reject_null_handles(tcm):
     mixed = lib.qlinear_create_mixed
     h = ctypes.c_void_p()
     assert mixed(ctypes.byref(h), 64, 256, 64, 2, 3, 16, 1, code, None, 0, None, None, 1.0) == tcm.QL_E_ARG
+
+
+def test_forward_noalloc_rejects_bad_arguments_on_the_host(tcm):
+    lib = tcm.raw_library()
+    assert lib.qlinear_forward_noalloc(None, None, 1, None, tcm.QL_F32, None) == tcm.QL_E_ARG
+    assert tcm.qlinear_strerror(tcm.QL_E_SCRATCH).startswith("request exceeds the fixed scratch")
+    header = open(os.path.join(ROOT, "include", "qlinear.h")).read()
+    assert re.search(r"#define QL_NOALLOC_SCRATCH_BYTES \(2 \* 1024 \* 1024\)", header)
+    assert tcm.QL_NOALLOC_SCRATCH_BYTES == 2 * 1024 * 1024

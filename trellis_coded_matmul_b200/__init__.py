@@ -28,6 +28,8 @@ QL_E_CUDA = -3
 QL_E_OOM = -4
 QL_E_TIMEOUT = -5
 QL_E_DEVICE = -6
+QL_E_SCRATCH = -7
+QL_NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
 QL_CODE_1MAD = 0
 QL_CODE_3INST = 1
 QL_CODE_HYB = 2
@@ -37,7 +39,8 @@ QL_F16 = 1
 # Every function include/qlinear.h declares (checked by the CPU tests).
 ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
-               "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read")
+               "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
+               "qlinear_forward_noalloc")
 
 
 class ql_code_t(ctypes.Structure):
@@ -56,6 +59,7 @@ _lib.qlinear_create_mixed.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _
                                       _vp, _f]
 _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
+_lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
 _lib.qlinear_eval_code.argtypes = [ql_code_t, _i, _i, _vp, _i, _vp, _vp]
 _lib.qlinear_get_status.argtypes = [_vp]
@@ -186,6 +190,22 @@ def qlinear_forward_host(h: QLinearHandle, x, y=None, out_dtype=None, stream=Non
         raise ValueError("y must be a CPU fp32/fp16 tensor [batch, m]")
     ydt = QL_F16 if y.dtype == torch.float16 else QL_F32
     _check(_lib.qlinear_forward_host(h.ptr, _ptr(x), batch, _ptr(y), ydt, _stream(stream)), "qlinear_forward_host")
+    return y
+
+
+def qlinear_forward_noalloc(h: QLinearHandle, x, y, stream=None):
+    """As qlinear_forward for batch <= 8, with the library's fixed scratch array
+    instead of allocated scratch; the caller provides y (CUDA fp32/fp16 [batch, m])."""
+    import torch
+    _cuda(x, "x", torch.float16)
+    if x.dim() != 2 or x.shape[1] != h.n:
+        raise ValueError("x must be [batch, n]")
+    _cuda(y, "y", (torch.float32, torch.float16))
+    if tuple(y.shape) != (x.shape[0], h.m):
+        raise ValueError("y must be [batch, m]")
+    ydt = QL_F16 if y.dtype == torch.float16 else QL_F32
+    _check(_lib.qlinear_forward_noalloc(h.ptr, _ptr(x), x.shape[0], _ptr(y), ydt, _stream(stream)),
+           "qlinear_forward_noalloc")
     return y
 
 

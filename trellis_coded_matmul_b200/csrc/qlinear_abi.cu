@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "internal.h"
@@ -486,9 +487,86 @@ const char* qlinear_strerror(int status) {
         case QL_E_OOM: return "device allocation failed";
         case QL_E_TIMEOUT: return "bounded device wait expired";
         case QL_E_DEVICE: return "device-side check failed";
+        case QL_E_SCRATCH: return "request exceeds the fixed scratch of qlinear_forward_noalloc";
         default: return "unknown status";
     }
 }
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Forward without allocation.
+//
+// Some callers cannot let a library allocate device memory while they run:
+// cudaMalloc and cudaFree may synchronise the whole device, which stalls every
+// other stream of a serving process in the middle of its step, and runtimes
+// that carve nearly all free HBM into their own pools at start-up (weights and
+// a key/value cache) leave no room for a late allocation.  For them,
+// qlinear_forward_noalloc keeps the decode-GEMV's scratch (x' and the fp32
+// accumulator z) in one fixed array in the library's static device memory.
+// The array is shared by every handle on a device, so calls that overlap in
+// time (two streams, or two host threads) race on it; calls issued in order
+// on one stream do not.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_base[kNoAllocMaxDevices];
+
+// The array's address on `device` (current on entry).  Looked up once per
+// device, on that device's first call; the lookup may load the library's
+// device code, which is why the first call belongs before any stream capture.
+int noalloc_scratch(int device, void** base) {
+    if (device < 0 || device >= kNoAllocMaxDevices) return QL_E_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_base[device]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return QL_E_CUDA;
+        }
+        g_noalloc_base[device] = p;
+    }
+    *base = g_noalloc_base[device];
+    return QL_OK;
+}
+
+}  // namespace
+
+extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream) {
+    if (!h || batch < 0 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
+    if (batch == 0) return QL_OK;
+    if (!x || !y) return QL_E_ARG;
+    if (batch > kGemvMaxBatch) return QL_E_UNSUPPORTED;
+    Layer& L = h->L;
+    const size_t xp_bytes = ((size_t)batch * L.n * 2 + 255) / 256 * 256;
+    const size_t z_bytes = (size_t)batch * L.m * 4;
+    if (xp_bytes + z_bytes > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_E_SCRATCH;
+    DeviceGuard g(L.device);
+    if (!g.ok) return QL_E_CUDA;
+    void* base = nullptr;
+    const int rc = noalloc_scratch(L.device, &base);
+    if (rc != QL_OK) return rc;
+    char* xp = (char*)base;
+    float* z = (float*)(xp + xp_bytes);
+    cudaStream_t st = (cudaStream_t)stream;
+
+    const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
+    // z must start at zero; another handle's failed call may have left sums there.
+    cudaError_t e = cudaMemsetAsync(z, 0, z_bytes, st);
+    if (e == cudaSuccess && !pl.xsmem) e = launch_rht_in_frag(L, x, batch, xp, st);
+    for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) {
+        const GemvPlan pi = i == 0 ? pl : plan_gemv(L, L.parts[i], batch);
+        e = launch_gemv(L, L.parts[i], pi, x, xp, batch, z, st);
+    }
+    if (e == cudaSuccess) e = launch_rht_out(L, z, batch, y, y_dtype, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    L.last_launches = L.nparts + 1 + (pl.xsmem ? 0 : 1);
+    return QL_OK;
+}
