@@ -1,28 +1,45 @@
 // gemm_tc.cu -- decode-to-shared-memory + tcgen05 tensor-core GEMM for
-// batches above 8: z[b][row] = sum_c W_hat[row][c] x'[b][c].
+// batches above 8: z[b][row] += sum_c W_hat[row][c] x'[b][c].
 //
-// The contraction is dense (M = 128 rows of W_hat per CTA, N = batch padded
+// The contraction is dense (M = 128 rows of W_hat per tile, N = batch padded
 // to 16, K = n), so it runs on the 5th-generation tensor cores: fp16 A and B
 // operands in shared memory (K-major, 128-byte swizzle), fp32 accumulator in
 // tensor memory, one thread issuing tcgen05.mma.  The A operand is produced
 // on the fly by decoder warps from the trellis code words (QTIP discussion:
 // decode with computed codes or a small table; the bitshift trellis makes any
 // run of steps decodable from the bits around it), so decoded weights never
-// reach HBM.  Warp roles, one 128-row tile per CTA:
-//   MMA warp       allocates tensor memory; one lane issues the MMAs of a
-//                  stage (4 x K=16) and commits them to the stages' "empty"
-//                  barriers;
-//   x' producer    bulk copy of the x' tile of each 64-column K stage (x' is
-//                  stored pre-swizzled, one copy per stage);
-//   code producer  bulk copies of the code words, one 256-column block of 8
-//                  row tiles at a time, up to 4 blocks ahead;
-//   16 decoders    two groups of 8 that take alternate stages; a warp decodes
-//                  16 rows x 64 columns of its stage (lane = one row, 32
-//                  consecutive trellis steps) into the A stage;
-//   all warps      at the end read the accumulator back and store z.
-// Every wait on an mbarrier is bounded; on expiry the CTA records
-// kStatusTimeout in the handle's status word, abandons its tile and frees its
-// tensor memory.
+// reach HBM.
+//
+// Work split (stream-K): the (128-row tile, 256-column block) units of the
+// layer are cut into one contiguous run per CTA, one CTA per SM, so every SM
+// decodes the same number of weights whatever the tile count.  A CTA's run
+// falls into segments of consecutive blocks of one tile; each segment is
+// accumulated in tensor memory and added into z with fp32 reductions (z is
+// all-zero when the kernel starts, so tiles split between CTAs sum up).
+//
+// Warp roles (a warp runs on SM sub-partition warp % 4, and may only touch
+// tensor-memory lanes 32 * (warp % 4) .. + 31):
+//   16 decoders    four groups of 4; group g decodes quarter g (64 columns) of
+//                  every 256-column block, i.e. every 4th stage; warp w of a
+//                  group covers rows 32 (w % 4) .. + 31 of the tile, one row
+//                  per lane, 64 consecutive trellis steps per lane, and writes
+//                  the decoded fp16 pairs straight into the stage's A slot in
+//                  tensor memory (tcgen05.st): decoded weights never touch
+//                  shared memory.  At the end of a segment the decoders read
+//                  the accumulator back and reduce it into z;
+//   MMA warp       allocates tensor memory (accumulator in columns [0, 256),
+//                  A slots of 32 columns from 256 on); one lane issues the 4
+//                  MMAs (K = 16 each, A from tensor memory, x' from shared
+//                  memory) of a stage and commits them to the stage's "empty"
+//                  barrier, and the last of a segment to "acc_full";
+//   x' producer    bulk copy of each stage's x' tile (x' is stored
+//                  pre-swizzled) into the stage's shared-memory slot;
+//   code producer  bulk copies of the code words, one 256-column block of the
+//                  tile's row tiles at a time, into a ring of blocks.
+// A stage has one "full" barrier (4 decoder arrivals and the x' bytes) and
+// one "empty" barrier (the MMA commit).  Every wait is bounded; on expiry the
+// CTA records kStatusTimeout in the handle's status word, abandons its work
+// and still frees its tensor memory.
 #include <cuda_fp16.h>
 
 #include "codes.cuh"
@@ -34,23 +51,32 @@ namespace qlk {
 
 constexpr int kTcRows = 128;         // M of one tile
 constexpr int kTcK = 64;             // K of one stage (one 128-byte swizzled row of fp16)
-constexpr int kTcDecoders = 16;      // decoder warps: two groups of 8 decode alternate stages
-constexpr int kTcGroup = 8;          // decoder warps per group (one per 16-row tile)
-constexpr int kTcWarps = 20;         // 5 per SM sub-partition (a warp runs on sub-partition warp % 4)
+constexpr int kTcDecoders = 16;      // decoder warps: four groups of 4, group g decodes quarter g of each block
+constexpr int kTcGroup = 4;          // decoder warps per group (one per 32-row lane quarter)
+constexpr int kTcWarps = 20;
 constexpr int kTcThreads = kTcWarps * 32;
-// Warp roles.  The MMA issuer shares its sub-partition only with the two
-// producers and one decoder, so its short instruction sequence per stage is
-// not starved of issue slots by the decoders.
-constexpr int kWarpMma = 0, kWarpXProd = 4, kWarpCodeProd = 8, kWarpSpare = 16;
-__device__ __forceinline__ int decoder_index(int w) {  // 0..15 for decoder warps, -1 otherwise
-    if (w == kWarpMma || w == kWarpXProd || w == kWarpCodeProd || w == kWarpSpare) return -1;
-    return w - 1 - (w > kWarpXProd) - (w > kWarpCodeProd) - (w > kWarpSpare);
-}
-constexpr int kTcAStages = 4;      // decoded A tiles in flight
-constexpr int kTcMaxBStages = 8;   // x' tiles in flight (as many as shared memory allows)
-constexpr int kTcMaxCodeSlots = 4;
+constexpr int kWarpMma = 16, kWarpXProd = 17, kWarpCodeProd = 18;  // warp 19 only joins set-up and teardown
+constexpr int kTcMaxStages = 8;      // stage slots (A in tensor memory, x' tile in shared memory)
+constexpr uint32_t kTcTmemCols = 512;  // accumulator [0, 256) and up to 8 A slots of 32 columns
+constexpr uint32_t kTcTmemA = 256;     // first A-slot column
+constexpr int kTcMaxCodeSlots = 4;   // code-word blocks in flight
+#ifndef QL_TC_XSPLIT
+#define QL_TC_XSPLIT 1
+#endif
+constexpr int kTcXSplit = QL_TC_XSPLIT;  // bulk copies per x' tile (npad * 128 bytes, a multiple of 2 KB)
+static_assert(kTcXSplit == 1 || kTcXSplit == 2 || kTcXSplit == 4 || kTcXSplit == 8, "x' split");
 constexpr int kTcWaitTries = 4096;           // try_wait calls of up to kTcSuspendNs each (a few seconds in all)
 constexpr uint32_t kTcSuspendNs = 1000000;   // before a wait is declared expired
+// barriers: code_full[C], code_empty[C], full[S], empty[S], acc_full, acc_empty
+static_assert(2 * kTcMaxCodeSlots + 2 * kTcMaxStages + 2 <= 60, "barrier area");
+
+// decoder group (0..3 = the block quarter it decodes) and lane quarter of warp w
+__device__ __forceinline__ bool decoder_role(int w, int& grp, int& qtr) {
+    if (w >= kTcDecoders) return false;
+    grp = w >> 2;
+    qtr = w & 3;
+    return true;
+}
 
 struct TcPart {
     const uint32_t* words;  // kernel layout
@@ -64,6 +90,7 @@ struct GemmArgs {
     TcPart part[2];
     int nparts;
     int nb;                 // 256-column blocks per row
+    int units;              // (tile, block) units of the layer: sum over parts of tiles * nb
     uint32_t lmask;
     int qshift;
     const uint32_t* lut;
@@ -71,30 +98,66 @@ struct GemmArgs {
     const uint8_t* xt;      // x' tiles: [n / 64][npad][128 B, swizzled]
     int npad;               // MMA N: batch padded to a multiple of 16 (<= 256)
     int batch;              // valid columns
-    float* z;               // [batch][m]
+    float* z;               // [batch][m], all-zero on entry
     int m;
     int* status;
-    int a_stages;           // depth of the A (decoded tile) ring
-    int b_stages;           // depth of the B (x' tile) ring
+    int stages;             // stage slots
     int code_slots;         // depth of the code-word ring
     int code_slot_words;    // words of one code-ring slot (8 units at the largest k)
-    uint32_t tmem_cols;
 };
 
 struct TcSmem {  // offsets in bytes from the 1024-aligned dynamic shared memory base
-    int a, b, code, lut, bar, total;
+    int b, code, lut, bar, total;
 };
 
-__host__ __device__ inline TcSmem tc_smem_layout(int a_stages, int b_stages, int code_slots, int npad,
-                                                  int code_slot_words, int lut_entries) {
+__host__ __device__ inline TcSmem tc_smem_layout(int stages, int code_slots, int npad, int code_slot_words,
+                                                  int lut_entries) {
     TcSmem s;
-    s.a = 0;
-    s.b = s.a + a_stages * kTcRows * 128;
-    s.code = s.b + b_stages * npad * 128;
+    s.b = 0;
+    s.code = s.b + stages * npad * 128;
     s.lut = s.code + code_slots * code_slot_words * 4;
     s.bar = s.lut + lut_entries * 32 * 4;
-    s.total = s.bar + 512;  // up to 33 mbarriers, the TMEM base address and the abort flag
+    s.total = s.bar + 512;  // mbarriers, the TMEM base address and the abort flag
     return s;
+}
+
+// A CTA's run of units in order, walked without divisions (the roles' loops
+// are latency-bound chains; the MMA issuer's especially).
+struct TcWalk {
+    int u, gt, j;  // unit, global 128-row tile, block
+    __device__ __forceinline__ TcWalk(const GemmArgs& p, int u0) : u(u0), gt(u0 / p.nb), j(u0 - (u0 / p.nb) * p.nb) {}
+    __device__ __forceinline__ void next(const GemmArgs& p) {
+        ++u;
+        if (++j == p.nb) {
+            j = 0;
+            ++gt;
+        }
+    }
+    __device__ __forceinline__ int part(const GemmArgs& p) const { return (p.nparts > 1 && gt >= p.part[0].tiles) ? 1 : 0; }
+    __device__ __forceinline__ int tile(const GemmArgs& p) const { return part(p) ? gt - p.part[0].tiles : gt; }
+};
+
+// Slot and phase parity of a ring position, advanced without divisions.
+struct TcRing {
+    int slot;
+    uint32_t phase;
+    __device__ __forceinline__ TcRing(int pos, int n) : slot(pos), phase(0) {
+        while (slot >= n) {
+            slot -= n;
+            phase ^= 1u;
+        }
+    }
+    __device__ __forceinline__ void advance(int by, int n) {
+        slot += by;
+        while (slot >= n) {
+            slot -= n;
+            phase ^= 1u;
+        }
+    }
+};
+__device__ __forceinline__ int tc_tiles16(const TcPart& pt, int tile) {  // row tiles present (ragged last tile)
+    const int n = pt.rt - tile * (kTcRows / kRowTile);
+    return n < kTcRows / kRowTile ? n : kTcRows / kRowTile;
 }
 
 // One decoder thread's 32 weights of a stage: row r of its row tile, trellis
@@ -126,34 +189,6 @@ __device__ __forceinline__ void decode_run32(const uint32_t (&cw)[K + 1], uint32
     }
 }
 
-// Decode one stage (quarter q of the block whose 8 units sit at shared address
-// `code`) for row tile `tdx` of the CTA into the swizzled A stage at `a_stage`.
-template <int CODE, int K, int V, bool L16>
-__device__ __forceinline__ void decode_stage(uint32_t code, uint32_t a_stage, int tdx, int q, int lane,
-                                             uint32_t lmask, const uint32_t* lut_lane, int qshift) {
-    using UL = UnitLayout<K>;
-    const uint32_t unit = code + tdx * UL::UW * 4;
-    const int r = lane & 15, hq = lane >> 4;
-    const int h = r >> 3, g = r & 7;
-    auto word = [&](int slot_lane, int e) -> uint32_t {
-        return lds32(unit + 4 * (((h * UL::NV + e / UL::VW) * 32 + slot_lane) * UL::VW + (e % UL::VW)));
-    };
-    uint32_t cw[K + 1];
-    const int own = 4 * g + q;
-    cw[0] = hq ? word(own, K - 1) : word(4 * g + ((q + 3) & 3), 2 * K - 1);
-#pragma unroll
-    for (int e = 0; e < K; ++e) cw[1 + e] = word(own, hq * K + e);
-    uint32_t out[16];
-    decode_run32<CODE, K, V, L16>(cw, lmask, lut_lane, qshift, out);
-    const int row = tdx * 16 + r;
-    const uint32_t rowp = a_stage + row * 128;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int chunk = (4 * hq + i) ^ (row & 7);
-        sts128(rowp + chunk * 16, out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
-    }
-}
-
 // Bounded wait; returns false (and raises the CTA's abort flag) on expiry.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
     if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspension
@@ -166,57 +201,81 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
+// One decoder thread's share of a stage: row r = 32 qtr + lane of the tile,
+// quarter q (64 steps) of the block whose row-tile units sit at shared address
+// `code`.  The quarter's 2K words of the row are loaded with vector loads,
+// plus the last word of the previous quarter (cyclically: tail-biting), then
+// decoded in two runs of 32 steps; run hq becomes 16 packed fp16 pairs stored
+// to tensor-memory columns a_col + 16 hq .. + 15 of the thread's lane.
+template <int CODE, int K, int V, bool L16>
+__device__ __forceinline__ void decode_stage_tmem(uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
+                                                  uint32_t lmask, const uint32_t* lut_lane, int qshift) {
+    using UL = UnitLayout<K>;
+    const int r = 32 * qtr + lane;
+    const int h = (r >> 3) & 1, g = r & 7;
+    const uint32_t unit = code + (r >> 4) * UL::UW * 4;
+    const int own = 4 * g + q;
+    auto addr = [&](int slot_lane, int e) -> uint32_t {  // word e of (row half h, lane slot) in the unit layout
+        return unit + 4 * (((h * UL::NV + e / UL::VW) * 32 + slot_lane) * UL::VW + (e % UL::VW));
+    };
+    uint32_t w[2 * K + 1];
+    w[0] = lds32(addr(4 * g + ((q + 3) & 3), 2 * K - 1));
+#pragma unroll
+    for (int c = 0; c < 2 * K / UL::VW; ++c) {
+        if (UL::VW == 4)
+            lds128(addr(own, 4 * c), w[1 + 4 * c], w[2 + 4 * c], w[3 + 4 * c], w[4 + 4 * c]);
+        else
+            lds64(addr(own, 2 * c), w[1 + 2 * c], w[2 + 2 * c]);
+    }
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+        uint32_t cw[K + 1];
+#pragma unroll
+        for (int e = 0; e <= K; ++e) cw[e] = w[hq * K + e];
+        uint32_t out[16];
+        decode_run32<CODE, K, V, L16>(cw, lmask, lut_lane, qshift, out);
+        tmem_st16(a_taddr + 16 * hq, out);
+    }
+}
+
 template <int CODE, int V, bool L16>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived by indexing the shared array so that
     // accesses through it stay shared-memory accesses
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const TcSmem L = tc_smem_layout(p.a_stages, p.b_stages, p.code_slots, p.npad, p.code_slot_words, p.lut_entries);
+    const TcSmem L = tc_smem_layout(p.stages, p.code_slots, p.npad, p.code_slot_words, p.lut_entries);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
-    // barrier slots: code_full[C], code_empty[C], a_full[SA], a_empty[SA], b_full[SB],
-    // b_empty[SB], mma_done; then the tmem base address and the abort flag
-    const int SA = p.a_stages, SB = p.b_stages, C = p.code_slots;
+    const int S = p.stages, C = p.code_slots;
     const uint32_t bar0 = smem_u32(bars);
     auto code_full = [&](int i) { return bar0 + 8 * i; };
     auto code_empty = [&](int i) { return bar0 + 8 * (C + i); };
-    auto a_full = [&](int i) { return bar0 + 8 * (2 * C + i); };
-    auto a_empty = [&](int i) { return bar0 + 8 * (2 * C + SA + i); };
-    auto b_full = [&](int i) { return bar0 + 8 * (2 * C + 2 * SA + i); };
-    auto b_empty = [&](int i) { return bar0 + 8 * (2 * C + 2 * SA + SB + i); };
-    const uint32_t mma_done = bar0 + 8 * (2 * C + 2 * SA + 2 * SB);
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * C + 2 * SA + 2 * SB + 1);
+    auto full = [&](int i) { return bar0 + 8 * (2 * C + i); };
+    auto empty = [&](int i) { return bar0 + 8 * (2 * C + S + i); };
+    const uint32_t acc_full = bar0 + 8 * (2 * C + 2 * S);
+    const uint32_t acc_empty = acc_full + 8;
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * C + 2 * S + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // which part and tile
-    int pi = 0, tile = blockIdx.x;
-    if (p.nparts > 1 && tile >= p.part[0].tiles) {
-        tile -= p.part[0].tiles;
-        pi = 1;
-    }
-    const TcPart part = p.part[pi];
-    const int R0 = tile * (kTcRows / kRowTile);        // first row tile of this CTA
-    int ntiles16 = part.rt - R0;                        // row tiles present (ragged last tile)
-    if (ntiles16 > kTcRows / kRowTile) ntiles16 = kTcRows / kRowTile;
-    const int k = part.k;
-    const int unit_words = 128 * k;
-    const int nstages = p.nb * 4;
+    // this CTA's run of units
+    const int u0 = (int)((long long)blockIdx.x * p.units / gridDim.x);
+    const int u1 = (int)((long long)(blockIdx.x + 1) * p.units / gridDim.x);
+    const uint32_t b_base = smem_u32(smem + L.b);
+    const uint32_t code_base = smem_u32(smem + L.code);
+    const uint32_t b_bytes = (uint32_t)p.npad * 128;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C; ++i) {
             mbar_init(code_full(i), 1);
             mbar_init(code_empty(i), kTcDecoders);  // every decoder warp releases each block once
         }
-        for (int i = 0; i < SA; ++i) {
-            mbar_init(a_full(i), kTcGroup);  // one group fills a stage
-            mbar_init(a_empty(i), 1);        // MMA commit
+        for (int i = 0; i < S; ++i) {
+            mbar_init(full(i), kTcGroup + 1);  // one decoder group and the x' producer
+            mbar_init(empty(i), 1);            // MMA commit
         }
-        for (int i = 0; i < SB; ++i) {
-            mbar_init(b_full(i), 1);
-            mbar_init(b_empty(i), 1);
-        }
-        mbar_init(mma_done, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kTcDecoders);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -224,7 +283,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
     if (CODE == kCodeHYB)
         for (int i = threadIdx.x; i < p.lut_entries * 32; i += blockDim.x) lut_smem[i] = p.lut[i >> 5];
     if (warp == kWarpMma) {
-        tmem_alloc(smem_u32(tmem_base_smem), p.tmem_cols);
+        tmem_alloc(smem_u32(tmem_base_smem), kTcTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -232,32 +291,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
 
-    const int dec = decoder_index(warp);
+    int grp = 0, qtr = 0;
     if (warp == kWarpXProd) {
         // ---------------- x' producer ----------------
         grid_dependency_wait();  // x' comes from the previous kernel
-        for (int s = 0; s < nstages && !*abort_flag; ++s) {
-            const int st = s % SB, round = s / SB;
-            if (!wait_bar(b_empty(st), (round & 1) ^ 1, abort_flag, p.status)) break;
-            if (lane == 0) {
-                const uint32_t bytes = (uint32_t)p.npad * 128;
-                mbar_arrive_expect_tx(b_full(st), bytes);
-                bulk_g2s(smem_u32(smem + L.b) + st * bytes, p.xt + (size_t)s * bytes, bytes, b_full(st));
+        TcRing r(0, S);
+        bool ok = true;
+        for (TcWalk w(p, u0); w.u < u1 && ok; w.next(p)) {
+            const int j = w.j;
+            for (int q = 0; q < 4; ++q, r.advance(1, S)) {
+                const int st = r.slot;
+                if (!wait_bar(empty(st), r.phase ^ 1u, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                // The tile goes in kTcXSplit pieces, one per lane, so that several
+                // bulk copies are in flight at once.
+                if (lane == 0) mbar_arrive_expect_tx(full(st), b_bytes);
+                __syncwarp();
+                if (lane < kTcXSplit) {
+                    const uint32_t piece = b_bytes / kTcXSplit;
+                    bulk_g2s(b_base + st * b_bytes + lane * piece,
+                             p.xt + (size_t)(4 * j + q) * b_bytes + (size_t)lane * piece, piece, full(st));
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
     } else if (warp == kWarpCodeProd) {
         // ---------------- code-word producer ----------------
-        const uint8_t* code_src = reinterpret_cast<const uint8_t*>(part.words);
-        for (int j = 0; j < p.nb && !*abort_flag; ++j) {
-            const int slot = j % C, round = j / C;
-            if (!wait_bar(code_empty(slot), (round & 1) ^ 1, abort_flag, p.status)) break;
+        TcRing r(0, C);
+        for (TcWalk w(p, u0); w.u < u1; w.next(p), r.advance(1, C)) {
+            const int slot = r.slot;
+            const TcPart& pt = p.part[w.part(p)];
+            const int tile = w.tile(p);
+            const int ntiles16 = tc_tiles16(pt, tile);
+            const int unit_words = 128 * pt.k;
+            if (!wait_bar(code_empty(slot), r.phase ^ 1u, abort_flag, p.status)) break;
             if (lane == 0) mbar_arrive_expect_tx(code_full(slot), (uint32_t)(ntiles16 * unit_words * 4));
             __syncwarp();
             if (lane < ntiles16) {
-                const size_t unit = (size_t)(R0 + lane) * p.nb + j;
-                bulk_g2s(smem_u32(smem + L.code) + (uint32_t)(slot * p.code_slot_words + lane * unit_words) * 4,
-                         code_src + unit * unit_words * 4, (uint32_t)unit_words * 4, code_full(slot));
+                const size_t unit = (size_t)(tile * (kTcRows / kRowTile) + lane) * p.nb + w.j;
+                bulk_g2s(code_base + (uint32_t)(slot * p.code_slot_words + lane * unit_words) * 4,
+                         reinterpret_cast<const uint8_t*>(pt.words) + unit * unit_words * 4,
+                         (uint32_t)unit_words * 4, code_full(slot));
             }
             __syncwarp();
         }
@@ -267,81 +343,104 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
         // field (low word, 16-byte units, no carry out of it below 256 KB):
         // build the words once and step the low word.
         const uint32_t idesc = idesc_f16_f32(kTcRows, p.npad);
-        const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(smem + L.a));
-        const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(smem + L.b));
-        const uint32_t a_hi = (uint32_t)(a_desc0 >> 32), b_hi = (uint32_t)(b_desc0 >> 32);
-        const uint32_t a_lo0 = (uint32_t)a_desc0, b_lo0 = (uint32_t)b_desc0;
-        const uint32_t b_step = (uint32_t)p.npad * 128 / 16;
-        int sa = 0, sb = 0, pa = 0, pb = 0;
-        for (int s = 0; s < nstages; ++s) {
-            if (!wait_bar(a_full(sa), pa, abort_flag, p.status)) break;
-            if (!wait_bar(b_full(sb), pb, abort_flag, p.status)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t a_lo = a_lo0 + (uint32_t)sa * (kTcRows * 128 / 16);
-                const uint32_t b_lo = b_lo0 + (uint32_t)sb * b_step;
-#pragma unroll
-                for (int kk = 0; kk < kTcK / 16; ++kk) {
-                    tc_mma_f16(tmem, ((uint64_t)a_hi << 32) | (a_lo + kk * 2), ((uint64_t)b_hi << 32) | (b_lo + kk * 2),
-                               idesc, (s > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t b_desc0 = smem_desc_k_sw128(b_base);
+        const uint32_t b_hi = (uint32_t)(b_desc0 >> 32), b_lo0 = (uint32_t)b_desc0;
+        const uint32_t b_step = b_bytes / 16;
+        TcRing r(0, S);
+        int seg = 0;
+        for (TcWalk w(p, u0); w.u < u1; w.next(p)) {
+            const bool first = w.u == u0 || w.j == 0;  // first block of a segment
+            const bool last = w.u + 1 == u1 || w.j + 1 == p.nb;
+            // the epilogue of the previous segment must have read the accumulator
+            if (first && seg > 0 && !wait_bar(acc_empty, (seg - 1) & 1, abort_flag, p.status)) break;
+            bool ok = true;
+            for (int q = 0; q < 4; ++q, r.advance(1, S)) {
+                const int st = r.slot;
+                if (!wait_bar(full(st), r.phase, abort_flag, p.status)) {
+                    ok = false;
+                    break;
                 }
-                tc_commit(a_empty(sa));
-                tc_commit(b_empty(sb));
-                if (s == nstages - 1) tc_commit(mma_done);
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a_t = tmem + kTcTmemA + (uint32_t)st * (kTcK / 2);
+                    const uint32_t b_lo = b_lo0 + (uint32_t)st * b_step;
+#pragma unroll
+                    for (int kk = 0; kk < kTcK / 16; ++kk)
+                        tc_mma_f16_ts(tmem, a_t + kk * 8, ((uint64_t)b_hi << 32) | (b_lo + kk * 2), idesc,
+                                      (first && q == 0 && kk == 0) ? 0u : 1u);
+                    tc_commit(empty(st));
+                    if (last && q == 3) tc_commit(acc_full);
+                }
+                __syncwarp();
             }
-            __syncwarp();
-            if (++sa == SA) sa = 0, pa ^= 1;
-            if (++sb == SB) sb = 0, pb ^= 1;
+            if (!ok) break;
+            if (last) ++seg;
         }
-    } else if (dec >= 0) {
-        // ---------------- decoders ----------------
-        const int grp = dec / kTcGroup, tdx = dec % kTcGroup;
+    } else if (decoder_role(warp, grp, qtr)) {
+        // ---------------- decoders, and the epilogue of every segment ----------------
         const uint32_t* lut_lane = lut_smem + lane;
-        const uint32_t code_base = smem_u32(smem + L.code);
-        for (int s = grp; s < nstages && !*abort_flag; s += 2) {
-            const int j = s >> 2, q = s & 3;
-            const int slot = j % C;
-            if (q < 2 && !wait_bar(code_full(slot), (j / C) & 1, abort_flag, p.status)) break;
-            const int st = s % SA, round = s / SA;
-            if (!wait_bar(a_empty(st), (round & 1) ^ 1, abort_flag, p.status)) break;
-            if (tdx < ntiles16) {
-                const uint32_t code = code_base + slot * p.code_slot_words * 4;
-                const uint32_t a_stage = smem_u32(smem + L.a) + st * kTcRows * 128;
-                switch (k) {
-                    case 1: decode_stage<CODE, 1, V, L16>(code, a_stage, tdx, q, lane, p.lmask, lut_lane, p.qshift); break;
-                    case 2: decode_stage<CODE, 2, V, L16>(code, a_stage, tdx, q, lane, p.lmask, lut_lane, p.qshift); break;
-                    case 3: decode_stage<CODE, 3, V, L16>(code, a_stage, tdx, q, lane, p.lmask, lut_lane, p.qshift); break;
-                    default: decode_stage<CODE, 4, V, L16>(code, a_stage, tdx, q, lane, p.lmask, lut_lane, p.qshift); break;
+        const int share = warp >> 2;   // 4 warps per lane quarter split the accumulator columns
+        const int chunks = p.npad / 16;
+        const uint32_t lane_base = (uint32_t)(qtr * 32) << 16;
+        int seg = 0;
+        bool z_ready = false;
+        TcRing rc(0, C), rs(grp, S);  // code block i, stage 4 i + grp
+        for (TcWalk w(p, u0); w.u < u1; w.next(p), rc.advance(1, C), rs.advance(4, S)) {
+            const int slot = rc.slot;
+            const TcPart& pt = p.part[w.part(p)];
+            const uint32_t code = code_base + slot * p.code_slot_words * 4;
+            if (!wait_bar(code_full(slot), rc.phase, abort_flag, p.status)) break;
+            bool ok = true;
+            {
+                const int st = rs.slot;
+                if (!wait_bar(empty(st), rs.phase ^ 1u, abort_flag, p.status)) {
+                    ok = false;
+                } else {
+                    tc_fence_after();  // the MMAs that read this A slot have completed
+                    // Rows of row tiles beyond a ragged last tile decode whatever the
+                    // slot holds; their accumulator rows are never stored.
+                    const uint32_t a_taddr = tmem + lane_base + kTcTmemA + (uint32_t)st * (kTcK / 2);
+                    switch (pt.k) {
+                        case 1: decode_stage_tmem<CODE, 1, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
+                        case 2: decode_stage_tmem<CODE, 2, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
+                        case 3: decode_stage_tmem<CODE, 3, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
+                        default: decode_stage_tmem<CODE, 4, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full(st));
                 }
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(a_full(st));
-                if (q >= 2) mbar_arrive(code_empty(slot));  // this group's last stage of the block
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(code_empty(slot));
+            if (w.u + 1 < u1 && w.j + 1 < p.nb) continue;
+            // ---- end of a segment: accumulator -> z (fp32 reductions) ----
+            if (!z_ready) {
+                grid_dependency_wait();  // z was last touched by the previous kernels
+                z_ready = true;
             }
-        }
-    }
-    // ---------------- epilogue (all warps): TMEM -> z ----------------
-    grid_dependency_wait();
-    if (wait_bar(mma_done, 0, abort_flag, p.status)) {
-        tc_fence_after();
-        const int quarter = warp & 3;        // TMEM lanes this warp may read
-        const int share = warp >> 2;         // kTcWarps / 4 warps per quarter split the columns
-        const int per = kTcWarps / 4;
-        const int row = part.row0 + R0 * kRowTile + quarter * 32 + lane;
-        const bool row_ok = (R0 * kRowTile + quarter * 32 + lane) < part.rt * kRowTile;
-        const int chunks = p.npad / 16;      // 16-column TMEM loads
-        for (int ci = share * chunks / per; ci < (share + 1) * chunks / per; ++ci) {
-            const int c0 = ci * 16;
-            uint32_t v[16];
-            tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v);
-            tmem_ld_wait();
-            if (row_ok) {
+            if (!wait_bar(acc_full, seg & 1, abort_flag, p.status)) break;
+            tc_fence_after();
+            const int rloc = qtr * 32 + lane;  // row within the tile
+            const int tile = w.tile(p);
+            const int row = pt.row0 + tile * kTcRows + rloc;
+            const bool row_ok = tile * kTcRows + rloc < pt.rt * kRowTile;
+            for (int ci = share * chunks / 4; ci < (share + 1) * chunks / 4; ++ci) {
+                const int c0 = ci * 16;
+                uint32_t v[16];
+                tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
+                tmem_ld_wait();
+                if (row_ok) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (c0 + i < p.batch) p.z[(size_t)(c0 + i) * p.m + row] = __uint_as_float(v[i]);
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e < p.batch) red_add_f32(p.z + (size_t)(c0 + e) * p.m + row, __uint_as_float(v[e]));
+                }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            ++seg;
         }
     }
     grid_launch_dependents();
@@ -349,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, p.tmem_cols);
+        tmem_dealloc(tmem, kTcTmemCols);
     }
 }
 
@@ -365,27 +464,24 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaS
     return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, a);
 }
 
-// Ring depths: 4 A stages, then the deepest code ring (4..2 slots) and the
-// deepest x' ring (8..2 stages) that fit in shared memory.
-size_t tc_smem_bytes(const Layer& L, int npad, int* a_stages, int* b_stages, int* code_slots) {
+// Ring depths: the most stage slots (up to kTcMaxStages), then the deepest
+// code ring (up to kTcMaxCodeSlots blocks) that fit in shared memory.
+size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
     int kmax = 0;
     for (int i = 0; i < L.nparts; ++i) kmax = L.parts[i].k > kmax ? L.parts[i].k : kmax;
     const int code_slot_words = (kTcRows / kRowTile) * 128 * kmax;
     const int lut_entries = L.code == kCodeHYB ? (1 << L.Q) : 0;
-    for (int sa = kTcAStages; sa >= 2; --sa) {
+    for (int s = kTcMaxStages; s >= 2; --s) {
         for (int c = kTcMaxCodeSlots; c >= 2; --c) {
-            for (int sb = kTcMaxBStages; sb >= 2; --sb) {
-                const TcSmem lay = tc_smem_layout(sa, sb, c, npad, code_slot_words, lut_entries);
-                if (lay.total + 1024 <= kTcMaxSmem && (sb >= 4 || c == 2)) {
-                    *a_stages = sa;
-                    *b_stages = sb;
-                    *code_slots = c;
-                    return (size_t)lay.total + 1024;
-                }
+            const TcSmem lay = tc_smem_layout(s, c, npad, code_slot_words, lut_entries);
+            if (lay.total + 1024 <= kTcMaxSmem) {
+                *stages = s;
+                *code_slots = c;
+                return (size_t)lay.total + 1024;
             }
         }
     }
-    *a_stages = *b_stages = *code_slots = 0;
+    *stages = *code_slots = 0;
     return 0;
 }
 
@@ -393,7 +489,8 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     GemmArgs a;
     int kmax = 0;
     a.nparts = L.nparts;
-    int grid = 0;
+    a.nb = L.n / kT;
+    int tiles = 0;
     for (int i = 0; i < L.nparts; ++i) {
         const Part& pt = L.parts[i];
         a.part[i].words = L.words + pt.word_off;
@@ -401,11 +498,11 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
         a.part[i].row0 = pt.row0;
         a.part[i].k = pt.k;
         a.part[i].tiles = (pt.rows + kTcRows - 1) / kTcRows;
-        grid += a.part[i].tiles;
+        tiles += a.part[i].tiles;
         kmax = pt.k > kmax ? pt.k : kmax;
     }
     if (L.nparts == 1) a.part[1] = a.part[0];
-    a.nb = L.n / kT;
+    a.units = tiles * a.nb;
     a.lmask = (1u << L.L) - 1u;
     a.qshift = 32 - L.Q;
     a.lut = L.lut;
@@ -417,11 +514,9 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     a.m = L.m;
     a.status = L.status;
     a.code_slot_words = (kTcRows / kRowTile) * 128 * kmax;
-    uint32_t cols = 32;
-    while (cols < (uint32_t)npad) cols <<= 1;
-    a.tmem_cols = cols;
-    const size_t smem = tc_smem_bytes(L, npad, &a.a_stages, &a.b_stages, &a.code_slots);
+    const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots);
     if (smem == 0) return cudaErrorInvalidValue;
+    const int grid = a.units < L.num_sms ? a.units : L.num_sms;
     const bool l16 = L.L == 16;
     if (L.code == kCode1MAD) return l16 ? launch_gemm_t<kCode1MAD, 1, true>(a, grid, smem, st)
                                         : launch_gemm_t<kCode1MAD, 1, false>(a, grid, smem, st);

@@ -119,8 +119,9 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch);
 cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
                         int batch, float* z, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
-// z[b][row] = W_hat x' for all parts, x' in tensor-core tiles with npad (multiple
-// of 16, <= 256) rows, b < batch; one 128-row tile per CTA.
+// z[b][row] += W_hat x' for all parts (z all-zero on entry), x' in tensor-core
+// tiles with npad (multiple of 16, <= 256) rows, b < batch; the (128-row tile,
+// 256-column block) units are split evenly over one CTA per SM.
 cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st);
 cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words,
                              const uint32_t* states, int count, void* out, cudaStream_t st);

@@ -200,7 +200,7 @@ int ensure(void** buf, size_t* have, size_t bytes) {
 
 // The z accumulator is all-zero between forwards: it is zeroed when
 // allocated, and the output-transform kernel re-zeroes what it consumed (the
-// tensor-core GEMM overwrites z, which keeps the same invariant).
+// tensor-core GEMM adds into z, which needs and keeps the same invariant).
 int prepare_z(Layer& L, size_t bytes, cudaStream_t st) {
     if (L.z_bytes >= bytes && !L.z_dirty) return QL_OK;
     int rc = ensure((void**)&L.z, &L.z_bytes, bytes);
