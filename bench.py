@@ -382,7 +382,7 @@ def run_ours(args):
             peak = pk["bf16_tflops_sustained"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": _traffic(f"gemm_{sp.name}_b{batch}", 1),
-                    "kernel": "gemm_tc_kernel (trellis decode to shared memory + tcgen05 MMA, fp16 in, fp32 TMEM)",
+                    "kernel": "gemm_tc_kernel (trellis decode into tensor memory + tcgen05 MMA, fp16 in, fp32 accumulate)",
                     "kernel_us": kern_s * 1e6,
                     "peak_kind": pk_kind + " bf16_tflops_sustained (fp16 dense rate = bf16 dense rate)",
                     "alg_flops_per_launch": flops, "timing": timing}

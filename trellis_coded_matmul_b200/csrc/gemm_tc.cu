@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0) {
+                if (elect_one()) {
                     const uint32_t a_t = tmem + kTcTmemA + (uint32_t)st * (kTcK / 2);
                     const uint32_t b_lo = b_lo0 + (uint32_t)st * b_step;
 #pragma unroll
