@@ -54,6 +54,9 @@ def parse_args():
     p.add_argument("--batch", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--instances", type=int, default=None,
+                   help="layer instances to rotate through (default: enough code words for 4x L2); a smaller "
+                        "count is for profiler captures only, and the line then says its inputs may sit in L2")
     a = p.parse_args()
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -72,8 +75,11 @@ def config_dict(sp, batch, n_inst, extra=None):
     d = {"workload": f"{sp.name}: m={sp.m} n={sp.n} bits/weight={sp.bits_per_weight:g} L={sp.L} V={sp.V} "
                      f"code={wl.CODE_NAMES[sp.code]}" + (f" Q={sp.Q}" if sp.Q else ""),
          "global_batch": batch, "seq_len": 1, "parallelism": "independent layer instances per GPU",
-         "l2": f"inputs larger than L2: rotating {n_inst} layer instances "
-               f"({n_inst * sp.stream_bytes / 2**20:.0f} MiB of code words)"}
+         "l2": (f"inputs larger than L2: rotating {n_inst} layer instances "
+                f"({n_inst * sp.stream_bytes / 2**20:.0f} MiB of code words)")
+               if n_inst * sp.stream_bytes >= 4 * L2_BYTES else
+               f"PROFILING CASE, not a benchmark: {n_inst} layer instances "
+               f"({n_inst * sp.stream_bytes / 2**20:.0f} MiB of code words) may stay in L2"}
     if extra:
         d.update(extra)
     return d
@@ -261,6 +267,8 @@ def run_ours(args):
     sp = wl.WORKLOADS[args.workload]
     batch = args.batch or sp.batches[0]
     n_inst = int(min(512, max(1, math.ceil(4 * L2_BYTES / sp.stream_bytes))))
+    if args.instances:
+        n_inst = max(1, min(n_inst, args.instances))
     handles = [make_handle(wl.make_layer(sp, instance=1 + rank * 4096 + i)) for i in range(n_inst)]
     xs = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).cuda() for i in range(n_inst)]
     ys = [torch.empty((batch, sp.m), dtype=torch.float32, device="cuda") for _ in range(n_inst)]
