@@ -14,12 +14,16 @@ namespace qlk {
 __device__ __forceinline__ bool sign_neg(const uint32_t* bits, int i) { return (bits[i >> 5] >> (i & 31)) & 1u; }
 __device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
 
+// One radix-2^LOGR pass at stride h = 2^logh: group gi holds the entries
+// base + q h, q < 2^LOGR (h and B are powers of two, so no divisions).
 template <int LOGR>
-__device__ __forceinline__ void fwht_pass(float* buf, int B, int h, int tid, int nthreads) {
+__device__ __forceinline__ void fwht_pass(float* buf, int B, int logh, int tid, int nthreads) {
     constexpr int R = 1 << LOGR;
     const int groups = B >> LOGR;
+    const int hmask = (1 << logh) - 1;
     for (int gi = tid; gi < groups; gi += nthreads) {
-        const int base = (gi / h) * (h << LOGR) + (gi % h);
+        const int base = ((gi >> logh) << (logh + LOGR)) + (gi & hmask);
+        const int h = 1 << logh;
         float v[R];
 #pragma unroll
         for (int q = 0; q < R; ++q) v[q] = buf[pad16(base + q * h)];
@@ -44,21 +48,22 @@ __device__ __forceinline__ void fwht_pass(float* buf, int B, int h, int tid, int
 // CTA barrier after every pass.
 // Threads with active == false touch no memory but take part in every barrier.
 __device__ __forceinline__ void fwht_smem_passes(float* buf, int B, int h0, int tid, int nthreads, bool active) {
-    int h = h0;
-    while (h < B) {
-        const int rem = 31 - __clz(B / h);  // log2(B / h)
+    int logh = 31 - __clz(h0);
+    const int logb = 31 - __clz(B);
+    while (logh < logb) {
+        const int rem = logb - logh;
         if (rem >= 4) {
-            if (active) fwht_pass<4>(buf, B, h, tid, nthreads);
-            h <<= 4;
+            if (active) fwht_pass<4>(buf, B, logh, tid, nthreads);
+            logh += 4;
         } else if (rem == 3) {
-            if (active) fwht_pass<3>(buf, B, h, tid, nthreads);
-            h <<= 3;
+            if (active) fwht_pass<3>(buf, B, logh, tid, nthreads);
+            logh += 3;
         } else if (rem == 2) {
-            if (active) fwht_pass<2>(buf, B, h, tid, nthreads);
-            h <<= 2;
+            if (active) fwht_pass<2>(buf, B, logh, tid, nthreads);
+            logh += 2;
         } else {
-            if (active) fwht_pass<1>(buf, B, h, tid, nthreads);
-            h <<= 1;
+            if (active) fwht_pass<1>(buf, B, logh, tid, nthreads);
+            logh += 1;
         }
         __syncthreads();
     }

@@ -166,56 +166,70 @@ struct GemvArgs {
     const __half* x;  // [batch][n]
     const uint32_t* sin_bits;
     int n, B_n;
-    int groups_in;    // thread groups (B_n/16 threads each) of the in-kernel input transform
+    int groups_in;    // thread groups (B_n/8 threads each) of the in-kernel input transform
 };
 
 // x' = H_n diag(s_in) x for every column and batch row, fp16, into the
-// fragment layout in shared memory.  Groups of B_n/16 threads take one
+// fragment layout in shared memory.  Groups of B_n/kXinE threads take one
 // (batch row, Hadamard block) at a time; all threads run the same rounds.
-__device__ __forceinline__ void input_transform_smem(const GemvArgs& p, __half* xs, float* fw) {
-    const int B = p.B_n, T = B / 16;
-    const int G = p.groups_in;  // groups with their own FWHT scratch; spare threads only join barriers
-    const int grp = threadIdx.x / T, tid = threadIdx.x % T;
-    const int per_row = p.n / B, total = p.batch * per_row;
-    const float scale = rsqrtf((float)B);
-    for (int r0 = 0; r0 < total; r0 += G) {
-        const int item = r0 + grp;
-        const bool active = grp < G && item < total;
-        const int b = active ? item / per_row : 0;
-        const int col = (active ? (item % per_row) * B : 0) + tid * 16;
-        float v[16];
-        if (active) {
-            const __half* src = p.x + (size_t)b * p.n + col;
-            const uint32_t sw = p.sin_bits[col >> 5] >> (col & 31);
-#pragma unroll
-            for (int q = 0; q < 16; q += 8) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(src + q);
+// prepare() runs before the wait for the previous kernel (the sign bits are
+// written once at create time); run() reads x, which that kernel may produce.
+constexpr int kXinE = 8;  // entries per thread of the in-kernel input transform
+struct InputTransform {
+    int B, T, G, grp, tid, per_row, total;
+    uint32_t sw0;  // sign bits of the thread's entries in the first round
+    __device__ __forceinline__ void prepare(const GemvArgs& p) {
+        B = p.B_n;
+        T = B / kXinE;
+        G = p.groups_in;  // groups with their own FWHT scratch; spare threads only join barriers
+        grp = threadIdx.x / T;
+        tid = threadIdx.x - grp * T;
+        per_row = p.n / B;
+        total = p.batch * per_row;
+        sw0 = 0;
+        if (grp < G && grp < total) {
+            const int col = (grp % per_row) * B + tid * kXinE;
+            sw0 = p.sin_bits[col >> 5] >> (col & 31);
+        }
+    }
+    __device__ __forceinline__ void run(const GemvArgs& p, __half* xs, float* fw) const {
+        const float scale = rsqrtf((float)B);
+        for (int r0 = 0; r0 < total; r0 += G) {
+            const int item = r0 + grp;
+            const bool active = grp < G && item < total;
+            const int b = active ? item / per_row : 0;
+            const int col = (active ? (item % per_row) * B : 0) + tid * kXinE;
+            float v[kXinE];
+            if (active) {
+                const __half* src = p.x + (size_t)b * p.n + col;
+                const uint32_t sw = r0 == 0 ? sw0 : p.sin_bits[col >> 5] >> (col & 31);
+                const uint4 raw = *reinterpret_cast<const uint4*>(src);
                 const __half* hv = reinterpret_cast<const __half*>(&raw);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int e = 0; e < kXinE; ++e) {
                     const float f = __half2float(hv[e]);
-                    v[q + e] = ((sw >> (q + e)) & 1u) ? -f : f;
+                    v[e] = ((sw >> e) & 1u) ? -f : f;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < kXinE; ++e) v[e] = 0.f;
+            }
+            fwht_block<kXinE>(v, B, tid, T, fw + (size_t)(grp < G ? grp : 0) * (B + B / 16), grp < G);
+            if (active) {
+#pragma unroll
+                for (int q = 0; q < kXinE; q += 4) {
+                    const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
+                    const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
+                    uint2 w;
+                    w.x = *reinterpret_cast<const uint32_t*>(&lo);
+                    w.y = *reinterpret_cast<const uint32_t*>(&hi);
+                    *reinterpret_cast<uint2*>(xs + frag_index4(col + q, b, p.batch)) = w;
                 }
             }
-        } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] = 0.f;
+            __syncthreads();
         }
-        fwht_block<16>(v, B, tid, T, fw + (size_t)(grp < G ? grp : 0) * (B + B / 16), grp < G);
-        if (active) {
-#pragma unroll
-            for (int q = 0; q < 16; q += 4) {
-                const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
-                const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
-                uint2 w;
-                w.x = *reinterpret_cast<const uint32_t*>(&lo);
-                w.y = *reinterpret_cast<const uint32_t*>(&hi);
-                *reinterpret_cast<uint2*>(xs + frag_index4(col + q, b, p.batch)) = w;
-            }
-        }
-        __syncthreads();
     }
-}
+};
 
 // One CTA per SM.  CTA i takes units [U*i/G, U*(i+1)/G) of the part (G CTAs)
 // and splits them evenly over its warps; the launcher sizes the CTA so that
@@ -247,11 +261,14 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p,
 
     uint32_t nxt[2][2 * K];
     if (u0 < u1) load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
-    // Programmatic dependent launch: the code words (and the HYB table) are
-    // written once at create time, so they are fetched before waiting for the
-    // previous kernel (the producer of x or x', the consumer of the last z).
+    // Programmatic dependent launch: the code words, the HYB table and the
+    // sign bits are written once at create time, so they are fetched before
+    // waiting for the previous kernel (the producer of x or x', the consumer
+    // of the last z).
+    InputTransform xin;
+    if (XSMEM) xin.prepare(p);
     grid_dependency_wait();
-    if (XSMEM) input_transform_smem(p, xs, fw);
+    if (XSMEM) xin.run(p, xs, fw);
     grid_launch_dependents();
 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -464,7 +481,7 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
     int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
     const int lut_words = L.code == kCodeHYB ? (32 << L.Q) : 0;
     const int budget = kGemvMaxSmem / 4 - lut_words;
-    const int t_in = L.B_n / 16;
+    const int t_in = L.B_n / kXinE;
     const int xs_words = batch * L.n / 2;
     pl.xsmem = L.L == 16 && L.nparts == 1 && (long long)batch * L.n <= kFuseInElems &&
                t_in <= kGemvMaxWarps * 32;
@@ -472,7 +489,7 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
     pl.groups_in = 0;
     if (pl.xsmem) {
         if (threads < t_in) threads = t_in;
-        // thread groups of B_n/16 threads; a group of more than a warp needs
+        // thread groups of B_n/kXinE threads; a group of more than a warp needs
         // its own FWHT scratch (B_n + B_n/16 floats)
         int g = threads / t_in;
         const int work = batch * (L.n / L.B_n);
