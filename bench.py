@@ -214,6 +214,25 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(values, device):
+    """Each value's maximum over all ranks (the values unchanged on one rank).
+    Every rank must call this with the same number of values."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(world, steps, batch, secs):
+    """Whole-job throughput: every rank ran `steps` forwards of `batch` tokens
+    (weak scaling), timed as the slowest rank's `secs`."""
+    return world * steps * batch / secs
+
+
 # ------------------------------------------------------------------ CUDA arm
 def _source_hash():
     h = hashlib.sha256()
@@ -338,9 +357,7 @@ def run_ours(args):
         tcm.qlinear_profile_enable(h, 0)
     kern_s = kern_ms * 1e-3 / max(1, kern_n)
     if world > 1:
-        t = torch.tensor([secs, kern_s], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs, kern_s = float(t[0]), float(t[1])
+        secs, kern_s = max_over_ranks([secs, kern_s], "cuda")
 
     # end to end through the public API with host buffers (pinned)
     e2e = None
@@ -362,17 +379,15 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_s = es.elapsed_time(ee) * 1e-3
         if world > 1:
-            t = torch.tensor([e2e_s], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_s = float(t[0])
-        e2e = {"value": world * e2e_steps * batch / e2e_s, "unit": "tokens/s",
+            e2e_s = max_over_ranks([e2e_s], "cuda")[0]
+        e2e = {"value": job_tokens_per_s(world, e2e_steps, batch, e2e_s), "unit": "tokens/s",
                "h2d_bytes_per_step": batch * sp.n * 2, "d2h_bytes_per_step": batch * sp.m * 4,
                "steps": e2e_steps}
 
     line = None
     if rank == 0:
         pk, pk_kind = peaks()
-        value = world * args.steps * batch / secs
+        value = job_tokens_per_s(world, args.steps, batch, secs)
         launches_per_step = tcm.qlinear_info(handles[0])["last_launches"]
         timing = (f"CUDA events around the kernel in a replay of {prof_steps} steps "
                   f"({prof_secs / prof_steps * 1e6:.2f} us/step with the events)")

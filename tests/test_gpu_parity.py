@@ -227,3 +227,17 @@ def test_forward_in_cuda_graph_with_profiling():
     ms, slots = tcm.qlinear_profile_read(h)
     assert slots == 4 and ms > 0
     tcm.qlinear_profile_enable(h, 0)
+
+
+# ---------------------------------------------------------------- largest Hadamard blocks
+# B = 16384 and 32768 run the transforms with 1024-thread CTAs (16 and 32
+# entries per thread); B_n = 32768 also takes the separate input-transform
+# kernel at batch 1 (batch * n above the in-kernel limit).
+@pytest.mark.parametrize("m,n", [(32768, 256), (16384, 256), (16, 32768)], ids=lambda v: str(v))
+def test_forward_largest_hadamard_blocks(m, n):
+    li = wl.random_layer(m, n, 2, 16, 1, wl.CODE_3INST, seed=7 + m + n, alpha=0.25)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, 2, instance=9)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_GEMV

@@ -487,6 +487,7 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
                t_in <= kGemvMaxWarps * 32;
     int fw = 0;
     pl.groups_in = 0;
+    const int threads_decode = threads;
     if (pl.xsmem) {
         if (threads < t_in) threads = t_in;
         // thread groups of B_n/kXinE threads; a group of more than a warp needs
@@ -502,6 +503,10 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
         }
         pl.groups_in = g;
         if (xs_words + fw > budget) pl.xsmem = false, fw = 0, pl.groups_in = 0;
+        // every CTA runs the transform before its first MMA: only worth it when
+        // it takes a single round (one group per (batch row, Hadamard block))
+        if (g < work) pl.xsmem = false, fw = 0, pl.groups_in = 0;
+        if (!pl.xsmem) threads = threads_decode;
     }
     pl.threads = threads;
     pl.sm.lut_words = lut_words;

@@ -14,7 +14,10 @@ constexpr int kMaxHadamard = 32768;
 
 constexpr int kGemvMaxWarps = 24;        // decode-GEMV: warps of its one CTA per SM (<= 85 registers/thread)
 constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
-constexpr int kFuseInElems = 16384;  // batch * n up to which the GEMV computes x' itself
+#ifndef QL_FUSE_IN_ELEMS
+#define QL_FUSE_IN_ELEMS 16384
+#endif
+constexpr int kFuseInElems = QL_FUSE_IN_ELEMS;  // batch * n up to which the GEMV computes x' itself
 constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
 constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
 constexpr int kTcMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA

@@ -35,7 +35,7 @@ struct RhtGeometry {
     int tpg;      // threads per group (B / E)
 };
 
-// E = 16 entries per thread (32 for B = 32768, to stay within 1024 threads).
+// E entries per thread (B / E <= 1024 threads).
 static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
     RhtGeometry g;
     g.B = B;
@@ -58,11 +58,13 @@ __device__ __forceinline__ size_t umma_tile_index4(int col, int b, int npad) {
     return (((size_t)s * npad + b) * 128 + chunk * 16 + (kin & 7) * 2) / 2;  // in halves
 }
 
+// B / E threads for one Hadamard block: up to 1024 threads per CTA for
+// E >= 16 (the launch bound keeps those within 64 registers per thread), up
+// to 512 for E = 8.
 template <int MODE, int E>
-__global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, RhtGeometry geo,
+__global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_in_kernel(const __half* __restrict__ x, int batch, int n, RhtGeometry geo,
                               const uint32_t* __restrict__ sin_bits, __half* __restrict__ out, int npad) {
     extern __shared__ float smem[];
-    grid_dependency_wait();
     const int B = geo.B;
     const int grp = threadIdx.x / geo.tpg, tid = threadIdx.x % geo.tpg;
     const int item = blockIdx.x * geo.groups + grp;
@@ -70,10 +72,12 @@ __global__ void rht_in_kernel(const __half* __restrict__ x, int batch, int n, Rh
     float* buf = smem + (size_t)grp * (B + B / 16);
     const int b = active ? item / geo.per_row : 0;
     const int col = (active ? (item % geo.per_row) * B : 0) + tid * E;
+    // the sign bits are written once at create time: read before the wait
+    const uint32_t sw = active ? sin_bits[col >> 5] >> (col & 31) : 0u;  // E <= 32 consecutive sign bits
+    grid_dependency_wait();
     float v[E];
     if (active) {
         const __half* xs = x + (size_t)b * n + col;
-        const uint32_t sw = sin_bits[col >> 5] >> (col & 31);  // E <= 32 consecutive sign bits
 #pragma unroll
         for (int q = 0; q < E; q += 8) {
             const uint4 raw = *reinterpret_cast<const uint4*>(xs + q);
@@ -141,10 +145,9 @@ cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npa
 
 // Entries per thread of the output transform: B_m may be as small as 16.
 template <bool F16, int E>
-__global__ void rht_out_kernel(float* __restrict__ z, int batch, int m, RhtGeometry geo,
+__global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_out_kernel(float* __restrict__ z, int batch, int m, RhtGeometry geo,
                                const uint32_t* __restrict__ sout_bits, float alpha, void* __restrict__ y) {
     extern __shared__ float smem[];
-    grid_dependency_wait();
     const int B = geo.B;
     const int grp = threadIdx.x / geo.tpg, tid = threadIdx.x % geo.tpg;
     const int item = blockIdx.x * geo.groups + grp;
@@ -152,6 +155,10 @@ __global__ void rht_out_kernel(float* __restrict__ z, int batch, int m, RhtGeome
     float* buf = smem + (size_t)grp * (B + B / 16);
     const int b = active ? item / geo.per_row : 0;
     const int row = (active ? (item % geo.per_row) * B : 0) + tid * E;
+    // the sign bits are written once at create time: read before the wait
+    const uint32_t sw = active ? sout_bits[row >> 5] >> (row & 31) : 0u;
+    const float scale = alpha * rsqrtf((float)B);
+    grid_dependency_wait();
     float v[E];
     if (active) {
         float* zs = z + (size_t)b * m + row;
@@ -171,8 +178,6 @@ __global__ void rht_out_kernel(float* __restrict__ z, int batch, int m, RhtGeome
     fwht_block<E>(v, B, tid, geo.tpg, buf);
     grid_launch_dependents();
     if (!active) return;
-    const float scale = alpha * rsqrtf((float)B);
-    const uint32_t sw = sout_bits[row >> 5] >> (row & 31);
 #pragma unroll
     for (int q = 0; q < E; ++q) v[q] = ((sw >> q) & 1u) ? -v[q] * scale : v[q] * scale;
     if (F16) {
@@ -212,8 +217,10 @@ static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y
 
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st) {
     const bool f16 = y_dtype == QL_F16;
+    // 8 entries per thread up to blocks of 4096 (512 threads): shorter chains per thread
     if (L.B_m > 16384) return f16 ? launch_rht_out_e<true, 32>(L, z, batch, y, st) : launch_rht_out_e<false, 32>(L, z, batch, y, st);
-    return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
+    if (L.B_m > 4096) return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
+    return f16 ? launch_rht_out_e<true, 8>(L, z, batch, y, st) : launch_rht_out_e<false, 8>(L, z, batch, y, st);
 }
 
 }  // namespace qlk
