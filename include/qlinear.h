@@ -100,6 +100,7 @@ typedef struct {
     size_t lut_bytes;          /* HYB table: 2^Q * V * 2 bytes                   */
     size_t scratch_bytes;      /* device scratch currently held by the handle    */
     int last_launches;         /* kernels launched by the most recent forward    */
+    int nparts;                /* row parts (1 uniform, 2 half-TCQ, up to 8)     */
 } ql_info_t;
 
 /* Create a uniform-bitrate layer.
@@ -123,6 +124,23 @@ int qlinear_create(qlinear_t* out, int m, int n, int k, int L, int V, ql_code_t 
  * k_bot bits.  m_top % 16 == 0, 0 < m_top < m.  n_words = (m_top*k_top +
  * (m - m_top)*k_bot) * n / 32.  Otherwise as qlinear_create. */
 int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int k_bot,
+                         int L, int V, ql_code_t code,
+                         const uint32_t* packed_codes, size_t n_words,
+                         const int8_t* s_in, const int8_t* s_out, float alpha);
+
+/* Create a layer of several row parts, each with its own bitwidth: layers
+ * that share their input fused along m (Q-Palette page: layer fusion of
+ * layers that read the same input, and a palette of TCQ quantizers of
+ * different bitwidths).  Part i covers rows [sum of part_rows[0..i), +
+ * part_rows[i]) at part_k[i] bits; the parts' streams follow one another in
+ * packed_codes, each in the stream format above.  One sign vector each for
+ * the input and the (fused) output, one Hadamard transform of the fused m.
+ *   nparts:     1..8;  part_rows, part_k: host arrays of nparts entries,
+ *               part_rows[i] % 16 == 0, sum(part_rows) == m, part_k[i] in 1..4.
+ *   n_words:    sum over parts of part_rows[i] * n * part_k[i] / 32.
+ * Otherwise as qlinear_create (qlinear_create_mixed is the two-part case).
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED, QL_E_OOM, QL_E_CUDA. */
+int qlinear_create_parts(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k,
                          int L, int V, ql_code_t code,
                          const uint32_t* packed_codes, size_t n_words,
                          const int8_t* s_in, const int8_t* s_out, float alpha);

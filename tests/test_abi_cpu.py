@@ -93,3 +93,26 @@ def test_forward_noalloc_rejects_bad_arguments_on_the_host(tcm):
     header = open(os.path.join(ROOT, "include", "qlinear.h")).read()
     assert re.search(r"#define QL_NOALLOC_SCRATCH_BYTES \(2 \* 1024 \* 1024\)", header)
     assert tcm.QL_NOALLOC_SCRATCH_BYTES == 2 * 1024 * 1024
+
+
+
+def test_create_parts_rejects_bad_arguments_on_the_host(tcm):
+    lib = tcm.raw_library()
+    code = tcm.ql_code_t(0, 0, None)
+
+    def create(rows, ks, m=None, n=256, n_words=None):
+        h = ctypes.c_void_p()
+        m = sum(rows) if m is None else m
+        nw = sum(r * n * k for r, k in zip(rows, ks)) // 32 if n_words is None else n_words
+        r = (ctypes.c_int * max(1, len(rows)))(*rows)
+        k = (ctypes.c_int * max(1, len(ks)))(*ks)
+        return lib.qlinear_create_parts(ctypes.byref(h), m, n, len(rows), r, k, 16, 1, code, None, nw, None, None, 1.0)
+
+    assert create([], []) == tcm.QL_E_ARG                          # no parts
+    assert create([16] * 9, [2] * 9) == tcm.QL_E_ARG               # more than 8 parts
+    assert create([16, 24], [2, 3]) == tcm.QL_E_UNSUPPORTED        # m = 40: not a multiple of 16
+    assert create([16, 16], [2, 3], m=48) == tcm.QL_E_ARG          # parts do not add up to m
+    assert create([16, 8, 8], [2, 3, 3]) == tcm.QL_E_ARG           # part rows not a multiple of 16
+    assert create([16, 16], [2, 5]) == tcm.QL_E_UNSUPPORTED        # k out of range
+    assert create([16, 16], [2, 3], n_words=7) == tcm.QL_E_ARG     # wrong stream length
+    assert create([16, 16], [2, 3]) == tcm.QL_E_ARG                # valid shape, null device pointers

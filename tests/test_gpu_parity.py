@@ -168,18 +168,19 @@ def test_info_reports_the_bit_accounting():
 
 # ---------------------------------------------------------------- full-size workloads
 FULL = [("tiny", 1), ("attn4096", 1), ("mlp_up", 8), ("mlp_down", 4), ("large", 4), ("large", 16),
-        ("halftcq", 64), ("halftcq", 256)]
+        ("halftcq", 64), ("halftcq", 256), ("qkv_fused", 1), ("qkv_fused", 16)]
 
 
-@pytest.mark.parametrize("name", ["tiny", "attn4096", "mlp_up", "mlp_down", "large", "halftcq"])
+@pytest.mark.parametrize("name", ["tiny", "attn4096", "mlp_up", "mlp_down", "large", "halftcq", "qkv_fused"])
 def test_full_decode_sampled_rows_bit_exact(name):
     sp = wl.WORKLOADS[name]
     li = wl.make_layer(sp)
     h = make_handle(li)
     w = tcm.qlinear_decode(h)
     rng = np.random.default_rng(42)
+    bounds = [r0 for r0, _, _ in sp.row_parts()[1:]]  # first rows of the later parts
     rows = np.unique(np.concatenate([[0, sp.m - 1], rng.integers(0, sp.m, 10),
-                                     [sp.m_top - 1, sp.m_top] if sp.mixed else []])).astype(np.int64)
+                                     [b - 1 for b in bounds] + bounds])).astype(np.int64)
     ref = oq.Layer.from_inputs(li).decode_bits(rows)
     got = _bits(w[torch.from_numpy(rows).cuda()])
     assert np.array_equal(got, ref)
@@ -241,3 +242,30 @@ def test_forward_largest_hadamard_blocks(m, n):
     y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
     y_ref = oq.Layer.from_inputs(li).forward(x)
     assert rel_err(y.cpu().numpy(), y_ref) <= TOL_GEMV
+
+
+# ---------------------------------------------------------------- layers of several row parts
+PARTS = [((32, 2), (48, 3), (16, 4)), ((16, 1), (16, 2), (32, 3), (16, 4), (16, 2))]
+
+
+@pytest.mark.parametrize("split", PARTS, ids=lambda v: "-".join(f"{r}k{k}" for r, k in v))
+def test_parts_decode_bit_exact(split):
+    m = sum(r for r, _ in split)
+    li = wl.random_layer(m, 512, 0, 16, 1, wl.CODE_3INST, seed=21 + m, alpha=0.5, row_split=split)
+    h = make_handle(li)
+    assert tcm.qlinear_info(h)["nparts"] == len(split)
+    w = tcm.qlinear_decode(h)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(w), oq.Layer.from_inputs(li).decode_bits(np.arange(m)))
+
+
+@pytest.mark.parametrize("split", PARTS, ids=lambda v: "-".join(f"{r}k{k}" for r, k in v))
+@pytest.mark.parametrize("batch", [1, 3, 16, 40])
+def test_parts_forward(split, batch):
+    m = sum(r for r, _ in split)
+    li = wl.random_layer(m, 512, 0, 16, 1, wl.CODE_1MAD, seed=31 + m, alpha=0.5, row_split=split)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=11)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= (TOL_GEMV if batch <= 8 else TOL_TC)

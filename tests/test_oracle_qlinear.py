@@ -113,3 +113,22 @@ def test_mixed_layer_decodes_each_part_with_its_own_k():
     W = layer.decode_rows(np.arange(32))
     assert np.array_equal(W[:16], top.decode_rows(np.arange(16)))
     assert np.array_equal(W[16:], bot.decode_rows(np.arange(16)))
+
+
+def test_layer_of_several_parts_is_the_stack_of_its_parts():
+    """A layer fused along m from parts of different bitwidths: its weight rows
+    are those of the single-part layers decoded from the consecutive
+    sub-streams (each part's blocks keep their own tail-biting)."""
+    split = ((16, 2), (32, 4), (16, 1))
+    li = wl.random_layer(64, 512, 0, 16, 1, wl.CODE_1MAD, 5, row_split=split)
+    layer = qlinear.Layer.from_inputs(li)
+    W = layer.decode_rows(np.arange(64))
+    off, r0 = 0, 0
+    for rows, k in split:
+        words = li.codes[off: off + rows * 512 * k // 32]
+        single = qlinear.Layer(rows, 512, [(0, rows, k)], 16, 1, wl.CODE_1MAD, words, li.s_in,
+                               li.s_out[r0:r0 + rows], 1.0)
+        assert np.array_equal(W[r0:r0 + rows], single.decode_rows(np.arange(rows)))
+        off += rows * 512 * k // 32
+        r0 += rows
+    assert off == len(li.codes) and li.spec.bits_per_weight == (16 * 2 + 32 * 4 + 16 * 1) / 64

@@ -37,7 +37,7 @@ QL_F32 = 0
 QL_F16 = 1
 
 # Every function include/qlinear.h declares (checked by the CPU tests).
-ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_forward", "qlinear_forward_host",
+ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts", "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
                "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
                "qlinear_forward_noalloc")
@@ -50,13 +50,15 @@ class ql_code_t(ctypes.Structure):
 class ql_info_t(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int) for f in ("m", "n", "L", "V", "code", "Q", "k_top", "k_bot", "m_top", "B_n", "B_m")] + \
                [(f, ctypes.c_size_t) for f in ("stream_bytes", "sign_bytes", "lut_bytes", "scratch_bytes")] + \
-               [("last_launches", ctypes.c_int)]
+               [("last_launches", ctypes.c_int), ("nparts", ctypes.c_int)]
 
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
 _lib.qlinear_create.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, ql_code_t, _vp, _sz, _vp, _vp, _f]
 _lib.qlinear_create_mixed.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _i, _i, ql_code_t, _vp, _sz, _vp,
                                       _vp, _f]
+_lib.qlinear_create_parts.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _i,
+                                      ql_code_t, _vp, _sz, _vp, _vp, _f]
 _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
@@ -158,6 +160,24 @@ def qlinear_create_mixed(m, n, m_top, k_top, k_bot, L, V, kind, codes, s_in, s_o
     _check(_lib.qlinear_create_mixed(ctypes.byref(out), m, n, m_top, k_top, k_bot, L, V, _code(kind, Q, lut),
                                      _ptr(codes), codes.numel(), _ptr(s_in), _ptr(s_out), float(alpha)),
            "qlinear_create_mixed")
+    return QLinearHandle(out.value, m, n)
+
+
+def qlinear_create_parts(m, n, part_rows, part_k, L, V, kind, codes, s_in, s_out, alpha, Q=0,
+                         lut=None) -> QLinearHandle:
+    """A layer of several row parts (layers fused along m), part i at part_k[i] bits."""
+    import torch
+    _cuda(codes, "codes", (torch.int32, torch.uint32))
+    _cuda(s_in, "s_in", torch.int8)
+    _cuda(s_out, "s_out", torch.int8)
+    if len(part_rows) != len(part_k):
+        raise ValueError("part_rows and part_k must have the same length")
+    rows = (ctypes.c_int * max(1, len(part_rows)))(*part_rows)
+    ks = (ctypes.c_int * max(1, len(part_k)))(*part_k)
+    out = _vp()
+    _check(_lib.qlinear_create_parts(ctypes.byref(out), m, n, len(part_rows), rows, ks, L, V, _code(kind, Q, lut),
+                                     _ptr(codes), codes.numel(), _ptr(s_in), _ptr(s_out), float(alpha)),
+           "qlinear_create_parts")
     return QLinearHandle(out.value, m, n)
 
 

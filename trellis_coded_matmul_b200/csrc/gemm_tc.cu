@@ -87,7 +87,7 @@ struct TcPart {
 };
 
 struct GemmArgs {
-    TcPart part[2];
+    TcPart part[kMaxParts];
     int nparts;
     int nb;                 // 256-column blocks per row
     int units;              // (tile, block) units of the layer: sum over parts of tiles * nb
@@ -122,19 +122,28 @@ __host__ __device__ inline TcSmem tc_smem_layout(int stages, int code_slots, int
 }
 
 // A CTA's run of units in order, walked without divisions (the roles' loops
-// are latency-bound chains; the MMA issuer's especially).
+// are latency-bound chains; the MMA issuer's especially).  Units are numbered
+// part by part, tile by tile, block by block.
 struct TcWalk {
-    int u, gt, j;  // unit, global 128-row tile, block
-    __device__ __forceinline__ TcWalk(const GemmArgs& p, int u0) : u(u0), gt(u0 / p.nb), j(u0 - (u0 / p.nb) * p.nb) {}
+    int u, pt, t, j;  // unit, part, 128-row tile within the part, block
+    __device__ __forceinline__ TcWalk(const GemmArgs& p, int u0) : u(u0), pt(0), j(0) {
+        int gt = u0 / p.nb;
+        j = u0 - gt * p.nb;
+        while (pt + 1 < p.nparts && gt >= p.part[pt].tiles) gt -= p.part[pt++].tiles;
+        t = gt;
+    }
     __device__ __forceinline__ void next(const GemmArgs& p) {
         ++u;
         if (++j == p.nb) {
             j = 0;
-            ++gt;
+            if (++t == p.part[pt].tiles && pt + 1 < p.nparts) {
+                t = 0;
+                ++pt;
+            }
         }
     }
-    __device__ __forceinline__ int part(const GemmArgs& p) const { return (p.nparts > 1 && gt >= p.part[0].tiles) ? 1 : 0; }
-    __device__ __forceinline__ int tile(const GemmArgs& p) const { return part(p) ? gt - p.part[0].tiles : gt; }
+    __device__ __forceinline__ int part(const GemmArgs&) const { return pt; }
+    __device__ __forceinline__ int tile(const GemmArgs&) const { return t; }
 };
 
 // Slot and phase parity of a ring position, advanced without divisions.
@@ -501,7 +510,7 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
         tiles += a.part[i].tiles;
         kmax = pt.k > kmax ? pt.k : kmax;
     }
-    if (L.nparts == 1) a.part[1] = a.part[0];
+    for (int i = L.nparts; i < kMaxParts; ++i) a.part[i] = a.part[0];
     a.units = tiles * a.nb;
     a.lmask = (1u << L.L) - 1u;
     a.qshift = 32 - L.Q;

@@ -18,6 +18,7 @@ constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory l
 #define QL_FUSE_IN_ELEMS 16384
 #endif
 constexpr int kFuseInElems = QL_FUSE_IN_ELEMS;  // batch * n up to which the GEMV computes x' itself
+constexpr int kMaxParts = 8;          // row parts of one layer (layers fused along m, own bitwidth each)
 constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
 constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
 constexpr int kTcMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA
@@ -44,7 +45,7 @@ struct Layer {
     float alpha;
     int B_n, B_m;
     int nparts;
-    Part parts[2];
+    Part parts[kMaxParts];
     uint32_t* words;      // all parts, kernel layout
     uint32_t* sin_bits;   // bit i set <=> s_in[i] == -1
     uint32_t* sout_bits;

@@ -86,7 +86,7 @@ int check_code(const ql_code_t& code, int V) {
     return QL_OK;
 }
 
-// Shared by both create calls. parts: [(rows, k)].
+// Shared by the create calls. parts: [(rows, k)], host arrays.
 int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k, int L,
                   int V, ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
                   const int8_t* s_out, float alpha) {
@@ -96,15 +96,18 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (V != 1 && V != 2) return QL_E_ARG;
     if (n % kT != 0 || m % kRowTile != 0) return QL_E_UNSUPPORTED;
     if (pow2_block(n) > kMaxHadamard || pow2_block(m) > kMaxHadamard) return QL_E_UNSUPPORTED;
+    if (nparts < 1 || nparts > kMaxParts || !part_rows || !part_k) return QL_E_ARG;
     size_t expect_words = 0;
+    long long rows_sum = 0;
     for (int i = 0; i < nparts; ++i) {
         const int k = part_k[i];
         if (k < 1 || k > 4) return QL_E_UNSUPPORTED;
         if (L < k * V || L > 16) return QL_E_UNSUPPORTED;
         if (part_rows[i] <= 0 || part_rows[i] % kRowTile != 0) return QL_E_ARG;
         expect_words += (size_t)part_rows[i] * n * k / 32;
+        rows_sum += part_rows[i];
     }
-    if (n_words != expect_words) return QL_E_ARG;
+    if (rows_sum != m || n_words != expect_words) return QL_E_ARG;
     int rc = check_code(code, V);
     if (rc != QL_OK) return rc;
     if (!is_device_pointer(packed_codes) || !is_device_pointer(s_in) || !is_device_pointer(s_out))
@@ -304,6 +307,14 @@ int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int
     return create_common(out, m, n, 2, rows, ks, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
 }
 
+int qlinear_create_parts(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k, int L,
+                         int V, ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
+                         const int8_t* s_out, float alpha) {
+    if (!out) return QL_E_ARG;
+    *out = nullptr;
+    return create_common(out, m, n, nparts, part_rows, part_k, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+}
+
 int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream) {
     if (!h || batch < 0 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
     if (batch == 0) return QL_OK;
@@ -419,6 +430,7 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->lut_bytes = L.code == QL_CODE_HYB ? ((size_t)1 << L.Q) * L.V * 2 : 0;
     info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
     info->last_launches = L.last_launches;
+    info->nparts = L.nparts;
     return QL_OK;
 }
 

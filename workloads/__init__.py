@@ -23,7 +23,7 @@ cast), activations x ~ N(0,1) cast to fp16.
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -51,14 +51,22 @@ class LayerSpec:
     k_top: Optional[int] = None
     k_bot: Optional[int] = None
     batches: Sequence[int] = (1,)
+    row_split: Optional[Tuple[Tuple[int, int], ...]] = None  # ((rows, k), ...): layers fused along m
 
     @property
     def mixed(self) -> bool:
-        return self.m_top is not None
+        return self.m_top is not None or self.row_split is not None
 
     def row_parts(self):
         """[(row0, rows, k)] in stream order."""
-        if self.mixed:
+        if self.row_split is not None:
+            out, r0 = [], 0
+            for rows, k in self.row_split:
+                out.append((r0, rows, k))
+                r0 += rows
+            assert r0 == self.m
+            return out
+        if self.m_top is not None:
             return [(0, self.m_top, self.k_top), (self.m_top, self.m - self.m_top, self.k_bot)]
         return [(0, self.m, self.k)]
 
@@ -83,6 +91,10 @@ WORKLOADS = {
     "large": LayerSpec("large", 28672, 8192, 4, 16, 1, CODE_1MAD, 0.01, seed=3, batches=(1, 4, 16)),
     "halftcq": LayerSpec("halftcq", 14336, 4096, 0, 16, 1, CODE_3INST, 1.0, seed=4,
                          m_top=7168, k_top=2, k_bot=3, batches=(64, 256)),
+    # Q, K and V projections of a 4096-wide attention block fused along m (they
+    # read the same input), each with its own bitwidth: 2, 3 and 4 bits.
+    "qkv_fused": LayerSpec("qkv_fused", 12288, 4096, 0, 16, 1, CODE_3INST, 0.02, seed=5,
+                           row_split=((4096, 2), (4096, 3), (4096, 4)), batches=(1, 16)),
 }
 
 # The up and down projections of the MLP pair draw from one seeded stream
@@ -135,8 +147,11 @@ def make_x(spec: LayerSpec, batch: int, instance: int = 0) -> np.ndarray:
 
 
 def random_layer(m: int, n: int, k: int, L: int, V: int, code: int, seed: int,
-                 alpha: float = 1.0, Q: int = 9, m_top=None, k_top=None, k_bot=None) -> LayerInputs:
-    """A small seeded layer of any supported shape (tests of ragged/edge shapes)."""
-    spec = LayerSpec(f"rand_{m}x{n}_k{k}", m, n, k if m_top is None else 0, L, V, code, alpha,
-                     seed, Q=Q if code == CODE_HYB else 0, m_top=m_top, k_top=k_top, k_bot=k_bot)
+                 alpha: float = 1.0, Q: int = 9, m_top=None, k_top=None, k_bot=None, row_split=None) -> LayerInputs:
+    """A small seeded layer of any supported shape (tests of ragged/edge shapes); row_split
+    ((rows, k), ...) makes a layer of several row parts (layers fused along m)."""
+    uniform = m_top is None and row_split is None
+    spec = LayerSpec(f"rand_{m}x{n}_k{k}", m, n, k if uniform else 0, L, V, code, alpha,
+                     seed, Q=Q if code == CODE_HYB else 0, m_top=m_top, k_top=k_top, k_bot=k_bot,
+                     row_split=tuple(tuple(r) for r in row_split) if row_split is not None else None)
     return make_layer(spec)
