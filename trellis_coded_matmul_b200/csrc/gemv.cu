@@ -321,6 +321,191 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p,
     if (u0 < u1) flush(curR);
 }
 
+// ---- decode-GEMV over all row parts of a layer in one launch ----
+// Units are numbered part by part (each part's row tiles x blocks, as in the
+// single-part kernel); a warp's contiguous range may cross into the next part,
+// whose bitwidth it dispatches per unit.  x' comes in the fragment layout from
+// the separate input-transform kernel.
+struct GemvPartArgs {
+    const uint32_t* words;  // the part's words, kernel layout
+    int rt;                 // row tiles
+    int row0;               // first layer row
+    int k;                  // bits per weight
+};
+struct GemvMultiArgs {
+    GemvPartArgs part[kMaxParts];
+    int nparts, nb;
+    uint32_t lmask;
+    int qshift;
+    const uint32_t* lut;
+    int lut_entries;
+    const uint2* xf;
+    int batch;
+    float* z;
+    int m;
+};
+
+// Two thread-rows of one unit at k bits per weight into w[h][0 .. 2k-1].
+__device__ __forceinline__ void load_unit_k(uint32_t (&w)[2][8], const uint32_t* unit_base, int k, int lane) {
+    uint32_t t1[2][2], t2[2][4], t3[2][6], t4[2][8];
+    switch (k) {
+        case 1: load_unit<1>(t1, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 2; ++i) w[h][i] = t1[h][i]; break;
+        case 2: load_unit<2>(t2, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 4; ++i) w[h][i] = t2[h][i]; break;
+        case 3: load_unit<3>(t3, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 6; ++i) w[h][i] = t3[h][i]; break;
+        default: load_unit<4>(t4, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 8; ++i) w[h][i] = t4[h][i]; break;
+    }
+}
+
+// One unit at K bits: take its words from nxt, start the next unit's load
+// into nxt, then decode and multiply.
+template <int CODE, int K, int V, bool L16>
+__device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k, int lane,
+                                          int src_lane, const GemvMultiArgs& p, const uint32_t* lut_lane,
+                                          size_t xoff, bool use_x, float (&acc)[4]) {
+    uint32_t cw[2][2 * K + 1];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = nxt[h][i];
+    if (next_base) load_unit_k(nxt, next_base, next_k, lane);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
+    for_each_mma<CODE, K, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
+        uint2 bv = make_uint2(0u, 0u);
+        if (use_x) bv = __ldg(p.xf + xoff + (size_t)u * p.batch * 4);
+        mma_16816(acc, a, bv.x, bv.y);
+    });
+}
+
+template <int CODE, int V, bool L16>
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvMultiArgs p) {
+    extern __shared__ uint32_t smem[];
+    const int lane = threadIdx.x & 31;
+    if (CODE == kCodeHYB) {
+        fill_lut_smem(smem, p.lut, p.lut_entries);
+        __syncthreads();
+    }
+    const uint32_t* lut_lane = smem + lane;
+    const int nb = p.nb;
+    long long U = 0;
+    for (int i = 0; i < p.nparts; ++i) U += (long long)p.part[i].rt * nb;
+    const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
+    const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
+    const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
+    const int g = lane >> 2, c = lane & 3;
+    const int src_lane = (lane & ~3) | ((c + 3) & 3);
+    const int batch = p.batch;
+
+    // walker: part pt, row tile t within it, block j
+    int pt = 0;
+    long long rest = u0;
+    while (pt + 1 < p.nparts && rest >= (long long)p.part[pt].rt * nb) rest -= (long long)p.part[pt++].rt * nb;
+    int t = (int)(rest / nb), j = (int)(rest % nb);
+    auto unit_base = [&](int part, int tile, int blk) {
+        return p.part[part].words + ((size_t)tile * nb + blk) * 128 * p.part[part].k;
+    };
+    uint32_t nxt[2][8];
+    if (u0 < u1) load_unit_k(nxt, unit_base(pt, t, j), p.part[pt].k, lane);
+    grid_dependency_wait();  // x' from the input transform; z consumed by the last output transform
+    grid_launch_dependents();
+
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int cur_pt = pt, cur_t = t;
+    auto flush = [&](int part, int tile) {
+        const int row = p.part[part].row0 + tile * kRowTile + g;
+        const int b0 = 2 * c, b1 = 2 * c + 1;
+        if (b0 < batch) {
+            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
+            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
+        }
+        if (b1 < batch) {
+            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
+            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
+        }
+    };
+    for (long long unit = u0; unit < u1; ++unit) {
+        // the unit after this one, for the prefetch
+        int npt = pt, nt = t, nj = j + 1;
+        if (nj == nb) {
+            nj = 0;
+            if (++nt == p.part[npt].rt && npt + 1 < p.nparts) {
+                nt = 0;
+                ++npt;
+            }
+        }
+        const uint32_t* next_base = unit + 1 < u1 ? unit_base(npt, nt, nj) : nullptr;
+        if (pt != cur_pt || t != cur_t) {
+            flush(cur_pt, cur_t);
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            cur_pt = pt;
+            cur_t = t;
+        }
+        const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
+        const bool use_x = g < batch;
+        switch (p.part[pt].k) {
+            case 1: gemv_unit<CODE, 1, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+            case 2: gemv_unit<CODE, 2, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+            case 3: gemv_unit<CODE, 3, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+            default: gemv_unit<CODE, 4, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        }
+        pt = npt;
+        t = nt;
+        j = nj;
+    }
+    if (u0 < u1) flush(cur_pt, cur_t);
+}
+
+template <int CODE, int V, bool L16>
+static cudaError_t launch_gemv_multi_t(const GemvMultiArgs& a, int grid, int threads, size_t smem, cudaStream_t st) {
+    auto kern = gemv_multi_kernel<CODE, V, L16>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a);
+}
+
+cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, float* z, cudaStream_t st) {
+    GemvMultiArgs a;
+    a.nparts = L.nparts;
+    a.nb = L.n / kT;
+    long long units = 0;
+    for (int i = 0; i < kMaxParts; ++i) {
+        const Part& pt = L.parts[i < L.nparts ? i : 0];
+        a.part[i].words = L.words + pt.word_off;
+        a.part[i].rt = pt.rows / kRowTile;
+        a.part[i].row0 = pt.row0;
+        a.part[i].k = pt.k;
+        if (i < L.nparts) units += (long long)a.part[i].rt * a.nb;
+    }
+    a.lmask = (1u << L.L) - 1u;
+    a.qshift = 32 - L.Q;
+    a.lut = L.lut;
+    a.lut_entries = L.code == kCodeHYB ? (1 << L.Q) : 0;
+    a.xf = (const uint2*)xp_frag;
+    a.batch = batch;
+    a.z = z;
+    a.m = L.m;
+    // one CTA per SM, warps sized so that every warp gets the same whole number of units
+    const int grid = (int)(units < L.num_sms ? units : L.num_sms);
+    const long long per_cta = (units + grid - 1) / grid;
+    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
+    const int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
+    const size_t smem = (size_t)a.lut_entries * 32 * 4;
+    const bool l16 = L.L == 16;
+    if (L.code == kCode1MAD && L.V == 1) return l16 ? launch_gemv_multi_t<kCode1MAD, 1, true>(a, grid, threads, smem, st)
+                                                    : launch_gemv_multi_t<kCode1MAD, 1, false>(a, grid, threads, smem, st);
+    if (L.code == kCode3INST && L.V == 1) return l16 ? launch_gemv_multi_t<kCode3INST, 1, true>(a, grid, threads, smem, st)
+                                                     : launch_gemv_multi_t<kCode3INST, 1, false>(a, grid, threads, smem, st);
+    if (L.code == kCodeHYB && L.V == 1) return l16 ? launch_gemv_multi_t<kCodeHYB, 1, true>(a, grid, threads, smem, st)
+                                                   : launch_gemv_multi_t<kCodeHYB, 1, false>(a, grid, threads, smem, st);
+    if (L.code == kCodeHYB && L.V == 2) return l16 ? launch_gemv_multi_t<kCodeHYB, 2, true>(a, grid, threads, smem, st)
+                                                   : launch_gemv_multi_t<kCodeHYB, 2, false>(a, grid, threads, smem, st);
+    return cudaErrorInvalidValue;
+}
+
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
 template <int CODE, int K, int V, bool L16>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {

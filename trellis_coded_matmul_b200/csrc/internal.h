@@ -122,6 +122,8 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch);
 // with pl.xsmem x' is computed from x in-kernel, else read from xp_frag.
 cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
                         int batch, float* z, cudaStream_t st);
+// The same for all row parts of a layer in one launch (nparts > 1), x' from xp_frag.
+cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, float* z, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
 // z[b][row] += W_hat x' for all parts (z all-zero on entry), x' in tensor-core
 // tiles with npad (multiple of 16, <= 256) rows, b < batch; the (128-row tile,

@@ -222,17 +222,17 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
     int rc = ensure(&L.xp, &L.xp_bytes, (size_t)batch * L.n * 2);
     if (rc == QL_OK) rc = prepare_z(L, (size_t)batch * L.m * 4, st);
     if (rc != QL_OK) return rc;
-    // One plan for all parts (a half-TCQ layer never fuses the input transform).
+    // A layer of several row parts runs all parts in one launch (x' from the
+    // separate input transform); a uniform layer may fuse the input transform.
     const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
+    const bool multi = L.nparts > 1;
+    const bool xsmem = !multi && pl.xsmem;
     cudaError_t e = cudaSuccess;
-    L.last_launches = L.nparts + 1 + (pl.xsmem ? 0 : 1);
-    if (!pl.xsmem) e = launch_rht_in_frag(L, x, batch, L.xp, st);
+    L.last_launches = 2 + (xsmem ? 0 : 1);
+    if (!xsmem) e = launch_rht_in_frag(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-    for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) {
-        const GemvPlan pi = i == 0 ? pl : plan_gemv(L, L.parts[i], batch);
-        e = launch_gemv(L, L.parts[i], pi, x, L.xp, batch, L.z, st);
-    }
+    if (e == cudaSuccess) e = multi ? launch_gemv_multi(L, L.xp, batch, L.z, st) : launch_gemv(L, L.parts[0], pl, x, L.xp, batch, L.z, st);
     if (e == cudaSuccess && slot >= 0) {
         e = record_event(L.prof_ev[2 * slot + 1], st);
         L.prof_next = (L.prof_next + 1) % L.prof_cap;
@@ -567,18 +567,17 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     cudaStream_t st = (cudaStream_t)stream;
 
     const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
+    const bool multi = L.nparts > 1;
+    const bool xsmem = !multi && pl.xsmem;
     // z must start at zero; another handle's failed call may have left sums there.
     cudaError_t e = cudaMemsetAsync(z, 0, z_bytes, st);
-    if (e == cudaSuccess && !pl.xsmem) e = launch_rht_in_frag(L, x, batch, xp, st);
-    for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) {
-        const GemvPlan pi = i == 0 ? pl : plan_gemv(L, L.parts[i], batch);
-        e = launch_gemv(L, L.parts[i], pi, x, xp, batch, z, st);
-    }
+    if (e == cudaSuccess && !xsmem) e = launch_rht_in_frag(L, x, batch, xp, st);
+    if (e == cudaSuccess) e = multi ? launch_gemv_multi(L, xp, batch, z, st) : launch_gemv(L, L.parts[0], pl, x, xp, batch, z, st);
     if (e == cudaSuccess) e = launch_rht_out(L, z, batch, y, y_dtype, st);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.last_launches = L.nparts + 1 + (pl.xsmem ? 0 : 1);
+    L.last_launches = 2 + (xsmem ? 0 : 1);
     return QL_OK;
 }
