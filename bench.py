@@ -234,10 +234,18 @@ def job_tokens_per_s(world, steps, batch, secs):
 
 
 # ------------------------------------------------------------------ CUDA arm
-def _source_hash():
+# the sources each profiled kernel is built from (its DRAM-traffic capture is
+# valid while these are unchanged)
+KERNEL_SOURCES = {
+    "gemv": ("gemv.cu", "codes.cuh", "layout.cuh", "fwht.cuh", "internal.h"),
+    "gemm": ("gemm_tc.cu", "codes.cuh", "layout.cuh", "tc_ptx.cuh", "internal.h"),
+}
+
+
+def _source_hash(kind):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "trellis_coded_matmul_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kind]:
         h.update(name.encode())
         h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
@@ -245,12 +253,12 @@ def _source_hash():
 
 def _traffic(kernel_key, launch_units):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    on the current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(kernel_key)
-    if not d or d.get("source_hash") != _source_hash():
+    if not d or d.get("source_hash") != _source_hash(kernel_key.split("_")[0]):
         return None
     return d["dram_bytes"] * launch_units / d["units"]
 
