@@ -217,9 +217,12 @@ static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y
 
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st) {
     const bool f16 = y_dtype == QL_F16;
-    // 8 entries per thread up to blocks of 4096 (512 threads): shorter chains per thread
+    // Small batches (a few CTAs, latency-bound): 8 entries per thread up to blocks
+    // of 4096 (512 threads), shorter chains per thread.  Large batches (many
+    // CTAs, bandwidth-bound): 16, fewer and fuller CTAs.
     if (L.B_m > 16384) return f16 ? launch_rht_out_e<true, 32>(L, z, batch, y, st) : launch_rht_out_e<false, 32>(L, z, batch, y, st);
-    if (L.B_m > 4096) return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
+    if (L.B_m > 4096 || batch > kGemvMaxBatch)
+        return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
     return f16 ? launch_rht_out_e<true, 8>(L, z, batch, y, st) : launch_rht_out_e<false, 8>(L, z, batch, y, st);
 }
 
