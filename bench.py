@@ -204,7 +204,8 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_dict(sp, batch, 1, {"step": f"{bps} blocks of 256 columns of W_hat per step "
+            "config": config_dict(sp, batch, 1, {"l2": "CPU oracle: no GPU caches involved",
+                                                 "step": f"{bps} blocks of 256 columns of W_hat per step "
                                                          f"(1/{sp.m * nb / bps:g} of a forward)"}),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
