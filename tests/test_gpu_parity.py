@@ -269,3 +269,31 @@ def test_parts_forward(split, batch):
     y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
     y_ref = oq.Layer.from_inputs(li).forward(x)
     assert rel_err(y.cpu().numpy(), y_ref) <= (TOL_GEMV if batch <= 8 else TOL_TC)
+
+
+# ---------------------------------------------------------------- tensor-core path over every small case
+# (L < 16, L = kV, HYB V = 1 and 2, 1-4 bits, ragged row tiles) at two batch sizes
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}_k{c[2]}_L{c[3]}_V{c[4]}_c{c[5]}")
+@pytest.mark.parametrize("batch", [16, 40])
+def test_forward_small_tensor_core_path(case, batch):
+    li = _small_layer(*case)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=13)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    assert tcm.qlinear_info(h)["last_launches"] == 3  # input transform, GEMM, output transform
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_TC
+
+
+@pytest.mark.parametrize("batch", [2, 24])
+def test_parts_with_the_hyb_code(batch):
+    split = ((16, 2), (32, 3), (16, 4))
+    li = wl.random_layer(64, 512, 0, 16, 2, wl.CODE_HYB, seed=41, alpha=0.5, Q=9, row_split=split)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=17)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= (TOL_GEMV if batch <= 8 else TOL_TC)
+    w = tcm.qlinear_decode(h)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(w), oq.Layer.from_inputs(li).decode_bits(np.arange(64)))
