@@ -1,0 +1,116 @@
+"""Pins for the trellis-coded quantization oracle (oracle/encode.py).
+
+- The exact tail-biting Viterbi is the true minimum: it equals brute force over
+  every bit string of tiny blocks.
+- The two-pass search is never better than the exact minimum.
+- With L = kV (no memory, plain kV-bit V-dimensional VQ: "When L = KV, TCQ
+  becomes K bit V dim VQ") both reduce to the nearest codeword at every step.
+- The encoded chunks, packed MSB-first into a block of the stream format, decode
+  through the layer oracle to the reconstruction the encoder scored.
+- On an i.i.d. N(0,1) source the distortion lies between the Gaussian
+  rate-distortion bound D(k) = 2^(-2k) and the optimal k-bit scalar (Lloyd-Max)
+  quantizer's distortion (0.3634 for 1 bit, 0.1175 for 2 bits: textbook
+  values), as the discussion's "Table 1" replies describe; a larger trellis
+  does better ("Larger trellises improve quality").
+- The two-pass search's costs follow its float32 rule."""
+import itertools
+
+import numpy as np
+import pytest
+
+import workloads as wl
+from oracle import bitstream, codes, encode, qlinear
+
+LLOYD_MAX = {1: 1.0 - 2.0 / np.pi, 2: 0.1175}
+
+
+def _brute_force(x, L, k, V, code, lut=None):
+    T = x.shape[0]
+    kV = k * V
+    best = None
+    for bits in itertools.product((0, 1), repeat=T * kV):
+        chunks = np.array([int("".join(map(str, bits[t * kV:(t + 1) * kV])), 2) for t in range(T)])
+        err = float(np.sum((x - encode.reconstruct(chunks, L, kV, code, V, lut)) ** 2))
+        if best is None or err < best:
+            best = err
+    return best
+
+
+@pytest.mark.parametrize("L,k,V,code,T", [(4, 1, 1, wl.CODE_3INST, 8), (4, 2, 1, wl.CODE_1MAD, 4),
+                                          (6, 1, 2, wl.CODE_HYB, 4), (5, 1, 1, wl.CODE_1MAD, 9)])
+def test_exact_viterbi_equals_brute_force(L, k, V, code, T):
+    rng = np.random.default_rng(L * 100 + k * 10 + V + T)
+    lut = wl.hyb_table(4, V, 7) if code == wl.CODE_HYB else None
+    for _ in range(3):
+        x = rng.standard_normal((T, V))
+        chunks, err = encode.encode_exact(x, L, k, V, code, lut)
+        assert err == pytest.approx(_brute_force(x, L, k, V, code, lut), rel=1e-12, abs=1e-12)
+        recon = encode.reconstruct(chunks, L, k * V, code, V, lut)
+        assert float(np.sum((x - recon) ** 2)) == pytest.approx(err, rel=1e-12, abs=1e-12)
+
+
+def test_two_pass_is_never_better_than_the_exact_minimum():
+    rng = np.random.default_rng(3)
+    for L, k in [(6, 1), (6, 2), (8, 2)]:
+        for _ in range(4):
+            x = rng.standard_normal((32, 1))
+            _, exact = encode.encode_exact(x, L, k, 1, wl.CODE_3INST)
+            _, two = encode.encode_two_pass(x, L, k, 1, wl.CODE_3INST)
+            assert two >= exact * (1 - 1e-6)
+
+
+@pytest.mark.parametrize("k,V,code", [(2, 1, wl.CODE_3INST), (3, 1, wl.CODE_1MAD), (2, 2, wl.CODE_HYB)])
+def test_memoryless_trellis_is_nearest_codeword_vq(k, V, code):
+    L = k * V
+    lut = wl.hyb_table(4, V, 5) if code == wl.CODE_HYB else None
+    rng = np.random.default_rng(k + V)
+    x = rng.standard_normal((40, V))
+    book = codes.evaluate(code, np.arange(1 << L), V, lut)                  # [2^L, V]
+    nearest = np.argmin(((x[:, None, :] - book[None, :, :]) ** 2).sum(-1), axis=1)
+    for enc in (encode.encode_exact, encode.encode_two_pass):
+        chunks, _ = enc(x, L, k, V, code, lut)
+        assert np.array_equal(chunks, nearest)
+
+
+def test_encoded_block_decodes_through_the_layer_format():
+    L, k, V, code = 16, 2, 1, wl.CODE_3INST
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((256, 1))                    # one 256-column block
+    chunks, err = encode.encode_two_pass(x, L, k, V, code)
+    bits = "".join(format(int(c), f"0{k * V}b") for c in chunks)
+    words = bitstream.bits_to_words(bits)
+    layer = qlinear.Layer(1, 256, [(0, 1, k)], L, V, code, words, np.ones(256, np.int8), np.ones(1, np.int8), 1.0)
+    w = layer.decode_rows(np.arange(1))[0]
+    assert np.array_equal(w, encode.reconstruct(chunks, L, k * V, code, V).reshape(-1))
+    x32 = x[:, 0].astype(np.float32).astype(np.float64)  # the two-pass search takes the source as float32
+    assert float(np.sum((x32 - w) ** 2)) == pytest.approx(err, rel=1e-12)
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_gaussian_distortion_between_the_bound_and_scalar_quantization(k):
+    rng = np.random.default_rng(20 + k)
+    x = rng.standard_normal((4, 256, 1))
+    mse = np.mean([encode.encode_two_pass(b, 12, k, 1, wl.CODE_3INST)[1] / b.size for b in x])
+    assert 2.0 ** (-2 * k) < mse < LLOYD_MAX[k]
+
+
+def test_larger_trellis_lowers_the_distortion():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((2, 256, 1))
+    mse = {L: np.mean([encode.encode_two_pass(b, L, 2, 1, wl.CODE_3INST)[1] / b.size for b in x]) for L in (8, 16)}
+    assert mse[16] < mse[8]
+    assert mse[16] > 2.0 ** -4
+
+
+def test_two_pass_costs_follow_the_float32_rule():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((3, 2))
+    values = rng.standard_normal((5, 2))
+    d = encode._step_costs(x, values, np.float32)
+    for t in range(3):
+        for s in range(5):
+            acc = np.float32(0)
+            for e in range(2):
+                diff = np.float32(np.float32(x[t, e]) - np.float32(values[s, e]))
+                acc = np.float32(acc + np.float32(diff * diff))
+            assert d[t, s] == acc
