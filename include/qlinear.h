@@ -193,6 +193,31 @@ int qlinear_decode(qlinear_t h, void* w_hat, void* stream);
 int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int count, void* out,
                       void* stream);
 
+/* Trellis-coded quantization: for each block of 256 source values, the bits
+ * whose tail-biting walk on the bitshift trellis reproduces the block with the
+ * least squared error (QTIP discussion: encoding searches the fixed-length
+ * walks of the trellis for the least distortion; the discussion's "Table 1"
+ * replies on i.i.d. Gaussian sources).  The search is a two-pass tail-biting
+ * Viterbi: a free-start pass fixes the block's wrap-around L-kV bits from its
+ * best final state, a second pass with both ends tied to them gives the bits;
+ * float32 costs, every operation rounded to nearest, ties to the smallest
+ * predecessor and final state.
+ *   x:      device pointer, float32 [blocks][256] source values (e.g. a row-major
+ *           m x n weight after incoherence processing and scaling, n % 256 == 0:
+ *           its blocks in stream order).
+ *   words:  device pointer, out, uint32 [blocks][256 k / 32] in the stream format
+ *           (for a row-major m x n source, exactly qlinear_create's packed_codes).
+ *   err:    device pointer or null, out, float32 [blocks]: squared error of each
+ *           block's reconstruction.
+ *   L <= 14 (both cost vectors and the code values sit in one CTA's shared
+ *   memory), k*V <= 8; code as in qlinear_create (HYB: the fp16 table is read).
+ * Allocates scratch (256/V * 2^(L-kV) bytes per SM) and returns when the
+ * result is ready (synchronises the stream).
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED (L > 14, or too large for shared memory),
+ * QL_E_OOM, QL_E_CUDA, QL_E_DEVICE (non-finite source values). */
+int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int blocks, uint32_t* words, float* err,
+                   void* stream);
+
 /* Read the handle's device status word (synchronises the device).  Returns
  * QL_OK, or QL_E_DEVICE / QL_E_TIMEOUT if a kernel recorded a failed check or
  * an expired bounded wait since the last call; reading clears the word. */

@@ -1,0 +1,94 @@
+"""The GPU trellis-coded quantizer (qlinear_encode) against the oracle's two-pass
+search, through the C ABI: the same float32 rule, so the same bits.
+
+Source blocks are i.i.d. N(0,1) float32 (the discussion's "Table 1" setting).
+The encoded words also round-trip through a layer: qlinear_create on them and
+qlinear_decode give the oracle's reconstruction of the chosen walks."""
+import time
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only hosts
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import trellis_coded_matmul_b200 as tcm  # noqa: E402
+import workloads as wl  # noqa: E402
+from oracle import bitstream, encode, fp16 as ofp16  # noqa: E402
+
+CASES = [
+    # L, k, V, code, Q
+    (10, 1, 1, wl.CODE_1MAD, 0),
+    (12, 2, 1, wl.CODE_3INST, 0),
+    (12, 2, 2, wl.CODE_HYB, 6),
+    (14, 2, 1, wl.CODE_3INST, 0),
+    (13, 3, 1, wl.CODE_HYB, 9),
+]
+
+
+def _source(blocks, seed):
+    return np.random.default_rng(seed).standard_normal((blocks, 256)).astype(np.float32)
+
+
+def _oracle_words(x, L, k, V, code, lut):
+    out = []
+    for blk in x:
+        chunks, _ = encode.encode_two_pass(blk.reshape(-1, V), L, k, V, code, lut)
+        bits = "".join(format(int(c), f"0{k * V}b") for c in chunks)
+        out.append(bitstream.bits_to_words(bits))
+    return np.stack(out)
+
+
+@pytest.mark.parametrize("L,k,V,code,Q", CASES, ids=lambda v: str(v))
+def test_encode_matches_the_oracle_bit_for_bit(L, k, V, code, Q):
+    lut_np = wl.hyb_table(Q, V, 3) if code == wl.CODE_HYB else None
+    lut = torch.from_numpy(lut_np.copy()).cuda() if lut_np is not None else None
+    x = _source(3, seed=L * 10 + k)
+    words, err = tcm.qlinear_encode(code, L, k, V, torch.from_numpy(x).cuda(), Q=Q, lut=lut, with_error=True)
+    torch.cuda.synchronize()
+    ref = _oracle_words(x, L, k, V, code, lut_np)
+    assert np.array_equal(words.cpu().numpy().view(np.uint32), ref)
+    for b in range(3):
+        chunks = np.array([int(c, 2) for c in (lambda s: [s[i:i + k * V] for i in range(0, len(s), k * V)])(
+            "".join(format(int(w), "032b") for w in ref[b]))])
+        recon = encode.reconstruct(chunks, L, k * V, code, V, lut_np).reshape(-1)
+        assert float(err[b]) == pytest.approx(float(np.sum((x[b].astype(np.float64) - recon) ** 2)), rel=1e-4)
+
+
+def test_encoded_words_round_trip_through_a_layer():
+    L, k, V, code = 12, 2, 1, wl.CODE_1MAD
+    m, n = 32, 512
+    x = _source(m * n // 256, seed=5).reshape(m, n)
+    words = tcm.qlinear_encode(code, L, k, V, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    codes = words.reshape(-1)
+    ones = torch.ones(n, dtype=torch.int8, device="cuda")
+    h = tcm.qlinear_create(m, n, k, L, V, code, codes, ones, torch.ones(m, dtype=torch.int8, device="cuda"), 1.0)
+    w = tcm.qlinear_decode(h)
+    torch.cuda.synchronize()
+    ref = _oracle_words(x.reshape(-1, 256), L, k, V, code, None)
+    recon = []
+    for row in ref:
+        bits = "".join(format(int(wd), "032b") for wd in row)
+        chunks = np.array([int(bits[i:i + k * V], 2) for i in range(0, len(bits), k * V)])
+        recon.append(encode.reconstruct(chunks, L, k * V, code, V).reshape(-1))
+    recon = np.concatenate(recon).reshape(m, n)
+    assert np.array_equal(w.cpu().numpy().view(np.uint16), ofp16.encode(recon))
+    tcm.qlinear_destroy(h)
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_gaussian_distortion_at_L14(k):
+    x = _source(64, seed=40 + k)
+    xt = torch.from_numpy(x).cuda()
+    tcm.qlinear_encode(wl.CODE_3INST, 14, k, 1, xt[:2])  # warm-up
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    _, err = tcm.qlinear_encode(wl.CODE_3INST, 14, k, 1, xt, with_error=True)
+    secs = time.perf_counter() - t0
+    mse = float(err.sum()) / x.size
+    print(f"L=14 k={k}: mse {mse:.4f}, {x.shape[0] / secs:.0f} blocks/s")
+    assert 2.0 ** (-2 * k) < mse < {1: 1.0 - 2.0 / np.pi, 2: 0.1175}[k]

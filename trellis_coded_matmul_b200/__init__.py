@@ -40,7 +40,7 @@ QL_F16 = 1
 ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts", "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
                "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
-               "qlinear_forward_noalloc")
+               "qlinear_forward_noalloc", "qlinear_encode")
 
 
 class ql_code_t(ctypes.Structure):
@@ -62,6 +62,7 @@ _lib.qlinear_create_parts.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, ctypes.PO
 _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
+_lib.qlinear_encode.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp]
 _lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
 _lib.qlinear_eval_code.argtypes = [ql_code_t, _i, _i, _vp, _i, _vp, _vp]
 _lib.qlinear_get_status.argtypes = [_vp]
@@ -227,6 +228,22 @@ def qlinear_forward_noalloc(h: QLinearHandle, x, y, stream=None):
     _check(_lib.qlinear_forward_noalloc(h.ptr, _ptr(x), x.shape[0], _ptr(y), ydt, _stream(stream)),
            "qlinear_forward_noalloc")
     return y
+
+
+def qlinear_encode(kind, L, k, V, x, Q=0, lut=None, with_error=False, stream=None):
+    """Trellis-coded quantization of x (CUDA float32, [..., 256*j] rows whose
+    length is a multiple of 256): the stream-format words (int32 [blocks, 8k])
+    and, with with_error, each block's squared reconstruction error."""
+    import torch
+    _cuda(x, "x", torch.float32)
+    if x.numel() % 256:
+        raise ValueError("x must hold whole blocks of 256 values")
+    blocks = x.numel() // 256
+    words = torch.empty((blocks, 8 * k), dtype=torch.int32, device=x.device)
+    err = torch.empty(blocks, dtype=torch.float32, device=x.device) if with_error else None
+    _check(_lib.qlinear_encode(_code(kind, Q, lut), L, k, V, _ptr(x), blocks, _ptr(words),
+                               _ptr(err) if err is not None else None, _stream(stream)), "qlinear_encode")
+    return (words, err) if with_error else words
 
 
 def qlinear_decode(h: QLinearHandle, w_hat=None, stream=None):

@@ -27,6 +27,7 @@ constexpr int kTcMaxSmem = 232448;    // 227 KB of dynamic shared memory per CTA
 constexpr int kStatusBadSign = 1;
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusBounds = 4;
+constexpr int kStatusBadInput = 8;   // the encoder found no finite walk (non-finite source values)
 
 // One run of rows sharing a bitrate.  Its code words are stored re-laid out
 // for the decode kernels (see layout.cuh) starting at word `word_off` of the
@@ -96,6 +97,14 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 cudaError_t launch_relayout(const uint32_t* src, uint32_t* dst, const Part& part, int n, cudaStream_t st);
 cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* status, cudaStream_t st);
 cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
+
+// Trellis-coded quantization of `blocks` blocks of 256 source values (two-pass
+// tail-biting Viterbi, L <= 14): words [blocks][8k] in the stream format, the
+// squared error of each block's reconstruction into err (may be null).
+// choice: grid * (256/V) * 2^(L-kV) bytes of scratch.
+size_t encode_smem_bytes(int L, int V, int code, int Q);
+cudaError_t launch_encode(int code, int L, int k, int V, int Q, const uint32_t* lut, const float* x, int blocks,
+                          uint32_t* words, float* err, uint8_t* choice, int grid, int* status, cudaStream_t st);
 
 // x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);

@@ -393,6 +393,51 @@ int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int 
     return QL_OK;
 }
 
+int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int blocks, uint32_t* words, float* err,
+                   void* stream) {
+    if (blocks < 0) return QL_E_ARG;
+    if (k < 1 || k > 4 || V < 1 || V > 2) return QL_E_UNSUPPORTED;
+    if (L < k * V || L > 14 || k * V > 8) return QL_E_UNSUPPORTED;
+    int rc = check_code(code, V);
+    if (rc != QL_OK) return rc;
+    if (blocks == 0) return QL_OK;
+    if (!is_device_pointer(x) || !is_device_pointer(words) || (err && !is_device_pointer(err))) return QL_E_ARG;
+    const int Q = code.kind == QL_CODE_HYB ? code.Q : 0;
+    if (encode_smem_bytes(L, V, code.kind, Q) > (size_t)kTcMaxSmem) return QL_E_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QL_E_CUDA;
+    }
+    const int grid = blocks < sms ? blocks : sms;
+    const size_t choice_bytes = (size_t)grid * (256 / V) * ((size_t)1 << (L - k * V));
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* choice = nullptr;
+    uint32_t* lut_words = nullptr;
+    int* status = nullptr;
+    if (cudaMalloc(&choice, choice_bytes) != cudaSuccess || cudaMalloc(&status, sizeof(int)) != cudaSuccess ||
+        (code.kind == QL_CODE_HYB && cudaMalloc(&lut_words, ((size_t)1 << Q) * 4) != cudaSuccess)) {
+        cudaGetLastError();
+        cudaFree(choice);
+        cudaFree(status);
+        cudaFree(lut_words);
+        return QL_E_OOM;
+    }
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+    if (e == cudaSuccess && code.kind == QL_CODE_HYB) e = launch_copy_lut(code.lut, Q, V, lut_words, st);
+    if (e == cudaSuccess)
+        e = launch_encode(code.kind, L, k, V, Q, lut_words, x, blocks, words, err, choice, grid, status, st);
+    int dev_status = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&dev_status, status, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) cudaGetLastError();
+    cudaFree(choice);
+    cudaFree(status);
+    cudaFree(lut_words);
+    if (e != cudaSuccess) return QL_E_CUDA;
+    return dev_status ? QL_E_DEVICE : QL_OK;
+}
+
 int qlinear_get_status(qlinear_t h) {
     if (!h) return QL_E_ARG;
     DeviceGuard g(h->L.device);
