@@ -54,6 +54,9 @@ def parse_args():
     p.add_argument("--batch", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--encode", action="store_true",
+                   help="time the trellis-coded quantizer (qlinear_encode, L = 14, k = 2, 3INST) on an N(0,1) "
+                        "source instead of the forward")
     p.add_argument("--instances", type=int, default=None,
                    help="layer instances to rotate through (default: enough code words for 4x L2); a smaller "
                         "count is for profiler captures only, and the line then says its inputs may sit in L2")
@@ -264,6 +267,36 @@ def _traffic(kernel_key, launch_units):
     return d["dram_bytes"] * launch_units / d["units"]
 
 
+def run_encode(args):
+    """The GPU trellis-coded quantizer on an i.i.d. N(0,1) source: blocks of 256
+    values, L = 14, k = 2, V = 1, 3INST; each step is one qlinear_encode call
+    (scratch allocation and the stream synchronisation included)."""
+    import torch
+    import trellis_coded_matmul_b200 as tcm
+    L, k, V, code = 14, 2, 1, wl.CODE_3INST
+    blocks = 148 * 8
+    x = torch.randn((blocks, 256), generator=torch.Generator().manual_seed(7)).cuda()
+    for _ in range(args.warmup):
+        tcm.qlinear_encode(code, L, k, V, x)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        _, err = tcm.qlinear_encode(code, L, k, V, x, with_error=True)
+    end.record()
+    torch.cuda.synchronize()
+    secs = start.elapsed_time(end) * 1e-3
+    line = {"metric": "trellis-coded quantization (two-pass tail-biting Viterbi) source weights/s",
+            "value": blocks * 256 * args.steps / secs, "unit": "weights/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"encode: {blocks} blocks of 256 N(0,1) values, L={L} k={k} V={V} code=3INST",
+                       "mse": float(err.sum()) / (blocks * 256)},
+            "roofline": None, "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -449,6 +482,8 @@ def main():
         return subprocess.call(cmd)
     if args.impl == "reference":
         return run_reference(args)
+    if args.encode:
+        return run_encode(args)
     return run_ours(args)
 
 
