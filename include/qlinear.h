@@ -62,7 +62,7 @@ extern "C" {
 
 #define QL_OK 0
 #define QL_E_ARG (-1)          /* invalid argument (null pointer, bad size, bad value)   */
-#define QL_E_UNSUPPORTED (-2)  /* valid for the format but not implemented by this build */
+#define QL_E_UNSUPPORTED (-2)  /* valid for the format but not implemented by this library */
 #define QL_E_CUDA (-3)         /* a CUDA runtime call failed                              */
 #define QL_E_OOM (-4)          /* device allocation failed                                */
 #define QL_E_TIMEOUT (-5)      /* a bounded device-side wait gave up                      */
