@@ -18,10 +18,13 @@ Modules:
   bitstream MSB-first bit access and the canonical stream layout
   trellis   the bitshift-trellis state walk (QTIP discussion, "Figure 2 (Q4)")
   codes     the 1MAD, 3INST and HYB codes ("Inference speed analysis", "HYB
-            Uniqueness", "Bit Accounting")
+            Uniqueness", "Bit Accounting") and the table code of the palette
+            quantizers (VQ / NUQ, Q-Palette page)
   hadamard  dense normalised Walsh-Hadamard blocks and the random-sign RHT
             (QuIP# Fig. 2; QTIP discussion, "Incoherence Processing (W2)")
-  qlinear   decode of W_hat and the forward pass (dense, naive)
+  qlinear   decode of W_hat and the forward pass (dense, naive), at whole or
+            half-integer bits per weight
+  encode    trellis-coded quantization (tail-biting Viterbi)
   stats     the statistics the pins use (moments, neighbour dependence)
 
 Parity status: every function here is pinned by a -m "not gpu" test against

@@ -33,18 +33,32 @@ def field(words: np.ndarray, p, width: int) -> np.ndarray:
     return out
 
 
-def row_base_bits(r, n: int, parts) -> np.ndarray:
-    """First bit of row r. parts = [(row0, rows, k)] in stream order."""
+def half_bits(k) -> int:
+    """2k as an integer (k is a whole or half number of bits per weight)."""
+    k2 = int(round(2 * k))
+    assert k2 > 0 and abs(2 * k - k2) < 1e-12, "k must be a multiple of 1/2"
+    return k2
+
+
+def bits(k, weights: int) -> int:
+    """Bits of `weights` weights at k bits each (a whole number)."""
+    b2 = half_bits(k) * weights
+    assert b2 % 2 == 0, "not a whole number of bits"
+    return b2 // 2
+
+
+def row_base_bits(r, n: int, parts):
+    """(first bit, 2k) of each row r. parts = [(row0, rows, k)] in stream order."""
     r = np.asarray(r, dtype=np.int64)
     base = np.zeros(r.shape, dtype=np.int64)
-    kk = np.zeros(r.shape, dtype=np.int64)
+    kk2 = np.zeros(r.shape, dtype=np.int64)
     offset = 0
     for row0, rows, k in parts:
         inside = (r >= row0) & (r < row0 + rows)
-        base = np.where(inside, offset + (r - row0) * n * k, base)
-        kk = np.where(inside, k, kk)
-        offset += rows * n * k
-    return base, kk
+        base = np.where(inside, offset + (r - row0) * bits(k, n), base)
+        kk2 = np.where(inside, half_bits(k), kk2)
+        offset += rows * bits(k, n)
+    return base, kk2
 
 
 def bits_to_words(bitstring: str) -> np.ndarray:

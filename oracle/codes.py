@@ -87,6 +87,15 @@ def hyb(state, lut: np.ndarray) -> np.ndarray:
     return np.concatenate([first[..., None], vals[..., 1:]], axis=-1)
 
 
+def table(state, lut: np.ndarray) -> np.ndarray:
+    """Table-code values, float64 [..., V]: entry `state` of lut (float16
+    [2^L, V]), read exactly."""
+    lut = np.asarray(lut)
+    s = np.asarray(state, dtype=np.int64)
+    assert np.all(s < lut.shape[0]), "state outside the table"
+    return fp16.decode_bits(lut.view(np.uint16).astype(np.int64))[s]
+
+
 def evaluate(code: int, state, V: int, lut=None) -> np.ndarray:
     """Code values of each state: float64 [..., V]."""
     if code == 0:
@@ -98,4 +107,7 @@ def evaluate(code: int, state, V: int, lut=None) -> np.ndarray:
     if code == 2:
         assert lut is not None and lut.shape[1] == V
         return hyb(state, lut)
+    if code == 3:
+        assert lut is not None and lut.shape[1] == V
+        return table(state, lut)
     raise ValueError(code)

@@ -70,20 +70,22 @@ def block_states(words: np.ndarray, rows: np.ndarray, n: int, parts, L: int, V: 
     """States of every step of the given blocks (default: all) of the given rows.
 
     Returns int [len(rows), len(blocks), T/V].  Each row's k is taken from
-    `parts` (half-TCQ layers carry two k values).
+    `parts` (half-TCQ layers carry two k values; k may be a half number of
+    bits, e.g. 2.5 with V = 2 is a 5-bit step).
     """
     T = bitstream.T
     rows = np.asarray(rows, dtype=np.int64)
-    base, kk = bitstream.row_base_bits(rows, n, parts)
+    base, kk2 = bitstream.row_base_bits(rows, n, parts)
     blocks = np.arange(n // T) if blocks is None else np.asarray(blocks, dtype=np.int64)
     nb = len(blocks)
     steps = T // V
     out = np.empty((len(rows), nb, steps), dtype=np.int64)
-    for k in np.unique(kk):
-        k = int(k)
-        sel = np.nonzero(kk == k)[0]
-        kV = k * V
-        S = T * k
+    for k2 in np.unique(kk2):
+        k2 = int(k2)
+        sel = np.nonzero(kk2 == k2)[0]
+        assert (k2 * V) % 2 == 0, "a step must carry a whole number of bits"
+        kV = k2 * V // 2
+        S = T * k2 // 2
         assert L >= kV, "a state must hold at least one step's bits"
         # bit offset of every block start: [rows_sel, nb]
         bstart = base[sel][:, None] + blocks[None, :] * S

@@ -15,10 +15,22 @@ OpenReview discussion times and evaluates; no weights or datasets are used):
   large     m=28672, n=8192,    k=4, L=16, V=1, 1MAD,  alpha=0.01, batch 1/4/16
   halftcq   m=14336, n=4096, rows [0,7168) k=2 and [7168,14336) k=3,
             L=16, V=1, 3INST, alpha=1, batch 64/256
+  qkv_fused m=12288, n=4096, three 4096-row parts at k=2, 3, 4, L=16, V=1, 3INST
+
+Palette workloads (the Q-Palette page's fractional bitwidths and its VQ / NUQ
+quantizers beside TCQ), all m=n=4096, batch 1/4/8:
+
+  tcq2p5    k=2.5 (5 bits per 2-value step), L=16, V=2, HYB Q=9
+  tcq2p75   rows [0,2048) at k=2.5 and [2048,4096) at k=3, L=16, V=2, HYB Q=9
+            (the page's 2.75-bit example: a 2.5-bit and a 3-bit quantizer)
+  vq2p5     k=2.5, L=5, V=2, table code: 32 codewords of 2 values
+  nuq3      k=3, L=3, V=1, table code: 8 levels
 
 Distributions: code words are uniform uint32, signs uniform +-1 (int8), the
 HYB table holds 2^Q x V standard normals rounded to fp16 (numpy's float16
-cast), activations x ~ N(0,1) cast to fp16.
+cast), the table code's codebook 2^L x V standard normals rounded to fp16
+(V = 1: sorted, as the levels of a scalar quantizer), activations x ~ N(0,1)
+cast to fp16.
 """
 from __future__ import annotations
 
@@ -30,7 +42,8 @@ import numpy as np
 CODE_1MAD = 0
 CODE_3INST = 1
 CODE_HYB = 2
-CODE_NAMES = {CODE_1MAD: "1MAD", CODE_3INST: "3INST", CODE_HYB: "HYB"}
+CODE_TABLE = 3
+CODE_NAMES = {CODE_1MAD: "1MAD", CODE_3INST: "3INST", CODE_HYB: "HYB", CODE_TABLE: "TABLE"}
 
 T_BLOCK = 256  # columns per independent trellis block (fixed by the format)
 
@@ -40,7 +53,7 @@ class LayerSpec:
     name: str
     m: int
     n: int
-    k: int                      # bits per weight (uniform layers)
+    k: float                    # bits per weight (uniform layers), a multiple of 1/2
     L: int
     V: int
     code: int
@@ -48,8 +61,8 @@ class LayerSpec:
     seed: int
     Q: int = 0                  # HYB table index bits
     m_top: Optional[int] = None  # half-TCQ: rows [0, m_top) at k_top, rest at k_bot
-    k_top: Optional[int] = None
-    k_bot: Optional[int] = None
+    k_top: Optional[float] = None
+    k_bot: Optional[float] = None
     batches: Sequence[int] = (1,)
     row_split: Optional[Tuple[Tuple[int, int], ...]] = None  # ((rows, k), ...): layers fused along m
 
@@ -70,9 +83,24 @@ class LayerSpec:
             return [(0, self.m_top, self.k_top), (self.m_top, self.m - self.m_top, self.k_bot)]
         return [(0, self.m, self.k)]
 
+    def part_kv(self):
+        """Bits per trellis step (kV) of each row part, in stream order."""
+        out = []
+        for _, _, k in self.row_parts():
+            kv2 = int(round(2 * k)) * self.V
+            assert kv2 % 2 == 0 and abs(2 * k - round(2 * k)) < 1e-12, "k*V must be a whole number of bits"
+            out.append(kv2 // 2)
+        return out
+
+    @property
+    def fractional(self) -> bool:
+        return any(kv % self.V for kv in self.part_kv())
+
     @property
     def n_words(self) -> int:
-        return sum(rows * self.n * k for _, rows, k in self.row_parts()) // 32
+        bits = sum(rows * self.n * kv // self.V for (_, rows, _), kv in zip(self.row_parts(), self.part_kv()))
+        assert bits % 32 == 0
+        return bits // 32
 
     @property
     def stream_bytes(self) -> int:
@@ -95,6 +123,11 @@ WORKLOADS = {
     # read the same input), each with its own bitwidth: 2, 3 and 4 bits.
     "qkv_fused": LayerSpec("qkv_fused", 12288, 4096, 0, 16, 1, CODE_3INST, 0.02, seed=5,
                            row_split=((4096, 2), (4096, 3), (4096, 4)), batches=(1, 16)),
+    "tcq2p5": LayerSpec("tcq2p5", 4096, 4096, 2.5, 16, 2, CODE_HYB, 1.0, seed=6, Q=9, batches=(1, 4, 8)),
+    "tcq2p75": LayerSpec("tcq2p75", 4096, 4096, 0, 16, 2, CODE_HYB, 1.0, seed=7, Q=9,
+                         m_top=2048, k_top=2.5, k_bot=3, batches=(1, 4, 8)),
+    "vq2p5": LayerSpec("vq2p5", 4096, 4096, 2.5, 5, 2, CODE_TABLE, 1.0, seed=8, batches=(1, 4, 8)),
+    "nuq3": LayerSpec("nuq3", 4096, 4096, 3, 3, 1, CODE_TABLE, 1.0, seed=9, batches=(1, 4, 8)),
 }
 
 # The up and down projections of the MLP pair draw from one seeded stream
@@ -108,7 +141,7 @@ class LayerInputs:
     codes: np.ndarray       # uint32 [n_words], canonical stream order
     s_in: np.ndarray        # int8 [n], +-1
     s_out: np.ndarray       # int8 [m], +-1
-    lut: Optional[np.ndarray]  # float16 [2^Q, V] for HYB, else None
+    lut: Optional[np.ndarray]  # float16 [2^Q, V] for HYB, [2^L, V] for the table code, else None
 
 
 def _rng(seed, instance, stream=0):
@@ -120,6 +153,13 @@ def _rng(seed, instance, stream=0):
 def hyb_table(Q: int, V: int, seed: int) -> np.ndarray:
     """2^Q x V standard-normal entries rounded to fp16 (numpy's float16 cast)."""
     return np.random.default_rng(seed).standard_normal((1 << Q, V)).astype(np.float16)
+
+
+def palette_table(L: int, V: int, seed: int) -> np.ndarray:
+    """The table code's codebook: 2^L x V standard normals rounded to fp16;
+    V = 1 sorted ascending (the levels of a non-uniform scalar quantizer)."""
+    t = np.random.default_rng([seed, 31]).standard_normal((1 << L, V)).astype(np.float16)
+    return np.sort(t, axis=0) if V == 1 else t
 
 
 def make_layer(spec: LayerSpec, instance: int = 0) -> LayerInputs:
@@ -137,6 +177,8 @@ def make_layer(spec: LayerSpec, instance: int = 0) -> LayerInputs:
     lut = None
     if spec.code == CODE_HYB:
         lut = hyb_table(spec.Q, spec.V, spec.seed + 1000 * instance)
+    elif spec.code == CODE_TABLE:
+        lut = palette_table(spec.L, spec.V, spec.seed + 1000 * instance)
     return LayerInputs(spec, codes, s_in, s_out, lut)
 
 
@@ -146,10 +188,11 @@ def make_x(spec: LayerSpec, batch: int, instance: int = 0) -> np.ndarray:
     return rng.standard_normal((batch, spec.n)).astype(np.float16)
 
 
-def random_layer(m: int, n: int, k: int, L: int, V: int, code: int, seed: int,
+def random_layer(m: int, n: int, k: float, L: int, V: int, code: int, seed: int,
                  alpha: float = 1.0, Q: int = 9, m_top=None, k_top=None, k_bot=None, row_split=None) -> LayerInputs:
     """A small seeded layer of any supported shape (tests of ragged/edge shapes); row_split
-    ((rows, k), ...) makes a layer of several row parts (layers fused along m)."""
+    ((rows, k), ...) makes a layer of several row parts (layers fused along m); k may be a
+    half number of bits when V = 2."""
     uniform = m_top is None and row_split is None
     spec = LayerSpec(f"rand_{m}x{n}_k{k}", m, n, k if uniform else 0, L, V, code, alpha,
                      seed, Q=Q if code == CODE_HYB else 0, m_top=m_top, k_top=k_top, k_bot=k_bot,
