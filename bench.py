@@ -319,6 +319,9 @@ def run_ours(args):
         s_in = torch.from_numpy(li.s_in.copy()).cuda()
         s_out = torch.from_numpy(li.s_out.copy()).cuda()
         lut = torch.from_numpy(li.lut.copy()).cuda() if li.lut is not None else None
+        if sp_.fractional:  # a half-integer bitwidth: parts given as bits per trellis step
+            return tcm.qlinear_create_kv(sp_.m, sp_.n, [r for _, r, _ in sp_.row_parts()], sp_.part_kv(), sp_.L,
+                                         sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
         if sp_.row_split is not None:
             return tcm.qlinear_create_parts(sp_.m, sp_.n, [r for r, _ in sp_.row_split], [k for _, k in sp_.row_split],
                                             sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)

@@ -12,15 +12,23 @@
  * the QuIP# page (Fig. 2) and in the QTIP OpenReview discussion ("Incoherence
  * Processing (W2)").  W_hat (m x n) is never stored: it is decoded on the fly
  * from a bitshift-trellis bit stream (QTIP discussion, "Figure 2 (Q4)" and
- * "Ablations and fast inference (W1 and W2)") through one of three codes
+ * "Ablations and fast inference (W1 and W2)") through one of four codes
  * (QTIP discussion, "Inference speed analysis (W2)" and the comment on HYB
- * cost, "Bit Accounting (Q2)"):
+ * cost, "Bit Accounting (Q2)"; the table code is the palette reading of the
+ * Q-Palette page):
  *
  *   QL_CODE_1MAD   x = A*s + B mod 2^32; value = fp16(C1 * (sum of the 4 bytes of x - 510))
  *   QL_CODE_3INST  x = A*s + B mod 2^32; m = (x & MASK) ^ XOR;
  *                  value = fp16(float16(m & 0xffff) + float16(m >> 16))
  *   QL_CODE_HYB    x = A*s + B mod 2^32; entry = lut[x >> (32 - Q)] (V fp16 values);
  *                  bit 15 of x negates the entry's first value
+ *   QL_CODE_TABLE  entry = lut[s] (V fp16 values of an explicit codebook of 2^L
+ *                  entries).  With L = kV each step's own kV bits index the
+ *                  codebook: vector quantization (V = 2) or a non-uniform
+ *                  scalar quantizer (V = 1), the VQ / NUQ members of the
+ *                  Q-Palette page's palette (a trellis with L = kV is plain
+ *                  k-bit, V-dimensional VQ, as the QTIP discussion's ablation
+ *                  reply notes); with L > kV, a trellis over the codebook.
  *
  * with the constants (A, B per code; C1 = 443 * 2^-16; MASK = 0x9CFF8FFF,
  * XOR = 0x20003000) fixed by this library's format.  Values are rounded to
@@ -32,6 +40,9 @@
  *     bit of each word first.
  *   - Every row is cut into blocks of T = 256 columns; block j of row r is an
  *     independent trellis of S = 256*k bits starting at bit r*n*k + j*S.
+ *     k is kV / V bits per weight: a whole number, or with V = 2 and an odd
+ *     kV a half number (the Q-Palette page's fractional bitwidths, e.g. 2.5
+ *     bits = 5 bits per 2-value step); S and r*n*k stay whole numbers.
  *   - Step t of a block carries bits [t*kV, (t+1)*kV); its L-bit state is the
  *     window of the block's bits ending at bit (t+1)*kV, read cyclically
  *     (tail-biting), and yields the V values of columns 256*j + t*V + e.
@@ -72,6 +83,7 @@ extern "C" {
 #define QL_CODE_1MAD 0
 #define QL_CODE_3INST 1
 #define QL_CODE_HYB 2
+#define QL_CODE_TABLE 3
 
 #define QL_F32 0
 #define QL_F16 1
@@ -79,11 +91,13 @@ extern "C" {
 typedef struct qlinear_s* qlinear_t;
 
 /* The code that maps a trellis state to V values.
- *   kind: QL_CODE_1MAD or QL_CODE_3INST (V must be 1), or QL_CODE_HYB (V = 1 or 2).
+ *   kind: QL_CODE_1MAD or QL_CODE_3INST (V must be 1), or QL_CODE_HYB or
+ *         QL_CODE_TABLE (V = 1 or 2).
  *   Q:    HYB only, table index bits, 1..9 (the discussion uses Q = 9; "you can
- *         go down to Q~6").
- *   lut:  HYB only, device pointer to 2^Q x V fp16 values, row-major
- *         (entry i = lut[i*V .. i*V+V-1]).  Copied by create. */
+ *         go down to Q~6").  Ignored by the table code, whose codebook has
+ *         2^L entries (L = 1..9).
+ *   lut:  HYB and table code, device pointer to 2^Q (table code: 2^L) x V fp16
+ *         values, row-major (entry i = lut[i*V .. i*V+V-1]).  Copied by create. */
 typedef struct {
     int kind;
     int Q;
@@ -93,14 +107,17 @@ typedef struct {
 /* Facts about a handle (qlinear_info). */
 typedef struct {
     int m, n, L, V, code, Q;
-    int k_top, k_bot, m_top;   /* uniform layers: k_top = k_bot = k, m_top = m */
+    int k_top, k_bot, m_top;   /* bits per weight of the first / last part (rounded
+                                  down: see part_kv), rows of the first part   */
     int B_n, B_m;              /* Hadamard block sizes                           */
-    size_t stream_bytes;       /* packed code words: m*n*k/8 (mixed: per part)   */
+    size_t stream_bytes;       /* packed code words: m*n*k/8 (summed over parts) */
     size_t sign_bytes;         /* bit-packed signs: (n + m) bits, word-padded    */
-    size_t lut_bytes;          /* HYB table: 2^Q * V * 2 bytes                   */
+    size_t lut_bytes;          /* HYB table / codebook: 2^Q (2^L) * V * 2 bytes  */
     size_t scratch_bytes;      /* device scratch currently held by the handle    */
     int last_launches;         /* kernels launched by the most recent forward    */
     int nparts;                /* row parts (1 uniform, 2 half-TCQ, up to 8)     */
+    int part_rows[8];          /* rows of each part (entries >= nparts are 0)    */
+    int part_kv[8];            /* bits per trellis step of each part (k = kv/V)  */
 } ql_info_t;
 
 /* Create a uniform-bitrate layer.
@@ -144,6 +161,19 @@ int qlinear_create_parts(qlinear_t* out, int m, int n, int nparts, const int* pa
                          int L, int V, ql_code_t code,
                          const uint32_t* packed_codes, size_t n_words,
                          const int8_t* s_in, const int8_t* s_out, float alpha);
+
+/* As qlinear_create_parts with each part's bitrate given as bits per trellis
+ * step: part i stores part_kv[i] bits per step of V values, so k = kv / V
+ * bits per weight, in [1, 4]; with V = 2 an odd kv gives a half-integer
+ * bitwidth (Q-Palette page: fractional bitwidths such as 2.5 bits, and
+ * half-TCQ's 2.75 bits from a 2.5-bit and a 3-bit quantizer).
+ *   part_kv:  host array of nparts entries, V <= part_kv[i] <= 4V, L >= part_kv[i].
+ *   n_words:  sum over parts of part_rows[i] * (n / V) * part_kv[i] / 32.
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED, QL_E_OOM, QL_E_CUDA. */
+int qlinear_create_kv(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_kv,
+                      int L, int V, ql_code_t code,
+                      const uint32_t* packed_codes, size_t n_words,
+                      const int8_t* s_in, const int8_t* s_out, float alpha);
 
 /* y = W x for a batch of inputs.
  *   x: device pointer, fp16 [batch][n] row-major.
@@ -210,7 +240,8 @@ int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int 
  *   err:    device pointer or null, out, float32 [blocks]: squared error of each
  *           block's reconstruction.
  *   L <= 14 (both cost vectors and the code values sit in one CTA's shared
- *   memory), k*V <= 8; code as in qlinear_create (HYB: the fp16 table is read).
+ *   memory), k*V <= 8; code as in qlinear_create (HYB and the table code: the
+ *   fp16 table is read; the table code with L = kV is nearest-codeword VQ / NUQ).
  * Allocates scratch (256/V * 2^(L-kV) bytes per SM) and returns when the
  * result is ready (synchronises the stream).
  * Errors: QL_E_ARG, QL_E_UNSUPPORTED (L > 14, or too large for shared memory),

@@ -24,6 +24,9 @@ def to_dev(li: wl.LayerInputs):
 def make_handle(li: wl.LayerInputs):
     sp = li.spec
     codes, s_in, s_out, lut = to_dev(li)
+    if sp.fractional:  # a half-integer bitwidth: parts given as bits per trellis step
+        return tcm.qlinear_create_kv(sp.m, sp.n, [r for _, r, _ in sp.row_parts()], sp.part_kv(), sp.L, sp.V,
+                                     sp.code, codes, s_in, s_out, sp.alpha, Q=sp.Q, lut=lut)
     if sp.row_split is not None:
         return tcm.qlinear_create_parts(sp.m, sp.n, [r for r, _ in sp.row_split], [k for _, k in sp.row_split],
                                         sp.L, sp.V, sp.code, codes, s_in, s_out, sp.alpha, Q=sp.Q, lut=lut)

@@ -118,6 +118,33 @@ def test_create_parts_rejects_bad_arguments_on_the_host(tcm):
     assert create([16, 16], [2, 3]) == tcm.QL_E_ARG                # valid shape, null device pointers
 
 
+def test_create_kv_rejects_bad_arguments_on_the_host(tcm):
+    """Bitrates as bits per trellis step: V <= kv <= 4V (1 to 4 bits per
+    weight, half numbers with V = 2), L >= kv; the stream holds rows * (n / V)
+    * kv bits per part; the table code's codebook has at most 2^9 entries."""
+    lib = tcm.raw_library()
+
+    def create(rows, kvs, V=2, L=16, kind=tcm.QL_CODE_HYB, Q=9, n=256, n_words=None):
+        h = ctypes.c_void_p()
+        nw = sum(r * (n // V) * kv for r, kv in zip(rows, kvs)) // 32 if n_words is None else n_words
+        r = (ctypes.c_int * max(1, len(rows)))(*rows)
+        k = (ctypes.c_int * max(1, len(kvs)))(*kvs)
+        code = tcm.ql_code_t(kind, Q, None)
+        return lib.qlinear_create_kv(ctypes.byref(h), sum(rows), n, len(rows), r, k, L, V, code, None, nw, None,
+                                     None, 1.0)
+
+    assert create([16], [1]) == tcm.QL_E_UNSUPPORTED               # 0.5 bits per weight
+    assert create([16], [9]) == tcm.QL_E_UNSUPPORTED               # 4.5 bits per weight
+    assert create([16], [5], L=4) == tcm.QL_E_UNSUPPORTED          # L < kV
+    assert create([16], [5], V=3) == tcm.QL_E_ARG                  # V is 1 or 2
+    assert create([16], [5], n_words=41) == tcm.QL_E_ARG           # 16 rows * 128 steps * 5 bits = 320 words
+    assert create([16], [5], n_words=320) == tcm.QL_E_ARG          # right length, null device pointers
+    assert create([16], [5], L=10, kind=tcm.QL_CODE_TABLE) == tcm.QL_E_UNSUPPORTED  # 2^10-entry codebook
+    assert create([16], [5], L=5, kind=tcm.QL_CODE_TABLE) == tcm.QL_E_ARG           # valid, null pointers
+    assert create([16], [3], V=1, kind=tcm.QL_CODE_1MAD) == tcm.QL_E_ARG            # 3 bits, V = 1
+    assert create([16, 16], [5, 6], n_words=320 + 384) == tcm.QL_E_ARG              # 2.5 + 3 bits
+
+
 def test_encode_rejects_bad_arguments_on_the_host(tcm):
     lib = tcm.raw_library()
     code = tcm.ql_code_t(1, 0, None)

@@ -33,11 +33,13 @@ QL_NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
 QL_CODE_1MAD = 0
 QL_CODE_3INST = 1
 QL_CODE_HYB = 2
+QL_CODE_TABLE = 3
 QL_F32 = 0
 QL_F16 = 1
 
 # Every function include/qlinear.h declares (checked by the CPU tests).
-ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts", "qlinear_forward", "qlinear_forward_host",
+ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts", "qlinear_create_kv",
+               "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
                "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
                "qlinear_forward_noalloc", "qlinear_encode")
@@ -50,7 +52,8 @@ class ql_code_t(ctypes.Structure):
 class ql_info_t(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int) for f in ("m", "n", "L", "V", "code", "Q", "k_top", "k_bot", "m_top", "B_n", "B_m")] + \
                [(f, ctypes.c_size_t) for f in ("stream_bytes", "sign_bytes", "lut_bytes", "scratch_bytes")] + \
-               [("last_launches", ctypes.c_int), ("nparts", ctypes.c_int)]
+               [("last_launches", ctypes.c_int), ("nparts", ctypes.c_int),
+                ("part_rows", ctypes.c_int * 8), ("part_kv", ctypes.c_int * 8)]
 
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -59,6 +62,8 @@ _lib.qlinear_create_mixed.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _
                                       _vp, _f]
 _lib.qlinear_create_parts.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _i,
                                       ql_code_t, _vp, _sz, _vp, _vp, _f]
+_lib.qlinear_create_kv.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _i,
+                                   ql_code_t, _vp, _sz, _vp, _vp, _f]
 _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
@@ -140,7 +145,8 @@ def _code(kind: int, Q: int = 0, lut=None) -> ql_code_t:
 
 
 def qlinear_create(m, n, k, L, V, kind, codes, s_in, s_out, alpha, Q=0, lut=None) -> QLinearHandle:
-    """codes: CUDA uint32/int32 [m*n*k/32]; s_in, s_out: CUDA int8 +-1; lut: CUDA fp16 [2^Q, V] (HYB)."""
+    """codes: CUDA uint32/int32 [m*n*k/32]; s_in, s_out: CUDA int8 +-1; lut: CUDA fp16
+    [2^Q, V] (HYB) or [2^L, V] (the table code's codebook)."""
     import torch
     _cuda(codes, "codes", (torch.int32, torch.uint32))
     _cuda(s_in, "s_in", torch.int8)
@@ -179,6 +185,26 @@ def qlinear_create_parts(m, n, part_rows, part_k, L, V, kind, codes, s_in, s_out
     _check(_lib.qlinear_create_parts(ctypes.byref(out), m, n, len(part_rows), rows, ks, L, V, _code(kind, Q, lut),
                                      _ptr(codes), codes.numel(), _ptr(s_in), _ptr(s_out), float(alpha)),
            "qlinear_create_parts")
+    return QLinearHandle(out.value, m, n)
+
+
+def qlinear_create_kv(m, n, part_rows, part_kv, L, V, kind, codes, s_in, s_out, alpha, Q=0,
+                      lut=None) -> QLinearHandle:
+    """A layer of row parts whose bitrates are given as bits per trellis step:
+    part i at part_kv[i] / V bits per weight (a half number when V = 2 and
+    part_kv[i] is odd, e.g. 5 bits per step = 2.5 bits per weight)."""
+    import torch
+    _cuda(codes, "codes", (torch.int32, torch.uint32))
+    _cuda(s_in, "s_in", torch.int8)
+    _cuda(s_out, "s_out", torch.int8)
+    if len(part_rows) != len(part_kv):
+        raise ValueError("part_rows and part_kv must have the same length")
+    rows = (ctypes.c_int * max(1, len(part_rows)))(*part_rows)
+    kvs = (ctypes.c_int * max(1, len(part_kv)))(*part_kv)
+    out = _vp()
+    _check(_lib.qlinear_create_kv(ctypes.byref(out), m, n, len(part_rows), rows, kvs, L, V, _code(kind, Q, lut),
+                                  _ptr(codes), codes.numel(), _ptr(s_in), _ptr(s_out), float(alpha)),
+           "qlinear_create_kv")
     return QLinearHandle(out.value, m, n)
 
 
@@ -274,7 +300,10 @@ def qlinear_get_status(h: QLinearHandle) -> int:
 def qlinear_info(h: QLinearHandle) -> dict:
     info = ql_info_t()
     _check(_lib.qlinear_info(h.ptr, ctypes.byref(info)), "qlinear_info")
-    return {f: getattr(info, f) for f, _ in ql_info_t._fields_}
+    d = {f: getattr(info, f) for f, _ in ql_info_t._fields_}
+    for f in ("part_rows", "part_kv"):
+        d[f] = list(d[f])[: info.nparts]
+    return d
 
 
 def qlinear_destroy(h: QLinearHandle) -> None:

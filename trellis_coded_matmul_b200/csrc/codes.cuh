@@ -5,6 +5,9 @@
 //   1MAD : x = A*s + B; value = fp16(C1 * (byte0 + byte1 + byte2 + byte3 - 510))
 //   3INST: x = A*s + B; m = (x & MASK) ^ XOR; value = fp16(half(m.lo) + half(m.hi))
 //   HYB  : x = A*s + B; entry = lut[x >> (32 - Q)]; bit 15 of x negates value 0
+//   TABLE: entry = lut[s]: the palette quantizers of the Q-Palette page (VQ for
+//          V = 2, NUQ for V = 1, when L = kV; a trellis over an explicit
+//          codebook when L > kV)
 // Every value is rounded to fp16 exactly once:
 //   * 1MAD: the byte sum is produced directly as the fp16 bit pattern of
 //     1536 + d (one dp4a whose accumulator is 0x6400 + 512 - 510; the
@@ -13,7 +16,7 @@
 //     rounding.  C1 = 443 * 2^-16 has 9 significant bits, so C1 and 1536*C1
 //     are exact halves.
 //   * 3INST: the two halves are finite normal halves; one fp16 add rounds once.
-//   * HYB: no arithmetic on values, only a sign-bit xor.
+//   * HYB: no arithmetic on values, only a sign-bit xor; TABLE: none at all.
 // The constants are part of the stream format; they were chosen by a seeded
 // search against the statistical properties the discussion states for the
 // codes (approximately N(0,1) at L = 16, successors of a state decorrelated).
@@ -30,6 +33,12 @@ namespace qlk {
 constexpr int kCode1MAD = 0;
 constexpr int kCode3INST = 1;
 constexpr int kCodeHYB = 2;
+constexpr int kCodeTable = 3;
+
+// Codes whose values come from a table in shared memory (2^Q entries; the
+// table code's Q is L).
+__host__ __device__ constexpr bool uses_table(int code) { return code == kCodeHYB || code == kCodeTable; }
+constexpr int kMaxTableBits = 9;  // 2^9 entries x 32 lanes x 4 bytes = 64 KiB replicated
 
 constexpr uint32_t kA1MAD = 0x61616D4Bu, kB1MAD = 0xE29B5692u;
 constexpr uint32_t kA3INST = 0x6C9FB67Bu, kB3INST = 0xA1E8CAB9u;
@@ -112,9 +121,18 @@ __device__ __forceinline__ uint32_t code_pair<kCodeHYB>(uint32_t sa, uint32_t sb
     return __byte_perm(ea, eb, 0x5410);
 }
 
-// HYB with V = 2: one state -> one table word (value 0 low, value 1 high).
-__device__ __forceinline__ uint32_t code_hyb_v2(uint32_t s, const uint32_t* lut_lane, int qshift) {
-    return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
+// Table code with V = 1: entry s of the table, value in the low half.
+template <>
+__device__ __forceinline__ uint32_t code_pair<kCodeTable>(uint32_t sa, uint32_t sb, const uint32_t* lut_lane, int) {
+    return __byte_perm(lut_lane[sa * 32u], lut_lane[sb * 32u], 0x5410);
+}
+
+// V = 2 (HYB or the table code): one state -> one table word (value 0 low, value 1 high).
+template <int CODE>
+__device__ __forceinline__ uint32_t code_v2(uint32_t s, const uint32_t* lut_lane, int qshift) {
+    static_assert(CODE == kCodeHYB || CODE == kCodeTable, "V = 2 needs a table code");
+    if (CODE == kCodeHYB) return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
+    return lut_lane[s * 32u];
 }
 
 // Bits [a, a + 32) of a thread-row's bit string (most significant bit first):

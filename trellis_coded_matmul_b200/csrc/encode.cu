@@ -32,7 +32,7 @@ constexpr int kEncMaxL = 14;
 
 struct EncodeArgs {
     int code, L, kV, V, Q;
-    const uint32_t* lut;    // HYB table, 2^Q words
+    const uint32_t* lut;    // HYB table or codebook, 2^Q words (codebook: Q = L)
     const float* x;         // [blocks][256]
     int blocks;
     uint32_t* words;        // [blocks][256 k / 32], stream format
@@ -44,7 +44,8 @@ struct EncodeArgs {
 // Code values of state s into v[0..V).
 __device__ __forceinline__ void code_values(const EncodeArgs& p, const uint32_t* lut_lane, uint32_t s, float* v) {
     if (p.V == 2) {
-        const uint32_t w = code_hyb_v2(s, lut_lane, 32 - p.Q);
+        const uint32_t w = p.code == kCodeTable ? code_v2<kCodeTable>(s, lut_lane, 0)
+                                                : code_v2<kCodeHYB>(s, lut_lane, 32 - p.Q);
         v[0] = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
         v[1] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
         return;
@@ -52,6 +53,7 @@ __device__ __forceinline__ void code_values(const EncodeArgs& p, const uint32_t*
     uint32_t w;
     if (p.code == kCode1MAD) w = code_pair<kCode1MAD>(s, s, lut_lane, 0);
     else if (p.code == kCode3INST) w = code_pair<kCode3INST>(s, s, lut_lane, 0);
+    else if (p.code == kCodeTable) w = code_pair<kCodeTable>(s, s, lut_lane, 0);
     else w = code_pair<kCodeHYB>(s, s, lut_lane, 32 - p.Q);
     v[0] = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
 }
@@ -93,9 +95,9 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(EncodeArgs p) {
     float* xs = vals + S * V;           // [256]
     float* red_v = xs + 256;            // [32]
     int* red_i = reinterpret_cast<int*>(red_v + 32);
-    uint32_t* lut_smem = reinterpret_cast<uint32_t*>(red_i + 32);  // HYB: 2^Q x 32 replicated words
+    uint32_t* lut_smem = reinterpret_cast<uint32_t*>(red_i + 32);  // table codes: 2^Q x 32 replicated words
     const int lane = threadIdx.x & 31;
-    if (p.code == kCodeHYB)
+    if (uses_table(p.code))
         for (int i = threadIdx.x; i < (32 << p.Q); i += blockDim.x) lut_smem[i] = p.lut[i >> 5];
     __syncthreads();
     const uint32_t* lut_lane = lut_smem + lane;
@@ -195,16 +197,16 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(EncodeArgs p) {
 size_t encode_smem_bytes(int L, int V, int code, int Q) {
     const size_t S = (size_t)1 << L;
     size_t b = (2 * S + S * V + 256 + 32) * 4 + 32 * 4;
-    if (code == kCodeHYB) b += ((size_t)32 << Q) * 4;
+    if (uses_table(code)) b += ((size_t)32 << Q) * 4;
     return b;
 }
 
-cudaError_t launch_encode(int code, int L, int k, int V, int Q, const uint32_t* lut, const float* x, int blocks,
+cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t* lut, const float* x, int blocks,
                           uint32_t* words, float* err, uint8_t* choice, int grid, int* status, cudaStream_t st) {
     EncodeArgs a;
     a.code = code;
     a.L = L;
-    a.kV = k * V;
+    a.kV = kv;
     a.V = V;
     a.Q = Q;
     a.lut = lut;

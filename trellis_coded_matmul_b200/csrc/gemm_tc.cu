@@ -82,7 +82,7 @@ struct TcPart {
     const uint32_t* words;  // kernel layout
     int rt;                 // row tiles of 16 rows
     int row0;               // first layer row
-    int k;                  // bits per weight
+    int k2;                 // 2k: bits per two weights
     int tiles;              // 128-row tiles
 };
 
@@ -103,7 +103,7 @@ struct GemmArgs {
     int* status;
     int stages;             // stage slots
     int code_slots;         // depth of the code-word ring
-    int code_slot_words;    // words of one code-ring slot (8 units at the largest k)
+    int code_slot_words;    // words of one code-ring slot (8 units at the largest k2)
 };
 
 struct TcSmem {  // offsets in bytes from the 1024-aligned dynamic shared memory base
@@ -170,31 +170,34 @@ __device__ __forceinline__ int tc_tiles16(const TcPart& pt, int tile) {  // row 
 }
 
 // One decoder thread's 32 weights of a stage: row r of its row tile, trellis
-// steps [32 hq / V, 32 (hq + 1) / V) of the quarter-block (64 columns).
-// cw[0] holds the 32 bits before the run, cw[1..K] its K words.  Output:
-// 16 half2 words, columns 2i and 2i + 1 of the run in word i.
-template <int CODE, int K, int V, bool L16>
-__device__ __forceinline__ void decode_run32(const uint32_t (&cw)[K + 1], uint32_t lmask, const uint32_t* lut_lane,
+// steps [HQ * NS, (HQ + 1) * NS) (NS = 32 / V) of its quarter-block (64
+// columns).  w[0] holds the 32 bits before the quarter, w[1..K2] its K2 words
+// (K2 = 2k; with a half-integer k a run starts inside a word).  Output: 16
+// half2 words, columns 2i and 2i + 1 of the run in word i.
+template <int CODE, int K2, int V, bool L16, int HQ>
+__device__ __forceinline__ void decode_run32(const uint32_t (&w)[K2 + 1], uint32_t lmask, const uint32_t* lut_lane,
                                              int qshift, uint32_t (&out)[16]) {
-    constexpr int kV = K * V;
+    static_assert((K2 * V) % 2 == 0, "a step carries a whole number of bits");
+    constexpr int kV = K2 * V / 2;
     constexpr int NS = 32 / V;
+    constexpr int T0 = HQ * NS;
     constexpr bool kPair = (16 % kV) == 0;
     constexpr int P = kPair ? 16 / kV : 1;
     uint32_t s[NS];
 #pragma unroll
     for (int t = 0; t < NS; ++t) {
         if (kPair) {
-            if (((t / P) & 1) == 0) state_pair<kV, L16>(cw, t, lmask, s[t], s[t + P]);
+            if (((t / P) & 1) == 0) state_pair<kV, L16>(w, T0 + t, lmask, s[t], s[t + P]);
         } else {
-            s[t] = state_one<kV, L16>(cw, t, lmask);
+            s[t] = state_one<kV, L16>(w, T0 + t, lmask);
         }
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        if (V == 1)
+        if constexpr (V == 1)
             out[i] = code_pair<CODE>(s[2 * i], s[2 * i + 1], lut_lane, qshift);
         else
-            out[i] = code_hyb_v2(s[i], lut_lane, qshift);
+            out[i] = code_v2<CODE>(s[i], lut_lane, qshift);
     }
 }
 
@@ -212,14 +215,14 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 
 // One decoder thread's share of a stage: row r = 32 qtr + lane of the tile,
 // quarter q (64 steps) of the block whose row-tile units sit at shared address
-// `code`.  The quarter's 2K words of the row are loaded with vector loads,
-// plus the last word of the previous quarter (cyclically: tail-biting), then
-// decoded in two runs of 32 steps; run hq becomes 16 packed fp16 pairs stored
-// to tensor-memory columns a_col + 16 hq .. + 15 of the thread's lane.
-template <int CODE, int K, int V, bool L16>
+// `code`.  The quarter's K2 = 2k words of the row are loaded with vector
+// loads, plus the last word of the previous quarter (cyclically: tail-biting),
+// then decoded in two runs of 32 columns; run hq becomes 16 packed fp16 pairs
+// stored to tensor-memory columns a_col + 16 hq .. + 15 of the thread's lane.
+template <int CODE, int K2, int V, bool L16>
 __device__ __forceinline__ void decode_stage_tmem(uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
                                                   uint32_t lmask, const uint32_t* lut_lane, int qshift) {
-    using UL = UnitLayout<K>;
+    using UL = UnitLayout<K2>;
     const int r = 32 * qtr + lane;
     const int h = (r >> 3) & 1, g = r & 7;
     const uint32_t unit = code + (r >> 4) * UL::UW * 4;
@@ -227,23 +230,36 @@ __device__ __forceinline__ void decode_stage_tmem(uint32_t code, uint32_t a_tadd
     auto addr = [&](int slot_lane, int e) -> uint32_t {  // word e of (row half h, lane slot) in the unit layout
         return unit + 4 * (((h * UL::NV + e / UL::VW) * 32 + slot_lane) * UL::VW + (e % UL::VW));
     };
-    uint32_t w[2 * K + 1];
-    w[0] = lds32(addr(4 * g + ((q + 3) & 3), 2 * K - 1));
+    uint32_t w[K2 + 1];
+    w[0] = lds32(addr(4 * g + ((q + 3) & 3), K2 - 1));
 #pragma unroll
-    for (int c = 0; c < 2 * K / UL::VW; ++c) {
+    for (int c = 0; c < K2 / UL::VW; ++c) {
         if (UL::VW == 4)
             lds128(addr(own, 4 * c), w[1 + 4 * c], w[2 + 4 * c], w[3 + 4 * c], w[4 + 4 * c]);
-        else
+        else if (UL::VW == 2)
             lds64(addr(own, 2 * c), w[1 + 2 * c], w[2 + 2 * c]);
+        else
+            w[1 + c] = lds32(addr(own, c));
     }
-#pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-        uint32_t cw[K + 1];
-#pragma unroll
-        for (int e = 0; e <= K; ++e) cw[e] = w[hq * K + e];
-        uint32_t out[16];
-        decode_run32<CODE, K, V, L16>(cw, lmask, lut_lane, qshift, out);
-        tmem_st16(a_taddr + 16 * hq, out);
+    uint32_t out[16];
+    decode_run32<CODE, K2, V, L16, 0>(w, lmask, lut_lane, qshift, out);
+    tmem_st16(a_taddr, out);
+    decode_run32<CODE, K2, V, L16, 1>(w, lmask, lut_lane, qshift, out);
+    tmem_st16(a_taddr + 16, out);
+}
+
+// The part's bitwidth picks the decoder (V = 1 has whole bitwidths only).
+template <int CODE, int V, bool L16>
+__device__ __forceinline__ void decode_stage_k2(int k2, uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
+                                                uint32_t lmask, const uint32_t* lut_lane, int qshift) {
+    switch (k2) {
+        case 2: decode_stage_tmem<CODE, 2, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        case 3: if constexpr (V == 2) decode_stage_tmem<CODE, 3, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        case 4: decode_stage_tmem<CODE, 4, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        case 5: if constexpr (V == 2) decode_stage_tmem<CODE, 5, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        case 6: decode_stage_tmem<CODE, 6, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        case 7: if constexpr (V == 2) decode_stage_tmem<CODE, 7, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
+        default: decode_stage_tmem<CODE, 8, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
     }
 }
 
@@ -289,7 +305,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
         mbar_fence_init();
     }
     uint32_t* lut_smem = reinterpret_cast<uint32_t*>(smem + L.lut);
-    if (CODE == kCodeHYB)
+    if (uses_table(CODE))
         for (int i = threadIdx.x; i < p.lut_entries * 32; i += blockDim.x) lut_smem[i] = p.lut[i >> 5];
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_base_smem), kTcTmemCols);
@@ -334,7 +350,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
             const TcPart& pt = p.part[w.part(p)];
             const int tile = w.tile(p);
             const int ntiles16 = tc_tiles16(pt, tile);
-            const int unit_words = 128 * pt.k;
+            const int unit_words = 64 * pt.k2;
             if (!wait_bar(code_empty(slot), r.phase ^ 1u, abort_flag, p.status)) break;
             if (lane == 0) mbar_arrive_expect_tx(code_full(slot), (uint32_t)(ntiles16 * unit_words * 4));
             __syncwarp();
@@ -409,12 +425,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
                     // Rows of row tiles beyond a ragged last tile decode whatever the
                     // slot holds; their accumulator rows are never stored.
                     const uint32_t a_taddr = tmem + lane_base + kTcTmemA + (uint32_t)st * (kTcK / 2);
-                    switch (pt.k) {
-                        case 1: decode_stage_tmem<CODE, 1, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
-                        case 2: decode_stage_tmem<CODE, 2, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
-                        case 3: decode_stage_tmem<CODE, 3, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
-                        default: decode_stage_tmem<CODE, 4, V, L16>(code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift); break;
-                    }
+                    decode_stage_k2<CODE, V, L16>(pt.k2, code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
@@ -476,10 +487,10 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaS
 // Ring depths: the most stage slots (up to kTcMaxStages), then the deepest
 // code ring (up to kTcMaxCodeSlots blocks) that fit in shared memory.
 size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
-    int kmax = 0;
-    for (int i = 0; i < L.nparts; ++i) kmax = L.parts[i].k > kmax ? L.parts[i].k : kmax;
-    const int code_slot_words = (kTcRows / kRowTile) * 128 * kmax;
-    const int lut_entries = L.code == kCodeHYB ? (1 << L.Q) : 0;
+    int k2max = 0;
+    for (int i = 0; i < L.nparts; ++i) k2max = L.parts[i].k2 > k2max ? L.parts[i].k2 : k2max;
+    const int code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
+    const int lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
     for (int s = kTcMaxStages; s >= 2; --s) {
         for (int c = kTcMaxCodeSlots; c >= 2; --c) {
             const TcSmem lay = tc_smem_layout(s, c, npad, code_slot_words, lut_entries);
@@ -496,7 +507,7 @@ size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
 
 cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st) {
     GemmArgs a;
-    int kmax = 0;
+    int k2max = 0;
     a.nparts = L.nparts;
     a.nb = L.n / kT;
     int tiles = 0;
@@ -505,24 +516,24 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
         a.part[i].words = L.words + pt.word_off;
         a.part[i].rt = pt.rows / kRowTile;
         a.part[i].row0 = pt.row0;
-        a.part[i].k = pt.k;
+        a.part[i].k2 = pt.k2;
         a.part[i].tiles = (pt.rows + kTcRows - 1) / kTcRows;
         tiles += a.part[i].tiles;
-        kmax = pt.k > kmax ? pt.k : kmax;
+        k2max = pt.k2 > k2max ? pt.k2 : k2max;
     }
     for (int i = L.nparts; i < kMaxParts; ++i) a.part[i] = a.part[0];
     a.units = tiles * a.nb;
     a.lmask = (1u << L.L) - 1u;
     a.qshift = 32 - L.Q;
     a.lut = L.lut;
-    a.lut_entries = L.code == kCodeHYB ? (1 << L.Q) : 0;
+    a.lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
     a.xt = (const uint8_t*)xt;
     a.npad = npad;
     a.batch = batch;
     a.z = z;
     a.m = L.m;
     a.status = L.status;
-    a.code_slot_words = (kTcRows / kRowTile) * 128 * kmax;
+    a.code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
     const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots);
     if (smem == 0) return cudaErrorInvalidValue;
     const int grid = a.units < L.num_sms ? a.units : L.num_sms;
@@ -531,6 +542,11 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
                                         : launch_gemm_t<kCode1MAD, 1, false>(a, grid, smem, st);
     if (L.code == kCode3INST) return l16 ? launch_gemm_t<kCode3INST, 1, true>(a, grid, smem, st)
                                          : launch_gemm_t<kCode3INST, 1, false>(a, grid, smem, st);
+    if (L.code == kCodeTable) {
+        if (l16) return cudaErrorInvalidValue;  // codebooks hold at most 2^9 entries
+        return L.V == 1 ? launch_gemm_t<kCodeTable, 1, false>(a, grid, smem, st)
+                        : launch_gemm_t<kCodeTable, 2, false>(a, grid, smem, st);
+    }
     if (L.V == 1) return l16 ? launch_gemm_t<kCodeHYB, 1, true>(a, grid, smem, st)
                              : launch_gemm_t<kCodeHYB, 1, false>(a, grid, smem, st);
     return l16 ? launch_gemm_t<kCodeHYB, 2, true>(a, grid, smem, st) : launch_gemm_t<kCodeHYB, 2, false>(a, grid, smem, st);

@@ -48,10 +48,16 @@ __device__ __forceinline__ uint2 ldg_stream_v2(const uint32_t* p) {
     return r;
 }
 
-// Load lane's two thread-rows of one unit into w[h][0 .. 2K-1].
-template <int K>
-__device__ __forceinline__ void load_unit(uint32_t (&w)[2][2 * K], const uint32_t* unit_base, int lane) {
-    using UL = UnitLayout<K>;
+__device__ __forceinline__ uint32_t ldg_stream_v1(const uint32_t* p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
+// Load lane's two thread-rows of one unit into w[h][0 .. K2-1] (K2 = 2k).
+template <int K2>
+__device__ __forceinline__ void load_unit(uint32_t (&w)[2][K2], const uint32_t* unit_base, int lane) {
+    using UL = UnitLayout<K2>;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -63,16 +69,18 @@ __device__ __forceinline__ void load_unit(uint32_t (&w)[2][2 * K], const uint32_
                 w[h][q * 4 + 1] = v.y;
                 w[h][q * 4 + 2] = v.z;
                 w[h][q * 4 + 3] = v.w;
-            } else {
+            } else if (UL::VW == 2) {
                 const uint2 v = ldg_stream_v2(p);
                 w[h][q * 2 + 0] = v.x;
                 w[h][q * 2 + 1] = v.y;
+            } else {
+                w[h][q] = ldg_stream_v1(p);
             }
         }
     }
 }
 
-// Fill the per-lane replicated HYB table in shared memory.
+// Fill the per-lane replicated table (HYB, or the table code's codebook) in shared memory.
 __device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lut, int entries) {
     for (int i = threadIdx.x; i < entries * 32; i += blockDim.x) smem[i] = lut[i >> 5];
 }
@@ -84,14 +92,16 @@ __device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lu
 //   a[1] = row g+8, columns 4u, 4u+1    a[3] = row g+8, columns 4u+2, 4u+3
 // Paired extraction (16 % kV == 0): steps t and t + 16/kV share one funnel
 // shift, which pairs MMA u with MMA u + MP (MP = 16/kV/steps-per-MMA).
-template <int CODE, int K, int V, bool L16>
+// K2 = 2k bits per two weights (k may be a half number when V = 2).
+template <int CODE, int K2, int V, bool L16>
 struct UnitDecoder {
-    static constexpr int kV = K * V;
+    static_assert((K2 * V) % 2 == 0, "a step carries a whole number of bits");
+    static constexpr int kV = K2 * V / 2;
     static constexpr int SPM = 4 / V;                  // steps per MMA per thread-row
     static constexpr bool kPair = (16 % kV) == 0;
     static constexpr int P = kPair ? 16 / kV : 1;      // step distance of paired windows
     static constexpr int MP = kPair ? P / SPM : 1;     // MMA distance of paired MMAs
-    static constexpr int NW = 2 * K + 1;
+    static constexpr int NW = K2 + 1;
 
     // states of steps [t0, t0 + SPM) into s[0..SPM) and, when paired, of
     // [t0 + P, t0 + P + SPM) into s2[0..SPM)
@@ -108,12 +118,12 @@ struct UnitDecoder {
 
     static __device__ __forceinline__ void codes(const uint32_t (&s)[SPM], uint32_t& lo, uint32_t& hi,
                                                  const uint32_t* lut_lane, int qshift) {
-        if (V == 1) {
+        if constexpr (V == 1) {
             lo = code_pair<CODE>(s[0], s[1], lut_lane, qshift);
             hi = code_pair<CODE>(s[2], s[3], lut_lane, qshift);
         } else {
-            lo = code_hyb_v2(s[0], lut_lane, qshift);
-            hi = code_hyb_v2(s[SPM - 1], lut_lane, qshift);
+            lo = code_v2<CODE>(s[0], lut_lane, qshift);
+            hi = code_v2<CODE>(s[SPM - 1], lut_lane, qshift);
         }
     }
 
@@ -133,10 +143,10 @@ struct UnitDecoder {
 
 // Calls f(u, a) for u = 0..15 with the A operands of MMA u, in the order
 // that lets paired extraction share its funnel shifts.
-template <int CODE, int K, int V, bool L16, typename F>
-__device__ __forceinline__ void for_each_mma(const uint32_t (&cw)[2][2 * K + 1], uint32_t lmask,
+template <int CODE, int K2, int V, bool L16, typename F>
+__device__ __forceinline__ void for_each_mma(const uint32_t (&cw)[2][K2 + 1], uint32_t lmask,
                                              const uint32_t* lut_lane, int qshift, F&& f) {
-    using D = UnitDecoder<CODE, K, V, L16>;
+    using D = UnitDecoder<CODE, K2, V, L16>;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         if (D::kPair && ((u / D::MP) & 1)) continue;  // produced together with MMA u - MP
@@ -236,15 +246,15 @@ struct InputTransform {
 // every warp gets the same whole number of units (to within one), which keeps
 // every SM and every warp equally loaded.  Every thread runs every phase (no
 // early exit), since the in-kernel transforms use CTA barriers.
-template <int CODE, int K, int V, bool L16, bool XSMEM>
+template <int CODE, int K2, int V, bool L16, bool XSMEM>
 __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p, GemvSmem sm) {
     extern __shared__ uint32_t smem[];
-    using UL = UnitLayout<K>;
+    using UL = UnitLayout<K2>;
     uint32_t* lut_smem = smem;
     __half* xs = reinterpret_cast<__half*>(smem + sm.lut_words);
     float* fw = reinterpret_cast<float*>(smem + sm.lut_words + sm.xs_words);
     const int lane = threadIdx.x & 31;
-    if (CODE == kCodeHYB) {
+    if (uses_table(CODE)) {
         fill_lut_smem(lut_smem, p.dec.lut, p.dec.lut_entries);
         __syncthreads();
     }
@@ -259,9 +269,9 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p,
     const int src_lane = (lane & ~3) | ((c + 3) & 3);
     const int batch = p.batch;
 
-    uint32_t nxt[2][2 * K];
-    if (u0 < u1) load_unit<K>(nxt, p.dec.words + u0 * UL::UW, lane);
-    // Programmatic dependent launch: the code words, the HYB table and the
+    uint32_t nxt[2][K2];
+    if (u0 < u1) load_unit<K2>(nxt, p.dec.words + u0 * UL::UW, lane);
+    // Programmatic dependent launch: the code words, the table and the
     // sign bits are written once at create time, so they are fetched before
     // waiting for the previous kernel (the producer of x or x', the consumer
     // of the last z).
@@ -288,22 +298,22 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p,
     };
 
     for (long long unit = u0; unit < u1; ++unit) {
-        uint32_t cw[2][2 * K + 1];
+        uint32_t cw[2][K2 + 1];
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = nxt[h][i];
-        if (unit + 1 < u1) load_unit<K>(nxt, p.dec.words + (unit + 1) * UL::UW, lane);
+            for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
+        if (unit + 1 < u1) load_unit<K2>(nxt, p.dec.words + (unit + 1) * UL::UW, lane);
         if (R != curR) {
             flush(curR);
             acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
             curR = R;
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
+        for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
 
         const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
-        for_each_mma<CODE, K, V, L16>(cw, p.dec.lmask, lut_lane, p.dec.qshift, [&](int u, const uint32_t(&a)[4]) {
+        for_each_mma<CODE, K2, V, L16>(cw, p.dec.lmask, lut_lane, p.dec.qshift, [&](int u, const uint32_t(&a)[4]) {
             uint2 bv = make_uint2(0u, 0u);
             if (g < batch) {
                 if (XSMEM)
@@ -330,7 +340,7 @@ struct GemvPartArgs {
     const uint32_t* words;  // the part's words, kernel layout
     int rt;                 // row tiles
     int row0;               // first layer row
-    int k;                  // bits per weight
+    int k2;                 // 2k: bits per two weights
 };
 struct GemvMultiArgs {
     GemvPartArgs part[kMaxParts];
@@ -345,43 +355,70 @@ struct GemvMultiArgs {
     int m;
 };
 
-// Two thread-rows of one unit at k bits per weight into w[h][0 .. 2k-1].
-__device__ __forceinline__ void load_unit_k(uint32_t (&w)[2][8], const uint32_t* unit_base, int k, int lane) {
-    uint32_t t1[2][2], t2[2][4], t3[2][6], t4[2][8];
-    switch (k) {
-        case 1: load_unit<1>(t1, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 2; ++i) w[h][i] = t1[h][i]; break;
-        case 2: load_unit<2>(t2, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 4; ++i) w[h][i] = t2[h][i]; break;
-        case 3: load_unit<3>(t3, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 6; ++i) w[h][i] = t3[h][i]; break;
-        default: load_unit<4>(t4, unit_base, lane); for (int h = 0; h < 2; ++h) for (int i = 0; i < 8; ++i) w[h][i] = t4[h][i]; break;
-    }
-}
-
-// One unit at K bits: take its words from nxt, start the next unit's load
-// into nxt, then decode and multiply.
-template <int CODE, int K, int V, bool L16>
-__device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k, int lane,
-                                          int src_lane, const GemvMultiArgs& p, const uint32_t* lut_lane,
-                                          size_t xoff, bool use_x, float (&acc)[4]) {
-    uint32_t cw[2][2 * K + 1];
+// Two thread-rows of one unit at K2 = 2k into w[h][0 .. K2-1].
+template <int K2>
+__device__ __forceinline__ void load_unit_into(uint32_t (&w)[2][8], const uint32_t* unit_base, int lane) {
+    uint32_t t[2][K2];
+    load_unit<K2>(t, unit_base, lane);
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = nxt[h][i];
-    if (next_base) load_unit_k(nxt, next_base, next_k, lane);
+        for (int i = 0; i < K2; ++i) w[h][i] = t[h][i];
+}
+__device__ __forceinline__ void load_unit_k2(uint32_t (&w)[2][8], const uint32_t* unit_base, int k2, int lane) {
+    switch (k2) {
+        case 2: load_unit_into<2>(w, unit_base, lane); break;
+        case 3: load_unit_into<3>(w, unit_base, lane); break;
+        case 4: load_unit_into<4>(w, unit_base, lane); break;
+        case 5: load_unit_into<5>(w, unit_base, lane); break;
+        case 6: load_unit_into<6>(w, unit_base, lane); break;
+        case 7: load_unit_into<7>(w, unit_base, lane); break;
+        default: load_unit_into<8>(w, unit_base, lane); break;
+    }
+}
+
+// One unit at K2 = 2k: take its words from nxt, start the next unit's load
+// into nxt, then decode and multiply.
+template <int CODE, int K2, int V, bool L16>
+__device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2, int lane,
+                                          int src_lane, const GemvMultiArgs& p, const uint32_t* lut_lane,
+                                          size_t xoff, bool use_x, float (&acc)[4]) {
+    uint32_t cw[2][K2 + 1];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][2 * K], src_lane);
-    for_each_mma<CODE, K, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
+    if (next_base) load_unit_k2(nxt, next_base, next_k2, lane);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
+    for_each_mma<CODE, K2, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
         uint2 bv = make_uint2(0u, 0u);
         if (use_x) bv = __ldg(p.xf + xoff + (size_t)u * p.batch * 4);
         mma_16816(acc, a, bv.x, bv.y);
     });
 }
 
+// The unit's bitwidth picks the decoder (V = 1 has whole bitwidths only).
+template <int CODE, int V, bool L16>
+__device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2,
+                                             int lane, int src_lane, const GemvMultiArgs& p,
+                                             const uint32_t* lut_lane, size_t xoff, bool use_x, float (&acc)[4]) {
+    switch (k2) {
+        case 2: gemv_unit<CODE, 2, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        case 3: if constexpr (V == 2) gemv_unit<CODE, 3, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        case 4: gemv_unit<CODE, 4, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        case 5: if constexpr (V == 2) gemv_unit<CODE, 5, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        case 6: gemv_unit<CODE, 6, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        case 7: if constexpr (V == 2) gemv_unit<CODE, 7, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+        default: gemv_unit<CODE, 8, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
+    }
+}
+
 template <int CODE, int V, bool L16>
 __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvMultiArgs p) {
     extern __shared__ uint32_t smem[];
     const int lane = threadIdx.x & 31;
-    if (CODE == kCodeHYB) {
+    if (uses_table(CODE)) {
         fill_lut_smem(smem, p.lut, p.lut_entries);
         __syncthreads();
     }
@@ -402,10 +439,10 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvM
     while (pt + 1 < p.nparts && rest >= (long long)p.part[pt].rt * nb) rest -= (long long)p.part[pt++].rt * nb;
     int t = (int)(rest / nb), j = (int)(rest % nb);
     auto unit_base = [&](int part, int tile, int blk) {
-        return p.part[part].words + ((size_t)tile * nb + blk) * 128 * p.part[part].k;
+        return p.part[part].words + ((size_t)tile * nb + blk) * 64 * p.part[part].k2;
     };
     uint32_t nxt[2][8];
-    if (u0 < u1) load_unit_k(nxt, unit_base(pt, t, j), p.part[pt].k, lane);
+    if (u0 < u1) load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
     grid_dependency_wait();  // x' from the input transform; z consumed by the last output transform
     grid_launch_dependents();
 
@@ -442,12 +479,8 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvM
         }
         const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
         const bool use_x = g < batch;
-        switch (p.part[pt].k) {
-            case 1: gemv_unit<CODE, 1, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-            case 2: gemv_unit<CODE, 2, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-            case 3: gemv_unit<CODE, 3, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-            default: gemv_unit<CODE, 4, V, L16>(nxt, next_base, p.part[npt].k, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        }
+        gemv_unit_k2<CODE, V, L16>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p, lut_lane, xoff,
+                                   use_x, acc);
         pt = npt;
         t = nt;
         j = nj;
@@ -477,13 +510,13 @@ cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, fl
         a.part[i].words = L.words + pt.word_off;
         a.part[i].rt = pt.rows / kRowTile;
         a.part[i].row0 = pt.row0;
-        a.part[i].k = pt.k;
+        a.part[i].k2 = pt.k2;
         if (i < L.nparts) units += (long long)a.part[i].rt * a.nb;
     }
     a.lmask = (1u << L.L) - 1u;
     a.qshift = 32 - L.Q;
     a.lut = L.lut;
-    a.lut_entries = L.code == kCodeHYB ? (1 << L.Q) : 0;
+    a.lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
     a.xf = (const uint2*)xp_frag;
     a.batch = batch;
     a.z = z;
@@ -503,16 +536,18 @@ cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, fl
                                                    : launch_gemv_multi_t<kCodeHYB, 1, false>(a, grid, threads, smem, st);
     if (L.code == kCodeHYB && L.V == 2) return l16 ? launch_gemv_multi_t<kCodeHYB, 2, true>(a, grid, threads, smem, st)
                                                    : launch_gemv_multi_t<kCodeHYB, 2, false>(a, grid, threads, smem, st);
+    if (L.code == kCodeTable && !l16) return L.V == 1 ? launch_gemv_multi_t<kCodeTable, 1, false>(a, grid, threads, smem, st)
+                                                      : launch_gemv_multi_t<kCodeTable, 2, false>(a, grid, threads, smem, st);
     return cudaErrorInvalidValue;
 }
 
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
-template <int CODE, int K, int V, bool L16>
+template <int CODE, int K2, int V, bool L16>
 __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
     extern __shared__ uint32_t lut_smem[];
-    using UL = UnitLayout<K>;
+    using UL = UnitLayout<K2>;
     const int lane = threadIdx.x & 31;
-    if (CODE == kCodeHYB) {
+    if (uses_table(CODE)) {
         fill_lut_smem(lut_smem, p.lut, p.lut_entries);
         __syncthreads();
     }
@@ -523,17 +558,17 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __res
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); unit < U;
          unit += nwarps) {
-        uint32_t w[2][2 * K];
-        load_unit<K>(w, p.words + unit * UL::UW, lane);
-        uint32_t cw[2][2 * K + 1];
+        uint32_t w[2][K2];
+        load_unit<K2>(w, p.words + unit * UL::UW, lane);
+        uint32_t cw[2][K2 + 1];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int i = 0; i < 2 * K; ++i) cw[h][i + 1] = w[h][i];
-            cw[h][0] = __shfl_sync(0xffffffffu, w[h][2 * K - 1], src_lane);
+            for (int i = 0; i < K2; ++i) cw[h][i + 1] = w[h][i];
+            cw[h][0] = __shfl_sync(0xffffffffu, w[h][K2 - 1], src_lane);
         }
         const int R = (int)(unit / p.nb), j = (int)(unit % p.nb);
-        for_each_mma<CODE, K, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
+        for_each_mma<CODE, K2, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const size_t row = (size_t)row0 + R * kRowTile + 8 * h + g;
@@ -550,14 +585,14 @@ __global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count,
                                  const uint32_t* __restrict__ lut, int lut_entries, __half* __restrict__ out) {
     extern __shared__ uint32_t lut_smem[];
     const int lane = threadIdx.x & 31;
-    if (CODE == kCodeHYB) {
+    if (uses_table(CODE)) {
         fill_lut_smem(lut_smem, lut, lut_entries);
         __syncthreads();
     }
     const uint32_t* lut_lane = lut_smem + lane;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (V == 2) {
-        if (t < count) ((uint32_t*)out)[t] = code_hyb_v2(states[t] & lmask, lut_lane, qshift);
+    if constexpr (V == 2) {
+        if (t < count) ((uint32_t*)out)[t] = code_v2<CODE>(states[t] & lmask, lut_lane, qshift);
     } else {
         const int i0 = 2 * t;
         if (i0 >= count) return;
@@ -572,43 +607,43 @@ __global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count,
 
 // ---- dispatch ----
 template <template <int, int, int, bool> class F, bool L16, typename... Args>
-static cudaError_t dispatch_l(int code, int k, int V, Args&&... args);
+static cudaError_t dispatch_l(int code, int k2, int V, Args&&... args);
 
 template <template <int, int, int, bool> class F, typename... Args>
-static cudaError_t dispatch(int code, int k, int V, bool l16, Args&&... args) {
-    return l16 ? dispatch_l<F, true>(code, k, V, args...) : dispatch_l<F, false>(code, k, V, args...);
+static cudaError_t dispatch(int code, int k2, int V, bool l16, Args&&... args) {
+    return l16 ? dispatch_l<F, true>(code, k2, V, args...) : dispatch_l<F, false>(code, k2, V, args...);
+}
+
+// (code, k2 = 2k, V) -> the kernel instance.  V = 1 takes whole bitwidths
+// (k2 even), V = 2 also half ones; the table code has no L = 16 instance
+// (its codebook holds at most 2^9 entries).
+template <template <int, int, int, bool> class F, int CODE, int V, bool L16, typename... Args>
+static cudaError_t dispatch_k2(int k2, Args&&... args) {
+    switch (k2) {
+        case 2: return F<CODE, 2, V, L16>::run(args...);
+        case 4: return F<CODE, 4, V, L16>::run(args...);
+        case 6: return F<CODE, 6, V, L16>::run(args...);
+        case 8: return F<CODE, 8, V, L16>::run(args...);
+    }
+    if constexpr (V == 2) {
+        switch (k2) {
+            case 3: return F<CODE, 3, V, L16>::run(args...);
+            case 5: return F<CODE, 5, V, L16>::run(args...);
+            case 7: return F<CODE, 7, V, L16>::run(args...);
+        }
+    }
+    return cudaErrorInvalidValue;
 }
 
 template <template <int, int, int, bool> class F, bool L16, typename... Args>
-static cudaError_t dispatch_l(int code, int k, int V, Args&&... args) {
-    if (code == kCode1MAD && V == 1) {
-        switch (k) {
-            case 1: return F<kCode1MAD, 1, 1, L16>::run(args...);
-            case 2: return F<kCode1MAD, 2, 1, L16>::run(args...);
-            case 3: return F<kCode1MAD, 3, 1, L16>::run(args...);
-            case 4: return F<kCode1MAD, 4, 1, L16>::run(args...);
-        }
-    } else if (code == kCode3INST && V == 1) {
-        switch (k) {
-            case 1: return F<kCode3INST, 1, 1, L16>::run(args...);
-            case 2: return F<kCode3INST, 2, 1, L16>::run(args...);
-            case 3: return F<kCode3INST, 3, 1, L16>::run(args...);
-            case 4: return F<kCode3INST, 4, 1, L16>::run(args...);
-        }
-    } else if (code == kCodeHYB && V == 1) {
-        switch (k) {
-            case 1: return F<kCodeHYB, 1, 1, L16>::run(args...);
-            case 2: return F<kCodeHYB, 2, 1, L16>::run(args...);
-            case 3: return F<kCodeHYB, 3, 1, L16>::run(args...);
-            case 4: return F<kCodeHYB, 4, 1, L16>::run(args...);
-        }
-    } else if (code == kCodeHYB && V == 2) {
-        switch (k) {
-            case 1: return F<kCodeHYB, 1, 2, L16>::run(args...);
-            case 2: return F<kCodeHYB, 2, 2, L16>::run(args...);
-            case 3: return F<kCodeHYB, 3, 2, L16>::run(args...);
-            case 4: return F<kCodeHYB, 4, 2, L16>::run(args...);
-        }
+static cudaError_t dispatch_l(int code, int k2, int V, Args&&... args) {
+    if (code == kCode1MAD && V == 1) return dispatch_k2<F, kCode1MAD, 1, L16>(k2, args...);
+    if (code == kCode3INST && V == 1) return dispatch_k2<F, kCode3INST, 1, L16>(k2, args...);
+    if (code == kCodeHYB && V == 1) return dispatch_k2<F, kCodeHYB, 1, L16>(k2, args...);
+    if (code == kCodeHYB && V == 2) return dispatch_k2<F, kCodeHYB, 2, L16>(k2, args...);
+    if constexpr (!L16) {
+        if (code == kCodeTable && V == 1) return dispatch_k2<F, kCodeTable, 1, false>(k2, args...);
+        if (code == kCodeTable && V == 2) return dispatch_k2<F, kCodeTable, 2, false>(k2, args...);
     }
     return cudaErrorInvalidValue;
 }
@@ -621,27 +656,31 @@ static DecodeArgs make_decode_args(const Layer& L, const Part& part) {
     d.lmask = (1u << L.L) - 1u;
     d.qshift = 32 - L.Q;
     d.lut = L.lut;
-    d.lut_entries = (L.code == kCodeHYB) ? (1 << L.Q) : 0;
+    d.lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
     return d;
 }
 
-template <int CODE, int K, int V, bool L16>
+// The in-kernel input transform has instances for L = 16 and for the table code.
+template <int CODE, int K2, int V, bool L16>
 struct GemvLaunch {
     static cudaError_t run(const GemvArgs& a, const GemvSmem& sm, bool xsmem, int grid, int threads,
                            cudaStream_t st) {
         const size_t smem = (size_t)(sm.lut_words + sm.xs_words + sm.fw_words) * 4;
         if (xsmem) {
-            if (!L16) return cudaErrorInvalidValue;
-            auto kern = gemv_kernel<CODE, K, V, true, true>;
-            static bool attr_set = false;
-            if (!attr_set) {
-                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
-                if (e != cudaSuccess) return e;
-                attr_set = true;
+            if constexpr (L16 || CODE == kCodeTable) {
+                auto kern = gemv_kernel<CODE, K2, V, L16, true>;
+                static bool attr_set = false;
+                if (!attr_set) {
+                    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
+                    if (e != cudaSuccess) return e;
+                    attr_set = true;
+                }
+                return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
+            } else {
+                return cudaErrorInvalidValue;
             }
-            return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
         }
-        auto kern = gemv_kernel<CODE, K, V, L16, false>;
+        auto kern = gemv_kernel<CODE, K2, V, L16, false>;
         static bool attr_set = false;
         if (!attr_set) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
@@ -664,11 +703,11 @@ GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
     const long long per_cta = (units + pl.grid - 1) / pl.grid;
     const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
     int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
-    const int lut_words = L.code == kCodeHYB ? (32 << L.Q) : 0;
+    const int lut_words = uses_table(L.code) ? (32 << L.Q) : 0;
     const int budget = kGemvMaxSmem / 4 - lut_words;
     const int t_in = L.B_n / kXinE;
     const int xs_words = batch * L.n / 2;
-    pl.xsmem = L.L == 16 && L.nparts == 1 && (long long)batch * L.n <= kFuseInElems &&
+    pl.xsmem = (L.L == 16 || L.code == kCodeTable) && L.nparts == 1 && (long long)batch * L.n <= kFuseInElems &&
                t_in <= kGemvMaxWarps * 32;
     int fw = 0;
     pl.groups_in = 0;
@@ -714,14 +753,14 @@ cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, co
     a.n = L.n;
     a.B_n = L.B_n;
     a.groups_in = pl.groups_in;
-    return dispatch<GemvLaunch>(L.code, part.k, L.V, L.L == 16, a, pl.sm, pl.xsmem, pl.grid, pl.threads, st);
+    return dispatch<GemvLaunch>(L.code, part.k2, L.V, L.L == 16, a, pl.sm, pl.xsmem, pl.grid, pl.threads, st);
 }
 
-template <int CODE, int K, int V, bool L16>
+template <int CODE, int K2, int V, bool L16>
 struct DecodeLaunch {
     static cudaError_t run(const DecodeArgs& d, __half* w, int n, int row0, int grid, cudaStream_t st) {
         const size_t smem = (size_t)d.lut_entries * 32 * 4;
-        auto kern = decode_kernel<CODE, K, V, L16>;
+        auto kern = decode_kernel<CODE, K2, V, L16>;
         static bool attr_set = false;
         if (smem > 48 * 1024 && !attr_set) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
@@ -738,14 +777,15 @@ cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStr
     const long long units = (long long)d.rt * d.nb;
     long long grid = (units + 7) / 8;
     if (grid > (long long)L.num_sms * 8) grid = (long long)L.num_sms * 8;
-    return dispatch<DecodeLaunch>(L.code, part.k, L.V, L.L == 16, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
+    return dispatch<DecodeLaunch>(L.code, part.k2, L.V, L.L == 16, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
 }
 
-template <int CODE, int K, int V, bool L16>
+template <int CODE, int K2, int V, bool L16>
 struct EvalLaunch {
     static cudaError_t run(const uint32_t* states, int count, uint32_t lmask, int qshift, const uint32_t* lut,
                            int entries, __half* out, cudaStream_t st) {
-        if (K != 1 || !L16) return cudaErrorInvalidValue;  // one instance suffices: the code ignores k and L
+        // one instance per (code, V) suffices: the code ignores k and L
+        if (K2 != 2 || L16 == (CODE == kCodeTable)) return cudaErrorInvalidValue;
         const size_t smem = (size_t)entries * 32 * 4;
         auto kern = eval_code_kernel<CODE, V>;
         static bool attr_set = false;
@@ -763,8 +803,9 @@ struct EvalLaunch {
 cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words, const uint32_t* states,
                              int count, void* out, cudaStream_t st) {
     const uint32_t lmask = (1u << L) - 1u;
-    const int entries = code == kCodeHYB ? (1 << Q) : 0;
-    return dispatch<EvalLaunch>(code, 1, V, true, states, count, lmask, 32 - Q, lut_words, entries, (__half*)out, st);
+    const int entries = uses_table(code) ? (1 << Q) : 0;
+    return dispatch<EvalLaunch>(code, 2, V, code != kCodeTable, states, count, lmask, 32 - Q, lut_words, entries,
+                                (__half*)out, st);
 }
 
 }  // namespace qlk

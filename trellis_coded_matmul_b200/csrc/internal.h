@@ -31,18 +31,21 @@ constexpr int kStatusBadInput = 8;   // the encoder found no finite walk (non-fi
 
 // One run of rows sharing a bitrate.  Its code words are stored re-laid out
 // for the decode kernels (see layout.cuh) starting at word `word_off` of the
-// handle's word buffer.
+// handle's word buffer.  The bitrate k = kv / V bits per weight may be a half
+// number; the kernels take it as k2 = 2k (a whole number of bits per two
+// weights, which is also the code words of one thread-row of a unit).
 struct Part {
     int row0;
     int rows;
-    int k;
+    int kv;       // bits per trellis step
+    int k2;       // 2k = 2 kv / V
     size_t word_off;
     size_t n_words;
 };
 
 struct Layer {
     int device;
-    int m, n, L, V, code, Q;
+    int m, n, L, V, code, Q;  // Q: table index bits of HYB and of the table code (= L), else 0
     float alpha;
     int B_n, B_m;
     int nparts;
@@ -50,7 +53,8 @@ struct Layer {
     uint32_t* words;      // all parts, kernel layout
     uint32_t* sin_bits;   // bit i set <=> s_in[i] == -1
     uint32_t* sout_bits;
-    uint32_t* lut;        // HYB: 2^Q words (V = 2: value 0 low half, value 1 high; V = 1: low half)
+    uint32_t* lut;        // HYB / table code: 2^Q words (table code: Q = L) (V = 2: value 0 low half,
+                          // value 1 high; V = 1: low half)
     int* status;          // device status word
     // scratch, grown on demand
     void* xp;             // transformed input x' (fp16)
@@ -99,11 +103,11 @@ cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* s
 cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
 
 // Trellis-coded quantization of `blocks` blocks of 256 source values (two-pass
-// tail-biting Viterbi, L <= 14): words [blocks][8k] in the stream format, the
-// squared error of each block's reconstruction into err (may be null).
-// choice: grid * (256/V) * 2^(L-kV) bytes of scratch.
+// tail-biting Viterbi, L <= 14, kv bits per step): words [blocks][8 kv / V] in
+// the stream format, the squared error of each block's reconstruction into
+// err (may be null).  choice: grid * (256/V) * 2^(L-kv) bytes of scratch.
 size_t encode_smem_bytes(int L, int V, int code, int Q);
-cudaError_t launch_encode(int code, int L, int k, int V, int Q, const uint32_t* lut, const float* x, int blocks,
+cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t* lut, const float* x, int blocks,
                           uint32_t* words, float* err, uint8_t* choice, int grid, int* status, cudaStream_t st);
 
 // x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.

@@ -7,6 +7,7 @@
 #include <mutex>
 #include <new>
 
+#include "codes.cuh"
 #include "internal.h"
 
 using namespace qlk;
@@ -77,17 +78,25 @@ void free_layer(Layer& L) {
     std::memset(&L, 0, sizeof(L));
 }
 
-int check_code(const ql_code_t& code, int V) {
+int check_code(const ql_code_t& code, int V, int L) {
     if (code.kind == QL_CODE_1MAD || code.kind == QL_CODE_3INST) return V == 1 ? QL_OK : QL_E_UNSUPPORTED;
-    if (code.kind != QL_CODE_HYB) return QL_E_ARG;
+    if (code.kind != QL_CODE_HYB && code.kind != QL_CODE_TABLE) return QL_E_ARG;
     if (V != 1 && V != 2) return QL_E_ARG;
-    if (code.Q < 1 || code.Q > 9) return QL_E_UNSUPPORTED;
+    if (code.kind == QL_CODE_HYB && (code.Q < 1 || code.Q > kMaxTableBits)) return QL_E_UNSUPPORTED;
+    if (code.kind == QL_CODE_TABLE && (L < 1 || L > kMaxTableBits)) return QL_E_UNSUPPORTED;
     if (!is_device_pointer(code.lut)) return QL_E_ARG;
     return QL_OK;
 }
 
-// Shared by the create calls. parts: [(rows, k)], host arrays.
-int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k, int L,
+// Index bits of the code's table (the table code's codebook has 2^L entries).
+int table_bits(const ql_code_t& code, int L) {
+    return code.kind == QL_CODE_HYB ? code.Q : code.kind == QL_CODE_TABLE ? L : 0;
+}
+
+// Shared by the create calls. parts: [(rows, kv)], host arrays; kv = bits per
+// trellis step, k = kv / V bits per weight in [1, 4] (a half number when
+// V = 2 and kv is odd).
+int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_kv, int L,
                   int V, ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
                   const int8_t* s_out, float alpha) {
     if (!out) return QL_E_ARG;
@@ -96,19 +105,19 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (V != 1 && V != 2) return QL_E_ARG;
     if (n % kT != 0 || m % kRowTile != 0) return QL_E_UNSUPPORTED;
     if (pow2_block(n) > kMaxHadamard || pow2_block(m) > kMaxHadamard) return QL_E_UNSUPPORTED;
-    if (nparts < 1 || nparts > kMaxParts || !part_rows || !part_k) return QL_E_ARG;
+    if (nparts < 1 || nparts > kMaxParts || !part_rows || !part_kv) return QL_E_ARG;
     size_t expect_words = 0;
     long long rows_sum = 0;
     for (int i = 0; i < nparts; ++i) {
-        const int k = part_k[i];
-        if (k < 1 || k > 4) return QL_E_UNSUPPORTED;
-        if (L < k * V || L > 16) return QL_E_UNSUPPORTED;
+        const int kv = part_kv[i];
+        if (kv < V || kv > 4 * V) return QL_E_UNSUPPORTED;
+        if (L < kv || L > 16) return QL_E_UNSUPPORTED;
         if (part_rows[i] <= 0 || part_rows[i] % kRowTile != 0) return QL_E_ARG;
-        expect_words += (size_t)part_rows[i] * n * k / 32;
+        expect_words += (size_t)part_rows[i] * n / V * kv / 32;  // n / V: whole steps per row
         rows_sum += part_rows[i];
     }
     if (rows_sum != m || n_words != expect_words) return QL_E_ARG;
-    int rc = check_code(code, V);
+    int rc = check_code(code, V, L);
     if (rc != QL_OK) return rc;
     if (!is_device_pointer(packed_codes) || !is_device_pointer(s_in) || !is_device_pointer(s_out))
         return QL_E_ARG;
@@ -124,7 +133,7 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     Ly.L = L;
     Ly.V = V;
     Ly.code = code.kind;
-    Ly.Q = code.kind == QL_CODE_HYB ? code.Q : 0;
+    Ly.Q = table_bits(code, L);
     Ly.alpha = alpha;
     Ly.B_n = pow2_block(n);
     Ly.B_m = pow2_block(m);
@@ -134,9 +143,10 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     for (int i = 0; i < nparts; ++i) {
         Ly.parts[i].row0 = row0;
         Ly.parts[i].rows = part_rows[i];
-        Ly.parts[i].k = part_k[i];
+        Ly.parts[i].kv = part_kv[i];
+        Ly.parts[i].k2 = 2 * part_kv[i] / V;
         Ly.parts[i].word_off = off;
-        Ly.parts[i].n_words = (size_t)part_rows[i] * n * part_k[i] / 32;
+        Ly.parts[i].n_words = (size_t)part_rows[i] * n / V * part_kv[i] / 32;
         off += Ly.parts[i].n_words;
         row0 += part_rows[i];
     }
@@ -145,7 +155,7 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (rc == QL_OK) rc = dev_alloc(&Ly.sin_bits, (size_t)((n + 31) / 32) * 4);
     if (rc == QL_OK) rc = dev_alloc(&Ly.sout_bits, (size_t)((m + 31) / 32) * 4);
     if (rc == QL_OK) rc = dev_alloc(&Ly.status, sizeof(int));
-    if (rc == QL_OK && Ly.code == QL_CODE_HYB) rc = dev_alloc(&Ly.lut, ((size_t)1 << Ly.Q) * 4);
+    if (rc == QL_OK && uses_table(Ly.code)) rc = dev_alloc(&Ly.lut, ((size_t)1 << Ly.Q) * 4);
     if (rc != QL_OK) {
         free_layer(Ly);
         delete h;
@@ -157,7 +167,7 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
         e = launch_relayout(packed_codes + Ly.parts[i].word_off, Ly.words, Ly.parts[i], n, st);
     if (e == cudaSuccess) e = launch_pack_signs(s_in, n, Ly.sin_bits, Ly.status, st);
     if (e == cudaSuccess) e = launch_pack_signs(s_out, m, Ly.sout_bits, Ly.status, st);
-    if (e == cudaSuccess && Ly.code == QL_CODE_HYB) e = launch_copy_lut(code.lut, Ly.Q, V, Ly.lut, st);
+    if (e == cudaSuccess && uses_table(Ly.code)) e = launch_copy_lut(code.lut, Ly.Q, V, Ly.lut, st);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     int status = 0;
     if (e == cudaSuccess) e = cudaMemcpy(&status, Ly.status, sizeof(int), cudaMemcpyDeviceToHost);
@@ -291,9 +301,13 @@ extern "C" {
 
 int qlinear_create(qlinear_t* out, int m, int n, int k, int L, int V, ql_code_t code, const uint32_t* packed_codes,
                    size_t n_words, const int8_t* s_in, const int8_t* s_out, float alpha) {
+    if (!out) return QL_E_ARG;
+    *out = nullptr;
+    if (k < 1 || k > 4) return QL_E_UNSUPPORTED;
+    if (V != 1 && V != 2) return QL_E_ARG;
     const int rows[1] = {m};
-    const int ks[1] = {k};
-    return create_common(out, m, n, 1, rows, ks, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+    const int kvs[1] = {k * V};
+    return create_common(out, m, n, 1, rows, kvs, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
 }
 
 int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int k_bot, int L, int V,
@@ -302,9 +316,11 @@ int qlinear_create_mixed(qlinear_t* out, int m, int n, int m_top, int k_top, int
     if (!out) return QL_E_ARG;
     *out = nullptr;
     if (m_top <= 0 || m_top >= m) return QL_E_ARG;
+    if (k_top < 1 || k_top > 4 || k_bot < 1 || k_bot > 4) return QL_E_UNSUPPORTED;
+    if (V != 1 && V != 2) return QL_E_ARG;
     const int rows[2] = {m_top, m - m_top};
-    const int ks[2] = {k_top, k_bot};
-    return create_common(out, m, n, 2, rows, ks, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+    const int kvs[2] = {k_top * V, k_bot * V};
+    return create_common(out, m, n, 2, rows, kvs, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
 }
 
 int qlinear_create_parts(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_k, int L,
@@ -312,7 +328,22 @@ int qlinear_create_parts(qlinear_t* out, int m, int n, int nparts, const int* pa
                          const int8_t* s_out, float alpha) {
     if (!out) return QL_E_ARG;
     *out = nullptr;
-    return create_common(out, m, n, nparts, part_rows, part_k, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+    if (nparts < 1 || nparts > kMaxParts || !part_rows || !part_k) return QL_E_ARG;
+    if (V != 1 && V != 2) return QL_E_ARG;
+    int kvs[kMaxParts];
+    for (int i = 0; i < nparts; ++i) {
+        if (part_k[i] < 1 || part_k[i] > 4) return QL_E_UNSUPPORTED;
+        kvs[i] = part_k[i] * V;
+    }
+    return create_common(out, m, n, nparts, part_rows, kvs, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
+}
+
+int qlinear_create_kv(qlinear_t* out, int m, int n, int nparts, const int* part_rows, const int* part_kv, int L,
+                      int V, ql_code_t code, const uint32_t* packed_codes, size_t n_words, const int8_t* s_in,
+                      const int8_t* s_out, float alpha) {
+    if (!out) return QL_E_ARG;
+    *out = nullptr;
+    return create_common(out, m, n, nparts, part_rows, part_kv, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
 }
 
 int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream) {
@@ -367,24 +398,25 @@ int qlinear_decode(qlinear_t h, void* w_hat, void* stream) {
 
 int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int count, void* out, void* stream) {
     if (count < 0 || L < 1 || L > 16) return QL_E_ARG;
-    int rc = check_code(code, V);
+    int rc = check_code(code, V, L);
     if (rc != QL_OK) return rc;
     if (count == 0) return QL_OK;
     if (!states || !out) return QL_E_ARG;
     uint32_t* lut_words = nullptr;
     cudaStream_t st = (cudaStream_t)stream;
-    if (code.kind == QL_CODE_HYB) {
-        if (cudaMallocAsync((void**)&lut_words, ((size_t)1 << code.Q) * 4, st) != cudaSuccess) {
+    const int Q = table_bits(code, L);
+    if (uses_table(code.kind)) {
+        if (cudaMallocAsync((void**)&lut_words, ((size_t)1 << Q) * 4, st) != cudaSuccess) {
             cudaGetLastError();
             return QL_E_OOM;
         }
-        if (launch_copy_lut(code.lut, code.Q, V, lut_words, st) != cudaSuccess) {
+        if (launch_copy_lut(code.lut, Q, V, lut_words, st) != cudaSuccess) {
             cudaGetLastError();
             cudaFreeAsync(lut_words, st);
             return QL_E_CUDA;
         }
     }
-    cudaError_t e = launch_eval_code(code.kind, L, V, code.Q, lut_words, states, count, out, st);
+    cudaError_t e = launch_eval_code(code.kind, L, V, Q, lut_words, states, count, out, st);
     if (lut_words) cudaFreeAsync(lut_words, st);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -398,11 +430,11 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
     if (blocks < 0) return QL_E_ARG;
     if (k < 1 || k > 4 || V < 1 || V > 2) return QL_E_UNSUPPORTED;
     if (L < k * V || L > 14 || k * V > 8) return QL_E_UNSUPPORTED;
-    int rc = check_code(code, V);
+    int rc = check_code(code, V, L);
     if (rc != QL_OK) return rc;
     if (blocks == 0) return QL_OK;
     if (!is_device_pointer(x) || !is_device_pointer(words) || (err && !is_device_pointer(err))) return QL_E_ARG;
-    const int Q = code.kind == QL_CODE_HYB ? code.Q : 0;
+    const int Q = table_bits(code, L);
     if (encode_smem_bytes(L, V, code.kind, Q) > (size_t)kTcMaxSmem) return QL_E_UNSUPPORTED;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -416,7 +448,7 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
     uint32_t* lut_words = nullptr;
     int* status = nullptr;
     if (cudaMalloc(&choice, choice_bytes) != cudaSuccess || cudaMalloc(&status, sizeof(int)) != cudaSuccess ||
-        (code.kind == QL_CODE_HYB && cudaMalloc(&lut_words, ((size_t)1 << Q) * 4) != cudaSuccess)) {
+        (uses_table(code.kind) && cudaMalloc(&lut_words, ((size_t)1 << Q) * 4) != cudaSuccess)) {
         cudaGetLastError();
         cudaFree(choice);
         cudaFree(status);
@@ -424,9 +456,9 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
         return QL_E_OOM;
     }
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
-    if (e == cudaSuccess && code.kind == QL_CODE_HYB) e = launch_copy_lut(code.lut, Q, V, lut_words, st);
+    if (e == cudaSuccess && uses_table(code.kind)) e = launch_copy_lut(code.lut, Q, V, lut_words, st);
     if (e == cudaSuccess)
-        e = launch_encode(code.kind, L, k, V, Q, lut_words, x, blocks, words, err, choice, grid, status, st);
+        e = launch_encode(code.kind, L, k * V, V, Q, lut_words, x, blocks, words, err, choice, grid, status, st);
     int dev_status = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&dev_status, status, sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -463,8 +495,8 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->V = L.V;
     info->code = L.code;
     info->Q = L.Q;
-    info->k_top = L.parts[0].k;
-    info->k_bot = L.parts[L.nparts - 1].k;
+    info->k_top = L.parts[0].kv / L.V;
+    info->k_bot = L.parts[L.nparts - 1].kv / L.V;
     info->m_top = L.parts[0].rows;
     info->B_n = L.B_n;
     info->B_m = L.B_m;
@@ -472,10 +504,14 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     for (int i = 0; i < L.nparts; ++i) words += L.parts[i].n_words;
     info->stream_bytes = words * 4;
     info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
-    info->lut_bytes = L.code == QL_CODE_HYB ? ((size_t)1 << L.Q) * L.V * 2 : 0;
+    info->lut_bytes = uses_table(L.code) ? ((size_t)1 << L.Q) * L.V * 2 : 0;
     info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
     info->last_launches = L.last_launches;
     info->nparts = L.nparts;
+    for (int i = 0; i < L.nparts; ++i) {
+        info->part_rows[i] = L.parts[i].rows;
+        info->part_kv[i] = L.parts[i].kv;
+    }
     return QL_OK;
 }
 
