@@ -55,8 +55,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--encode", action="store_true",
-                   help="time the trellis-coded quantizer (qlinear_encode, L = 14, k = 2, 3INST) on an N(0,1) "
+                   help="time the trellis-coded quantizer (qlinear_encode, k = 2, 3INST) on an N(0,1) "
                         "source instead of the forward")
+    p.add_argument("--encode-L", type=int, default=16, help="state bits of the --encode run (at most 16)")
     p.add_argument("--instances", type=int, default=None,
                    help="layer instances to rotate through (default: enough code words for 4x L2); a smaller "
                         "count is for profiler captures only, and the line then says its inputs may sit in L2")
@@ -269,11 +270,12 @@ def _traffic(kernel_key, launch_units):
 
 def run_encode(args):
     """The GPU trellis-coded quantizer on an i.i.d. N(0,1) source: blocks of 256
-    values, L = 14, k = 2, V = 1, 3INST; each step is one qlinear_encode call
-    (scratch allocation and the stream synchronisation included)."""
+    values, L = --encode-L (16 by default), k = 2, V = 1, 3INST; each step is one
+    qlinear_encode call (scratch allocation and the stream synchronisation
+    included)."""
     import torch
     import trellis_coded_matmul_b200 as tcm
-    L, k, V, code = 14, 2, 1, wl.CODE_3INST
+    L, k, V, code = args.encode_L, 2, 1, wl.CODE_3INST
     blocks = 148 * 8
     x = torch.randn((blocks, 256), generator=torch.Generator().manual_seed(7)).cuda()
     for _ in range(args.warmup):

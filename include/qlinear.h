@@ -239,12 +239,15 @@ int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int 
  *           (for a row-major m x n source, exactly qlinear_create's packed_codes).
  *   err:    device pointer or null, out, float32 [blocks]: squared error of each
  *           block's reconstruction.
- *   L <= 14 (both cost vectors and the code values sit in one CTA's shared
- *   memory), k*V <= 8; code as in qlinear_create (HYB and the table code: the
+ *   L <= 16, k*V <= 8; code as in qlinear_create (HYB and the table code: the
  *   fp16 table is read; the table code with L = kV is nearest-codeword VQ / NUQ).
- * Allocates scratch (256/V * 2^(L-kV) bytes per SM) and returns when the
- * result is ready (synchronises the stream).
- * Errors: QL_E_ARG, QL_E_UNSUPPORTED (L > 14, or too large for shared memory),
+ *   Up to L = 14 one CTA holds a block's whole dynamic programme in its shared
+ *   memory; at L = 15 and 16 a thread-block cluster of 2 or 4 CTAs shares it
+ *   (16384 states per CTA, predecessors' costs read from the other CTAs'
+ *   shared memory).
+ * Allocates scratch (256/V * 2^(L-kV) bytes per CTA or cluster that runs at
+ * once) and returns when the result is ready (synchronises the stream).
+ * Errors: QL_E_ARG, QL_E_UNSUPPORTED (L > 16, or too large for shared memory),
  * QL_E_OOM, QL_E_CUDA, QL_E_DEVICE (non-finite source values). */
 int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int blocks, uint32_t* words, float* err,
                    void* stream);

@@ -149,7 +149,7 @@ def test_encode_rejects_bad_arguments_on_the_host(tcm):
     lib = tcm.raw_library()
     code = tcm.ql_code_t(1, 0, None)
     assert lib.qlinear_encode(code, 12, 2, 1, None, -1, None, None, None) == tcm.QL_E_ARG
-    assert lib.qlinear_encode(code, 16, 2, 1, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # L > 14
+    assert lib.qlinear_encode(code, 17, 2, 1, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # L > 16
     assert lib.qlinear_encode(code, 12, 5, 1, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # k > 4
     assert lib.qlinear_encode(code, 3, 2, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED   # L < kV
     assert lib.qlinear_encode(code, 12, 2, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # 3INST: V = 1

@@ -26,6 +26,11 @@ CASES = [
     (12, 2, 2, wl.CODE_HYB, 6),
     (14, 2, 1, wl.CODE_3INST, 0),
     (13, 3, 1, wl.CODE_HYB, 9),
+    # L = 15, 16: the dynamic programme shared by a cluster of 2 or 4 CTAs
+    (16, 2, 1, wl.CODE_3INST, 0),
+    (15, 1, 1, wl.CODE_1MAD, 0),
+    (16, 1, 2, wl.CODE_HYB, 9),
+    (16, 3, 1, wl.CODE_HYB, 9),
 ]
 
 
@@ -78,6 +83,30 @@ def test_encoded_words_round_trip_through_a_layer():
     recon = np.concatenate(recon).reshape(m, n)
     assert np.array_equal(w.cpu().numpy().view(np.uint16), ofp16.encode(recon))
     tcm.qlinear_destroy(h)
+
+
+def test_cluster_encoder_loops_over_more_blocks_than_clusters():
+    """80 blocks at L = 16: more than the clusters that run at once, so every
+    cluster encodes several blocks in turn; sampled blocks match the oracle."""
+    L, k, V, code = 16, 2, 1, wl.CODE_3INST
+    x = _source(80, seed=77)
+    words = tcm.qlinear_encode(code, L, k, V, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    got = words.cpu().numpy().view(np.uint32)
+    for b in (0, 1, 36, 37, 38, 79):
+        assert np.array_equal(got[b], _oracle_words(x[b:b + 1], L, k, V, code, None)[0]), b
+
+
+def test_gaussian_distortion_at_L16_beats_L14():
+    """The discussion's setting (L = 16, k = 2): distortion between the Gaussian
+    rate-distortion bound and the 2-bit Lloyd-Max quantizer, and below L = 14's
+    on the same source ("larger trellises improve quality")."""
+    x = torch.from_numpy(_source(128, seed=60)).cuda()
+    mse = {}
+    for L in (14, 16):
+        _, err = tcm.qlinear_encode(wl.CODE_3INST, L, 2, 1, x, with_error=True)
+        mse[L] = float(err.sum()) / x.numel()
+    assert 2.0 ** -4 < mse[16] < mse[14] < 0.1175
 
 
 @pytest.mark.parametrize("k", [1, 2])
