@@ -103,11 +103,18 @@ def reconstruct(chunks: np.ndarray, L: int, kV: int, code: int, V: int, lut=None
     return codes.evaluate(code, states, V, lut)
 
 
-def encode_exact(x, L: int, k: int, V: int, code: int, lut=None):
+def _bits_per_step(k, V: int) -> int:
+    """kV as an integer: k may be a half number of bits when V = 2."""
+    kV = int(round(k * V))
+    assert abs(k * V - kV) < 1e-12, "k*V must be a whole number of bits"
+    return kV
+
+
+def encode_exact(x, L: int, k, V: int, code: int, lut=None):
     """Minimum-squared-error tail-biting encoding of one block, float64.
     x: [T, V] source values (T steps).  Returns (chunks [T], squared error)."""
     x = np.asarray(x, dtype=np.float64).reshape(-1, V)
-    kV = k * V
+    kV = _bits_per_step(k, V)
     keep = L - kV
     pred = _predecessors(L, kV)
     values = codes.evaluate(code, np.arange(1 << L), V, lut)
@@ -121,12 +128,12 @@ def encode_exact(x, L: int, k: int, V: int, code: int, lut=None):
     return states & ((1 << kV) - 1), float(best[0])
 
 
-def encode_two_pass(x, L: int, k: int, V: int, code: int, lut=None):
+def encode_two_pass(x, L: int, k, V: int, code: int, lut=None):
     """The two-pass tail-biting encoding (module docstring), float32 costs; the
     source is taken as float32.  Returns (chunks [T], squared error of the
     reconstruction against that source, in float64)."""
     x = np.asarray(x, dtype=np.float32).reshape(-1, V)
-    kV = k * V
+    kV = _bits_per_step(k, V)
     keep = L - kV
     pred = _predecessors(L, kV)
     values = codes.evaluate(code, np.arange(1 << L), V, lut)

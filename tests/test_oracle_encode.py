@@ -26,7 +26,7 @@ LLOYD_MAX = {1: 1.0 - 2.0 / np.pi, 2: 0.1175}
 
 def _brute_force(x, L, k, V, code, lut=None):
     T = x.shape[0]
-    kV = k * V
+    kV = int(k * V)
     best = None
     for bits in itertools.product((0, 1), repeat=T * kV):
         chunks = np.array([int("".join(map(str, bits[t * kV:(t + 1) * kV])), 2) for t in range(T)])
@@ -36,16 +36,27 @@ def _brute_force(x, L, k, V, code, lut=None):
     return best
 
 
+def _lut(code, L, V, seed):
+    if code == wl.CODE_HYB:
+        return wl.hyb_table(4, V, seed)
+    if code == wl.CODE_TABLE:
+        return wl.palette_table(L, V, seed)
+    return None
+
+
 @pytest.mark.parametrize("L,k,V,code,T", [(4, 1, 1, wl.CODE_3INST, 8), (4, 2, 1, wl.CODE_1MAD, 4),
-                                          (6, 1, 2, wl.CODE_HYB, 4), (5, 1, 1, wl.CODE_1MAD, 9)])
+                                          (6, 1, 2, wl.CODE_HYB, 4), (5, 1, 1, wl.CODE_1MAD, 9),
+                                          (5, 1.5, 2, wl.CODE_HYB, 4), (6, 1.5, 2, wl.CODE_TABLE, 4),
+                                          (4, 1, 1, wl.CODE_TABLE, 7)])
 def test_exact_viterbi_equals_brute_force(L, k, V, code, T):
-    rng = np.random.default_rng(L * 100 + k * 10 + V + T)
-    lut = wl.hyb_table(4, V, 7) if code == wl.CODE_HYB else None
+    rng = np.random.default_rng(int(L * 100 + k * 10 + V + T))
+    lut = _lut(code, L, V, 7)
+    kV = int(k * V)
     for _ in range(3):
         x = rng.standard_normal((T, V))
         chunks, err = encode.encode_exact(x, L, k, V, code, lut)
         assert err == pytest.approx(_brute_force(x, L, k, V, code, lut), rel=1e-12, abs=1e-12)
-        recon = encode.reconstruct(chunks, L, k * V, code, V, lut)
+        recon = encode.reconstruct(chunks, L, kV, code, V, lut)
         assert float(np.sum((x - recon) ** 2)) == pytest.approx(err, rel=1e-12, abs=1e-12)
 
 
@@ -59,11 +70,14 @@ def test_two_pass_is_never_better_than_the_exact_minimum():
             assert two >= exact * (1 - 1e-6)
 
 
-@pytest.mark.parametrize("k,V,code", [(2, 1, wl.CODE_3INST), (3, 1, wl.CODE_1MAD), (2, 2, wl.CODE_HYB)])
+@pytest.mark.parametrize("k,V,code", [(2, 1, wl.CODE_3INST), (3, 1, wl.CODE_1MAD), (2, 2, wl.CODE_HYB),
+                                      (2.5, 2, wl.CODE_TABLE), (3, 1, wl.CODE_TABLE)])
 def test_memoryless_trellis_is_nearest_codeword_vq(k, V, code):
-    L = k * V
-    lut = wl.hyb_table(4, V, 5) if code == wl.CODE_HYB else None
-    rng = np.random.default_rng(k + V)
+    """L = kV: every state is its own chunk, so both searches pick the nearest
+    codeword at every step (VQ at V = 2, NUQ at V = 1 with the table code)."""
+    L = int(k * V)
+    lut = wl.hyb_table(4, V, 5) if code == wl.CODE_HYB else (wl.palette_table(L, V, 5) if code == wl.CODE_TABLE else None)
+    rng = np.random.default_rng(int(2 * k) + V)
     x = rng.standard_normal((40, V))
     book = codes.evaluate(code, np.arange(1 << L), V, lut)                  # [2^L, V]
     nearest = np.argmin(((x[:, None, :] - book[None, :, :]) ** 2).sum(-1), axis=1)
@@ -83,6 +97,24 @@ def test_encoded_block_decodes_through_the_layer_format():
     w = layer.decode_rows(np.arange(1))[0]
     assert np.array_equal(w, encode.reconstruct(chunks, L, k * V, code, V).reshape(-1))
     x32 = x[:, 0].astype(np.float32).astype(np.float64)  # the two-pass search takes the source as float32
+    assert float(np.sum((x32 - w) ** 2)) == pytest.approx(err, rel=1e-12)
+
+
+def test_fractional_block_decodes_through_the_layer_format():
+    """A 2.5-bit block (V = 2, 5 bits per step) packed MSB-first decodes
+    through the layer oracle to the reconstruction the encoder scored."""
+    L, k, V, code = 12, 2.5, 2, wl.CODE_HYB
+    lut = wl.hyb_table(9, V, 4)
+    x = np.random.default_rng(13).standard_normal((128, 2))
+    chunks, err = encode.encode_two_pass(x, L, k, V, code, lut)
+    bits = "".join(format(int(c), "05b") for c in chunks)
+    assert len(bits) == 640
+    words = bitstream.bits_to_words(bits)
+    layer = qlinear.Layer(1, 256, [(0, 1, k)], L, V, code, words, np.ones(256, np.int8), np.ones(1, np.int8), 1.0,
+                          lut)
+    w = layer.decode_rows(np.arange(1))[0]
+    assert np.array_equal(w, encode.reconstruct(chunks, L, 5, code, V, lut).reshape(-1))
+    x32 = x.astype(np.float32).astype(np.float64).reshape(-1)
     assert float(np.sum((x32 - w) ** 2)) == pytest.approx(err, rel=1e-12)
 
 
