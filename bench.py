@@ -272,7 +272,14 @@ def run_encode(args):
     """The GPU trellis-coded quantizer on an i.i.d. N(0,1) source: blocks of 256
     values, L = --encode-L (16 by default), k = 2, V = 1, 3INST; each step is one
     qlinear_encode call (scratch allocation and the stream synchronisation
-    included)."""
+    included).
+
+    Roofline: the search is plain fp32 ALU work.  Per block it updates 2^L
+    states at each of the T = 256 / V steps of both passes, and a state update
+    is 3V + (C - 1) / C operations (V subtractions, V multiplications, V - 1
+    additions over the values, one addition to the path cost, and one C-way
+    minimum per group of C = 2^kV states).  The peak is the SM array's fp32
+    lane rate at the highest SM clock seen (128 lanes per SM per clock)."""
     import torch
     import trellis_coded_matmul_b200 as tcm
     L, k, V, code = args.encode_L, 2, 1, wl.CODE_3INST
@@ -281,20 +288,46 @@ def run_encode(args):
     for _ in range(args.warmup):
         tcm.qlinear_encode(code, L, k, V, x)
     torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for _ in range(args.steps):
         _, err = tcm.qlinear_encode(code, L, k, V, x, with_error=True)
     end.record()
     torch.cuda.synchronize()
+    clk = clocks.stop()
     secs = start.elapsed_time(end) * 1e-3
+    C = 1 << (k * V)
+    ops_per_block = 2 * (256 // V) * (1 << L) * (3 * V + (C - 1) / C)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    max_mhz = clk["sm_max_mhz"] if clk else 1965.0
+    peak = sms * 128 * max_mhz * 1e6 / 1e12
+    achieved = ops_per_block * blocks * args.steps / secs / 1e12
     line = {"metric": "trellis-coded quantization (two-pass tail-biting Viterbi) source weights/s",
             "value": blocks * 256 * args.steps / secs, "unit": "weights/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"encode: {blocks} blocks of 256 N(0,1) values, L={L} k={k} V={V} code=3INST",
                        "mse": float(err.sum()) / (blocks * 256)},
-            "roofline": None, "gpu_launches": args.steps}
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Top/s", "frac": achieved / peak,
+                         "traffic": None, "ops_per_block": ops_per_block,
+                         "peak_kind": f"derived: {sms} SMs x 128 fp32 lanes x {max_mhz:.0f} MHz"},
+            "gpu_launches": args.steps, "clocks": clk}
+    if not args.no_cpu_baseline:
+        from oracle import encode as oenc
+        xs = x[:4].cpu().numpy()
+        t0 = time.perf_counter()
+        done = 0
+        for blk in xs:
+            oenc.encode_two_pass(blk.reshape(-1, V), L, k, V, code)
+            done += 1
+            if time.perf_counter() - t0 > 20.0:
+                break
+        cs = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": done * 256 / cs, "unit": "weights/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{done} blocks of 256 values: oracle.encode.encode_two_pass (numpy "
+                                          f"element-wise, one thread; float32 costs), {cs:.1f} s"}
     print(json.dumps(line), flush=True)
     return 0
 

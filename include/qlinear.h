@@ -252,6 +252,15 @@ int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int 
 int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int blocks, uint32_t* words, float* err,
                    void* stream);
 
+/* As qlinear_encode with the bitrate given as kv bits per trellis step
+ * (V <= kv <= min(4V, 8), L >= kv): with V = 2 an odd kv is a half-integer
+ * bitwidth (kv = 5: 2.5 bits per weight), the layout qlinear_create_kv reads.
+ *   words: device pointer, out, uint32 [blocks][(256 / V) * kv / 32].
+ * With the table code and L = kv this is nearest-codeword vector (V = 2) or
+ * non-uniform scalar (V = 1) quantization.  Errors as qlinear_encode. */
+int qlinear_encode_kv(ql_code_t code, int L, int kv, int V, const float* x, int blocks, uint32_t* words, float* err,
+                      void* stream);
+
 /* Read the handle's device status word (synchronises the device).  Returns
  * QL_OK, or QL_E_DEVICE / QL_E_TIMEOUT if a kernel recorded a failed check or
  * an expired bounded wait since the last call; reading clears the word. */

@@ -155,3 +155,10 @@ def test_encode_rejects_bad_arguments_on_the_host(tcm):
     assert lib.qlinear_encode(code, 12, 2, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # 3INST: V = 1
     assert lib.qlinear_encode(code, 12, 2, 1, None, 0, None, None, None) == tcm.QL_OK             # nothing to do
     assert lib.qlinear_encode(code, 12, 2, 1, None, 4, None, None, None) == tcm.QL_E_ARG          # null pointers
+    hyb = tcm.ql_code_t(tcm.QL_CODE_HYB, 9, None)
+    enc_kv = lib.qlinear_encode_kv
+    assert enc_kv(hyb, 12, 5, 2, None, 4, None, None, None) == tcm.QL_E_ARG      # 2.5 bits: valid, null pointers
+    assert enc_kv(hyb, 12, 1, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # 0.5 bits
+    assert enc_kv(hyb, 12, 9, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # more than 8 bits per step
+    assert enc_kv(hyb, 4, 5, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED   # L < kV
+    assert enc_kv(code, 12, 3, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # 3INST: V = 1

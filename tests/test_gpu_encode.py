@@ -63,6 +63,79 @@ def test_encode_matches_the_oracle_bit_for_bit(L, k, V, code, Q):
         assert float(err[b]) == pytest.approx(float(np.sum((x[b].astype(np.float64) - recon) ** 2)), rel=1e-4)
 
 
+# bits per step (kv) instead of k: half-integer bitwidths and the palette's table code
+CASES_KV = [
+    # L, kv, V, code, Q
+    (12, 5, 2, wl.CODE_HYB, 9),      # 2.5-bit TCQ, one CTA per block
+    (16, 5, 2, wl.CODE_HYB, 9),      # 2.5-bit TCQ at L = 16, a cluster of 4 CTAs
+    (15, 7, 2, wl.CODE_HYB, 6),      # 3.5 bits, a cluster of 2 CTAs
+    (5, 5, 2, wl.CODE_TABLE, 0),     # 2.5-bit VQ: nearest codeword
+    (3, 3, 1, wl.CODE_TABLE, 0),     # 3-bit NUQ: nearest level
+    (8, 3, 2, wl.CODE_TABLE, 0),     # 1.5 bits, a trellis over a 256-entry codebook
+]
+
+
+def _table(code, L, V, Q, seed):
+    if code == wl.CODE_HYB:
+        return wl.hyb_table(Q, V, seed)
+    if code == wl.CODE_TABLE:
+        return wl.palette_table(L, V, seed)
+    return None
+
+
+def _oracle_words_kv(x, L, kv, V, code, lut):
+    out = []
+    for blk in x:
+        chunks, _ = encode.encode_two_pass(blk.reshape(-1, V), L, kv / V, V, code, lut)
+        out.append(bitstream.bits_to_words("".join(format(int(c), f"0{kv}b") for c in chunks)))
+    return np.stack(out)
+
+
+@pytest.mark.parametrize("L,kv,V,code,Q", CASES_KV, ids=lambda v: str(v))
+def test_encode_kv_matches_the_oracle_bit_for_bit(L, kv, V, code, Q):
+    lut_np = _table(code, L, V, Q, 8)
+    lut = torch.from_numpy(lut_np.copy()).cuda() if lut_np is not None else None
+    x = _source(3, seed=L * 10 + kv)
+    words, err = tcm.qlinear_encode_kv(code, L, kv, V, torch.from_numpy(x).cuda(), Q=Q, lut=lut, with_error=True)
+    torch.cuda.synchronize()
+    ref = _oracle_words_kv(x, L, kv, V, code, lut_np)
+    assert words.shape == (3, (256 // V) * kv // 32)
+    assert np.array_equal(words.cpu().numpy().view(np.uint32), ref)
+
+
+def test_fractional_vq_round_trips_through_a_layer():
+    """2.5-bit VQ of a 32 x 512 source: the encoder's words, given to
+    qlinear_create_kv, decode to the oracle's reconstruction, which is the
+    nearest codeword of (nearly) every pair: with L = kV the search only adds
+    per-step costs, so it departs from the nearest codeword only where two
+    codewords' costs tie after rounding against the running path cost."""
+    L, kv, V, code = 5, 5, 2, wl.CODE_TABLE
+    m, n = 32, 512
+    book = wl.palette_table(L, V, 9)
+    lut = torch.from_numpy(book.copy()).cuda()
+    x = _source(m * n // 256, seed=15).reshape(m, n)
+    words = tcm.qlinear_encode_kv(code, L, kv, V, torch.from_numpy(x).cuda(), lut=lut)
+    torch.cuda.synchronize()
+    ones_n = torch.ones(n, dtype=torch.int8, device="cuda")
+    ones_m = torch.ones(m, dtype=torch.int8, device="cuda")
+    h = tcm.qlinear_create_kv(m, n, [m], [kv], L, V, code, words.reshape(-1), ones_n, ones_m, 1.0, lut=lut)
+    w = tcm.qlinear_decode(h).cpu().numpy()
+    ref = _oracle_words_kv(x.reshape(-1, 256), L, kv, V, code, book)
+    recon = []
+    for row in ref:
+        bits = "".join(format(int(wd), "032b") for wd in row)
+        chunks = np.array([int(bits[i:i + kv], 2) for i in range(0, len(bits), kv)])
+        recon.append(encode.reconstruct(chunks, L, kv, code, V, book).reshape(-1))
+    recon = np.concatenate(recon).reshape(m, n)
+    assert np.array_equal(w.view(np.uint16), ofp16.encode(recon))
+    cb = book.astype(np.float32)
+    pairs = x.reshape(m, n // 2, 2)
+    d = (pairs[:, :, None, 0] - cb[None, None, :, 0]) ** 2 + (pairs[:, :, None, 1] - cb[None, None, :, 1]) ** 2
+    nearest = cb[np.argmin(d, axis=-1)].astype(np.float64)
+    assert np.mean(np.all(w.astype(np.float64).reshape(m, n // 2, 2) == nearest, axis=-1)) > 0.999
+    tcm.qlinear_destroy(h)
+
+
 def test_encoded_words_round_trip_through_a_layer():
     L, k, V, code = 12, 2, 1, wl.CODE_1MAD
     m, n = 32, 512

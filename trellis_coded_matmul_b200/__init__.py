@@ -18,7 +18,7 @@ from typing import Optional
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
 if not os.path.exists(_LIB_PATH):
-    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m trellis_coded_matmul_b200.build`")
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python trellis_coded_matmul_b200/build.py`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
 QL_OK = 0
@@ -42,7 +42,7 @@ ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts",
                "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
                "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
-               "qlinear_forward_noalloc", "qlinear_encode")
+               "qlinear_forward_noalloc", "qlinear_encode", "qlinear_encode_kv")
 
 
 class ql_code_t(ctypes.Structure):
@@ -68,6 +68,7 @@ _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_encode.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp]
+_lib.qlinear_encode_kv.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp]
 _lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
 _lib.qlinear_eval_code.argtypes = [ql_code_t, _i, _i, _vp, _i, _vp, _vp]
 _lib.qlinear_get_status.argtypes = [_vp]
@@ -269,6 +270,23 @@ def qlinear_encode(kind, L, k, V, x, Q=0, lut=None, with_error=False, stream=Non
     err = torch.empty(blocks, dtype=torch.float32, device=x.device) if with_error else None
     _check(_lib.qlinear_encode(_code(kind, Q, lut), L, k, V, _ptr(x), blocks, _ptr(words),
                                _ptr(err) if err is not None else None, _stream(stream)), "qlinear_encode")
+    return (words, err) if with_error else words
+
+
+def qlinear_encode_kv(kind, L, kv, V, x, Q=0, lut=None, with_error=False, stream=None):
+    """As qlinear_encode with kv bits per trellis step (odd kv with V = 2: a
+    half-integer bitwidth): words int32 [blocks, (256 // V) * kv // 32]."""
+    import torch
+    _cuda(x, "x", torch.float32)
+    if x.numel() % 256:
+        raise ValueError("x must hold whole blocks of 256 values")
+    if V not in (1, 2):
+        raise ValueError("V must be 1 or 2")
+    blocks = x.numel() // 256
+    words = torch.empty((blocks, (256 // V) * kv // 32), dtype=torch.int32, device=x.device)
+    err = torch.empty(blocks, dtype=torch.float32, device=x.device) if with_error else None
+    _check(_lib.qlinear_encode_kv(_code(kind, Q, lut), L, kv, V, _ptr(x), blocks, _ptr(words),
+                                  _ptr(err) if err is not None else None, _stream(stream)), "qlinear_encode_kv")
     return (words, err) if with_error else words
 
 

@@ -1,6 +1,6 @@
 """Build libqlinear.so (the C ABI of include/qlinear.h) in-tree for sm_100a.
 
-    python -m trellis_coded_matmul_b200.build [--force]
+    python trellis_coded_matmul_b200/build.py [--force]
 
 nvcc cross-compiles without a GPU.  The CUDA runtime is linked statically,
 so the shared library only needs the driver at run time.

@@ -429,7 +429,14 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
                    void* stream) {
     if (blocks < 0) return QL_E_ARG;
     if (k < 1 || k > 4 || V < 1 || V > 2) return QL_E_UNSUPPORTED;
-    if (L < k * V || L > 16 || k * V > 8) return QL_E_UNSUPPORTED;
+    return qlinear_encode_kv(code, L, k * V, V, x, blocks, words, err, stream);
+}
+
+int qlinear_encode_kv(ql_code_t code, int L, int kv, int V, const float* x, int blocks, uint32_t* words, float* err,
+                      void* stream) {
+    if (blocks < 0) return QL_E_ARG;
+    if (V < 1 || V > 2 || kv < V || kv > 4 * V || kv > 8) return QL_E_UNSUPPORTED;
+    if (L < kv || L > 16) return QL_E_UNSUPPORTED;
     int rc = check_code(code, V, L);
     if (rc != QL_OK) return rc;
     if (blocks == 0) return QL_OK;
@@ -442,11 +449,11 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
         return QL_E_CUDA;
     }
     int workers = 0;
-    if (encode_workers(L, k * V, V, blocks, sms, &workers) != cudaSuccess) {
+    if (encode_workers(L, kv, V, blocks, sms, &workers) != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    const size_t choice_bytes = (size_t)workers * (256 / V) * ((size_t)1 << (L - k * V));
+    const size_t choice_bytes = (size_t)workers * (256 / V) * ((size_t)1 << (L - kv));
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* choice = nullptr;
     uint32_t* lut_words = nullptr;
@@ -462,7 +469,7 @@ int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int bloc
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
     if (e == cudaSuccess && uses_table(code.kind)) e = launch_copy_lut(code.lut, Q, V, lut_words, st);
     if (e == cudaSuccess)
-        e = launch_encode(code.kind, L, k * V, V, Q, lut_words, x, blocks, words, err, choice, workers, status, st);
+        e = launch_encode(code.kind, L, kv, V, Q, lut_words, x, blocks, words, err, choice, workers, status, st);
     int dev_status = 0;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&dev_status, status, sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
