@@ -467,8 +467,29 @@ def run_ours(args):
                "h2d_bytes_per_step": batch * sp.n * 2, "d2h_bytes_per_step": batch * sp.m * 4,
                "steps": e2e_steps}
 
+    def cold_call_us():
+        """Latency of one forward whose code words are not in L2 (a buffer of
+        twice the L2 size is written first), median of 3; None if it fails."""
+        try:
+            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            out = []
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    flush.zero_()
+                    ev0.record(stream)
+                    tcm.qlinear_forward(handles[i % n_inst], xs[i % n_inst], ys[i % n_inst])
+                    ev1.record(stream)
+                    torch.cuda.synchronize()
+                    out.append(ev0.elapsed_time(ev1) * 1e3)
+            del flush
+            return statistics.median(out)
+        except Exception:
+            return None
+
     line = None
     if rank == 0:
+        cold = cold_call_us()  # rank 0 only, no collective inside
         pk, pk_kind = peaks()
         value = job_tokens_per_s(world, args.steps, batch, secs)
         launches_per_step = tcm.qlinear_info(handles[0])["last_launches"]
@@ -497,6 +518,7 @@ def run_ours(args):
                 "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
                 "config": config_dict(sp, batch, n_inst),
                 "hbm_gbs_step": sp.stream_bytes * args.steps * world / secs / 1e9,
+                "cold_call_us": cold,
                 "roofline": roof,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk, "e2e": e2e}
