@@ -162,3 +162,33 @@ def test_encode_rejects_bad_arguments_on_the_host(tcm):
     assert enc_kv(hyb, 12, 9, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # more than 8 bits per step
     assert enc_kv(hyb, 4, 5, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED   # L < kV
     assert enc_kv(code, 12, 3, 2, None, 4, None, None, None) == tcm.QL_E_UNSUPPORTED  # 3INST: V = 1
+
+
+def test_info_struct_layout_matches_the_header(tcm, tmp_path):
+    """The binding's ctypes mirror of ql_info_t has the C struct's size and
+    field offsets (compiled from include/qlinear.h with the host compiler)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = [f for f, _ in tcm.ql_info_t._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"qlinear.h\"\nint main(void) {\n"
+                   "  printf(\"%zu\\n\", sizeof(ql_info_t));\n"
+                   + "".join(f"  printf(\"%zu\\n\", offsetof(ql_info_t, {f}));\n" for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(tcm.ql_info_t)
+    assert out[1:] == [getattr(tcm.ql_info_t, f).offset for f in fields]
+    code = tmp_path / "code.c"
+    code.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"qlinear.h\"\nint main(void) {\n"
+                    "  printf(\"%zu %zu %zu %zu\\n\", sizeof(ql_code_t), offsetof(ql_code_t, kind),"
+                    " offsetof(ql_code_t, Q), offsetof(ql_code_t, lut));\n  return 0;\n}\n")
+    exe2 = tmp_path / "code"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(code), "-o", str(exe2)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe2)], check=True, capture_output=True, text=True).stdout.split()]
+    assert got == [ctypes.sizeof(tcm.ql_code_t), tcm.ql_code_t.kind.offset, tcm.ql_code_t.Q.offset,
+                   tcm.ql_code_t.lut.offset]
