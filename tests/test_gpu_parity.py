@@ -297,3 +297,24 @@ def test_parts_with_the_hyb_code(batch):
     w = tcm.qlinear_decode(h)
     torch.cuda.synchronize()
     assert np.array_equal(_bits(w), oq.Layer.from_inputs(li).decode_bits(np.arange(64)))
+
+
+# ---------------------------------------------------------------- every output element written
+@pytest.mark.parametrize("case", [SMALL[1], SMALL[4], SMALL[9]], ids=lambda c: f"{c[0]}x{c[1]}_k{c[2]}_L{c[3]}_V{c[4]}")
+def test_outputs_are_fully_written_over_a_nan_sentinel(case):
+    """y and W_hat buffers pre-filled with NaN come back without any NaN (the
+    codes' values and the outputs are finite), on both forward paths; the
+    fp16 output too."""
+    li = _small_layer(*case)
+    h = make_handle(li)
+    for batch in (3, 16):
+        x = torch.from_numpy(wl.make_x(li.spec, batch, instance=21)).cuda()
+        for dtype in (torch.float32, torch.float16):
+            y = torch.full((batch, li.spec.m), float("nan"), dtype=dtype, device="cuda")
+            tcm.qlinear_forward(h, x, y)
+            torch.cuda.synchronize()
+            assert not torch.isnan(y).any()
+    w = torch.full((li.spec.m, li.spec.n), float("nan"), dtype=torch.float16, device="cuda")
+    tcm.qlinear_decode(h, w)
+    torch.cuda.synchronize()
+    assert not torch.isnan(w).any()
