@@ -245,7 +245,8 @@ def test_forward_largest_hadamard_blocks(m, n):
 
 
 # ---------------------------------------------------------------- layers of several row parts
-PARTS = [((32, 2), (48, 3), (16, 4)), ((16, 1), (16, 2), (32, 3), (16, 4), (16, 2))]
+PARTS = [((32, 2), (48, 3), (16, 4)), ((16, 1), (16, 2), (32, 3), (16, 4), (16, 2)),
+         ((16, 1), (16, 2), (16, 3), (16, 4), (32, 2), (16, 3), (16, 1), (16, 4))]  # the most parts: 8
 
 
 @pytest.mark.parametrize("split", PARTS, ids=lambda v: "-".join(f"{r}k{k}" for r, k in v))
