@@ -30,6 +30,7 @@
 #include <math.h>
 
 #include "codes.cuh"
+#include "encode.h"
 #include "internal.h"
 
 namespace cg = cooperative_groups;

@@ -103,15 +103,12 @@ cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* s
 cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
 
 // Trellis-coded quantization of `blocks` blocks of 256 source values (two-pass
-// tail-biting Viterbi, L <= 16, kv bits per step): words [blocks][8 kv / V] in
+// tail-biting Viterbi, L <= 14, kv bits per step): words [blocks][8 kv / V] in
 // the stream format, the squared error of each block's reconstruction into
-// err (may be null).  Blocks are shared out over `workers` (CTAs up to L = 14,
-// clusters of 2^(L-14) CTAs above; encode_workers gives how many run at
-// once); choice: workers * (256/V) * 2^(L-kv) bytes of scratch.
+// err (may be null).  choice: grid * (256/V) * 2^(L-kv) bytes of scratch.
 size_t encode_smem_bytes(int L, int V, int code, int Q);
-cudaError_t encode_workers(int L, int kv, int V, int blocks, int num_sms, int* workers);
 cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t* lut, const float* x, int blocks,
-                          uint32_t* words, float* err, uint8_t* choice, int workers, int* status, cudaStream_t st);
+                          uint32_t* words, float* err, uint8_t* choice, int grid, int* status, cudaStream_t st);
 
 // x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);

@@ -8,6 +8,7 @@
 #include <new>
 
 #include "codes.cuh"
+#include "encode.h"
 #include "internal.h"
 
 using namespace qlk;
