@@ -134,6 +134,20 @@ def test_larger_trellis_lowers_the_distortion():
     assert mse[16] > 2.0 ** -4
 
 
+@pytest.mark.parametrize("k,levels,mse", [(1, [-0.7979, 0.7979], 1.0 - 2.0 / np.pi),
+                                          (2, [-1.5104, -0.4528, 0.4528, 1.5104], 0.1175)])
+def test_nuq_with_lloyd_max_levels_reaches_the_lloyd_max_distortion(k, levels, mse):
+    """The palette's NUQ member (table code, L = kV, V = 1) with the optimal
+    k-bit scalar quantizer's levels for N(0,1) as its codebook (textbook
+    Lloyd-Max values, rounded to fp16) quantizes N(0,1) samples to its
+    textbook distortion, within four standard errors of the sample mean."""
+    book = np.array(levels, dtype=np.float16).reshape(-1, 1)
+    x = np.random.default_rng(30 + k).standard_normal((400, 256, 1)).astype(np.float32)
+    per_block = np.array([encode.encode_two_pass(b, k, k, 1, wl.CODE_TABLE, book)[1] / b.size for b in x])
+    sem = per_block.std(ddof=1) / np.sqrt(len(per_block))
+    assert abs(per_block.mean() - mse) < 4 * sem + 1e-3
+
+
 def test_two_pass_costs_follow_the_float32_rule():
     rng = np.random.default_rng(9)
     x = rng.standard_normal((3, 2))
