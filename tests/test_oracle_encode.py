@@ -148,6 +148,33 @@ def test_nuq_with_lloyd_max_levels_reaches_the_lloyd_max_distortion(k, levels, m
     assert abs(per_block.mean() - mse) < 4 * sem + 1e-3
 
 
+def test_vq_with_a_product_codebook_is_per_dimension_scalar_quantization():
+    """The palette's VQ member (table code, L = kV, V = 2) with the product of
+    the 2-bit Lloyd-Max quantizer (first value of a pair) and the 1-bit one
+    (second value) as its 8-pair codebook, 1.5 bits per weight: the nearest
+    pair is the pair of per-dimension nearest levels, so the reconstruction
+    matches per-dimension scalar quantization, and the distortion per weight
+    is the mean of the two Lloyd-Max values.  The two coordinates use
+    different level sets, so a pair read in the wrong order fails."""
+    lv2 = np.array([-1.5104, -0.4528, 0.4528, 1.5104], dtype=np.float16)
+    lv1 = np.array([-0.7979, 0.7979], dtype=np.float16)
+    book = np.array([[a, b] for a in lv2 for b in lv1], dtype=np.float16)      # entry 2i + j = (lv2[i], lv1[j])
+    x = np.random.default_rng(44).standard_normal((100, 128, 2)).astype(np.float32)
+    same, per_block = 0, []
+    for blk in x:
+        chunks, err = encode.encode_two_pass(blk, 3, 1.5, 2, wl.CODE_TABLE, book)
+        recon = encode.reconstruct(chunks, 3, 3, wl.CODE_TABLE, 2, book)
+        xb = blk.astype(np.float64)
+        n0 = lv2.astype(np.float64)[np.argmin(np.abs(xb[:, :1] - lv2.astype(np.float64)[None, :]), axis=1)]
+        n1 = lv1.astype(np.float64)[np.argmin(np.abs(xb[:, 1:] - lv1.astype(np.float64)[None, :]), axis=1)]
+        same += int(np.sum((recon[:, 0] == n0) & (recon[:, 1] == n1)))
+        per_block.append(err / blk.size)
+    assert same / (x.shape[0] * x.shape[1]) > 0.999
+    per_block = np.array(per_block)
+    want = (0.1175 + (1.0 - 2.0 / np.pi)) / 2
+    assert abs(per_block.mean() - want) < 4 * per_block.std(ddof=1) / np.sqrt(len(per_block)) + 1e-3
+
+
 def test_two_pass_costs_follow_the_float32_rule():
     rng = np.random.default_rng(9)
     x = rng.standard_normal((3, 2))
