@@ -70,3 +70,46 @@ def test_absolute_instead_of_squared_error_is_caught(monkeypatch):
         return d
     monkeypatch.setattr(encode, "_step_costs", step_costs)
     _fails(t_encode.test_exact_viterbi_equals_brute_force, 4, 1, 1, wl.CODE_3INST, 8)
+
+
+def test_round_half_up_instead_of_to_even_is_caught(monkeypatch):
+    """fp16 rounding with ties away from zero (floor(x + 1/2)) instead of to even."""
+    from oracle import fp16
+    import test_oracle_fp16 as t_fp16
+
+    def round_half_up(v):
+        v = np.asarray(v, dtype=np.float64)
+        a = np.abs(v)
+        mant, ex = np.frexp(np.where(a > 0, a, 1.0))
+        q = np.exp2((np.maximum(ex - 1, -14) - 10).astype(np.float64))
+        r = np.where(a == 0, 0.0, np.floor(a / q + 0.5) * q)
+        r = np.where(a >= 65520.0, np.inf, r)
+        return np.copysign(r, v)
+    monkeypatch.setattr(fp16, "round_rne", round_half_up)
+    _fails(t_fp16.test_round_ties_to_even_and_overflow)
+
+
+def test_reversed_steps_inside_a_block_are_caught(monkeypatch):
+    """Decoded values placed at column 256 j + (T/V - 1 - t) V + e instead of 256 j + t V + e."""
+    def decode_rows(self, rows, blocks=None):
+        rows = np.asarray(rows, dtype=np.int64)
+        from oracle import trellis
+        states = trellis.block_states(self.words, rows, self.n, self.parts, self.L, self.V, blocks)
+        vals = codes.evaluate(self.code, states, self.V, self.lut)[:, :, ::-1, :]
+        return vals.reshape(len(rows), -1)
+    monkeypatch.setattr(qlinear.Layer, "decode_rows", decode_rows)
+    _fails(t_qlinear.test_element_order_inside_a_block)
+    _fails(t_palette.test_memoryless_table_code_is_a_field_lookup, 3, 1)
+
+
+def test_3inst_without_its_high_half_is_caught(monkeypatch):
+    """3INST taking only the low half (one fp16 value) instead of the sum of both halves."""
+    import test_oracle_codes as t_codes
+
+    def low_half_only(state):
+        from oracle import fp16
+        x = codes.lcg(state, codes.A_3INST, codes.B_3INST).astype(np.int64)
+        m = (x & codes.MASK_3INST) ^ codes.XOR_3INST
+        return fp16.round_rne(fp16.decode_bits(m & 0xFFFF))
+    monkeypatch.setattr(codes, "three_inst", low_half_only)
+    _fails(t_codes.test_computed_code_is_close_to_standard_normal, codes.three_inst)
