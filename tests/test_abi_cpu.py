@@ -192,3 +192,35 @@ def test_info_struct_layout_matches_the_header(tcm, tmp_path):
     got = [int(v) for v in subprocess.run([str(exe2)], check=True, capture_output=True, text=True).stdout.split()]
     assert got == [ctypes.sizeof(tcm.ql_code_t), tcm.ql_code_t.kind.offset, tcm.ql_code_t.Q.offset,
                    tcm.ql_code_t.lut.offset]
+
+
+def test_host_validation_never_accepts_null_buffers(tcm):
+    """Random shapes, bitrates, codes and stream lengths with null device
+    buffers: every create entry point rejects them on the host with QL_E_ARG
+    or QL_E_UNSUPPORTED (never QL_OK, never a crash), whatever else is wrong."""
+    hyp = pytest.importorskip("hypothesis")
+    st = pytest.importorskip("hypothesis.strategies")
+    lib = tcm.raw_library()
+    bad = {tcm.QL_E_ARG, tcm.QL_E_UNSUPPORTED}
+
+    @hyp.settings(max_examples=400, deadline=None, derandomize=True)
+    @hyp.given(m=st.integers(-16, 1 << 20), n=st.integers(-256, 1 << 20), k=st.integers(-1, 6),
+               L=st.integers(-1, 18), V=st.integers(0, 3), kind=st.integers(-1, 4), Q=st.integers(-1, 11),
+               nparts=st.integers(0, 9), kv=st.lists(st.integers(-1, 10), min_size=9, max_size=9),
+               rows=st.lists(st.integers(-16, 4096), min_size=9, max_size=9), exact=st.booleans())
+    def check(m, n, k, L, V, kind, Q, nparts, kv, rows, exact):
+        code = tcm.ql_code_t(kind, Q, None)
+        h = ctypes.c_void_p()
+        nw = (m * n * max(k, 0)) // 32 if exact and m > 0 and n > 0 else 7
+        assert lib.qlinear_create(ctypes.byref(h), m, n, k, L, V, code, None, max(nw, 0), None, None, 1.0) in bad
+        r = (ctypes.c_int * 9)(*rows)
+        kvs = (ctypes.c_int * 9)(*kv)
+        tot = sum(max(x, 0) * max(n, 0) // max(V, 1) * max(y, 0) for x, y in zip(rows[:nparts], kv[:nparts])) // 32
+        nw2 = tot if exact else 7
+        assert lib.qlinear_create_kv(ctypes.byref(h), sum(rows[:nparts]), n, nparts, r, kvs, L, V, code, None,
+                                     max(nw2, 0), None, None, 1.0) in bad
+        assert lib.qlinear_create_parts(ctypes.byref(h), sum(rows[:nparts]), n, nparts, r, kvs, L, V, code, None,
+                                        max(nw2, 0), None, None, 1.0) in bad
+        assert h.value is None
+
+    check()
