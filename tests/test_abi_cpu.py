@@ -224,3 +224,25 @@ def test_host_validation_never_accepts_null_buffers(tcm):
         assert h.value is None
 
     check()
+
+
+def test_encode_and_eval_validation_never_accept_null_buffers(tcm):
+    """Random encoder and code-evaluation arguments with null device buffers:
+    rejected on the host (QL_E_ARG / QL_E_UNSUPPORTED), or QL_OK only when
+    there is nothing to do (zero blocks or states) and the arguments are valid."""
+    hyp = pytest.importorskip("hypothesis")
+    st = pytest.importorskip("hypothesis.strategies")
+    lib = tcm.raw_library()
+    rejected = {tcm.QL_E_ARG, tcm.QL_E_UNSUPPORTED}
+
+    @hyp.settings(max_examples=400, deadline=None, derandomize=True)
+    @hyp.given(L=st.integers(-1, 18), kv=st.integers(-1, 10), k=st.integers(-1, 6), V=st.integers(0, 3),
+               kind=st.integers(-1, 4), Q=st.integers(-1, 11), count=st.integers(-2, 5))
+    def check(L, kv, k, V, kind, Q, count):
+        code = tcm.ql_code_t(kind, Q, None)
+        for rc in (lib.qlinear_encode_kv(code, L, kv, V, None, count, None, None, None),
+                   lib.qlinear_encode(code, L, k, V, None, count, None, None, None),
+                   lib.qlinear_eval_code(code, L, V, None, count, None, None)):
+            assert rc in rejected or (rc == tcm.QL_OK and count == 0)
+
+    check()
