@@ -32,16 +32,20 @@ def dense(B: int, normalised: bool = True, rows=None) -> np.ndarray:
     return H / np.sqrt(B) if normalised else H
 
 
-def apply_blockwise(v: np.ndarray, B: int, chunk_rows: int = 1024) -> np.ndarray:
-    """(I (x) H_B) applied along the last axis of v (float64), naive dense products."""
+def apply_blockwise(v: np.ndarray, B: int) -> np.ndarray:
+    """(I (x) H_B) applied along the last axis of v, in float64.
+
+    Output entry i of a block is the sum over j of H_B[i][j] * v[j], accumulated
+    in the order j = 0, 1, ..., B-1; column j of H_B is taken from the closed
+    form (H_B is symmetric, so it is row j)."""
     v = np.asarray(v, dtype=np.float64)
     d = v.shape[-1]
     assert d % B == 0
     blocks = v.reshape(v.shape[:-1] + (d // B, B))
-    out = np.empty_like(blocks)
-    for r0 in range(0, B, chunk_rows):
-        Hr = dense(B, rows=np.arange(r0, min(B, r0 + chunk_rows)))  # [rows, B]
-        out[..., r0:r0 + Hr.shape[0]] = blocks @ Hr.T
+    out = np.zeros_like(blocks)
+    for j in range(B):
+        col = dense(B, rows=[j])[0]
+        out += blocks[..., j:j + 1] * col
     return out.reshape(v.shape)
 
 

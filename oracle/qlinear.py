@@ -9,8 +9,8 @@ the V consecutive columns t*V .. t*V+V-1 of its block).  Each value is rounded
 once to fp16; the decoded matrix is the fp16 matrix the layer multiplies by.
 
 Every step is a plain dense computation in float64: the trellis walk state by
-state, the code on each state, the dense Hadamard blocks built explicitly,
-and a library matrix product for the contraction.
+state, the code on each state, the dense Hadamard blocks built explicitly, and
+the contraction as a sum of products accumulated column by column.
 """
 from __future__ import annotations
 
@@ -71,6 +71,20 @@ class Layer:
         x64 = np.asarray(x).astype(np.float64)
         return hadamard.rht(x64, self.s_in, self.B_n)
 
+    def contract(self, xp, rows) -> np.ndarray:
+        """z = W_hat x' at the listed rows, float64 [batch, len(rows)]: entry
+        (b, r) is the sum over columns c of W_hat[r][c] * x'[b][c], accumulated
+        in the order c = 0, 1, ..., n-1."""
+        return contract(self.decode_rows(rows), xp)
+
+    def output_transform(self, z, rows) -> np.ndarray:
+        """y = alpha * s_out * (H_m z) on whole output Hadamard blocks: `rows`
+        lists the blocks' rows in order and z holds W_hat x' on them."""
+        rows = np.asarray(rows, dtype=np.int64)
+        assert len(rows) % self.B_m == 0 and np.all(rows[::self.B_m] % self.B_m == 0)
+        yb = hadamard.apply_blockwise(z, self.B_m)  # H_m^T = H_m (symmetric)
+        return self.alpha * self.s_out[rows].astype(np.float64) * yb
+
     def forward_blocks(self, x, out_blocks) -> dict:
         """y on whole output Hadamard blocks: {block index: float64 [batch, B_m]}."""
         xp = self.input_transform(x)
@@ -78,10 +92,7 @@ class Layer:
         out = {}
         for b in out_blocks:
             rows = np.arange(b * Bm, (b + 1) * Bm)
-            W = self.decode_rows(rows)                  # [B_m, n]
-            z = xp @ W.T                                # [batch, B_m]
-            yb = hadamard.apply_blockwise(z, Bm)        # H_m^T = H_m (symmetric)
-            out[b] = self.alpha * self.s_out[rows].astype(np.float64) * yb
+            out[b] = self.output_transform(self.contract(xp, rows), rows)
         return out
 
     def forward(self, x) -> np.ndarray:
@@ -95,3 +106,15 @@ class Layer:
         Bm = self.B_m
         blocks = self.forward_blocks(x, sorted(set((rows // Bm).tolist())))
         return np.stack([blocks[r // Bm][:, r % Bm] for r in rows], axis=1)
+
+
+def contract(W, xp) -> np.ndarray:
+    """z[b][r] = sum over c of W[r][c] * xp[b][c], float64, accumulated column by
+    column in order (W: [rows, n], xp: [batch, n])."""
+    W = np.asarray(W, dtype=np.float64)
+    xp = np.asarray(xp, dtype=np.float64)
+    Wt = np.ascontiguousarray(W.T)   # column c of W as a contiguous vector
+    z = np.zeros((xp.shape[0], W.shape[0]))
+    for c in range(W.shape[1]):
+        z += xp[:, c:c + 1] * Wt[c]
+    return z

@@ -63,9 +63,12 @@ def test_blockwise_equals_kronecker_and_preserves_norm():
     assert np.allclose(back, v, atol=1e-12)
 
 
-def test_chunked_apply_matches_unchunked():
+def test_blockwise_apply_equals_the_dense_product():
+    """The ordered accumulation equals the dense matrix product (H_2048 built
+    by the Sylvester recursion, not the closed form) on random input."""
     rng = np.random.default_rng(1)
-    v = rng.standard_normal((2, 2048))
-    a = hadamard.apply_blockwise(v, 2048, chunk_rows=300)
-    b = v @ hadamard.dense(2048).T
+    v = rng.standard_normal((2, 4096))
+    a = hadamard.apply_blockwise(v, 2048)
+    H = _sylvester(2048) / np.sqrt(2048)
+    b = np.concatenate([v[:, :2048] @ H.T, v[:, 2048:] @ H.T], axis=1)
     assert np.allclose(a, b, atol=1e-12)
