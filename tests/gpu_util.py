@@ -39,14 +39,3 @@ def make_handle(li: wl.LayerInputs):
 def rel_err(y, y_ref):
     y = np.asarray(y, dtype=np.float64)
     return float(np.max(np.abs(y - y_ref)) / np.max(np.abs(y_ref)))
-
-
-def sample_rows(m, B_m, count, seed):
-    """Output rows to check on a full-size layer: the first and last row, and a
-    few random ones, restricted to at most `count` Hadamard blocks."""
-    rng = np.random.default_rng(seed)
-    blocks = sorted(set([0, m // B_m - 1] + list(rng.integers(0, m // B_m, max(count - 2, 0)))))[:count]
-    rows = []
-    for b in blocks:
-        rows += [b * B_m, b * B_m + B_m - 1] + list(b * B_m + rng.integers(0, B_m, 6))
-    return np.array(sorted(set(rows)))

@@ -18,7 +18,7 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only ho
 import trellis_coded_matmul_b200 as tcm  # noqa: E402
 import workloads as wl  # noqa: E402
 from oracle import codes as ocodes, fp16 as ofp16, qlinear as oq  # noqa: E402
-from gpu_util import TOL_GEMV, TOL_TC, make_handle, rel_err, sample_rows  # noqa: E402
+from gpu_util import TOL_GEMV, TOL_TC, make_handle, rel_err  # noqa: E402
 
 
 def _bits(t):
@@ -115,34 +115,3 @@ def test_fractional_create_rejects_bad_bitrates():
     with pytest.raises(tcm.QLinearError) as e:  # a 2^10-entry codebook is over the limit
         tcm.qlinear_create_kv(48, 512, [48], [5], 10, 2, wl.CODE_TABLE, codes, s_in, s_out, 1.0, lut=lut)
     assert e.value.status == tcm.QL_E_UNSUPPORTED
-
-
-# ---------------------------------------------------------------- full-size palette layers
-PALETTE_FULL = ["tcq2p5", "tcq2p75", "vq2p5", "nuq3"]
-
-
-@pytest.mark.parametrize("name", PALETTE_FULL)
-def test_palette_full_decode_sampled_rows_bit_exact(name):
-    sp = wl.WORKLOADS[name]
-    li = wl.make_layer(sp)
-    h = make_handle(li)
-    w = tcm.qlinear_decode(h)
-    rng = np.random.default_rng(7)
-    bounds = [r0 for r0, _, _ in sp.row_parts()[1:]]
-    rows = np.unique(np.concatenate([[0, sp.m - 1], rng.integers(0, sp.m, 10),
-                                     [b - 1 for b in bounds] + bounds])).astype(np.int64)
-    got = _bits(w[torch.from_numpy(rows).cuda()])
-    assert np.array_equal(got, oq.Layer.from_inputs(li).decode_bits(rows))
-
-
-@pytest.mark.parametrize("name", PALETTE_FULL)
-@pytest.mark.parametrize("batch", [1, 8, 64])
-def test_palette_full_forward_sampled_outputs(name, batch):
-    sp = wl.WORKLOADS[name]
-    li = wl.make_layer(sp)
-    h = make_handle(li)
-    x = wl.make_x(sp, batch)
-    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda()).cpu().numpy()
-    layer = oq.Layer.from_inputs(li)
-    rows = sample_rows(sp.m, layer.B_m, 1, seed=batch)
-    assert rel_err(y[:, rows], layer.forward_rows(x, rows)) <= (TOL_GEMV if batch <= 8 else TOL_TC)

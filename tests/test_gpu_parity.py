@@ -16,7 +16,7 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only ho
 import trellis_coded_matmul_b200 as tcm  # noqa: E402
 import workloads as wl  # noqa: E402
 from oracle import codes as ocodes, fp16 as ofp16, qlinear as oq  # noqa: E402
-from gpu_util import TOL_GEMV, TOL_TC, make_handle, rel_err, sample_rows  # noqa: E402
+from gpu_util import TOL_GEMV, TOL_TC, make_handle, rel_err  # noqa: E402
 
 L16 = 1 << 16
 
@@ -164,40 +164,6 @@ def test_info_reports_the_bit_accounting():
     assert info["sign_bytes"] * 8 >= sp.m + sp.n and info["sign_bytes"] * 8 < sp.m + sp.n + 64
     assert info["lut_bytes"] == 2048
     assert (info["B_n"], info["B_m"]) == (4096, 256)
-
-
-# ---------------------------------------------------------------- full-size workloads
-FULL = [("tiny", 1), ("attn4096", 1), ("mlp_up", 8), ("mlp_down", 4), ("large", 4), ("large", 16),
-        ("halftcq", 64), ("halftcq", 256), ("qkv_fused", 1), ("qkv_fused", 16)]
-
-
-@pytest.mark.parametrize("name", ["tiny", "attn4096", "mlp_up", "mlp_down", "large", "halftcq", "qkv_fused"])
-def test_full_decode_sampled_rows_bit_exact(name):
-    sp = wl.WORKLOADS[name]
-    li = wl.make_layer(sp)
-    h = make_handle(li)
-    w = tcm.qlinear_decode(h)
-    rng = np.random.default_rng(42)
-    bounds = [r0 for r0, _, _ in sp.row_parts()[1:]]  # first rows of the later parts
-    rows = np.unique(np.concatenate([[0, sp.m - 1], rng.integers(0, sp.m, 10),
-                                     [b - 1 for b in bounds] + bounds])).astype(np.int64)
-    ref = oq.Layer.from_inputs(li).decode_bits(rows)
-    got = _bits(w[torch.from_numpy(rows).cuda()])
-    assert np.array_equal(got, ref)
-
-
-@pytest.mark.parametrize("name,batch", FULL, ids=lambda v: str(v))
-def test_full_forward_sampled_outputs(name, batch):
-    sp = wl.WORKLOADS[name]
-    li = wl.make_layer(sp)
-    h = make_handle(li)
-    x = wl.make_x(sp, batch)
-    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda()).cpu().numpy()
-    layer = oq.Layer.from_inputs(li)
-    rows = sample_rows(sp.m, layer.B_m, 1 if layer.B_m >= 4096 else 3, seed=batch)
-    y_ref = layer.forward_rows(x, rows)
-    tol = TOL_GEMV if batch <= 8 else TOL_TC
-    assert rel_err(y[:, rows], y_ref) <= tol
 
 
 def test_forward_in_cuda_graph_with_profiling():
