@@ -54,10 +54,15 @@ def parse_args():
     p.add_argument("--batch", type=int, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="skip the per-configuration measurements of every benchmark (workload, batch) pair")
     p.add_argument("--encode", action="store_true",
                    help="time the trellis-coded quantizer (qlinear_encode, k = 2, 3INST) on an N(0,1) "
                         "source instead of the forward")
     p.add_argument("--encode-L", type=int, default=16, help="state bits of the --encode run (at most 16)")
+    p.add_argument("--record-counters", nargs=3, metavar=("NCU_CSV", "KEY", "CAPTURE"),
+                   help="store the counters of an ncu --csv log in profiles/counters.json under KEY (e.g. "
+                        "gemv_attn4096_b1) and exit; CAPTURE names the profile that gives the command")
     p.add_argument("--instances", type=int, default=None,
                    help="layer instances to rotate through (default: enough code words for 4x L2); a smaller "
                         "count is for profiler captures only, and the line then says its inputs may sit in L2")
@@ -157,7 +162,7 @@ def _oracle_chunked(sp, batch, blocks_per_step, steps, deadline=None):
             r, j0 = divmod(pos, nb)
             j1 = min(nb, j0 + left)
             W = layer.decode_rows([r], np.arange(j0, j1))
-            z[:, r] += xp[:, j0 * 256:j1 * 256] @ W[0]
+            z[:, r] += qlinear.contract(W, xp[:, j0 * 256:j1 * 256])[:, 0]
             left -= j1 - j0
             pos += j1 - j0
             done += j1 - j0
@@ -171,19 +176,11 @@ def _oracle_chunked(sp, batch, blocks_per_step, steps, deadline=None):
     return time.perf_counter() - t0, done
 
 
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    except Exception:
-        return 1
-
-
 def cpu_baseline(sp, batch, budget_s=15.0):
     nb = sp.n // 256
     secs, blocks = _oracle_chunked(sp, batch, 16 * nb, steps=10**9, deadline=budget_s)
     fwd = blocks / (sp.m * nb)
-    return {"value": batch * fwd / secs, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+    return {"value": batch * fwd / secs, "unit": "tokens/s", "cores": 1, "cpu_model": _cpu_model(), "kind": "oracle",
             "sample": f"{blocks // nb} of {sp.m} rows of W_hat ({fwd:.3f} forwards) of {sp.name} at batch {batch}: "
                       f"float64 trellis walk, code evaluation, dense Hadamard blocks, matrix product; "
                       f"{secs:.1f} s"}
@@ -212,7 +209,7 @@ def run_reference(args):
                                                  "step": f"{bps} blocks of 256 columns of W_hat per step "
                                                          f"(1/{sp.m * nb / bps:g} of a forward)"}),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "cpu_model": _cpu_model(), "kind": "oracle",
                              "sample": f"{done} blocks of 256 columns of W_hat in {args.steps} steps of {bps}"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -256,16 +253,39 @@ def _source_hash(kind):
     return h.hexdigest()[:16]
 
 
-def _traffic(kernel_key, launch_units):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current sources of that kernel; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
-        return None
-    d = json.load(open(path)).get(kernel_key)
-    if not d or d.get("source_hash") != _source_hash(kernel_key.split("_")[0]):
-        return None
-    return d["dram_bytes"] * launch_units / d["units"]
+_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "inst": 1, "": 1, "nsecond": 1e-9,
+          "usecond": 1e-6, "msecond": 1e-3}
+_COUNTER_METRICS = {"dram__bytes_read.sum": "dram_read", "dram__bytes_write.sum": "dram_write",
+                    "smsp__inst_executed.sum": "warp_inst", "smsp__thread_inst_executed.sum": "thread_inst",
+                    "gpu__time_duration.sum": "duration_s"}
+
+
+def record_counters(csv_path, key, capture):
+    """Store the counters of the first kernel launch in an ncu --csv log under
+    `key` in profiles/counters.json, stamped with the hash of that kernel's
+    sources (bench.py reports them only while the sources are unchanged)."""
+    import csv
+    rows = list(csv.reader(l for l in open(csv_path) if l.startswith('"')))
+    head = rows[0]
+    iid, iname, iunit, ival = (head.index(c) for c in ("ID", "Metric Name", "Metric Unit", "Metric Value"))
+    first = rows[1][iid]
+    vals = {}
+    for r in rows[1:]:
+        if r[iid] != first or r[iname] not in _COUNTER_METRICS:
+            continue
+        vals[_COUNTER_METRICS[r[iname]]] = float(r[ival].replace(",", "")) * _UNITS[r[iunit]]
+    entry = {"dram_bytes": vals.get("dram_read", 0) + vals.get("dram_write", 0),
+             "warp_inst": vals.get("warp_inst"), "thread_inst": vals.get("thread_inst"),
+             "duration_us_ncu": vals.get("duration_s", 0) * 1e6,
+             "source_hash": _source_hash(key.split("_")[0]), "capture": capture}
+    path = os.path.join(ROOT, "profiles", "counters.json")
+    d = json.load(open(path)) if os.path.exists(path) else {
+        "_note": "per-launch counters of one ncu capture per kernel and workload (dram bytes read + written, warp "
+                 "and thread instructions executed); bench.py uses an entry only while the kernel's sources hash "
+                 "to its source_hash"}
+    d[key] = entry
+    json.dump(d, open(path, "w"), indent=1, sort_keys=True)
+    print(json.dumps({key: entry}))
 
 
 def run_encode(args):
@@ -332,6 +352,223 @@ def run_encode(args):
     return 0
 
 
+# The (workload, batch) pairs the layer shapes are benchmarked at: the five
+# layer configurations of the workload list with their batches.
+PER_CONFIG = [("tiny", 1), ("attn4096", 1), ("mlp_up", 1), ("mlp_up", 4), ("mlp_up", 8), ("mlp_down", 1),
+              ("mlp_down", 4), ("mlp_down", 8), ("large", 1), ("large", 4), ("large", 16), ("halftcq", 64),
+              ("halftcq", 256)]
+
+
+def _counters(key):
+    """Per-launch counters of the kernel `key` from the committed ncu summary
+    (profiles/counters.json), if they were taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "counters.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(key)
+    if not d or d.get("source_hash") != _source_hash(key.split("_")[0]):
+        return None
+    return d
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def make_handle(tcm, torch, li):
+    sp_ = li.spec
+    codes = torch.from_numpy(li.codes.view(np.int32).copy()).cuda()
+    s_in = torch.from_numpy(li.s_in.copy()).cuda()
+    s_out = torch.from_numpy(li.s_out.copy()).cuda()
+    lut = torch.from_numpy(li.lut.copy()).cuda() if li.lut is not None else None
+    if sp_.fractional:  # a half-integer bitwidth: parts given as bits per trellis step
+        return tcm.qlinear_create_kv(sp_.m, sp_.n, [r for _, r, _ in sp_.row_parts()], sp_.part_kv(), sp_.L,
+                                     sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
+    if sp_.row_split is not None:
+        return tcm.qlinear_create_parts(sp_.m, sp_.n, [r for r, _ in sp_.row_split], [k for _, k in sp_.row_split],
+                                        sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
+    if sp_.mixed:
+        return tcm.qlinear_create_mixed(sp_.m, sp_.n, sp_.m_top, sp_.k_top, sp_.k_bot, sp_.L, sp_.V, sp_.code,
+                                        codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
+    return tcm.qlinear_create(sp_.m, sp_.n, sp_.k, sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha,
+                              Q=sp_.Q, lut=lut)
+
+
+class Runner:
+    """Times forwards of one workload at one batch on this rank's GPU: steps
+    rotate through enough independent layer instances that their code words
+    exceed four times the L2 (replayed from CUDA graphs), and a separate replay
+    with CUDA events around the layer's main kernel gives its duration."""
+
+    def __init__(self, torch, tcm, dist, world, rank, stream, sp, batch, n_inst):
+        self.torch, self.tcm, self.dist, self.world = torch, tcm, dist, world
+        self.stream, self.sp, self.batch, self.n_inst = stream, sp, batch, n_inst
+        self.handles = [make_handle(tcm, torch, wl.make_layer(sp, instance=1 + rank * 4096 + i)) for i in range(n_inst)]
+        self.xs = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).cuda() for i in range(n_inst)]
+        self.ys = [torch.empty((batch, sp.m), dtype=torch.float32, device="cuda") for _ in range(n_inst)]
+        self.graphs = []
+        with torch.cuda.stream(stream):
+            self.run_steps(n_inst)  # allocate per-handle scratch before capture
+        torch.cuda.synchronize()
+
+    def run_steps(self, count, start=0):
+        for s in range(start, start + count):
+            i = s % self.n_inst
+            self.tcm.qlinear_forward(self.handles[i], self.xs[i], self.ys[i])
+
+    def capture(self, count):
+        if count == 0:
+            return None
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, stream=self.stream):
+            self.run_steps(count)
+        self.graphs.append(g)
+        return g
+
+    def replay(self, steps, full, tail):
+        for _ in range(steps // self.n_inst):
+            full.replay()
+        if steps % self.n_inst:
+            tail.replay()
+
+    def timed(self, fn):
+        torch, dist = self.torch, self.dist
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if self.world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            start.record(self.stream)
+            fn()
+            end.record(self.stream)
+        torch.cuda.synchronize()
+        if self.world > 1:
+            dist.barrier()
+        return start.elapsed_time(end) * 1e-3
+
+    def throughput(self, steps, warmup):
+        """Seconds for `steps` forwards after `warmup` untimed ones."""
+        g_full, g_tail, g_warm = self.capture(self.n_inst), self.capture(steps % self.n_inst), \
+            self.capture(warmup % self.n_inst)
+        with self.torch.cuda.stream(self.stream):
+            self.replay(warmup, g_full, g_warm)
+        return self.timed(lambda: self.replay(steps, g_full, g_tail))
+
+    def kernel_seconds(self, steps):
+        """Average duration of the main kernel (decode-GEMV or tensor-core GEMM):
+        the same steps again from a graph whose forwards carry CUDA events
+        around that kernel (events between programmatically dependent launches
+        serialise them, so this pass is separate from the throughput one)."""
+        tcm = self.tcm
+        for h in self.handles:
+            tcm.qlinear_profile_enable(h, 1)
+        prof_steps = min(steps, 4 * self.n_inst)
+        g_prof, g_tail = self.capture(self.n_inst), self.capture(prof_steps % self.n_inst)
+        with self.torch.cuda.stream(self.stream):
+            g_prof.replay()
+        prof_secs = self.timed(lambda: self.replay(prof_steps, g_prof, g_tail))
+        ms, n = 0.0, 0
+        for h in self.handles:
+            a, b = tcm.qlinear_profile_read(h)
+            ms += a
+            n += b
+            tcm.qlinear_profile_enable(h, 0)
+        return ms * 1e-3 / max(1, n), prof_steps, prof_secs
+
+    def e2e(self, steps):
+        """Seconds for `steps` forwards through qlinear_forward_host (pinned host
+        x in, host y out, copies and the stream synchronisation in every step)."""
+        torch, tcm, sp, batch = self.torch, self.tcm, self.sp, self.batch
+        x_h = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).pin_memory() for i in range(4)]
+        y_h = [torch.empty((batch, sp.m), dtype=torch.float32).pin_memory() for _ in range(4)]
+        with torch.cuda.stream(self.stream):
+            for s in range(8):
+                tcm.qlinear_forward_host(self.handles[s % self.n_inst], x_h[s % 4], y_h[s % 4], stream=self.stream)
+
+        def body():
+            for s in range(steps):
+                tcm.qlinear_forward_host(self.handles[s % self.n_inst], x_h[s % 4], y_h[s % 4], stream=self.stream)
+        return self.timed(body)
+
+    def cold_call_us(self):
+        """Latency of one forward whose code words are not in L2 (a buffer of
+        twice the L2 size is written first), median of 3; None if it fails."""
+        torch = self.torch
+        try:
+            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            out = []
+            with torch.cuda.stream(self.stream):
+                for i in range(3):
+                    flush.zero_()
+                    ev0.record(self.stream)
+                    j = i % self.n_inst
+                    self.tcm.qlinear_forward(self.handles[j], self.xs[j], self.ys[j])
+                    ev1.record(self.stream)
+                    torch.cuda.synchronize()
+                    out.append(ev0.elapsed_time(ev1) * 1e3)
+            del flush
+            return statistics.median(out)
+        except Exception:
+            return None
+
+    def close(self):
+        for h in self.handles:
+            self.tcm.qlinear_destroy(h)
+        self.handles = []
+        self.graphs = []
+
+
+def n_instances(sp, override=None):
+    n = int(min(512, max(1, math.ceil(4 * L2_BYTES / sp.stream_bytes))))
+    return max(1, min(n, override)) if override else n
+
+
+def roofline(sp, batch, kern_s, pk, pk_kind, clk_mhz, sms, timing, burst_gemm):
+    """The main kernel's roofline: HBM on the algorithmic bytes (decode-GEMV,
+    batch <= 8) or the dense tensor rate (tensor-core GEMM), plus the issue
+    fraction from the committed instruction counters when they are current."""
+    weights = sp.m * sp.n
+    if batch <= GEMV_MAX_BATCH:
+        key = f"gemv_{sp.name}_b{batch}"
+        alg_bytes = sp.stream_bytes + batch * sp.n * 2 + batch * sp.m * 4
+        achieved = alg_bytes / kern_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "kernel": "trellis_gemv_kernel (fused trellis decode + MMA)",
+                "peak_kind": pk_kind + " hbm_gbs (copy)", "alg_bytes_per_launch": alg_bytes}
+    else:
+        key = f"gemm_{sp.name}_b{batch}"
+        flops = 2.0 * sp.m * sp.n * batch
+        achieved = flops / kern_s / 1e12
+        peak = pk["bf16_tflops"] if burst_gemm else pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "kernel": "trellis_gemm_kernel (trellis decode into tensor memory + tcgen05 MMA, fp16 in, "
+                          "fp32 accumulate)",
+                "peak_kind": pk_kind + (" bf16_tflops (burst: the kernel is timed in a sub-second loop)" if burst_gemm
+                                        else " bf16_tflops_sustained (seconds-long loop)")
+                + "; the fp16 dense rate equals the bf16 one",
+                "alg_flops_per_launch": flops}
+    c = _counters(key)
+    roof["traffic"] = c["dram_bytes"] if c else None
+    roof["kernel_us"] = kern_s * 1e6
+    roof["timing"] = timing
+    if c and c.get("warp_inst"):
+        roof["warp_inst_per_launch"] = c["warp_inst"]
+        roof["lane_inst_per_weight"] = c["thread_inst"] / weights
+        roof["issue_frac"] = c["warp_inst"] / kern_s / (sms * 4 * clk_mhz * 1e6)
+        roof["issue_note"] = (f"warp instructions per launch (ncu) / kernel time / ({sms} SMs x 4 issue slots x "
+                              f"{clk_mhz:.0f} MHz sampled)")
+    else:
+        roof["issue_frac"] = None
+    return roof
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -348,171 +585,68 @@ def run_ours(args):
 
     import trellis_coded_matmul_b200 as tcm
 
-    def make_handle(li):
-        sp_ = li.spec
-        codes = torch.from_numpy(li.codes.view(np.int32).copy()).cuda()
-        s_in = torch.from_numpy(li.s_in.copy()).cuda()
-        s_out = torch.from_numpy(li.s_out.copy()).cuda()
-        lut = torch.from_numpy(li.lut.copy()).cuda() if li.lut is not None else None
-        if sp_.fractional:  # a half-integer bitwidth: parts given as bits per trellis step
-            return tcm.qlinear_create_kv(sp_.m, sp_.n, [r for _, r, _ in sp_.row_parts()], sp_.part_kv(), sp_.L,
-                                         sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
-        if sp_.row_split is not None:
-            return tcm.qlinear_create_parts(sp_.m, sp_.n, [r for r, _ in sp_.row_split], [k for _, k in sp_.row_split],
-                                            sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
-        if sp_.mixed:
-            return tcm.qlinear_create_mixed(sp_.m, sp_.n, sp_.m_top, sp_.k_top, sp_.k_bot, sp_.L, sp_.V, sp_.code,
-                                            codes, s_in, s_out, sp_.alpha, Q=sp_.Q, lut=lut)
-        return tcm.qlinear_create(sp_.m, sp_.n, sp_.k, sp_.L, sp_.V, sp_.code, codes, s_in, s_out, sp_.alpha,
-                                  Q=sp_.Q, lut=lut)
-
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    stream = torch.cuda.Stream()
+    pk, pk_kind = peaks()
     sp = wl.WORKLOADS[args.workload]
     batch = args.batch or sp.batches[0]
-    n_inst = int(min(512, max(1, math.ceil(4 * L2_BYTES / sp.stream_bytes))))
-    if args.instances:
-        n_inst = max(1, min(n_inst, args.instances))
-    handles = [make_handle(wl.make_layer(sp, instance=1 + rank * 4096 + i)) for i in range(n_inst)]
-    xs = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).cuda() for i in range(n_inst)]
-    ys = [torch.empty((batch, sp.m), dtype=torch.float32, device="cuda") for _ in range(n_inst)]
-    stream = torch.cuda.Stream()
-
-    def run_steps(count, start=0):
-        for s in range(start, start + count):
-            i = s % n_inst
-            tcm.qlinear_forward(handles[i], xs[i], ys[i])
-
-    def capture(count):
-        if count == 0:
-            return None
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            run_steps(count)
-        return g
-
-    with torch.cuda.stream(stream):
-        run_steps(n_inst)  # allocate per-handle scratch before capture
-    torch.cuda.synchronize()
-    g_full, g_tail, g_warm = capture(n_inst), capture(args.steps % n_inst), capture(args.warmup % n_inst)
-
-    def replay(steps, full, tail_graph):
-        for _ in range(steps // n_inst):
-            full.replay()
-        if steps % n_inst:
-            tail_graph.replay()
-
-    def timed(fn):
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            fn()
-            end.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return start.elapsed_time(end) * 1e-3
+    n_inst = n_instances(sp, args.instances)
+    r = Runner(torch, tcm, dist, world, rank, stream, sp, batch, n_inst)
 
     clocks = ClockSampler(local)
-    with torch.cuda.stream(stream):
-        replay(args.warmup, g_full, g_warm)
-    secs = timed(lambda: replay(args.steps, g_full, g_tail))
+    secs = r.throughput(args.steps, args.warmup)
     clk = clocks.stop()
-
-    # The decode-GEMV kernel's own duration: the same steps again, from a graph
-    # whose forwards carry CUDA events around that kernel (events between
-    # programmatically dependent launches serialise them, so this pass is
-    # separate from the throughput measurement above).
-    for h in handles:
-        tcm.qlinear_profile_enable(h, 1)
-    prof_steps = min(args.steps, 4 * n_inst)
-    g_prof = capture(n_inst)
-    g_prof_tail = capture(prof_steps % n_inst)
-    with torch.cuda.stream(stream):
-        g_prof.replay()
-    prof_secs = timed(lambda: replay(prof_steps, g_prof, g_prof_tail))
-    kern_ms, kern_n = 0.0, 0
-    for h in handles:
-        ms, n = tcm.qlinear_profile_read(h)
-        kern_ms += ms
-        kern_n += n
-        tcm.qlinear_profile_enable(h, 0)
-    kern_s = kern_ms * 1e-3 / max(1, kern_n)
+    kern_s, prof_steps, prof_secs = r.kernel_seconds(args.steps)
     if world > 1:
         secs, kern_s = max_over_ranks([secs, kern_s], "cuda")
-
-    # end to end through the public API with host buffers (pinned)
     e2e = None
     if not args.no_e2e:
-        x_h = [torch.from_numpy(wl.make_x(sp, batch, instance=i)).pin_memory() for i in range(4)]
-        y_h = [torch.empty((batch, sp.m), dtype=torch.float32).pin_memory() for _ in range(4)]
         e2e_steps = min(args.steps, 2000)
-        with torch.cuda.stream(stream):
-            for s in range(8):
-                tcm.qlinear_forward_host(handles[s % n_inst], x_h[s % 4], y_h[s % 4], stream=stream)
-        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        es.record(stream)
-        for s in range(e2e_steps):
-            tcm.qlinear_forward_host(handles[s % n_inst], x_h[s % 4], y_h[s % 4], stream=stream)
-        ee.record(stream)
-        torch.cuda.synchronize()
-        e2e_s = es.elapsed_time(ee) * 1e-3
+        e2e_s = r.e2e(e2e_steps)
         if world > 1:
             e2e_s = max_over_ranks([e2e_s], "cuda")[0]
         e2e = {"value": job_tokens_per_s(world, e2e_steps, batch, e2e_s), "unit": "tokens/s",
                "h2d_bytes_per_step": batch * sp.n * 2, "d2h_bytes_per_step": batch * sp.m * 4,
                "steps": e2e_steps}
+    cold = r.cold_call_us() if rank == 0 else None  # rank 0 only, no collective inside
+    launches_per_step = tcm.qlinear_info(r.handles[0])["last_launches"]
+    r.close()
+    clk_mhz = (clk or {}).get("sm_mhz") or 1965.0
 
-    def cold_call_us():
-        """Latency of one forward whose code words are not in L2 (a buffer of
-        twice the L2 size is written first), median of 3; None if it fails."""
-        try:
-            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            out = []
-            with torch.cuda.stream(stream):
-                for i in range(3):
-                    flush.zero_()
-                    ev0.record(stream)
-                    tcm.qlinear_forward(handles[i % n_inst], xs[i % n_inst], ys[i % n_inst])
-                    ev1.record(stream)
-                    torch.cuda.synchronize()
-                    out.append(ev0.elapsed_time(ev1) * 1e3)
-            del flush
-            return statistics.median(out)
-        except Exception:
-            return None
+    # every benchmark configuration, each on its own rotating instances
+    per_config = None
+    if not args.no_per_config and not args.instances:
+        per_config = []
+        clocks_pc = ClockSampler(local)
+        for name, b in PER_CONFIG:
+            spc = wl.WORKLOADS[name]
+            ni = n_instances(spc)
+            rc = Runner(torch, tcm, dist, world, rank, stream, spc, b, ni)
+            steps_c = max(args.steps, 2 * ni, 200)
+            s_c = rc.throughput(steps_c, max(args.warmup, ni))
+            k_c, ps, pss = rc.kernel_seconds(steps_c)
+            if world > 1:
+                s_c, k_c = max_over_ranks([s_c, k_c], "cuda")
+            launches_c = tcm.qlinear_info(rc.handles[0])["last_launches"]
+            rc.close()
+            per_config.append({"workload": name, "batch": b, "steps": steps_c, "instances": ni,
+                               "ms_per_step": s_c / steps_c * 1e3,
+                               "tokens_per_s": job_tokens_per_s(world, steps_c, b, s_c),
+                               "stream_gbs_step": spc.stream_bytes * steps_c * world / s_c / 1e9,
+                               "launches_per_step": launches_c,
+                               "roofline": roofline(spc, b, k_c, pk, pk_kind, clk_mhz, sms,
+                                                    f"CUDA events around the kernel in a replay of {ps} steps",
+                                                    burst_gemm=True)})
+        clk_pc = clocks_pc.stop()
+        per_config.append({"clocks": clk_pc, "note": f"issue fractions use the headline run's median SM clock "
+                                                      f"({clk_mhz:.0f} MHz)"})
 
     line = None
     if rank == 0:
-        cold = cold_call_us()  # rank 0 only, no collective inside
-        pk, pk_kind = peaks()
         value = job_tokens_per_s(world, args.steps, batch, secs)
-        launches_per_step = tcm.qlinear_info(handles[0])["last_launches"]
         timing = (f"CUDA events around the kernel in a replay of {prof_steps} steps "
                   f"({prof_secs / prof_steps * 1e6:.2f} us/step with the events)")
-        if batch <= GEMV_MAX_BATCH:
-            alg_bytes = sp.stream_bytes + batch * sp.n * 2 + batch * sp.m * 4
-            achieved = alg_bytes / kern_s / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / pk["hbm_gbs"], "traffic": _traffic(f"gemv_{sp.name}_b{batch}", 1),
-                    "kernel": "gemv_kernel (fused trellis decode + m16n8k16 MMA)",
-                    "kernel_us": kern_s * 1e6, "peak_kind": pk_kind + " hbm_gbs (copy)",
-                    "alg_bytes_per_launch": alg_bytes, "timing": timing}
-        else:
-            flops = 2.0 * sp.m * sp.n * batch
-            achieved = flops / kern_s / 1e12
-            peak = pk["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": _traffic(f"gemm_{sp.name}_b{batch}", 1),
-                    "kernel": "gemm_tc_kernel (trellis decode into tensor memory + tcgen05 MMA, fp16 in, fp32 accumulate)",
-                    "kernel_us": kern_s * 1e6,
-                    "peak_kind": pk_kind + " bf16_tflops_sustained (fp16 dense rate = bf16 dense rate)",
-                    "alg_flops_per_launch": flops, "timing": timing}
+        roof = roofline(sp, batch, kern_s, pk, pk_kind, clk_mhz, sms, timing, burst_gemm=False)
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
@@ -521,13 +655,10 @@ def run_ours(args):
                 "cold_call_us": cold,
                 "roofline": roof,
                 "gpu_launches": launches_per_step * args.steps,
-                "clocks": clk, "e2e": e2e}
+                "clocks": clk, "e2e": e2e, "per_config": per_config}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(sp, batch)
         print(json.dumps(line), flush=True)
-    for h in handles:
-        tcm.qlinear_destroy(h)
-    del g_full, g_tail, g_warm, g_prof, g_prof_tail
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -536,6 +667,9 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.record_counters:
+        record_counters(*args.record_counters)
+        return 0
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
                "--master-addr", "127.0.0.1", "--master-port", "29517", __file__] + sys.argv[1:]

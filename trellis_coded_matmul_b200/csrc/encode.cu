@@ -18,13 +18,15 @@
 // for every group a, one minimum over its 2^kV predecessors (the choice h is
 // recorded per group), then the 2^kV successors' costs.
 //
-// Up to L = 14 one CTA encodes one block with both cost vectors and the code
-// values in its shared memory.  At L = 15 and 16 (the discussion's
-// experiments use L = 16) the 2^L states are split over a thread-block
-// cluster of 2 or 4 CTAs, 16384 states each: a CTA keeps its states' two cost
-// vectors and code values (fp16, which they are exactly) in its shared
-// memory, reads the predecessors' costs from the other CTAs' shared memory
-// (distributed shared memory), and the cluster synchronises once per step.
+// One CTA encodes one block whenever the group minima fit its shared memory
+// (every case but L = 16 with kV = 1): it stores only M_t(a) = min_h
+// cost_{t-1}(a + hG), 2^(L-kV) floats per buffer, and recomputes a state's
+// cost M_t(s >> kV) + d(t, s) when it reads it (the same float32 operations
+// as storing it), with the code values computed on the fly.  L = 16 with
+// kV = 1 splits the 2^16 states over a thread-block cluster of 4 CTAs,
+// 16384 states each, which keep their costs and code values (fp16, which they
+// are exactly) in shared memory and read the predecessors' costs from the
+// other CTAs' shared memory; the cluster synchronises once per step.
 #include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -38,7 +40,7 @@ namespace cg = cooperative_groups;
 namespace qlk {
 
 constexpr int kEncThreads = 1024;
-constexpr int kEncMaxL = 14;           // single-CTA kernel
+constexpr int kEncMaxL = 14;           // above: the cluster kernel when the group minima do not fit
 constexpr int kEncClusterStates = 16384;  // states per CTA of a cluster (L = 15, 16)
 
 struct EncodeArgs {
@@ -96,107 +98,121 @@ __device__ __forceinline__ void argmin_cta(float& val, int& idx, float* red_v, i
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(EncodeArgs p) {
-    extern __shared__ float esm[];
-    const int L = p.L, kV = p.kV, V = p.V;
-    const int S = 1 << L, G = S >> kV, C = 1 << kV;
-    const int T = 256 / V;
-    float* cost_a = esm;                // [S]
-    float* cost_b = cost_a + S;         // [S]
-    float* vals = cost_b + S;           // [S][V]
-    float* xs = vals + S * V;           // [256]
-    float* red_v = xs + 256;            // [32]
+// ---- group-minima search (one CTA per block): cost_t(s) = M_t(s >> kV) + d(t, s) ----
+// Only the group minima M_t(a) = min_h cost_{t-1}(a + hG) are stored (2^(L-kV)
+// floats per buffer); a state's cost is recomputed when it is read, with the
+// same float32 operations as the stored form, and the code values are
+// computed (or looked up in the replicated table) on the fly.
+// fp32 values of state s (V of them), fp16-exact
+template <int CODE, int V>
+__device__ __forceinline__ void values_of(uint32_t s, const uint32_t* lut_lane, int qshift, float (&v)[V]) {
+    uint32_t w;
+    if constexpr (V == 2) w = code_v2<CODE>(s, lut_lane, qshift);
+    else w = code_pair<CODE>(s, s, lut_lane, qshift);
+    v[0] = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
+    if constexpr (V == 2) v[1] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+
+template <int V>
+__device__ __forceinline__ float dist_of(const float* xt, const float (&v)[V]) {
+    const float d0 = __fsub_rn(xt[0], v[0]);
+    float d = __fmul_rn(d0, d0);
+    if constexpr (V == 2) {
+        const float d1 = __fsub_rn(xt[1], v[1]);
+        d = __fadd_rn(d, __fmul_rn(d1, d1));
+    }
+    return d;
+}
+
+template <int CODE, int KV, int V>
+__global__ void __launch_bounds__(1024, 1) encode_gm_kernel(EncodeArgs p) {
+    extern __shared__ __align__(16) unsigned char sm[];
+    constexpr int C = 1 << KV;
+    constexpr int T = 256 / V;
+    const int L = p.L;
+    const int S = 1 << L, G = S >> KV;  // p.kV == KV, p.V == V
+    const int qshift = 32 - p.Q;
+    float* Ma = reinterpret_cast<float*>(sm);
+    float* Mb = Ma + G;
+    float* xs = Mb + G;
+    float* red_v = xs + 256;
     int* red_i = reinterpret_cast<int*>(red_v + 32);
-    uint32_t* lut_smem = reinterpret_cast<uint32_t*>(red_i + 32);  // table codes: 2^Q x 32 replicated words
+    uint32_t* lut_smem = reinterpret_cast<uint32_t*>(red_i + 32);
     const int lane = threadIdx.x & 31;
-    if (uses_table(p.code))
+    if (uses_table(CODE))
         for (int i = threadIdx.x; i < (32 << p.Q); i += blockDim.x) lut_smem[i] = p.lut[i >> 5];
     __syncthreads();
     const uint32_t* lut_lane = lut_smem + lane;
-    for (int s = threadIdx.x; s < S; s += blockDim.x) {
-        float v[2];
-        code_values(p, lut_lane, (uint32_t)s, v);
-        for (int e = 0; e < V; ++e) vals[s * V + e] = v[e];
-    }
     uint8_t* choice = p.choice + (size_t)blockIdx.x * T * G;
     for (int blk = blockIdx.x; blk < p.blocks; blk += gridDim.x) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) xs[i] = p.x[(size_t)blk * 256 + i];
         __syncthreads();
-        // step cost of state s at step t (the float32 rule)
-        auto dist = [&](int t, int s) {
-            float d = 0.f;
-            for (int e = 0; e < V; ++e) {
-                const float diff = __fsub_rn(xs[t * V + e], vals[s * V + e]);
-                d = e ? __fadd_rn(d, __fmul_rn(diff, diff)) : __fmul_rn(diff, diff);
-            }
-            return d;
-        };
-        int prefix = 0;
-        int last = 0;
+        int prefix = 0, last = 0;
         for (int pass = 0; pass < 2; ++pass) {
-            float* old_c = cost_a;
-            float* new_c = cost_b;
-            for (int s = threadIdx.x; s < S; s += blockDim.x)
-                old_c[s] = (pass == 0 || (s >> kV) == prefix) ? dist(0, s) : INFINITY;
+            float* Mp = Ma;
+            float* Mn = Mb;
+            for (int a = threadIdx.x; a < G; a += blockDim.x) Mp[a] = (pass == 0 || a == prefix) ? 0.f : INFINITY;
             __syncthreads();
             for (int t = 1; t < T; ++t) {
+                const float* xt = xs + (t - 1) * V;
                 for (int a = threadIdx.x; a < G; a += blockDim.x) {
-                    float m = old_c[a];
+                    float m = INFINITY;
                     int hb = 0;
-                    for (int h = 1; h < C; ++h) {
-                        const float c = old_c[a + h * G];
+#pragma unroll (C <= 16 ? C : 4)
+                    for (int h = 0; h < C; ++h) {
+                        const uint32_t q = (uint32_t)(a + h * G);
+                        float v[V];
+                        values_of<CODE, V>(q, lut_lane, qshift, v);
+                        const float c = __fadd_rn(Mp[q >> KV], dist_of<V>(xt, v));
                         if (c < m) m = c, hb = h;
                     }
+                    Mn[a] = m;
                     if (pass == 1) choice[(size_t)t * G + a] = (uint8_t)hb;
-                    for (int c = 0; c < C; ++c) {
-                        const int s = a * C + c;
-                        new_c[s] = __fadd_rn(m, dist(t, s));
-                    }
                 }
                 __syncthreads();
-                float* tmp = old_c;
-                old_c = new_c;
-                new_c = tmp;
+                float* tmp = Mp;
+                Mp = Mn;
+                Mn = tmp;
             }
-            // best final state (pass 2: only those whose low bits are the prefix)
+            const float* xl = xs + (T - 1) * V;
             float bv = INFINITY;
             int bi = 0x7fffffff;
             for (int s = threadIdx.x; s < S; s += blockDim.x) {
                 if (pass == 1 && (s & (G - 1)) != prefix) continue;
-                const float c = old_c[s];
+                float v[V];
+                values_of<CODE, V>((uint32_t)s, lut_lane, qshift, v);
+                const float c = __fadd_rn(Mp[s >> KV], dist_of<V>(xl, v));
                 if (c < bv || (c == bv && s < bi)) bv = c, bi = s;
             }
             argmin_cta(bv, bi, red_v, red_i);
-            if (bi < 0 || bi >= S) {  // no finite walk (cannot happen for finite inputs)
+            if (bi < 0 || bi >= S) {
                 if (threadIdx.x == 0) atomicOr(p.status, kStatusBadInput);
                 bi = 0;
             }
             if (pass == 0) prefix = bi & (G - 1);
             last = bi;
         }
-        // trace back (one thread), pack the chunks MSB-first, score the reconstruction
-        __threadfence_block();
         __syncthreads();
         if (threadIdx.x == 0) {
-            const int words_per_block = T * kV / 32;
+            constexpr int words_per_block = T * KV / 32;
             uint32_t* out = p.words + (size_t)blk * words_per_block;
             for (int i = 0; i < words_per_block; ++i) out[i] = 0u;
             int s = last;
             float err = 0.f;
             for (int t = T - 1; t >= 0; --t) {
                 const uint32_t chunk = (uint32_t)(s & (C - 1));
-                const int bitpos = t * kV;  // chunk t covers bits [t kV, (t+1) kV) of the block
-                for (int b = 0; b < kV; ++b) {
-                    const int pos = bitpos + b;
-                    const uint32_t bit = (chunk >> (kV - 1 - b)) & 1u;
-                    out[pos >> 5] |= bit << (31 - (pos & 31));
+                for (int b = 0; b < KV; ++b) {
+                    const int pos = t * KV + b;
+                    out[pos >> 5] |= ((chunk >> (KV - 1 - b)) & 1u) << (31 - (pos & 31));
                 }
+                float v[V];
+                values_of<CODE, V>((uint32_t)s, lut_lane, qshift, v);
                 for (int e = 0; e < V; ++e) {
-                    const float diff = xs[t * V + e] - vals[s * V + e];
+                    const float diff = xs[t * V + e] - v[e];
                     err += diff * diff;
                 }
                 if (t) {
-                    const int a = s >> kV;
+                    const int a = s >> KV;
                     s = a + (int)choice[(size_t)t * G + a] * G;
                 }
             }
@@ -205,6 +221,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_kernel(EncodeArgs p) {
         __syncthreads();
     }
 }
+
 
 // ---- L = 15, 16: one cluster of nc CTAs per block ----
 
@@ -379,12 +396,19 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
     }
 }
 
-size_t encode_smem_bytes(int L, int V, int code, int Q) {
-    if (L > kEncMaxL) return (size_t)cluster_smem(V).total;
-    const size_t S = (size_t)1 << L;
-    size_t b = (2 * S + S * V + 256 + 32) * 4 + 32 * 4;
+static size_t gm_smem_bytes(int L, int kv, int code, int Q) {
+    const size_t G = (size_t)1 << (L - kv);
+    size_t b = (2 * G + 256 + 64) * 4;
     if (uses_table(code)) b += ((size_t)32 << Q) * 4;
     return b;
+}
+
+static bool use_gm(int L, int kv, int code, int Q) { return gm_smem_bytes(L, kv, code, Q) <= (size_t)kTcMaxSmem; }
+
+size_t encode_smem_bytes(int L, int kv, int V, int code, int Q) {
+    if (use_gm(L, kv, code, Q)) return gm_smem_bytes(L, kv, code, Q);
+    if (L > kEncMaxL) return (size_t)cluster_smem(V).total;  // the cluster kernel reads tables from global memory
+    return (size_t)-1;  // does not fit
 }
 
 static int encode_cluster_size(int L) { return L > kEncMaxL ? (1 << L) / kEncClusterStates : 1; }
@@ -392,13 +416,8 @@ static int encode_cluster_size(int L) { return L > kEncMaxL ? (1 << L) / kEncClu
 template <int KV>
 static cudaError_t cluster_config(int nc, int workers, size_t smem, cudaStream_t st, cudaLaunchConfig_t* cfg,
                                   cudaLaunchAttribute* attr) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(encode_cluster_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kTcMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = ensure_smem_limit<encode_cluster_kernel<KV>>(kTcMaxSmem);
+    if (e != cudaSuccess) return e;
     *cfg = cudaLaunchConfig_t{};
     cfg->gridDim = dim3(nc * workers);
     cfg->blockDim = dim3(kEncThreads);
@@ -432,9 +451,9 @@ static cudaError_t launch_cluster(const EncodeArgs& a, int workers, size_t smem,
     return cudaLaunchKernelEx(&cfg, encode_cluster_kernel<KV>, a);
 }
 
-cudaError_t encode_workers(int L, int kv, int V, int blocks, int num_sms, int* workers) {
+cudaError_t encode_workers(int L, int kv, int V, int code, int Q, int blocks, int num_sms, int* workers) {
     int w = num_sms;
-    if (L > kEncMaxL) {
+    if (!use_gm(L, kv, code, Q)) {
         const int nc = encode_cluster_size(L);
         const size_t smem = (size_t)cluster_smem(V).total;
         cudaError_t e = cudaErrorInvalidValue;
@@ -455,6 +474,40 @@ cudaError_t encode_workers(int L, int kv, int V, int blocks, int num_sms, int* w
     return cudaSuccess;
 }
 
+template <int CODE, int KV, int V>
+static cudaError_t launch_gm(const EncodeArgs& a, int workers, size_t smem, cudaStream_t st) {
+    auto kern = encode_gm_kernel<CODE, KV, V>;
+    cudaError_t e = ensure_smem_limit<encode_gm_kernel<CODE, KV, V>>(kTcMaxSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<workers, kEncThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+// (code, V, kv) -> the group-minima instance: V = 1 takes kv 1..4 (any code),
+// V = 2 kv 2..8 (the table codes)
+template <int CODE, int V>
+static cudaError_t launch_gm_kv(const EncodeArgs& a, int kv, int workers, size_t smem, cudaStream_t st) {
+    if constexpr (V == 1) {
+        switch (kv) {
+            case 1: return launch_gm<CODE, 1, 1>(a, workers, smem, st);
+            case 2: return launch_gm<CODE, 2, 1>(a, workers, smem, st);
+            case 3: return launch_gm<CODE, 3, 1>(a, workers, smem, st);
+            case 4: return launch_gm<CODE, 4, 1>(a, workers, smem, st);
+        }
+    } else {
+        switch (kv) {
+            case 2: return launch_gm<CODE, 2, 2>(a, workers, smem, st);
+            case 3: return launch_gm<CODE, 3, 2>(a, workers, smem, st);
+            case 4: return launch_gm<CODE, 4, 2>(a, workers, smem, st);
+            case 5: return launch_gm<CODE, 5, 2>(a, workers, smem, st);
+            case 6: return launch_gm<CODE, 6, 2>(a, workers, smem, st);
+            case 7: return launch_gm<CODE, 7, 2>(a, workers, smem, st);
+            case 8: return launch_gm<CODE, 8, 2>(a, workers, smem, st);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t* lut, const float* x, int blocks,
                           uint32_t* words, float* err, uint8_t* choice, int workers, int* status, cudaStream_t st) {
     EncodeArgs a;
@@ -471,28 +524,35 @@ cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t*
     a.choice = choice;
     a.status = status;
     a.nc = encode_cluster_size(L);
-    const size_t smem = encode_smem_bytes(L, V, code, Q);
-    if (L > kEncMaxL) {
-        switch (kv) {
-            case 1: return launch_cluster<1>(a, workers, smem, st);
-            case 2: return launch_cluster<2>(a, workers, smem, st);
-            case 3: return launch_cluster<3>(a, workers, smem, st);
-            case 4: return launch_cluster<4>(a, workers, smem, st);
-            case 5: return launch_cluster<5>(a, workers, smem, st);
-            case 6: return launch_cluster<6>(a, workers, smem, st);
-            case 7: return launch_cluster<7>(a, workers, smem, st);
-            case 8: return launch_cluster<8>(a, workers, smem, st);
+    if (use_gm(L, kv, code, Q)) {
+        const size_t smem = gm_smem_bytes(L, kv, code, Q);
+        if (V == 1) {
+            switch (code) {
+                case kCode1MAD: return launch_gm_kv<kCode1MAD, 1>(a, kv, workers, smem, st);
+                case kCode3INST: return launch_gm_kv<kCode3INST, 1>(a, kv, workers, smem, st);
+                case kCodeHYB: return launch_gm_kv<kCodeHYB, 1>(a, kv, workers, smem, st);
+                case kCodeTable: return launch_gm_kv<kCodeTable, 1>(a, kv, workers, smem, st);
+            }
+        } else {
+            switch (code) {
+                case kCodeHYB: return launch_gm_kv<kCodeHYB, 2>(a, kv, workers, smem, st);
+                case kCodeTable: return launch_gm_kv<kCodeTable, 2>(a, kv, workers, smem, st);
+            }
         }
         return cudaErrorInvalidValue;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
+    const size_t smem = (size_t)cluster_smem(V).total;
+    switch (kv) {
+        case 1: return launch_cluster<1>(a, workers, smem, st);
+        case 2: return launch_cluster<2>(a, workers, smem, st);
+        case 3: return launch_cluster<3>(a, workers, smem, st);
+        case 4: return launch_cluster<4>(a, workers, smem, st);
+        case 5: return launch_cluster<5>(a, workers, smem, st);
+        case 6: return launch_cluster<6>(a, workers, smem, st);
+        case 7: return launch_cluster<7>(a, workers, smem, st);
+        case 8: return launch_cluster<8>(a, workers, smem, st);
     }
-    encode_kernel<<<workers, kEncThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace qlk

@@ -264,7 +264,7 @@ __device__ __forceinline__ void decode_stage_k2(int k2, uint32_t code, uint32_t 
 }
 
 template <int CODE, int V, bool L16>
-__global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
+__global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived by indexing the shared array so that
     // accesses through it stay shared-memory accesses
@@ -474,13 +474,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(GemmArgs p) {
 
 template <int CODE, int V, bool L16>
 static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaStream_t st) {
-    auto kern = gemm_tc_kernel<CODE, V, L16>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    auto kern = trellis_gemm_kernel<CODE, V, L16>;
+    cudaError_t e = ensure_smem_limit<trellis_gemm_kernel<CODE, V, L16>>(kTcMaxSmem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, a);
 }
 

@@ -247,7 +247,7 @@ struct InputTransform {
 // every SM and every warp equally loaded.  Every thread runs every phase (no
 // early exit), since the in-kernel transforms use CTA barriers.
 template <int CODE, int K2, int V, bool L16, bool XSMEM>
-__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_kernel(GemvArgs p, GemvSmem sm) {
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(GemvArgs p, GemvSmem sm) {
     extern __shared__ uint32_t smem[];
     using UL = UnitLayout<K2>;
     uint32_t* lut_smem = smem;
@@ -415,7 +415,7 @@ __device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], cons
 }
 
 template <int CODE, int V, bool L16>
-__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvMultiArgs p) {
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_multi_kernel(GemvMultiArgs p) {
     extern __shared__ uint32_t smem[];
     const int lane = threadIdx.x & 31;
     if (uses_table(CODE)) {
@@ -490,13 +490,9 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_multi_kernel(GemvM
 
 template <int CODE, int V, bool L16>
 static cudaError_t launch_gemv_multi_t(const GemvMultiArgs& a, int grid, int threads, size_t smem, cudaStream_t st) {
-    auto kern = gemv_multi_kernel<CODE, V, L16>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    auto kern = trellis_gemv_multi_kernel<CODE, V, L16>;
+    cudaError_t e = ensure_smem_limit<trellis_gemv_multi_kernel<CODE, V, L16>>(kGemvMaxSmem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a);
 }
 
@@ -543,7 +539,7 @@ cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, fl
 
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
 template <int CODE, int K2, int V, bool L16>
-__global__ void __launch_bounds__(256) decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
+__global__ void __launch_bounds__(256) trellis_decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
     extern __shared__ uint32_t lut_smem[];
     using UL = UnitLayout<K2>;
     const int lane = threadIdx.x & 31;
@@ -668,25 +664,17 @@ struct GemvLaunch {
         const size_t smem = (size_t)(sm.lut_words + sm.xs_words + sm.fw_words) * 4;
         if (xsmem) {
             if constexpr (L16 || CODE == kCodeTable) {
-                auto kern = gemv_kernel<CODE, K2, V, L16, true>;
-                static bool attr_set = false;
-                if (!attr_set) {
-                    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
-                    if (e != cudaSuccess) return e;
-                    attr_set = true;
-                }
+                auto kern = trellis_gemv_kernel<CODE, K2, V, L16, true>;
+                cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, K2, V, L16, true>>(kGemvMaxSmem);
+                if (e != cudaSuccess) return e;
                 return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
             } else {
                 return cudaErrorInvalidValue;
             }
         }
-        auto kern = gemv_kernel<CODE, K2, V, L16, false>;
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
+        auto kern = trellis_gemv_kernel<CODE, K2, V, L16, false>;
+        cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, K2, V, L16, false>>(kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
     }
 };
@@ -760,12 +748,10 @@ template <int CODE, int K2, int V, bool L16>
 struct DecodeLaunch {
     static cudaError_t run(const DecodeArgs& d, __half* w, int n, int row0, int grid, cudaStream_t st) {
         const size_t smem = (size_t)d.lut_entries * 32 * 4;
-        auto kern = decode_kernel<CODE, K2, V, L16>;
-        static bool attr_set = false;
-        if (smem > 48 * 1024 && !attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
+        auto kern = trellis_decode_kernel<CODE, K2, V, L16>;
+        if (smem > 48 * 1024) {
+            cudaError_t e = ensure_smem_limit<trellis_decode_kernel<CODE, K2, V, L16>>(32 * 512 * 4);
             if (e != cudaSuccess) return e;
-            attr_set = true;
         }
         kern<<<grid, 256, smem, st>>>(d, w, n, row0);
         return cudaGetLastError();
@@ -788,11 +774,9 @@ struct EvalLaunch {
         if (K2 != 2 || L16 == (CODE == kCodeTable)) return cudaErrorInvalidValue;
         const size_t smem = (size_t)entries * 32 * 4;
         auto kern = eval_code_kernel<CODE, V>;
-        static bool attr_set = false;
-        if (smem > 48 * 1024 && !attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 512 * 4);
+        if (smem > 48 * 1024) {
+            cudaError_t e = ensure_smem_limit<eval_code_kernel<CODE, V>>(32 * 512 * 4);
             if (e != cudaSuccess) return e;
-            attr_set = true;
         }
         const int items = V == 2 ? count : (count + 1) / 2;
         kern<<<(items + 255) / 256, 256, smem, st>>>(states, count, lmask, qshift, lut, entries, out);

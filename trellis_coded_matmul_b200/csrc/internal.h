@@ -4,6 +4,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/qlinear.h"
 
 namespace qlk {
@@ -97,18 +99,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Raise kernel Kern's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute is per device context); devices
+// numbered 64 and above set it on every call.  Safe to call from several
+// host threads.
+template <auto Kern>
+cudaError_t ensure_smem_limit(int bytes) {
+    static std::atomic<unsigned long long> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_relayout(const uint32_t* src, uint32_t* dst, const Part& part, int n, cudaStream_t st);
 cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* status, cudaStream_t st);
 cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
-
-// Trellis-coded quantization of `blocks` blocks of 256 source values (two-pass
-// tail-biting Viterbi, L <= 14, kv bits per step): words [blocks][8 kv / V] in
-// the stream format, the squared error of each block's reconstruction into
-// err (may be null).  choice: grid * (256/V) * 2^(L-kv) bytes of scratch.
-size_t encode_smem_bytes(int L, int V, int code, int Q);
-cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t* lut, const float* x, int blocks,
-                          uint32_t* words, float* err, uint8_t* choice, int grid, int* status, cudaStream_t st);
 
 // x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
 cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);

@@ -443,14 +443,14 @@ int qlinear_encode_kv(ql_code_t code, int L, int kv, int V, const float* x, int 
     if (blocks == 0) return QL_OK;
     if (!is_device_pointer(x) || !is_device_pointer(words) || (err && !is_device_pointer(err))) return QL_E_ARG;
     const int Q = table_bits(code, L);
-    if (encode_smem_bytes(L, V, code.kind, Q) > (size_t)kTcMaxSmem) return QL_E_UNSUPPORTED;
+    if (encode_smem_bytes(L, kv, V, code.kind, Q) > (size_t)kTcMaxSmem) return QL_E_UNSUPPORTED;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
     int workers = 0;
-    if (encode_workers(L, kv, V, blocks, sms, &workers) != cudaSuccess) {
+    if (encode_workers(L, kv, V, code.kind, Q, blocks, sms, &workers) != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }

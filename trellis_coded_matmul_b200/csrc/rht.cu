@@ -117,13 +117,8 @@ static cudaError_t launch_rht_in_e(const Layer& L, const void* x, int batch, voi
     const RhtGeometry geo = rht_geometry(L.n, L.B_n, batch, E);
     const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
     auto kern = rht_in_kernel<MODE, E>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (kMaxHadamard + kMaxHadamard / 16) * 4);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = ensure_smem_limit<rht_in_kernel<MODE, E>>((kMaxHadamard + kMaxHadamard / 16) * 4);
+    if (e != cudaSuccess) return e;
     const int grid = (geo.total + geo.groups - 1) / geo.groups;
     return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, (const __half*)x, batch, L.n, geo,
                       (const uint32_t*)L.sin_bits, (__half*)xp, npad);
@@ -203,13 +198,8 @@ static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y
     const RhtGeometry geo = rht_geometry(L.m, L.B_m, batch, E);
     const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
     auto kern = rht_out_kernel<F16, E>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (kMaxHadamard + kMaxHadamard / 16) * 4);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = ensure_smem_limit<rht_out_kernel<F16, E>>((kMaxHadamard + kMaxHadamard / 16) * 4);
+    if (e != cudaSuccess) return e;
     const int grid = (geo.total + geo.groups - 1) / geo.groups;
     return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, z, batch, L.m, geo,
                       (const uint32_t*)L.sout_bits, L.alpha, y);
