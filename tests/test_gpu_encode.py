@@ -26,11 +26,15 @@ CASES = [
     (12, 2, 2, wl.CODE_HYB, 6),
     (14, 2, 1, wl.CODE_3INST, 0),
     (13, 3, 1, wl.CODE_HYB, 9),
-    # L = 15, 16: the dynamic programme shared by a cluster of 2 or 4 CTAs
+    (14, 2, 2, wl.CODE_HYB, 9),
+    # L = 15, 16: one CTA holds the group minima of the search whenever they fit
     (16, 2, 1, wl.CODE_3INST, 0),
     (15, 1, 1, wl.CODE_1MAD, 0),
     (16, 1, 2, wl.CODE_HYB, 9),
     (16, 3, 1, wl.CODE_HYB, 9),
+    # L = 16 at one bit per step: the dynamic programme shared by a cluster of 4 CTAs
+    (16, 1, 1, wl.CODE_HYB, 9),
+    (16, 1, 1, wl.CODE_3INST, 0),
 ]
 
 
@@ -67,8 +71,8 @@ def test_encode_matches_the_oracle_bit_for_bit(L, k, V, code, Q):
 CASES_KV = [
     # L, kv, V, code, Q
     (12, 5, 2, wl.CODE_HYB, 9),      # 2.5-bit TCQ, one CTA per block
-    (16, 5, 2, wl.CODE_HYB, 9),      # 2.5-bit TCQ at L = 16, a cluster of 4 CTAs
-    (15, 7, 2, wl.CODE_HYB, 6),      # 3.5 bits, a cluster of 2 CTAs
+    (16, 5, 2, wl.CODE_HYB, 9),      # 2.5-bit TCQ at L = 16
+    (15, 7, 2, wl.CODE_HYB, 6),      # 3.5 bits
     (5, 5, 2, wl.CODE_TABLE, 0),     # 2.5-bit VQ: nearest codeword
     (3, 3, 1, wl.CODE_TABLE, 0),     # 3-bit NUQ: nearest level
     (8, 3, 2, wl.CODE_TABLE, 0),     # 1.5 bits, a trellis over a 256-entry codebook
