@@ -178,8 +178,11 @@ int qlinear_create_kv(qlinear_t* out, int m, int n, int nparts, const int* part_
 /* y = W x for a batch of inputs.
  *   x: device pointer, fp16 [batch][n] row-major.
  *   y: device pointer, [batch][m] row-major, fp32 (y_dtype = QL_F32) or fp16 (QL_F16).
- *   batch >= 0 (0 is a no-op).  batch <= 8 runs the fused decode-GEMV kernels;
- *   larger batches run the decode-to-shared-memory tcgen05 GEMM.
+ *   batch >= 0 (0 is a no-op).  batch <= 8 runs the fused decode-GEMV kernel
+ *   (the whole forward in one launch when batch*n <= 16384, else after an
+ *   input-transform kernel); larger batches run the decode-to-tensor-memory
+ *   tcgen05 GEMM between the two transform kernels.  x and y must be 16-byte
+ *   aligned.
  * The first call with a batch larger than any before it allocates scratch;
  * make such a call before capturing forward into a CUDA graph.
  * Errors: QL_E_ARG, QL_E_OOM, QL_E_CUDA (launch failure). */
@@ -197,11 +200,13 @@ int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_hos
  * cannot let a library allocate while they run (cudaMalloc/cudaFree may
  * synchronise the whole device and stall a serving process's other streams;
  * runtimes that pre-carve all free HBM into their own pools leave no room).
- *   Scratch: x' and the fp32 accumulator z live in one fixed array of
+ *   Scratch: the output-block tickets, the fp32 accumulator z and (when the
+ *   input transform runs as its own kernel) x' live in one fixed array of
  *   QL_NOALLOC_SCRATCH_BYTES in the library's static device memory, per
- *   device: round_up(batch*n*2, 256) + batch*m*4 bytes must fit, else
- *   QL_E_SCRATCH (before any device work).  Every call clears its part of z
- *   on `stream` first.
+ *   device: round_up(4*m/B(m), 256) + round_up(4*batch*m, 256) bytes, plus
+ *   4*batch*n/V bytes of x' when batch*n > 16384, must fit, else
+ *   QL_E_SCRATCH (before any device work).  Every call clears its tickets
+ *   and z on `stream` first.
  *   Sharing: all handles on a device share the array, so calls that overlap
  *   in time (different streams or host threads) race and give wrong y; calls
  *   in order on one stream are safe.
@@ -222,6 +227,21 @@ int qlinear_decode(qlinear_t h, void* w_hat, void* stream);
  * exhaustively. */
 int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int count, void* out,
                       void* stream);
+
+/* Test hook for the tensor-core GEMM's bounded waits (no counterpart on the
+ * pages; the waits themselves are the failure detection of the GEMM's
+ * producer/consumer pipeline).  With enable != 0, every later forward with
+ * batch > 8 on this handle runs the GEMM with each mbarrier wait limited to
+ * wait_tries suspending tries (1..4096; each try suspends for at most about a
+ * millisecond) and with the x' producer withholding the first stage of every
+ * CTA, so the MMA issuer's wait on it runs out.  The CTAs then set
+ * QL_E_TIMEOUT in the handle's status word (read by qlinear_get_status), drop
+ * their work, free their tensor memory and exit: y of that forward is
+ * undefined, and the next forward after qlinear_get_status reported the
+ * timeout is correct again.  No fault and no unbounded wait is involved.
+ * enable = 0 restores the normal limit (a few seconds) and stops withholding.
+ * Errors: QL_E_ARG (null handle, wait_tries out of range when enabling). */
+int qlinear_test_stall(qlinear_t h, int enable, int wait_tries);
 
 /* Trellis-coded quantization: for each block of 256 source values, the bits
  * whose tail-biting walk on the bitshift trellis reproduces the block with the

@@ -70,7 +70,7 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(name, batch, dtype):
             tol = TOL_SAME_KERNELS if dtype == torch.float32 else 2 ** -10
             assert _same(y, y_ref) <= tol, (call, _same(y, y_ref))
         assert tcm.qlinear_get_status(h) == tcm.QL_OK
-        assert tcm.qlinear_info(h)["last_launches"] >= 2
+        assert tcm.qlinear_info(h)["last_launches"] >= 1
     finally:
         tcm.qlinear_destroy(h)
 
@@ -91,16 +91,23 @@ def test_noalloc_against_the_oracle():
         tcm.qlinear_destroy(h)
 
 
+def _noalloc_bytes(m, n, V, B_m, batch):
+    """Scratch of one call as the header states it: the output-block tickets,
+    z, and x' when the input transform runs as its own kernel."""
+    up = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    return up(4 * (m // B_m)) + up(4 * batch * m) + (0 if batch * n <= 16384 else 4 * batch * n // V)
+
+
 def test_noalloc_scratch_limit_and_batch_limit():
     # m = 81920 (Hadamard blocks of 16384), n = 256: batch 6 needs
-    # 3072 + 6*81920*4 = 1969152 bytes of scratch (fits in 2 MiB), batch 7
-    # needs 2296832 (does not).
+    # 256 + 6*81920*4 = 1966336 bytes of scratch (fits in 2 MiB), batch 7
+    # needs 2294016 (does not).
     m, n = 81920, 256
     li = wl.random_layer(m, n, 2, 16, 1, wl.CODE_3INST, seed=11, alpha=0.5)
     h = make_handle(li)
     try:
         limit = tcm.QL_NOALLOC_SCRATCH_BYTES
-        assert (6 * n * 2 + 255) // 256 * 256 + 6 * m * 4 <= limit < (7 * n * 2 + 255) // 256 * 256 + 7 * m * 4
+        assert _noalloc_bytes(m, n, 1, 16384, 6) <= limit < _noalloc_bytes(m, n, 1, 16384, 7)
 
         x6 = torch.from_numpy(wl.make_x(li.spec, 6)).cuda()
         y_ref = tcm.qlinear_forward(h, x6)

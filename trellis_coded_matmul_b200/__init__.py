@@ -42,7 +42,7 @@ ABI_SYMBOLS = ("qlinear_create", "qlinear_create_mixed", "qlinear_create_parts",
                "qlinear_forward", "qlinear_forward_host",
                "qlinear_decode", "qlinear_eval_code", "qlinear_get_status", "qlinear_info",
                "qlinear_destroy", "qlinear_strerror", "qlinear_profile_enable", "qlinear_profile_read",
-               "qlinear_forward_noalloc", "qlinear_encode", "qlinear_encode_kv")
+               "qlinear_forward_noalloc", "qlinear_encode", "qlinear_encode_kv", "qlinear_test_stall")
 
 
 class ql_code_t(ctypes.Structure):
@@ -72,6 +72,7 @@ _lib.qlinear_encode_kv.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp
 _lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
 _lib.qlinear_eval_code.argtypes = [ql_code_t, _i, _i, _vp, _i, _vp, _vp]
 _lib.qlinear_get_status.argtypes = [_vp]
+_lib.qlinear_test_stall.argtypes = [_vp, _i, _i]
 _lib.qlinear_info.argtypes = [_vp, ctypes.POINTER(ql_info_t)]
 _lib.qlinear_destroy.argtypes = [_vp]
 _lib.qlinear_strerror.argtypes = [_i]
@@ -313,6 +314,12 @@ def qlinear_eval_code(kind, L, V, states, Q=0, lut=None, out=None, stream=None):
 
 def qlinear_get_status(h: QLinearHandle) -> int:
     return _lib.qlinear_get_status(h.ptr)
+
+
+def qlinear_test_stall(h: QLinearHandle, enable: bool, wait_tries: int = 8) -> None:
+    """Test hook: make the handle's tensor-core GEMM withhold its first stage so
+    that its bounded waits expire after `wait_tries` tries (see the header)."""
+    _check(_lib.qlinear_test_stall(h.ptr, int(bool(enable)), wait_tries), "qlinear_test_stall")
 
 
 def qlinear_info(h: QLinearHandle) -> dict:

@@ -113,15 +113,4 @@ __device__ __forceinline__ void fwht_block(float (&v)[E], int B, int tid, int T,
     }
 }
 
-// Fragment layout of x' for the decode-GEMV: the 8-byte group
-//   frag[((j*16 + u) * batch + b) * 4 + c] = x'[b][256 j + 64 c + 4 u + 0..3]
-// is what lane (g = b, c) needs as its B operand for the u-th m16n8k16 MMA of
-// block j (see gemv.cu).  Returns the index of the first of the four halves.
-__device__ __forceinline__ size_t frag_index4(int col, int b, int batch) {
-    const int j = col >> 8, within = col & 255;
-    const int c = within >> 6, r = within & 63;
-    const int u = r >> 2;
-    return ((((size_t)j * 16 + u) * batch + b) * 4 + c) * 4;
-}
-
 }  // namespace qlk

@@ -101,6 +101,8 @@ struct GemmArgs {
     float* z;               // [batch][m], all-zero on entry
     int m;
     int* status;
+    int wait_tries;         // try_wait calls of up to kTcSuspendNs before a wait is declared expired
+    int withhold;           // test hook: the x' producer withholds its first stage (its waits then expire)
     int stages;             // stage slots
     int code_slots;         // depth of the code-word ring
     int code_slot_words;    // words of one code-ring slot (8 units at the largest k2)
@@ -201,10 +203,12 @@ __device__ __forceinline__ void decode_run32(const uint32_t (&w)[K2 + 1], uint32
     }
 }
 
-// Bounded wait; returns false (and raises the CTA's abort flag) on expiry.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// Bounded wait (at most `tries` suspending tries); returns false (and raises
+// the CTA's abort flag) on expiry.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                         int tries) {
     if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspension
-    for (int i = 0; i < kTcWaitTries; ++i) {
+    for (int i = 0; i < tries; ++i) {
         if (mbar_try_wait(bar, parity, kTcSuspendNs)) return true;
         if (*abort_flag) return false;
     }
@@ -326,10 +330,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             const int j = w.j;
             for (int q = 0; q < 4; ++q, r.advance(1, S)) {
                 const int st = r.slot;
-                if (!wait_bar(empty(st), r.phase ^ 1u, abort_flag, p.status)) {
+                if (!wait_bar(empty(st), r.phase ^ 1u, abort_flag, p.status, p.wait_tries)) {
                     ok = false;
                     break;
                 }
+                // Test hook: the first stage's x' never arrives, so the MMA issuer's
+                // wait on it expires (and with it every role's).
+                if (p.withhold && w.u == u0 && q == 0) continue;
                 // The tile goes in kTcXSplit pieces, one per lane, so that several
                 // bulk copies are in flight at once.
                 if (lane == 0) mbar_arrive_expect_tx(full(st), b_bytes);
@@ -351,7 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             const int tile = w.tile(p);
             const int ntiles16 = tc_tiles16(pt, tile);
             const int unit_words = 64 * pt.k2;
-            if (!wait_bar(code_empty(slot), r.phase ^ 1u, abort_flag, p.status)) break;
+            if (!wait_bar(code_empty(slot), r.phase ^ 1u, abort_flag, p.status, p.wait_tries)) break;
             if (lane == 0) mbar_arrive_expect_tx(code_full(slot), (uint32_t)(ntiles16 * unit_words * 4));
             __syncwarp();
             if (lane < ntiles16) {
@@ -377,11 +384,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             const bool first = w.u == u0 || w.j == 0;  // first block of a segment
             const bool last = w.u + 1 == u1 || w.j + 1 == p.nb;
             // the epilogue of the previous segment must have read the accumulator
-            if (first && seg > 0 && !wait_bar(acc_empty, (seg - 1) & 1, abort_flag, p.status)) break;
+            if (first && seg > 0 && !wait_bar(acc_empty, (seg - 1) & 1, abort_flag, p.status, p.wait_tries)) break;
             bool ok = true;
             for (int q = 0; q < 4; ++q, r.advance(1, S)) {
                 const int st = r.slot;
-                if (!wait_bar(full(st), r.phase, abort_flag, p.status)) {
+                if (!wait_bar(full(st), r.phase, abort_flag, p.status, p.wait_tries)) {
                     ok = false;
                     break;
                 }
@@ -414,11 +421,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             const int slot = rc.slot;
             const TcPart& pt = p.part[w.part(p)];
             const uint32_t code = code_base + slot * p.code_slot_words * 4;
-            if (!wait_bar(code_full(slot), rc.phase, abort_flag, p.status)) break;
+            if (!wait_bar(code_full(slot), rc.phase, abort_flag, p.status, p.wait_tries)) break;
             bool ok = true;
             {
                 const int st = rs.slot;
-                if (!wait_bar(empty(st), rs.phase ^ 1u, abort_flag, p.status)) {
+                if (!wait_bar(empty(st), rs.phase ^ 1u, abort_flag, p.status, p.wait_tries)) {
                     ok = false;
                 } else {
                     tc_fence_after();  // the MMAs that read this A slot have completed
@@ -440,7 +447,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
                 grid_dependency_wait();  // z was last touched by the previous kernels
                 z_ready = true;
             }
-            if (!wait_bar(acc_full, seg & 1, abort_flag, p.status)) break;
+            if (!wait_bar(acc_full, seg & 1, abort_flag, p.status, p.wait_tries)) break;
             tc_fence_after();
             const int rloc = qtr * 32 + lane;  // row within the tile
             const int tile = w.tile(p);
@@ -529,6 +536,8 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     a.z = z;
     a.m = L.m;
     a.status = L.status;
+    a.wait_tries = L.test_wait_tries > 0 ? L.test_wait_tries : kTcWaitTries;
+    a.withhold = L.test_withhold;
     a.code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
     const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots);
     if (smem == 0) return cudaErrorInvalidValue;
@@ -546,6 +555,20 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     if (L.V == 1) return l16 ? launch_gemm_t<kCodeHYB, 1, true>(a, grid, smem, st)
                              : launch_gemm_t<kCodeHYB, 1, false>(a, grid, smem, st);
     return l16 ? launch_gemm_t<kCodeHYB, 2, true>(a, grid, smem, st) : launch_gemm_t<kCodeHYB, 2, false>(a, grid, smem, st);
+}
+
+cudaError_t prepare_gemm_kernels(const Layer& L) {
+    const bool l16 = L.L == 16;
+#define QLK_PREP(C, V_, L_) preload_kernel<trellis_gemm_kernel<C, V_, L_>>(kTcMaxSmem)
+    if (L.code == kCode1MAD) return l16 ? QLK_PREP(kCode1MAD, 1, true) : QLK_PREP(kCode1MAD, 1, false);
+    if (L.code == kCode3INST) return l16 ? QLK_PREP(kCode3INST, 1, true) : QLK_PREP(kCode3INST, 1, false);
+    if (L.code == kCodeTable) {
+        if (l16) return cudaErrorInvalidValue;
+        return L.V == 1 ? QLK_PREP(kCodeTable, 1, false) : QLK_PREP(kCodeTable, 2, false);
+    }
+    if (L.V == 1) return l16 ? QLK_PREP(kCodeHYB, 1, true) : QLK_PREP(kCodeHYB, 1, false);
+    return l16 ? QLK_PREP(kCodeHYB, 2, true) : QLK_PREP(kCodeHYB, 2, false);
+#undef QLK_PREP
 }
 
 }  // namespace qlk

@@ -1,28 +1,57 @@
-// gemv.cu -- fused trellis decode + matrix-vector product for batch <= 8, and
-// the decode / eval_code test kernels built on the same device functions.
+// gemv.cu -- fused trellis decode + matrix-vector product for batch <= 8 (the
+// whole forward in one kernel when x is small), and the decode / eval_code
+// test kernels built on the same device functions.
 //
 // Decode follows the QTIP discussion: the bitshift trellis makes every state
 // a window of the stored bits, so a lane can decode any run of steps on its
 // own ("the bitshift trellis also enables parallel decoding"), and the codes
 // are computed in INT32 ALU (1MAD, 3INST) or with a small table in banked
-// shared memory (HYB).  Decoded weights stay in registers: they are the A
-// operand of m16n8k16 half-precision MMAs whose B operand is x' (batch padded
-// to 8 columns) and whose fp32 accumulators hold 16 rows x 8 batch columns.
+// shared memory (HYB, and the palette's table code).  Decoded weights stay in
+// registers: they are the A operand of m16n8k16 half-precision MMAs whose B
+// operand is x' (batch padded to 8 columns) and whose fp32 accumulators hold
+// 16 rows x 8 batch columns.
 //
-// Work split: the m x n matrix is a grid of units (16 rows x 256 columns).
-// Units are numbered row-tile-major; every warp of the grid takes one
-// contiguous, equally sized range of units, accumulates while the row tile is
-// unchanged and adds its partial sums into z with atomics when it moves on.
-// The k-slot order inside an MMA is free (both operands use it): lane c
-// feeds its own 4 consecutive columns per MMA, so every lane walks a
-// contiguous run of trellis steps and the matching x' values are one 8-byte
-// load (see the fragment layout in rht.cu).
+// One 32-bit A word per trellis step (xstep.cuh gives the matching B words):
+//   V = 2: the code's table word, the step's two fp16 weights;
+//   V = 1: the code's "split" word, two fp16 halves whose sum is the weight,
+//          so the MMA adds them (h0 x' + h1 x' = (h0 + h1) x') and the decode
+//          spends no instruction on the sum or on pairing weights:
+//            3INST  the masked word m itself (value = m.lo + m.hi);
+//            1MAD   one dp4a whose accumulator puts 1536 + d in the low half
+//                   and -1536 in the high half (sum d, the byte sum minus
+//                   510); the factor C1 is applied to z in the epilogue;
+//            HYB / table  the table word (value in the low half, 0 above).
+//   The product then carries the code value before its rounding to fp16
+//   (qlinear_decode still returns the fp16-rounded values); the difference
+//   is a relative 2^-12 per weight, independent from weight to weight.
+//
+// Work split: the m x n matrix is a grid of units (16 rows x 256 columns),
+// numbered part by part, row tile by row tile.  Every warp of the grid takes
+// one contiguous, equally sized range of units, accumulates while the row
+// tile is unchanged and adds its partial sums into z with atomics when it
+// moves on.  Lane (g, c) decodes rows g and g + 8 of a unit, one contiguous
+// run of 64 / V trellis steps of each (see layout.cuh).
+//
+// Forward in one launch (batch <= 8):
+//   1. code words of the first unit in flight, then the wait for the previous
+//      kernel (programmatic dependent launch);
+//   2. x' = H_n diag(s_in) x into shared memory when batch * n is small (every
+//      CTA computes all of it), else read from the input-transform kernel's
+//      output;
+//   3. decode + MMA over the warp's units, atomics into z;
+//   4. the output transform (QuIP# page, Fig. 2; QTIP discussion,
+//      "Incoherence Processing (W2)"): a CTA adds the units it finished in
+//      each output Hadamard block to that block's ticket; the CTA that
+//      completes a ticket owns the block, reads its z, applies
+//      y = alpha diag(s_out) H_B z, writes y and returns z and the ticket to
+//      zero for the next forward.  No CTA waits for another.
 #include <cuda_fp16.h>
 
 #include "codes.cuh"
 #include "fwht.cuh"
 #include "internal.h"
 #include "layout.cuh"
+#include "xstep.cuh"
 
 namespace qlk {
 
@@ -80,12 +109,482 @@ __device__ __forceinline__ void load_unit(uint32_t (&w)[2][K2], const uint32_t* 
     }
 }
 
+
 // Fill the per-lane replicated table (HYB, or the table code's codebook) in shared memory.
 __device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lut, int entries) {
     for (int i = threadIdx.x; i < entries * 32; i += blockDim.x) smem[i] = lut[i >> 5];
 }
 
-// A operands of the 16 m16n8k16 MMAs of one unit.  MMA u takes, for each
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The A operand paired with decode (qlinear_decode uses code_pair / code_v2 of
+// codes.cuh, which round each value to fp16; the forward uses these words).
+// 1MAD: {1536 + d, -1536} as two halves (0x6600 is 1536.0; 0xE600 is -1536.0).
+constexpr uint32_t kDp4aSplitAcc = 0xE6006600u - 510u;
+constexpr float kC1 = 443.0f / 65536.0f;  // the 1MAD scale
+
+template <int CODE, int V>
+__device__ __forceinline__ uint32_t step_word(uint32_t s, const uint32_t* lut_lane, int qshift) {
+    if constexpr (V == 2) {
+        return code_v2<CODE>(s, lut_lane, qshift);
+    } else if constexpr (CODE == kCode1MAD) {
+        return __dp4a(kA1MAD * s + kB1MAD, 0x01010101u, kDp4aSplitAcc);
+    } else if constexpr (CODE == kCode3INST) {
+        return ((kA3INST * s + kB3INST) & kMask3INST) ^ kXor3INST;
+    } else if constexpr (CODE == kCodeHYB) {
+        return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
+    } else {
+        return lut_lane[s * 32u];
+    }
+}
+
+// Decode + MMA of one unit: lane (g, c) holds, for thread-row h (row g + 8h),
+// the 32 bits before its run in cw[h][0] and its run's K2 words in
+// cw[h][1..K2].  MMA u takes the lane's steps 2u (K slots 2c, 2c+1) and 2u+1
+// (slots 2c+8, 2c+9) of rows g (a[0], a[2]) and g + 8 (a[1], a[3]); its B
+// words are word 2*(u%2) and 2*(u%2)+1 of the 16-byte group u/2.  When 16 is a
+// multiple of kV, the windows of steps t and t + 16/kV are the two halves of
+// one funnel shift, which pairs MMA u with MMA u + 8/kV.
+template <int CODE, int K2, int V, bool L16>
+struct StepMMAs {
+    static constexpr int kV = K2 * V / 2;
+    static constexpr bool kPair = (16 % kV) == 0;
+    static constexpr int MP = kPair ? 8 / kV : 0;   // MMA distance of paired windows
+    static constexpr bool kQuad = kPair && MP >= 2;  // an iteration covers MMAs u, u+1, u+MP, u+MP+1
+    static constexpr int NM = 32 / V;                // MMAs per unit
+    static constexpr int NW = K2 + 1;
+
+    template <bool XSMEM>
+    static __device__ __forceinline__ void run(const uint32_t (&cw)[2][NW], uint32_t lmask, const uint32_t* lut_lane,
+                                               int qshift, const uint4* xsrc, int xstride, bool use_x,
+                                               float (&acc)[4]) {
+#pragma unroll
+        for (int u = 0; u < NM; u += 2) {
+            if (kQuad && ((u / (kQuad ? MP : 1)) & 1)) continue;  // produced together with MMAs u - MP, u - MP + 1
+            uint32_t a[4][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = 2 * u + e;  // step of MMA u + e/2, register 2 (e % 2) + h
+                    const int q = e >> 1, r = 2 * (e & 1) + h;
+                    if constexpr (kQuad) {
+                        uint32_t s, s2;
+                        state_pair<kV, L16>(cw[h], t, lmask, s, s2);
+                        a[q][r] = step_word<CODE, V>(s, lut_lane, qshift);
+                        a[2 + q][r] = step_word<CODE, V>(s2, lut_lane, qshift);
+                    } else if constexpr (kPair) {  // MP == 1: step t pairs with step t + 2, of MMA u + 1
+                        if (e < 2) {
+                            uint32_t s, s2;
+                            state_pair<kV, L16>(cw[h], t, lmask, s, s2);
+                            a[0][r] = step_word<CODE, V>(s, lut_lane, qshift);
+                            a[1][r] = step_word<CODE, V>(s2, lut_lane, qshift);
+                        }
+                    } else {
+                        a[q][r] = step_word<CODE, V>(state_one<kV, L16>(cw[h], t, lmask), lut_lane, qshift);
+                    }
+                }
+            }
+            uint4 b0 = make_uint4(0u, 0u, 0u, 0u), b1 = b0;
+            if (use_x) {
+                b0 = XSMEM ? xsrc[(u >> 1) * xstride] : __ldg(xsrc + (u >> 1) * xstride);
+                if (kQuad) b1 = XSMEM ? xsrc[((u + MP) >> 1) * xstride] : __ldg(xsrc + ((u + MP) >> 1) * xstride);
+            }
+            mma_16816(acc, a[0], b0.x, b0.y);
+            mma_16816(acc, a[1], b0.z, b0.w);
+            if (kQuad) {
+                mma_16816(acc, a[2], b1.x, b1.y);
+                mma_16816(acc, a[3], b1.z, b1.w);
+            }
+        }
+    }
+};
+
+struct GemvPartArgs {
+    const uint32_t* words;  // the part's words, kernel layout
+    int rt;                 // row tiles
+    int row0;               // first layer row
+    int k2;                 // 2k: bits per two weights
+};
+
+struct GemvArgs {
+    GemvPartArgs part[kMaxParts];
+    int nparts;
+    int nb;                 // 256-column blocks per row
+    long long units;        // (row tile, block) units over all parts
+    uint32_t lmask;         // (1 << L) - 1
+    int qshift;             // HYB: 32 - Q
+    const uint32_t* lut;    // HYB / table code: 2^Q words
+    int lut_entries;
+    int batch;              // 1..8
+    int m, n;
+    const __half* x;        // [batch][n] (in-kernel input transform)
+    const uint32_t* sin_bits;
+    int B_n;
+    const uint4* xstep;     // x' step words from the input-transform kernel (else unused)
+    float* z;               // [batch][m], all-zero on entry and on exit
+    int* tickets;           // [m / B_m], all-zero on entry and on exit
+    int B_m;
+    const uint32_t* sout_bits;
+    float out_scale;        // alpha (times C1 for 1MAD) / sqrt(B_m)
+    void* y;                // [batch][m]
+    int y_f16;
+    int smem_floats;        // dynamic shared memory of the launch, in 4-byte words
+};
+
+// Load one unit's K2 words per thread-row into w[h][0 .. K2-1] (runtime K2 <= 8).
+template <int K2>
+__device__ __forceinline__ void load_unit_into(uint32_t (&w)[2][8], const uint32_t* unit_base, int lane) {
+    uint32_t t[2][K2];
+    load_unit<K2>(t, unit_base, lane);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < K2; ++i) w[h][i] = t[h][i];
+}
+__device__ __forceinline__ void load_unit_k2(uint32_t (&w)[2][8], const uint32_t* unit_base, int k2, int lane) {
+    switch (k2) {
+        case 2: load_unit_into<2>(w, unit_base, lane); break;
+        case 3: load_unit_into<3>(w, unit_base, lane); break;
+        case 4: load_unit_into<4>(w, unit_base, lane); break;
+        case 5: load_unit_into<5>(w, unit_base, lane); break;
+        case 6: load_unit_into<6>(w, unit_base, lane); break;
+        case 7: load_unit_into<7>(w, unit_base, lane); break;
+        default: load_unit_into<8>(w, unit_base, lane); break;
+    }
+}
+
+// One unit at K2 = 2k: take its words from nxt, start the next unit's load
+// into nxt (NXW = K2: a one-part layer; NXW = 8: the next unit's own K2),
+// then decode and multiply.
+template <int CODE, int K2, int V, bool L16, bool XSMEM, int NXW>
+__device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][NXW], const uint32_t* next_base, int next_k2, int lane,
+                                          int src_lane, const GemvArgs& p, const uint32_t* lut_lane, const uint4* xsrc,
+                                          int xstride, bool use_x, float (&acc)[4]) {
+    uint32_t cw[2][K2 + 1];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
+    if (next_base) {
+        if constexpr (NXW == K2)
+            load_unit<K2>(nxt, next_base, lane);
+        else
+            load_unit_k2(nxt, next_base, next_k2, lane);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
+    StepMMAs<CODE, K2, V, L16>::template run<XSMEM>(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
+}
+
+// The unit's bitwidth picks the decoder (V = 1 has whole bitwidths only).
+template <int CODE, int V, bool L16, bool XSMEM>
+__device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2,
+                                             int lane, int src_lane, const GemvArgs& p, const uint32_t* lut_lane,
+                                             const uint4* xsrc, int xstride, bool use_x, float (&acc)[4]) {
+#define QLK_UNIT(K) gemv_unit<CODE, K, V, L16, XSMEM, 8>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xsrc, \
+                                                         xstride, use_x, acc)
+    switch (k2) {
+        case 2: QLK_UNIT(2); break;
+        case 3: if constexpr (V == 2) QLK_UNIT(3); break;
+        case 4: QLK_UNIT(4); break;
+        case 5: if constexpr (V == 2) QLK_UNIT(5); break;
+        case 6: QLK_UNIT(6); break;
+        case 7: if constexpr (V == 2) QLK_UNIT(7); break;
+        default: QLK_UNIT(8); break;
+    }
+#undef QLK_UNIT
+}
+
+// x' = H_n diag(s_in) x for every batch row, as step words in shared memory
+// (fp32 transform in `work`, then one rounding to fp16).
+template <int V>
+__device__ __forceinline__ void input_transform_smem(const GemvArgs& p, uint32_t* xs_words, float* work) {
+    const int n = p.n, batch = p.batch;
+    const float scale = rsqrtf((float)p.B_n);
+    fwht_blocks_smem(
+        work, batch * n, p.B_n,
+        [&](int i, float (&v)[8]) {
+            const int b = i / n, col = i - b * n;
+            const uint4 raw = *reinterpret_cast<const uint4*>(p.x + (size_t)b * n + col);
+            const uint32_t sw = p.sin_bits[col >> 5] >> (col & 31);  // 8 consecutive sign bits (col % 8 == 0)
+            const __half* hv = reinterpret_cast<const __half*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float f = __half2float(hv[e]);
+                v[e] = ((sw >> e) & 1u) ? -f : f;
+            }
+        },
+        [&](int i, const float (&v)[4]) {
+            const int b = i / n, col = i - b * n;
+            const float w[4] = {v[0] * scale, v[1] * scale, v[2] * scale, v[3] * scale};
+            store_xstep4<V>(xs_words, col, b, batch, w);
+        });
+    __syncthreads();
+}
+
+// The output transform of Hadamard block hb for every batch row (as many rows
+// at once as `buf` holds): y = out_scale * s_out (H z); z returns to zero.
+__device__ __forceinline__ void output_transform_block(const GemvArgs& p, int hb, float* buf) {
+    const int B = p.B_m, m = p.m;
+    int rows = p.smem_floats / (B + B / 16);
+    rows = rows < 1 ? 1 : (rows > p.batch ? p.batch : rows);
+    for (int b0 = 0; b0 < p.batch; b0 += rows) {
+        const int nr = p.batch - b0 < rows ? p.batch - b0 : rows;
+        fwht_blocks_smem(
+            buf, nr * B, B,
+            [&](int i, float (&v)[8]) {
+                const int bb = b0 + i / B, r = hb * B + (i % B);
+                float4* zp = reinterpret_cast<float4*>(p.z + (size_t)bb * m + r);
+                const float4 t0 = __ldcg(zp), t1 = __ldcg(zp + 1);
+                __stcg(zp, make_float4(0.f, 0.f, 0.f, 0.f));
+                __stcg(zp + 1, make_float4(0.f, 0.f, 0.f, 0.f));
+                v[0] = t0.x, v[1] = t0.y, v[2] = t0.z, v[3] = t0.w;
+                v[4] = t1.x, v[5] = t1.y, v[6] = t1.z, v[7] = t1.w;
+            },
+            [&](int i, const float (&v)[4]) {
+                const int bb = b0 + i / B, r = hb * B + (i % B);
+                const uint32_t sw = p.sout_bits[r >> 5] >> (r & 31);  // r % 4 == 0
+                float o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) o[q] = ((sw >> q) & 1u) ? -v[q] * p.out_scale : v[q] * p.out_scale;
+                if (p.y_f16) {
+                    *reinterpret_cast<uint2*>((__half*)p.y + (size_t)bb * m + r) =
+                        make_uint2(half2_bits(o[0], o[1]), half2_bits(o[2], o[3]));
+                } else {
+                    *reinterpret_cast<float4*>((float*)p.y + (size_t)bb * m + r) = make_float4(o[0], o[1], o[2], o[3]);
+                }
+            });
+        __syncthreads();
+    }
+}
+
+// After the CTA's last atomics into z: count its units into the tickets of the
+// Hadamard blocks they touch and transform the blocks it completes.
+constexpr int kEpiOwnedMax = 32;
+__device__ __forceinline__ void output_epilogue(const GemvArgs& p, float* buf, long long c0, long long c1) {
+    __shared__ int owned[kEpiOwnedMax];
+    __shared__ int n_owned;
+    __threadfence();  // this thread's atomics into z are visible device-wide before the ticket
+    __syncthreads();
+    if (c0 >= c1) return;  // uniform over the CTA
+    const long long uph = (long long)(p.B_m / kRowTile) * p.nb;  // units per output Hadamard block
+    const int hb_first = (int)(c0 / uph), hb_last = (int)((c1 - 1) / uph);
+    for (int hb0 = hb_first; hb0 <= hb_last; hb0 += kEpiOwnedMax) {
+        if (threadIdx.x == 0) {
+            int cnt = 0;
+            for (int hb = hb0; hb <= hb_last && hb < hb0 + kEpiOwnedMax; ++hb) {
+                const long long lo = c0 > hb * uph ? c0 : hb * uph;
+                const long long hi = c1 < (hb + 1) * uph ? c1 : (hb + 1) * uph;
+                const int mine = (int)(hi - lo);
+                const int prev = atomicAdd(p.tickets + hb, mine);
+                if ((long long)(prev + mine) == uph) {
+                    owned[cnt++] = hb;
+                    p.tickets[hb] = 0;  // every unit of the block is in: no other CTA touches this ticket again
+                }
+            }
+            n_owned = cnt;
+            __threadfence();  // the other CTAs' z sums, published before their tickets, are read after this
+        }
+        __syncthreads();
+        const int cnt = n_owned;
+        for (int i = 0; i < cnt; ++i) output_transform_block(p, owned[i], buf);
+        __syncthreads();
+    }
+}
+
+// One CTA per SM (at most).  CTA i takes units [U*i/G, U*(i+1)/G) and splits
+// them evenly over its warps.  K2F: the bitwidth of a one-part layer (decoder
+// fixed at compile time), 0 for several parts (decoder per unit).  Every
+// thread runs every phase, since the transforms use CTA barriers.
+template <int CODE, int V, bool L16, bool XSMEM, int K2F>
+__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(GemvArgs p) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int NXW = K2F ? K2F : 8;
+    const int lane = threadIdx.x & 31;
+    const int lut_words = uses_table(CODE) ? p.lut_entries * 32 : 0;
+    uint32_t* xs_words = smem + lut_words;
+    float* work = reinterpret_cast<float*>(smem + lut_words + (XSMEM ? p.batch * p.n / V : 0));
+    if (uses_table(CODE)) fill_lut_smem(smem, p.lut, p.lut_entries);
+    const uint32_t* lut_lane = smem + lane;
+
+    const int nb = p.nb;
+    const long long U = p.units;
+    const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
+    const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
+    const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
+    const int g = lane >> 2, c = lane & 3;
+    const int src_lane = (lane & ~3) | ((c + 3) & 3);
+    const int batch = p.batch;
+
+    // walker over (part, row tile, block)
+    int pt = 0;
+    long long rest = u0;
+    while (pt + 1 < p.nparts && rest >= (long long)p.part[pt].rt * nb) rest -= (long long)p.part[pt++].rt * nb;
+    int t = (int)(rest / nb), j = (int)(rest % nb);
+    auto unit_base = [&](int part, int tile, int blk) {
+        return p.part[part].words + ((size_t)tile * nb + blk) * 64 * p.part[part].k2;
+    };
+    // Programmatic dependent launch: the code words, the tables and the sign
+    // bits are written once at create time, so the first unit's words are
+    // fetched before waiting for the previous kernel (the producer of x or x',
+    // the previous forward that used z).
+    uint32_t nxt[2][NXW];
+    if (u0 < u1) {
+        if constexpr (K2F != 0)
+            load_unit<K2F>(nxt, unit_base(pt, t, j), lane);
+        else
+            load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
+    }
+    grid_dependency_wait();
+    if constexpr (XSMEM)
+        input_transform_smem<V>(p, xs_words, work);  // ends with a CTA barrier (the table is filled too)
+    else if (uses_table(CODE))
+        __syncthreads();
+    grid_launch_dependents();
+
+    const uint4* xbase = XSMEM ? reinterpret_cast<const uint4*>(xs_words) : p.xstep;
+    const int xstride = batch * 4;  // uint4 groups between consecutive u2
+    const bool use_x = g < batch;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int cur_pt = pt, cur_t = t;
+    auto flush = [&](int part, int tile) {
+        const int row = p.part[part].row0 + tile * kRowTile + g;
+        const int b0 = 2 * c, b1 = 2 * c + 1;
+        if (b0 < batch) {
+            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
+            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
+        }
+        if (b1 < batch) {
+            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
+            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
+        }
+    };
+    for (long long unit = u0; unit < u1; ++unit) {
+        int npt = pt, nt = t, nj = j + 1;  // the unit after this one, for the prefetch
+        if (nj == nb) {
+            nj = 0;
+            if (++nt == p.part[npt].rt && npt + 1 < p.nparts) {
+                nt = 0;
+                ++npt;
+            }
+        }
+        const uint32_t* next_base = unit + 1 < u1 ? unit_base(npt, nt, nj) : nullptr;
+        if (pt != cur_pt || t != cur_t) {
+            flush(cur_pt, cur_t);
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            cur_pt = pt;
+            cur_t = t;
+        }
+        const uint4* xsrc = xbase + ((size_t)j * (16 / V) * batch + g) * 4 + c;
+        if constexpr (K2F != 0)
+            gemv_unit<CODE, K2F, V, L16, XSMEM, NXW>(nxt, next_base, K2F, lane, src_lane, p, lut_lane, xsrc, xstride,
+                                                     use_x, acc);
+        else
+            gemv_unit_k2<CODE, V, L16, XSMEM>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p,
+                                              lut_lane, xsrc, xstride, use_x, acc);
+        pt = npt;
+        t = nt;
+        j = nj;
+    }
+    if (u0 < u1) flush(cur_pt, cur_t);
+    output_epilogue(p, reinterpret_cast<float*>(smem), c0, c1);
+}
+
+// ---- the forward's launch plan and dispatch ----
+
+GemvPlan plan_gemv(const Layer& L, int batch) {
+    GemvPlan pl;
+    long long units = 0;
+    for (int i = 0; i < L.nparts; ++i) units += (long long)(L.parts[i].rows / kRowTile) * (L.n / kT);
+    pl.grid = (int)(units < L.num_sms ? units : L.num_sms);
+    const long long per_cta = (units + pl.grid - 1) / pl.grid;
+    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
+    pl.threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
+    const long long lut_words = uses_table(L.code) ? (32ll << L.Q) : 0;
+    const long long elems = (long long)batch * L.n;
+    const long long xs_words = elems / L.V;
+    const long long work_words = elems + elems / 16;
+    const long long budget = kGemvMaxSmem / 4;
+    pl.xsmem = elems <= kFuseInElems && lut_words + xs_words + work_words <= budget;
+    long long main_words = lut_words + (pl.xsmem ? xs_words + work_words : 0);
+    // the output transform: as many batch rows of one Hadamard block as fit
+    const long long row_words = L.B_m + L.B_m / 16;
+    long long rows = budget / row_words;
+    if (rows > batch) rows = batch;
+    if (rows < 1) rows = 1;
+    const long long epi_words = rows * row_words;
+    pl.smem_bytes = (int)((main_words > epi_words ? main_words : epi_words) * 4);
+    return pl;
+}
+
+size_t gemv_xstep_bytes(const Layer& L, int batch) { return (size_t)batch * L.n / L.V * 4; }
+
+template <int CODE, int K2, int V, bool L16>
+struct GemvLaunch {
+    template <bool XSMEM>
+    static cudaError_t go(const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
+        constexpr int K2F = K2 == 99 ? 0 : K2;
+        cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, V, L16, XSMEM, K2F>>(kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(trellis_gemv_kernel<CODE, V, L16, XSMEM, K2F>, dim3(pl.grid), dim3(pl.threads),
+                          (size_t)pl.smem_bytes, st, a);
+    }
+    static cudaError_t run(const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
+        return pl.xsmem ? go<true>(a, pl, st) : go<false>(a, pl, st);
+    }
+};
+
+template <int CODE, int K2, int V, bool L16>
+struct GemvPrepare {
+    static cudaError_t run() {
+        constexpr int K2F = K2 == 99 ? 0 : K2;
+        cudaError_t e = preload_kernel<trellis_gemv_kernel<CODE, V, L16, true, K2F>>(kGemvMaxSmem);
+        if (e == cudaSuccess) e = preload_kernel<trellis_gemv_kernel<CODE, V, L16, false, K2F>>(kGemvMaxSmem);
+        return e;
+    }
+};
+
+// A multi-part layer takes the per-unit decoder (the "K2 = 99" instance).
+template <int CODE, int V, bool L16>
+static cudaError_t gemv_multi_dispatch(const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
+    return GemvLaunch<CODE, 99, V, L16>::run(a, pl, st);
+}
+
+template <bool L16>
+static cudaError_t gemv_multi_prepare(int code, int V) {
+    if (code == kCode1MAD && V == 1) return GemvPrepare<kCode1MAD, 99, 1, L16>::run();
+    if (code == kCode3INST && V == 1) return GemvPrepare<kCode3INST, 99, 1, L16>::run();
+    if (code == kCodeHYB && V == 1) return GemvPrepare<kCodeHYB, 99, 1, L16>::run();
+    if (code == kCodeHYB && V == 2) return GemvPrepare<kCodeHYB, 99, 2, L16>::run();
+    if constexpr (!L16) {
+        if (code == kCodeTable && V == 1) return GemvPrepare<kCodeTable, 99, 1, false>::run();
+        if (code == kCodeTable && V == 2) return GemvPrepare<kCodeTable, 99, 2, false>::run();
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <bool L16>
+static cudaError_t gemv_multi_l(int code, int V, const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
+    if (code == kCode1MAD && V == 1) return gemv_multi_dispatch<kCode1MAD, 1, L16>(a, pl, st);
+    if (code == kCode3INST && V == 1) return gemv_multi_dispatch<kCode3INST, 1, L16>(a, pl, st);
+    if (code == kCodeHYB && V == 1) return gemv_multi_dispatch<kCodeHYB, 1, L16>(a, pl, st);
+    if (code == kCodeHYB && V == 2) return gemv_multi_dispatch<kCodeHYB, 2, L16>(a, pl, st);
+    if constexpr (!L16) {
+        if (code == kCodeTable && V == 1) return gemv_multi_dispatch<kCodeTable, 1, false>(a, pl, st);
+        if (code == kCodeTable && V == 2) return gemv_multi_dispatch<kCodeTable, 2, false>(a, pl, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// qlinear_decode: the fp16-rounded values of one unit in the order of 16
+// m16n8k16 A operands (two weights per register).  MMA u takes, for each
 // thread-row h (row g for h = 0, row g + 8 for h = 1), the lane's columns
 // 4u .. 4u+3 of its run, i.e. steps 4u .. 4u+3 (V = 1) or 2u, 2u+1 (V = 2):
 //   a[0] = row g, columns 4u, 4u+1      a[2] = row g, columns 4u+2, 4u+3
@@ -155,386 +654,6 @@ __device__ __forceinline__ void for_each_mma(const uint32_t (&cw)[2][K2 + 1], ui
         f(u, a);
         if (D::kPair) f(u + D::MP, a2);
     }
-}
-
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-struct GemvArgs {
-    DecodeArgs dec;
-    const uint2* xf;  // x' fragment layout in global memory (when x' is not computed in-kernel)
-    int batch;        // 1..8
-    float* z;         // [batch][m], all-zero on entry (the output transform re-zeroes it)
-    int m;
-    int row0;         // first layer row of the part
-    // input transform in-kernel (XSMEM): x' = H_n diag(s_in) x into shared memory
-    const __half* x;  // [batch][n]
-    const uint32_t* sin_bits;
-    int n, B_n;
-    int groups_in;    // thread groups (B_n/8 threads each) of the in-kernel input transform
-};
-
-// x' = H_n diag(s_in) x for every column and batch row, fp16, into the
-// fragment layout in shared memory.  Groups of B_n/kXinE threads take one
-// (batch row, Hadamard block) at a time; all threads run the same rounds.
-// prepare() runs before the wait for the previous kernel (the sign bits are
-// written once at create time); run() reads x, which that kernel may produce.
-constexpr int kXinE = 8;  // entries per thread of the in-kernel input transform
-struct InputTransform {
-    int B, T, G, grp, tid, per_row, total;
-    uint32_t sw0;  // sign bits of the thread's entries in the first round
-    __device__ __forceinline__ void prepare(const GemvArgs& p) {
-        B = p.B_n;
-        T = B / kXinE;
-        G = p.groups_in;  // groups with their own FWHT scratch; spare threads only join barriers
-        grp = threadIdx.x / T;
-        tid = threadIdx.x - grp * T;
-        per_row = p.n / B;
-        total = p.batch * per_row;
-        sw0 = 0;
-        if (grp < G && grp < total) {
-            const int col = (grp % per_row) * B + tid * kXinE;
-            sw0 = p.sin_bits[col >> 5] >> (col & 31);
-        }
-    }
-    __device__ __forceinline__ void run(const GemvArgs& p, __half* xs, float* fw) const {
-        const float scale = rsqrtf((float)B);
-        for (int r0 = 0; r0 < total; r0 += G) {
-            const int item = r0 + grp;
-            const bool active = grp < G && item < total;
-            const int b = active ? item / per_row : 0;
-            const int col = (active ? (item % per_row) * B : 0) + tid * kXinE;
-            float v[kXinE];
-            if (active) {
-                const __half* src = p.x + (size_t)b * p.n + col;
-                const uint32_t sw = r0 == 0 ? sw0 : p.sin_bits[col >> 5] >> (col & 31);
-                const uint4 raw = *reinterpret_cast<const uint4*>(src);
-                const __half* hv = reinterpret_cast<const __half*>(&raw);
-#pragma unroll
-                for (int e = 0; e < kXinE; ++e) {
-                    const float f = __half2float(hv[e]);
-                    v[e] = ((sw >> e) & 1u) ? -f : f;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < kXinE; ++e) v[e] = 0.f;
-            }
-            fwht_block<kXinE>(v, B, tid, T, fw + (size_t)(grp < G ? grp : 0) * (B + B / 16), grp < G);
-            if (active) {
-#pragma unroll
-                for (int q = 0; q < kXinE; q += 4) {
-                    const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
-                    const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
-                    uint2 w;
-                    w.x = *reinterpret_cast<const uint32_t*>(&lo);
-                    w.y = *reinterpret_cast<const uint32_t*>(&hi);
-                    *reinterpret_cast<uint2*>(xs + frag_index4(col + q, b, p.batch)) = w;
-                }
-            }
-            __syncthreads();
-        }
-    }
-};
-
-// One CTA per SM.  CTA i takes units [U*i/G, U*(i+1)/G) of the part (G CTAs)
-// and splits them evenly over its warps; the launcher sizes the CTA so that
-// every warp gets the same whole number of units (to within one), which keeps
-// every SM and every warp equally loaded.  Every thread runs every phase (no
-// early exit), since the in-kernel transforms use CTA barriers.
-template <int CODE, int K2, int V, bool L16, bool XSMEM>
-__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(GemvArgs p, GemvSmem sm) {
-    extern __shared__ uint32_t smem[];
-    using UL = UnitLayout<K2>;
-    uint32_t* lut_smem = smem;
-    __half* xs = reinterpret_cast<__half*>(smem + sm.lut_words);
-    float* fw = reinterpret_cast<float*>(smem + sm.lut_words + sm.xs_words);
-    const int lane = threadIdx.x & 31;
-    if (uses_table(CODE)) {
-        fill_lut_smem(lut_smem, p.dec.lut, p.dec.lut_entries);
-        __syncthreads();
-    }
-    const uint32_t* lut_lane = lut_smem + lane;
-    const int nb = p.dec.nb;
-    const long long U = (long long)p.dec.rt * nb;
-    const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
-    const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
-    const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
-
-    const int g = lane >> 2, c = lane & 3;
-    const int src_lane = (lane & ~3) | ((c + 3) & 3);
-    const int batch = p.batch;
-
-    uint32_t nxt[2][K2];
-    if (u0 < u1) load_unit<K2>(nxt, p.dec.words + u0 * UL::UW, lane);
-    // Programmatic dependent launch: the code words, the table and the
-    // sign bits are written once at create time, so they are fetched before
-    // waiting for the previous kernel (the producer of x or x', the consumer
-    // of the last z).
-    InputTransform xin;
-    if (XSMEM) xin.prepare(p);
-    grid_dependency_wait();
-    if (XSMEM) xin.run(p, xs, fw);
-    grid_launch_dependents();
-
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int R = (int)(u0 / nb), j = (int)(u0 % nb);
-    int curR = R;
-    auto flush = [&](int tile) {
-        const int row = p.row0 + tile * kRowTile + g;
-        const int b0 = 2 * c, b1 = 2 * c + 1;
-        if (b0 < batch) {
-            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
-            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
-        }
-        if (b1 < batch) {
-            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
-            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
-        }
-    };
-
-    for (long long unit = u0; unit < u1; ++unit) {
-        uint32_t cw[2][K2 + 1];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
-        if (unit + 1 < u1) load_unit<K2>(nxt, p.dec.words + (unit + 1) * UL::UW, lane);
-        if (R != curR) {
-            flush(curR);
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-            curR = R;
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
-
-        const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
-        for_each_mma<CODE, K2, V, L16>(cw, p.dec.lmask, lut_lane, p.dec.qshift, [&](int u, const uint32_t(&a)[4]) {
-            uint2 bv = make_uint2(0u, 0u);
-            if (g < batch) {
-                if (XSMEM)
-                    bv = reinterpret_cast<const uint2*>(xs)[xoff + (size_t)u * batch * 4];
-                else
-                    bv = __ldg(p.xf + xoff + (size_t)u * batch * 4);
-            }
-            mma_16816(acc, a, bv.x, bv.y);
-        });
-        if (++j == nb) {
-            j = 0;
-            ++R;
-        }
-    }
-    if (u0 < u1) flush(curR);
-}
-
-// ---- decode-GEMV over all row parts of a layer in one launch ----
-// Units are numbered part by part (each part's row tiles x blocks, as in the
-// single-part kernel); a warp's contiguous range may cross into the next part,
-// whose bitwidth it dispatches per unit.  x' comes in the fragment layout from
-// the separate input-transform kernel.
-struct GemvPartArgs {
-    const uint32_t* words;  // the part's words, kernel layout
-    int rt;                 // row tiles
-    int row0;               // first layer row
-    int k2;                 // 2k: bits per two weights
-};
-struct GemvMultiArgs {
-    GemvPartArgs part[kMaxParts];
-    int nparts, nb;
-    uint32_t lmask;
-    int qshift;
-    const uint32_t* lut;
-    int lut_entries;
-    const uint2* xf;
-    int batch;
-    float* z;
-    int m;
-};
-
-// Two thread-rows of one unit at K2 = 2k into w[h][0 .. K2-1].
-template <int K2>
-__device__ __forceinline__ void load_unit_into(uint32_t (&w)[2][8], const uint32_t* unit_base, int lane) {
-    uint32_t t[2][K2];
-    load_unit<K2>(t, unit_base, lane);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int i = 0; i < K2; ++i) w[h][i] = t[h][i];
-}
-__device__ __forceinline__ void load_unit_k2(uint32_t (&w)[2][8], const uint32_t* unit_base, int k2, int lane) {
-    switch (k2) {
-        case 2: load_unit_into<2>(w, unit_base, lane); break;
-        case 3: load_unit_into<3>(w, unit_base, lane); break;
-        case 4: load_unit_into<4>(w, unit_base, lane); break;
-        case 5: load_unit_into<5>(w, unit_base, lane); break;
-        case 6: load_unit_into<6>(w, unit_base, lane); break;
-        case 7: load_unit_into<7>(w, unit_base, lane); break;
-        default: load_unit_into<8>(w, unit_base, lane); break;
-    }
-}
-
-// One unit at K2 = 2k: take its words from nxt, start the next unit's load
-// into nxt, then decode and multiply.
-template <int CODE, int K2, int V, bool L16>
-__device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2, int lane,
-                                          int src_lane, const GemvMultiArgs& p, const uint32_t* lut_lane,
-                                          size_t xoff, bool use_x, float (&acc)[4]) {
-    uint32_t cw[2][K2 + 1];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
-    if (next_base) load_unit_k2(nxt, next_base, next_k2, lane);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
-    for_each_mma<CODE, K2, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
-        uint2 bv = make_uint2(0u, 0u);
-        if (use_x) bv = __ldg(p.xf + xoff + (size_t)u * p.batch * 4);
-        mma_16816(acc, a, bv.x, bv.y);
-    });
-}
-
-// The unit's bitwidth picks the decoder (V = 1 has whole bitwidths only).
-template <int CODE, int V, bool L16>
-__device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2,
-                                             int lane, int src_lane, const GemvMultiArgs& p,
-                                             const uint32_t* lut_lane, size_t xoff, bool use_x, float (&acc)[4]) {
-    switch (k2) {
-        case 2: gemv_unit<CODE, 2, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        case 3: if constexpr (V == 2) gemv_unit<CODE, 3, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        case 4: gemv_unit<CODE, 4, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        case 5: if constexpr (V == 2) gemv_unit<CODE, 5, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        case 6: gemv_unit<CODE, 6, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        case 7: if constexpr (V == 2) gemv_unit<CODE, 7, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-        default: gemv_unit<CODE, 8, V, L16>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xoff, use_x, acc); break;
-    }
-}
-
-template <int CODE, int V, bool L16>
-__global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_multi_kernel(GemvMultiArgs p) {
-    extern __shared__ uint32_t smem[];
-    const int lane = threadIdx.x & 31;
-    if (uses_table(CODE)) {
-        fill_lut_smem(smem, p.lut, p.lut_entries);
-        __syncthreads();
-    }
-    const uint32_t* lut_lane = smem + lane;
-    const int nb = p.nb;
-    long long U = 0;
-    for (int i = 0; i < p.nparts; ++i) U += (long long)p.part[i].rt * nb;
-    const long long c0 = U * blockIdx.x / gridDim.x, c1 = U * (blockIdx.x + 1) / gridDim.x;
-    const int wpb = blockDim.x >> 5, w = threadIdx.x >> 5;
-    const long long u0 = c0 + (c1 - c0) * w / wpb, u1 = c0 + (c1 - c0) * (w + 1) / wpb;
-    const int g = lane >> 2, c = lane & 3;
-    const int src_lane = (lane & ~3) | ((c + 3) & 3);
-    const int batch = p.batch;
-
-    // walker: part pt, row tile t within it, block j
-    int pt = 0;
-    long long rest = u0;
-    while (pt + 1 < p.nparts && rest >= (long long)p.part[pt].rt * nb) rest -= (long long)p.part[pt++].rt * nb;
-    int t = (int)(rest / nb), j = (int)(rest % nb);
-    auto unit_base = [&](int part, int tile, int blk) {
-        return p.part[part].words + ((size_t)tile * nb + blk) * 64 * p.part[part].k2;
-    };
-    uint32_t nxt[2][8];
-    if (u0 < u1) load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
-    grid_dependency_wait();  // x' from the input transform; z consumed by the last output transform
-    grid_launch_dependents();
-
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int cur_pt = pt, cur_t = t;
-    auto flush = [&](int part, int tile) {
-        const int row = p.part[part].row0 + tile * kRowTile + g;
-        const int b0 = 2 * c, b1 = 2 * c + 1;
-        if (b0 < batch) {
-            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
-            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
-        }
-        if (b1 < batch) {
-            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
-            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
-        }
-    };
-    for (long long unit = u0; unit < u1; ++unit) {
-        // the unit after this one, for the prefetch
-        int npt = pt, nt = t, nj = j + 1;
-        if (nj == nb) {
-            nj = 0;
-            if (++nt == p.part[npt].rt && npt + 1 < p.nparts) {
-                nt = 0;
-                ++npt;
-            }
-        }
-        const uint32_t* next_base = unit + 1 < u1 ? unit_base(npt, nt, nj) : nullptr;
-        if (pt != cur_pt || t != cur_t) {
-            flush(cur_pt, cur_t);
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-            cur_pt = pt;
-            cur_t = t;
-        }
-        const size_t xoff = (size_t)j * 16 * batch * 4 + g * 4 + c;
-        const bool use_x = g < batch;
-        gemv_unit_k2<CODE, V, L16>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p, lut_lane, xoff,
-                                   use_x, acc);
-        pt = npt;
-        t = nt;
-        j = nj;
-    }
-    if (u0 < u1) flush(cur_pt, cur_t);
-}
-
-template <int CODE, int V, bool L16>
-static cudaError_t launch_gemv_multi_t(const GemvMultiArgs& a, int grid, int threads, size_t smem, cudaStream_t st) {
-    auto kern = trellis_gemv_multi_kernel<CODE, V, L16>;
-    cudaError_t e = ensure_smem_limit<trellis_gemv_multi_kernel<CODE, V, L16>>(kGemvMaxSmem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a);
-}
-
-cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, float* z, cudaStream_t st) {
-    GemvMultiArgs a;
-    a.nparts = L.nparts;
-    a.nb = L.n / kT;
-    long long units = 0;
-    for (int i = 0; i < kMaxParts; ++i) {
-        const Part& pt = L.parts[i < L.nparts ? i : 0];
-        a.part[i].words = L.words + pt.word_off;
-        a.part[i].rt = pt.rows / kRowTile;
-        a.part[i].row0 = pt.row0;
-        a.part[i].k2 = pt.k2;
-        if (i < L.nparts) units += (long long)a.part[i].rt * a.nb;
-    }
-    a.lmask = (1u << L.L) - 1u;
-    a.qshift = 32 - L.Q;
-    a.lut = L.lut;
-    a.lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
-    a.xf = (const uint2*)xp_frag;
-    a.batch = batch;
-    a.z = z;
-    a.m = L.m;
-    // one CTA per SM, warps sized so that every warp gets the same whole number of units
-    const int grid = (int)(units < L.num_sms ? units : L.num_sms);
-    const long long per_cta = (units + grid - 1) / grid;
-    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
-    const int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
-    const size_t smem = (size_t)a.lut_entries * 32 * 4;
-    const bool l16 = L.L == 16;
-    if (L.code == kCode1MAD && L.V == 1) return l16 ? launch_gemv_multi_t<kCode1MAD, 1, true>(a, grid, threads, smem, st)
-                                                    : launch_gemv_multi_t<kCode1MAD, 1, false>(a, grid, threads, smem, st);
-    if (L.code == kCode3INST && L.V == 1) return l16 ? launch_gemv_multi_t<kCode3INST, 1, true>(a, grid, threads, smem, st)
-                                                     : launch_gemv_multi_t<kCode3INST, 1, false>(a, grid, threads, smem, st);
-    if (L.code == kCodeHYB && L.V == 1) return l16 ? launch_gemv_multi_t<kCodeHYB, 1, true>(a, grid, threads, smem, st)
-                                                   : launch_gemv_multi_t<kCodeHYB, 1, false>(a, grid, threads, smem, st);
-    if (L.code == kCodeHYB && L.V == 2) return l16 ? launch_gemv_multi_t<kCodeHYB, 2, true>(a, grid, threads, smem, st)
-                                                   : launch_gemv_multi_t<kCodeHYB, 2, false>(a, grid, threads, smem, st);
-    if (L.code == kCodeTable && !l16) return L.V == 1 ? launch_gemv_multi_t<kCodeTable, 1, false>(a, grid, threads, smem, st)
-                                                      : launch_gemv_multi_t<kCodeTable, 2, false>(a, grid, threads, smem, st);
-    return cudaErrorInvalidValue;
 }
 
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
@@ -656,94 +775,6 @@ static DecodeArgs make_decode_args(const Layer& L, const Part& part) {
     return d;
 }
 
-// The in-kernel input transform has instances for L = 16 and for the table code.
-template <int CODE, int K2, int V, bool L16>
-struct GemvLaunch {
-    static cudaError_t run(const GemvArgs& a, const GemvSmem& sm, bool xsmem, int grid, int threads,
-                           cudaStream_t st) {
-        const size_t smem = (size_t)(sm.lut_words + sm.xs_words + sm.fw_words) * 4;
-        if (xsmem) {
-            if constexpr (L16 || CODE == kCodeTable) {
-                auto kern = trellis_gemv_kernel<CODE, K2, V, L16, true>;
-                cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, K2, V, L16, true>>(kGemvMaxSmem);
-                if (e != cudaSuccess) return e;
-                return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
-            } else {
-                return cudaErrorInvalidValue;
-            }
-        }
-        auto kern = trellis_gemv_kernel<CODE, K2, V, L16, false>;
-        cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, K2, V, L16, false>>(kGemvMaxSmem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, a, sm);
-    }
-};
-
-// CTA shape: one CTA per SM, warps sized so every warp gets the same whole
-// number of units.  The input transform runs in-kernel (each CTA computes
-// x' into its shared memory while its first code words are in flight) when
-// x is small; otherwise a separate kernel writes x' to global memory.
-GemvPlan plan_gemv(const Layer& L, const Part& part, int batch) {
-    GemvPlan pl;
-    const long long nb = L.n / kT;
-    const long long units = (long long)(part.rows / kRowTile) * nb;
-    pl.grid = (int)(units < L.num_sms ? units : L.num_sms);
-    const long long per_cta = (units + pl.grid - 1) / pl.grid;
-    const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
-    int threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
-    const int lut_words = uses_table(L.code) ? (32 << L.Q) : 0;
-    const int budget = kGemvMaxSmem / 4 - lut_words;
-    const int t_in = L.B_n / kXinE;
-    const int xs_words = batch * L.n / 2;
-    pl.xsmem = (L.L == 16 || L.code == kCodeTable) && L.nparts == 1 && (long long)batch * L.n <= kFuseInElems &&
-               t_in <= kGemvMaxWarps * 32;
-    int fw = 0;
-    pl.groups_in = 0;
-    const int threads_decode = threads;
-    if (pl.xsmem) {
-        if (threads < t_in) threads = t_in;
-        // thread groups of B_n/kXinE threads; a group of more than a warp needs
-        // its own FWHT scratch (B_n + B_n/16 floats)
-        int g = threads / t_in;
-        const int work = batch * (L.n / L.B_n);
-        if (g > work) g = work;
-        if (g < 1) g = 1;
-        if (t_in > 32) {
-            const int per = L.B_n + L.B_n / 16;
-            while (g > 1 && xs_words + g * per > budget) --g;
-            fw = g * per;
-        }
-        pl.groups_in = g;
-        if (xs_words + fw > budget) pl.xsmem = false, fw = 0, pl.groups_in = 0;
-        // every CTA runs the transform before its first MMA: only worth it when
-        // it takes a single round (one group per (batch row, Hadamard block))
-        if (g < work) pl.xsmem = false, fw = 0, pl.groups_in = 0;
-        if (!pl.xsmem) threads = threads_decode;
-    }
-    pl.threads = threads;
-    pl.sm.lut_words = lut_words;
-    pl.sm.xs_words = pl.xsmem ? xs_words : 0;
-    pl.sm.fw_words = fw;
-    return pl;
-}
-
-cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
-                        int batch, float* z, cudaStream_t st) {
-    GemvArgs a;
-    a.dec = make_decode_args(L, part);
-    a.xf = (const uint2*)xp_frag;
-    a.batch = batch;
-    a.z = z;
-    a.m = L.m;
-    a.row0 = part.row0;
-    a.x = (const __half*)x;
-    a.sin_bits = L.sin_bits;
-    a.n = L.n;
-    a.B_n = L.B_n;
-    a.groups_in = pl.groups_in;
-    return dispatch<GemvLaunch>(L.code, part.k2, L.V, L.L == 16, a, pl.sm, pl.xsmem, pl.grid, pl.threads, st);
-}
-
 template <int CODE, int K2, int V, bool L16>
 struct DecodeLaunch {
     static cudaError_t run(const DecodeArgs& d, __half* w, int n, int row0, int grid, cudaStream_t st) {
@@ -765,6 +796,14 @@ cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStr
     if (grid > (long long)L.num_sms * 8) grid = (long long)L.num_sms * 8;
     return dispatch<DecodeLaunch>(L.code, part.k2, L.V, L.L == 16, d, (__half*)w_hat, L.n, part.row0, (int)grid, st);
 }
+
+template <int CODE, int K2, int V, bool L16>
+struct DecodePrepare {
+    static cudaError_t run() {
+        const bool big = uses_table(CODE) && (32 << kMaxTableBits) * 4 > 48 * 1024;
+        return preload_kernel<trellis_decode_kernel<CODE, K2, V, L16>>(big ? 32 * 512 * 4 : 0);
+    }
+};
 
 template <int CODE, int K2, int V, bool L16>
 struct EvalLaunch {
@@ -790,6 +829,53 @@ cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_
     const int entries = uses_table(code) ? (1 << Q) : 0;
     return dispatch<EvalLaunch>(code, 2, V, code != kCodeTable, states, count, lmask, 32 - Q, lut_words, entries,
                                 (__half*)out, st);
+}
+
+
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
+                        int* tickets, void* y, int y_dtype, cudaStream_t st) {
+    GemvArgs a;
+    a.nparts = L.nparts;
+    a.nb = L.n / kT;
+    a.units = 0;
+    for (int i = 0; i < kMaxParts; ++i) {
+        const Part& pt = L.parts[i < L.nparts ? i : 0];
+        a.part[i].words = L.words + pt.word_off;
+        a.part[i].rt = pt.rows / kRowTile;
+        a.part[i].row0 = pt.row0;
+        a.part[i].k2 = pt.k2;
+        if (i < L.nparts) a.units += (long long)a.part[i].rt * a.nb;
+    }
+    a.lmask = (1u << L.L) - 1u;
+    a.qshift = 32 - L.Q;
+    a.lut = L.lut;
+    a.lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
+    a.batch = batch;
+    a.m = L.m;
+    a.n = L.n;
+    a.x = (const __half*)x;
+    a.sin_bits = L.sin_bits;
+    a.B_n = L.B_n;
+    a.xstep = (const uint4*)xstep;
+    a.z = z;
+    a.tickets = tickets;
+    a.B_m = L.B_m;
+    a.sout_bits = L.sout_bits;
+    a.out_scale = L.alpha * (L.code == kCode1MAD ? kC1 : 1.0f) / sqrtf((float)L.B_m);
+    a.y = y;
+    a.y_f16 = y_dtype == QL_F16;
+    a.smem_floats = pl.smem_bytes / 4;
+    const bool l16 = L.L == 16;
+    if (L.nparts > 1) return l16 ? gemv_multi_l<true>(L.code, L.V, a, pl, st) : gemv_multi_l<false>(L.code, L.V, a, pl, st);
+    return dispatch<GemvLaunch>(L.code, L.parts[0].k2, L.V, l16, a, pl, st);
+}
+
+cudaError_t prepare_gemv_kernels(const Layer& L) {
+    const bool l16 = L.L == 16;
+    cudaError_t e = L.nparts > 1 ? (l16 ? gemv_multi_prepare<true>(L.code, L.V) : gemv_multi_prepare<false>(L.code, L.V))
+                                 : dispatch<GemvPrepare>(L.code, L.parts[0].k2, L.V, l16);
+    for (int i = 0; i < L.nparts && e == cudaSuccess; ++i) e = dispatch<DecodePrepare>(L.code, L.parts[i].k2, L.V, l16);
+    return e;
 }
 
 }  // namespace qlk

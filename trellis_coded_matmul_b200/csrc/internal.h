@@ -14,7 +14,7 @@ constexpr int kT = 256;            // columns per trellis block
 constexpr int kRowTile = 16;       // rows per decode tile (the m16n8k16 M dimension)
 constexpr int kMaxHadamard = 32768;
 
-constexpr int kGemvMaxWarps = 24;        // decode-GEMV: warps of its one CTA per SM (<= 85 registers/thread)
+constexpr int kGemvMaxWarps = 16;        // decode-GEMV: warps of its one CTA per SM (<= 128 registers/thread)
 constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
 #ifndef QL_FUSE_IN_ELEMS
 #define QL_FUSE_IN_ELEMS 16384
@@ -61,13 +61,18 @@ struct Layer {
     // scratch, grown on demand
     void* xp;             // transformed input x' (fp16)
     size_t xp_bytes;
-    float* z;             // W_hat x' before the output transform, fp32 [batch][m]; all-zero between forwards
-    size_t z_bytes;
-    int z_dirty;          // z may hold partial sums (a forward failed part-way)
+    void* acc;            // the output-block tickets (int [m / B_m], padded to 256 bytes), then z = W_hat x'
+                          // before the output transform (fp32 [batch][m]); all-zero between forwards
+    size_t acc_bytes;
+    int acc_dirty;        // z or a ticket may be non-zero (a forward failed part-way)
     int last_launches;    // kernels launched by the most recent forward
     void* host_stage;     // device staging for qlinear_forward_host (x then y)
     size_t host_stage_bytes;
     int num_sms;
+    // test hooks of the tensor-core GEMM (qlinear_test_stall): a shorter
+    // limit on its bounded waits and a stage that never arrives
+    int test_wait_tries;
+    int test_withhold;
     // profiling ring (qlinear_profile_enable)
     cudaEvent_t* prof_ev;  // 2 * prof_cap events
     int prof_cap;
@@ -116,43 +121,63 @@ cudaError_t ensure_smem_limit(int bytes) {
     return e;
 }
 
+// Load kernel Kern's code on the current device now and raise its
+// shared-memory limit to `smem_limit` bytes (0: leave it).  Under lazy module
+// loading a kernel is otherwise loaded at its first launch, which may
+// allocate device memory and must not happen inside a stream capture; create
+// calls this for every kernel a handle's forwards and decodes can launch.
+template <auto Kern>
+cudaError_t preload_kernel(int smem_limit) {
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, Kern);
+    if (e == cudaSuccess && smem_limit > 0) e = ensure_smem_limit<Kern>(smem_limit);
+    return e;
+}
+
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_relayout(const uint32_t* src, uint32_t* dst, const Part& part, int n, cudaStream_t st);
 cudaError_t launch_pack_signs(const int8_t* s, int count, uint32_t* bits, int* status, cudaStream_t st);
 cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cudaStream_t st);
 
-// x (fp16 [batch][n]) -> x' in the fragment layout of the decode-GEMV.
-cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st);
+// x (fp16 [batch][n]) -> x' as the decode-GEMV's step words (xstep.cuh).
+cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* xstep, cudaStream_t st);
 // x (fp16 [batch][n]) -> x' as tensor-core operand tiles: [n/64][npad][128 B],
 // the 16-byte chunk c of row b at chunk c ^ (b % 8) (rows >= batch untouched).
 cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st);
 // z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st);
 
-// How one decode-GEMV launch is shaped: grid and CTA size, its shared memory
-// (32-bit words: replicated HYB table, x' fragments, FWHT scratch), and
-// whether the input transform runs inside it (xsmem).
-struct GemvSmem {
-    int lut_words, xs_words, fw_words;
-};
+// How one decode-GEMV launch is shaped: grid and CTA size, whether the input
+// transform runs inside it (xsmem: x' computed by every CTA into its shared
+// memory), and its dynamic shared memory.
 struct GemvPlan {
     int grid, threads;
     bool xsmem;
-    int groups_in;
-    GemvSmem sm;
+    int smem_bytes;
 };
-GemvPlan plan_gemv(const Layer& L, const Part& part, int batch);
-// z[b][row0 + r] += sum_c W_hat[row0 + r][c] x'[b][c] for the part's rows, batch <= 8;
-// with pl.xsmem x' is computed from x in-kernel, else read from xp_frag.
-cudaError_t launch_gemv(const Layer& L, const Part& part, const GemvPlan& pl, const void* x, const void* xp_frag,
-                        int batch, float* z, cudaStream_t st);
-// The same for all row parts of a layer in one launch (nparts > 1), x' from xp_frag.
-cudaError_t launch_gemv_multi(const Layer& L, const void* xp_frag, int batch, float* z, cudaStream_t st);
+GemvPlan plan_gemv(const Layer& L, int batch);
+// Bytes of x' step words for `batch` rows (the input-transform kernel's output
+// when the plan does not compute x' in-kernel).
+size_t gemv_xstep_bytes(const Layer& L, int batch);
+// The whole forward for batch <= 8 after the input transform: decode-GEMV over
+// all row parts, z accumulation, and the output transform into y (fp32 or
+// fp16) by the CTA that completes each output Hadamard block.  z ([batch][m]
+// fp32) and tickets ([m / B_m] int) must be all-zero on entry and are all-zero
+// again when the kernel completes.  With pl.xsmem x' is computed from x
+// in-kernel, else read from xstep.
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
+                        int* tickets, void* y, int y_dtype, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
 // z[b][row] += W_hat x' for all parts (z all-zero on entry), x' in tensor-core
 // tiles with npad (multiple of 16, <= 256) rows, b < batch; the (128-row tile,
 // 256-column block) units are split evenly over one CTA per SM.
 cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st);
+// Preload (preload_kernel) every kernel a handle can launch: decode-GEMV
+// (both input-transform variants) and qlinear_decode (gemv.cu), the transform
+// kernels (rht.cu), the tensor-core GEMM (gemm_tc.cu).
+cudaError_t prepare_gemv_kernels(const Layer& L);
+cudaError_t prepare_rht_kernels(const Layer& L);
+cudaError_t prepare_gemm_kernels(const Layer& L);
 cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_words,
                              const uint32_t* states, int count, void* out, cudaStream_t st);
 

@@ -74,7 +74,7 @@ void free_layer(Layer& L) {
     cudaFree(L.lut);
     cudaFree(L.status);
     cudaFree(L.xp);
-    cudaFree(L.z);
+    cudaFree(L.acc);
     cudaFree(L.host_stage);
     std::memset(&L, 0, sizeof(L));
 }
@@ -183,6 +183,16 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
         delete h;
         return QL_E_ARG;
     }
+    // load every kernel this layer can launch now, not at its first launch
+    e = prepare_gemv_kernels(Ly);
+    if (e == cudaSuccess) e = prepare_rht_kernels(Ly);
+    if (e == cudaSuccess) e = prepare_gemm_kernels(Ly);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        free_layer(Ly);
+        delete h;
+        return QL_E_CUDA;
+    }
     *out = h;
     return QL_OK;
 }
@@ -212,47 +222,51 @@ int ensure(void** buf, size_t* have, size_t bytes) {
     return QL_OK;
 }
 
-// The z accumulator is all-zero between forwards: it is zeroed when
-// allocated, and the output-transform kernel re-zeroes what it consumed (the
-// tensor-core GEMM adds into z, which needs and keeps the same invariant).
-int prepare_z(Layer& L, size_t bytes, cudaStream_t st) {
-    if (L.z_bytes >= bytes && !L.z_dirty) return QL_OK;
-    int rc = ensure((void**)&L.z, &L.z_bytes, bytes);
+// Bytes of the ticket array at the start of the accumulator buffer.
+size_t ticket_bytes(const Layer& L) { return ((size_t)(L.m / L.B_m) * 4 + 255) / 256 * 256; }
+int* tickets_of(void* acc) { return (int*)acc; }
+float* z_of(const Layer& L, void* acc) { return (float*)((char*)acc + ticket_bytes(L)); }
+
+// The accumulator (tickets and z) is all-zero between forwards: it is zeroed
+// when allocated, and the kernel that consumes z re-zeroes it (the
+// decode-GEMV's output transform, or the output-transform kernel after the
+// tensor-core GEMM, which adds into z and needs the same invariant).
+int prepare_acc(Layer& L, size_t z_bytes, cudaStream_t st) {
+    const size_t bytes = ticket_bytes(L) + z_bytes;
+    if (L.acc_bytes >= bytes && !L.acc_dirty) return QL_OK;
+    int rc = ensure(&L.acc, &L.acc_bytes, bytes);
     if (rc != QL_OK) return rc;
-    if (cudaMemsetAsync(L.z, 0, L.z_bytes, st) != cudaSuccess) {
+    if (cudaMemsetAsync(L.acc, 0, L.acc_bytes, st) != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.z_dirty = 0;
+    L.acc_dirty = 0;
     return QL_OK;
 }
 
-// batch <= 8: decode-GEMV (input transform in-kernel for small x, else a
-// separate kernel), then the output transform.
+// batch <= 8: the decode-GEMV kernel does the whole forward (its input
+// transform in-kernel for small x, else after a separate input-transform
+// kernel; the output transform in its epilogue).
 int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
-    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)batch * L.n * 2);
-    if (rc == QL_OK) rc = prepare_z(L, (size_t)batch * L.m * 4, st);
+    const GemvPlan pl = plan_gemv(L, batch);
+    int rc = pl.xsmem ? QL_OK : ensure(&L.xp, &L.xp_bytes, gemv_xstep_bytes(L, batch));
+    if (rc == QL_OK) rc = prepare_acc(L, (size_t)batch * L.m * 4, st);
     if (rc != QL_OK) return rc;
-    // A layer of several row parts runs all parts in one launch (x' from the
-    // separate input transform); a uniform layer may fuse the input transform.
-    const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
-    const bool multi = L.nparts > 1;
-    const bool xsmem = !multi && pl.xsmem;
     cudaError_t e = cudaSuccess;
-    L.last_launches = 2 + (xsmem ? 0 : 1);
-    if (!xsmem) e = launch_rht_in_frag(L, x, batch, L.xp, st);
+    L.last_launches = pl.xsmem ? 1 : 2;
+    if (!pl.xsmem) e = launch_rht_in_xstep(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-    if (e == cudaSuccess) e = multi ? launch_gemv_multi(L, L.xp, batch, L.z, st) : launch_gemv(L, L.parts[0], pl, x, L.xp, batch, L.z, st);
+    if (e == cudaSuccess)
+        e = launch_gemv(L, pl, x, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
     if (e == cudaSuccess && slot >= 0) {
         e = record_event(L.prof_ev[2 * slot + 1], st);
         L.prof_next = (L.prof_next + 1) % L.prof_cap;
         if (L.prof_count < L.prof_cap) ++L.prof_count;
     }
-    if (e == cudaSuccess) e = launch_rht_out(L, L.z, batch, y, y_dtype, st);
     if (e != cudaSuccess) {
         cudaGetLastError();
-        L.z_dirty = 1;  // a partial forward may have left sums in z
+        L.acc_dirty = 1;  // a partial forward may have left sums in z or counts in the tickets
         return QL_E_CUDA;
     }
     return QL_OK;
@@ -264,8 +278,9 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
     const int chunk = batch < kTcMaxN ? batch : kTcMaxN;
     const int npad_max = (chunk + 15) / 16 * 16;
     int rc = ensure(&L.xp, &L.xp_bytes, (size_t)npad_max * L.n * 2);
-    if (rc == QL_OK) rc = prepare_z(L, (size_t)chunk * L.m * 4, st);
+    if (rc == QL_OK) rc = prepare_acc(L, (size_t)chunk * L.m * 4, st);
     if (rc != QL_OK) return rc;
+    float* z = z_of(L, L.acc);
     const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
     L.last_launches = 3 * ((batch + kTcMaxN - 1) / kTcMaxN);
     for (int b0 = 0; b0 < batch; b0 += kTcMaxN) {
@@ -276,16 +291,16 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
         cudaError_t e = launch_rht_in_umma(L, xb, nb, npad, L.xp, st);
         const int slot = L.prof_cap ? L.prof_next : -1;
         if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-        if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, L.z, st);
+        if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, z, st);
         if (e == cudaSuccess && slot >= 0) {
             e = record_event(L.prof_ev[2 * slot + 1], st);
             L.prof_next = (L.prof_next + 1) % L.prof_cap;
             if (L.prof_count < L.prof_cap) ++L.prof_count;
         }
-        if (e == cudaSuccess) e = launch_rht_out(L, L.z, nb, yb, y_dtype, st);
+        if (e == cudaSuccess) e = launch_rht_out(L, z, nb, yb, y_dtype, st);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            L.z_dirty = 1;
+            L.acc_dirty = 1;
             return QL_E_CUDA;
         }
     }
@@ -492,8 +507,18 @@ int qlinear_get_status(qlinear_t h) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    if (status & kStatusTimeout) return QL_E_TIMEOUT;
+    if (status & kStatusTimeout) {
+        h->L.acc_dirty = 1;  // an abandoned GEMM may have left partial sums in z
+        return QL_E_TIMEOUT;
+    }
     if (status) return QL_E_DEVICE;
+    return QL_OK;
+}
+
+int qlinear_test_stall(qlinear_t h, int enable, int wait_tries) {
+    if (!h || (enable && (wait_tries < 1 || wait_tries > 4096))) return QL_E_ARG;
+    h->L.test_withhold = enable ? 1 : 0;
+    h->L.test_wait_tries = enable ? wait_tries : 0;
     return QL_OK;
 }
 
@@ -517,7 +542,7 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->stream_bytes = words * 4;
     info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
     info->lut_bytes = uses_table(L.code) ? ((size_t)1 << L.Q) * L.V * 2 : 0;
-    info->scratch_bytes = L.xp_bytes + L.z_bytes + L.host_stage_bytes;
+    info->scratch_bytes = L.xp_bytes + L.acc_bytes + L.host_stage_bytes;
     info->last_launches = L.last_launches;
     info->nparts = L.nparts;
     for (int i = 0; i < L.nparts; ++i) {
@@ -647,30 +672,30 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     if (!x || !y) return QL_E_ARG;
     if (batch > kGemvMaxBatch) return QL_E_UNSUPPORTED;
     Layer& L = h->L;
-    const size_t xp_bytes = ((size_t)batch * L.n * 2 + 255) / 256 * 256;
-    const size_t z_bytes = (size_t)batch * L.m * 4;
-    if (xp_bytes + z_bytes > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_E_SCRATCH;
+    // array layout: output-block tickets, z, then x' when the input transform
+    // runs as its own kernel
+    const GemvPlan pl = plan_gemv(L, batch);
+    const size_t t_bytes = ticket_bytes(L);
+    const size_t z_bytes = ((size_t)batch * L.m * 4 + 255) / 256 * 256;
+    const size_t xp_bytes = pl.xsmem ? 0 : gemv_xstep_bytes(L, batch);
+    if (t_bytes + z_bytes + xp_bytes > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_E_SCRATCH;
     DeviceGuard g(L.device);
     if (!g.ok) return QL_E_CUDA;
     void* base = nullptr;
     const int rc = noalloc_scratch(L.device, &base);
     if (rc != QL_OK) return rc;
-    char* xp = (char*)base;
-    float* z = (float*)(xp + xp_bytes);
+    int* tickets = (int*)base;
+    float* z = (float*)((char*)base + t_bytes);
+    void* xp = (char*)base + t_bytes + z_bytes;
     cudaStream_t st = (cudaStream_t)stream;
-
-    const GemvPlan pl = plan_gemv(L, L.parts[0], batch);
-    const bool multi = L.nparts > 1;
-    const bool xsmem = !multi && pl.xsmem;
-    // z must start at zero; another handle's failed call may have left sums there.
-    cudaError_t e = cudaMemsetAsync(z, 0, z_bytes, st);
-    if (e == cudaSuccess && !xsmem) e = launch_rht_in_frag(L, x, batch, xp, st);
-    if (e == cudaSuccess) e = multi ? launch_gemv_multi(L, xp, batch, z, st) : launch_gemv(L, L.parts[0], pl, x, xp, batch, z, st);
-    if (e == cudaSuccess) e = launch_rht_out(L, z, batch, y, y_dtype, st);
+    // tickets and z must start at zero; another handle's failed call may have left sums there
+    cudaError_t e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
+    if (e == cudaSuccess && !pl.xsmem) e = launch_rht_in_xstep(L, x, batch, xp, st);
+    if (e == cudaSuccess) e = launch_gemv(L, pl, x, xp, batch, z, tickets, y, y_dtype, st);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.last_launches = 2 + (xsmem ? 0 : 1);
+    L.last_launches = pl.xsmem ? 1 : 2;
     return QL_OK;
 }

@@ -24,6 +24,7 @@
 
 #include "fwht.cuh"
 #include "internal.h"
+#include "xstep.cuh"
 
 namespace qlk {
 
@@ -47,10 +48,11 @@ static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
     return g;
 }
 
-// Output layouts of x': the decode-GEMV fragment layout, row-major [batch][n],
-// or the tensor-core operand tiles (64-column K stages of npad rows of 128
-// bytes, 16-byte chunk c of row b stored at chunk c ^ (b % 8)).
-enum { kXpFrag = 0, kXpRowMajor = 1, kXpUmma = 2 };
+// Output layouts of x': the decode-GEMV's step words for V = 1 or V = 2
+// (xstep.cuh), row-major [batch][n], or the tensor-core operand tiles
+// (64-column K stages of npad rows of 128 bytes, 16-byte chunk c of row b
+// stored at chunk c ^ (b % 8)).
+enum { kXpStep1 = 0, kXpRowMajor = 1, kXpUmma = 2, kXpStep2 = 3 };
 
 __device__ __forceinline__ size_t umma_tile_index4(int col, int b, int npad) {
     const int s = col >> 6, kin = col & 63;
@@ -98,14 +100,17 @@ __global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_in_kernel(const __hal
     const float scale = rsqrtf((float)B);
 #pragma unroll
     for (int q = 0; q < E; q += 4) {
+        if (MODE == kXpStep1 || MODE == kXpStep2) {
+            const float w4[4] = {v[q] * scale, v[q + 1] * scale, v[q + 2] * scale, v[q + 3] * scale};
+            store_xstep4<MODE == kXpStep1 ? 1 : 2>(reinterpret_cast<uint32_t*>(out), col + q, b, batch, w4);
+            continue;
+        }
         const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
         const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
         uint2 w;
         w.x = *reinterpret_cast<const uint32_t*>(&lo);
         w.y = *reinterpret_cast<const uint32_t*>(&hi);
-        if (MODE == kXpFrag)
-            *reinterpret_cast<uint2*>(out + frag_index4(col + q, b, batch)) = w;
-        else if (MODE == kXpUmma)
+        if (MODE == kXpUmma)
             *reinterpret_cast<uint2*>(out + umma_tile_index4(col + q, b, npad)) = w;
         else
             *reinterpret_cast<uint2*>(out + (size_t)b * n + col + q) = w;
@@ -130,8 +135,8 @@ static cudaError_t launch_rht_in(const Layer& L, const void* x, int batch, void*
                          : launch_rht_in_e<MODE, 16>(L, x, batch, xp, npad, st);
 }
 
-cudaError_t launch_rht_in_frag(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    return launch_rht_in<kXpFrag>(L, x, batch, xp, 0, st);
+cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
+    return L.V == 1 ? launch_rht_in<kXpStep1>(L, x, batch, xp, 0, st) : launch_rht_in<kXpStep2>(L, x, batch, xp, 0, st);
 }
 
 cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st) {
@@ -214,6 +219,31 @@ cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_d
     if (L.B_m > 4096 || batch > kGemvMaxBatch)
         return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
     return f16 ? launch_rht_out_e<true, 8>(L, z, batch, y, st) : launch_rht_out_e<false, 8>(L, z, batch, y, st);
+}
+
+template <int MODE>
+static cudaError_t prepare_rht_in(const Layer& L) {
+    const int limit = (kMaxHadamard + kMaxHadamard / 16) * 4;
+    return L.B_n > 16384 ? preload_kernel<rht_in_kernel<MODE, 32>>(limit) : preload_kernel<rht_in_kernel<MODE, 16>>(limit);
+}
+
+template <bool F16>
+static cudaError_t prepare_rht_out(const Layer& L) {
+    const int limit = (kMaxHadamard + kMaxHadamard / 16) * 4;
+    if (L.B_m > 16384) return preload_kernel<rht_out_kernel<F16, 32>>(limit);
+    cudaError_t e = preload_kernel<rht_out_kernel<F16, 16>>(limit);
+    if (e == cudaSuccess && L.B_m <= 4096) e = preload_kernel<rht_out_kernel<F16, 8>>(limit);
+    return e;
+}
+
+// The transform kernels launch_rht_in_xstep, launch_rht_in_umma and
+// launch_rht_out can pick for this layer.
+cudaError_t prepare_rht_kernels(const Layer& L) {
+    cudaError_t e = L.V == 1 ? prepare_rht_in<kXpStep1>(L) : prepare_rht_in<kXpStep2>(L);
+    if (e == cudaSuccess) e = prepare_rht_in<kXpUmma>(L);
+    if (e == cudaSuccess) e = prepare_rht_out<true>(L);
+    if (e == cudaSuccess) e = prepare_rht_out<false>(L);
+    return e;
 }
 
 }  // namespace qlk
