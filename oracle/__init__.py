@@ -17,6 +17,8 @@ Modules:
   fp16      IEEE binary16 decoding and round-to-nearest-even, from the definition
   bitstream MSB-first bit access and the canonical stream layout
   trellis   the bitshift-trellis state walk (QTIP discussion, "Figure 2 (Q4)")
+  e8p       an E8-lattice codebook of 2^16 eight-dimensional entries (QuIP#
+            page, abstract and Fig. captions: the E8P-style comparison VQ)
   codes     the 1MAD, 3INST and HYB codes ("Inference speed analysis", "HYB
             Uniqueness", "Bit Accounting") and the table code of the palette
             quantizers (VQ / NUQ, Q-Palette page)
@@ -32,4 +34,4 @@ values or properties fixed by the pages or by mathematics (tests/test_oracle_*.p
 The code constants themselves are a reading (the pages do not print them); what
 pins them is the set of properties the pages claim for the codes.
 """
-from . import fp16, bitstream, trellis, codes, hadamard, qlinear, stats  # noqa: F401
+from . import fp16, bitstream, trellis, e8p, codes, hadamard, qlinear, stats  # noqa: F401

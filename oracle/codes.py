@@ -22,7 +22,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import fp16
+from . import e8p, fp16
 
 MASK32 = 0xFFFFFFFF
 
@@ -110,4 +110,7 @@ def evaluate(code: int, state, V: int, lut=None) -> np.ndarray:
     if code == 3:
         assert lut is not None and lut.shape[1] == V
         return table(state, lut)
+    if code == 4:
+        assert V == 8
+        return e8p.e8p(state)
     raise ValueError(code)

@@ -113,3 +113,18 @@ def test_3inst_without_its_high_half_is_caught(monkeypatch):
         return fp16.round_rne(fp16.decode_bits(m & 0xFFFF))
     monkeypatch.setattr(codes, "three_inst", low_half_only)
     _fails(t_codes.test_computed_code_is_close_to_standard_normal, codes.three_inst)
+
+
+def test_e8_code_without_its_parity_sign_is_caught(monkeypatch):
+    """The sign of coordinate 7 taken from nowhere (always +) instead of the
+    even-sum rule: half the codewords leave the lattice."""
+    import test_oracle_e8p as t_e8p
+    from oracle import e8p
+
+    def no_parity(state):
+        s = np.asarray(state, dtype=np.int64)
+        T = e8p.shape_table()[s >> 8]
+        neg = np.stack([(s >> (i + 1)) & 1 for i in range(7)] + [np.zeros_like(s)], axis=-1)
+        return (1.0 - 2.0 * neg) * T + np.where(s & 1, 0.25, -0.25)[..., None]
+    monkeypatch.setattr(e8p, "codeword", no_parity)
+    _fails(t_e8p.test_every_codeword_is_a_shifted_e8_point_and_the_set_is_symmetric)

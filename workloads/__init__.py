@@ -25,6 +25,7 @@ quantizers beside TCQ), all m=n=4096, batch 1/4/8:
             (the page's 2.75-bit example: a 2.5-bit and a 3-bit quantizer)
   vq2p5     k=2.5, L=5, V=2, table code: 32 codewords of 2 values
   nuq3      k=3, L=3, V=1, table code: 8 levels
+  e8p2      k=2, L=16, V=8, the E8-lattice code: 2^16 codewords of 8 values
 
 Distributions: code words are uniform uint32, signs uniform +-1 (int8), the
 HYB table holds 2^Q x V standard normals rounded to fp16 (numpy's float16
@@ -43,7 +44,8 @@ CODE_1MAD = 0
 CODE_3INST = 1
 CODE_HYB = 2
 CODE_TABLE = 3
-CODE_NAMES = {CODE_1MAD: "1MAD", CODE_3INST: "3INST", CODE_HYB: "HYB", CODE_TABLE: "TABLE"}
+CODE_E8P = 4
+CODE_NAMES = {CODE_1MAD: "1MAD", CODE_3INST: "3INST", CODE_HYB: "HYB", CODE_TABLE: "TABLE", CODE_E8P: "E8P"}
 
 T_BLOCK = 256  # columns per independent trellis block (fixed by the format)
 
@@ -128,6 +130,9 @@ WORKLOADS = {
                          m_top=2048, k_top=2.5, k_bot=3, batches=(1, 4, 8)),
     "vq2p5": LayerSpec("vq2p5", 4096, 4096, 2.5, 5, 2, CODE_TABLE, 1.0, seed=8, batches=(1, 4, 8)),
     "nuq3": LayerSpec("nuq3", 4096, 4096, 3, 3, 1, CODE_TABLE, 1.0, seed=9, batches=(1, 4, 8)),
+    # the E8-lattice vector quantizer the trellis codes are compared with: 2 bits
+    # per weight, 8 weights per 16-bit step, L = kV = 16 (plain VQ)
+    "e8p2": LayerSpec("e8p2", 4096, 4096, 2, 16, 8, CODE_E8P, 0.02, seed=10, batches=(1, 4, 8)),
 }
 
 # The up and down projections of the MLP pair draw from one seeded stream
