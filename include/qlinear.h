@@ -29,6 +29,20 @@
  *                  Q-Palette page's palette (a trellis with L = kV is plain
  *                  k-bit, V-dimensional VQ, as the QTIP discussion's ablation
  *                  reply notes); with L > kV, a trellis over the codebook.
+ *   QL_CODE_E8P    the E8-lattice vector quantizer the QTIP discussion compares
+ *                  the trellis codes with (QuIP# page: abstract, Fig. 3
+ *                  caption; QTIP discussion, "Inference speed analysis
+ *                  (W2)": 2^16 E8-based entries of dimension 8, stored as 256
+ *                  table words): V = 8, L = kV = 16 (each step's own 16 bits
+ *                  index the codebook), k = 2.  State s: shape a = s >> 8,
+ *                  signs of coordinates 0..6 in bits 1..7 (set = negative),
+ *                  shift bit 0; codeword = sigma * T[a] + (bit 0 ? 1/4 : -1/4)
+ *                  in every coordinate, where T[a] is the a-th of the 256
+ *                  vectors of nonnegative half-odd-integer coordinates of
+ *                  smallest norm (ties: 2T in lexicographic order) and the
+ *                  sign of coordinate 7 makes sum(sigma * T[a]) even, i.e.
+ *                  sigma * T[a] lies in the E8 lattice.  The library builds
+ *                  the table; code.lut is not read.  One part only.
  *
  * with the constants (A, B per code; C1 = 443 * 2^-16; MASK = 0x9CFF8FFF,
  * XOR = 0x20003000) fixed by this library's format.  Values are rounded to
@@ -84,6 +98,7 @@ extern "C" {
 #define QL_CODE_3INST 1
 #define QL_CODE_HYB 2
 #define QL_CODE_TABLE 3
+#define QL_CODE_E8P 4
 
 #define QL_F32 0
 #define QL_F16 1
@@ -91,8 +106,8 @@ extern "C" {
 typedef struct qlinear_s* qlinear_t;
 
 /* The code that maps a trellis state to V values.
- *   kind: QL_CODE_1MAD or QL_CODE_3INST (V must be 1), or QL_CODE_HYB or
- *         QL_CODE_TABLE (V = 1 or 2).
+ *   kind: QL_CODE_1MAD or QL_CODE_3INST (V must be 1), QL_CODE_HYB or
+ *         QL_CODE_TABLE (V = 1 or 2), or QL_CODE_E8P (V = 8, L = 16, k = 2).
  *   Q:    HYB only, table index bits, 1..9 (the discussion uses Q = 9; "you can
  *         go down to Q~6").  Ignored by the table code, whose codebook has
  *         2^L entries (L = 1..9).
@@ -204,7 +219,8 @@ int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_hos
  *   input transform runs as its own kernel) x' live in one fixed array of
  *   QL_NOALLOC_SCRATCH_BYTES in the library's static device memory, per
  *   device: round_up(4*m/B(m), 256) + round_up(4*batch*m, 256) bytes, plus
- *   4*batch*n/V bytes of x' when batch*n > 16384, must fit, else
+ *   x' when batch*n > 16384 (4*batch*n bytes at V = 1, 2*batch*n at V = 2
+ *   or 8), must fit, else
  *   QL_E_SCRATCH (before any device work).  Every call clears its tickets
  *   and z on `stream` first.
  *   Sharing: all handles on a device share the array, so calls that overlap

@@ -41,6 +41,7 @@ FULL = {
     "tcq2p75": (1, 4, 8, 64),
     "vq2p5": (1, 4, 8, 64),
     "nuq3": (1, 4, 8, 64),
+    "e8p2": (1, 4, 8, 64),
 }
 CHUNK_WEIGHTS = 1 << 21  # weights per oracle task
 

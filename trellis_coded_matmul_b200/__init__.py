@@ -34,6 +34,7 @@ QL_CODE_1MAD = 0
 QL_CODE_3INST = 1
 QL_CODE_HYB = 2
 QL_CODE_TABLE = 3
+QL_CODE_E8P = 4
 QL_F32 = 0
 QL_F16 = 1
 

@@ -34,10 +34,13 @@ constexpr int kCode1MAD = 0;
 constexpr int kCode3INST = 1;
 constexpr int kCodeHYB = 2;
 constexpr int kCodeTable = 3;
+constexpr int kCodeE8P = 4;
 
-// Codes whose values come from a table in shared memory (2^Q entries; the
-// table code's Q is L).
-__host__ __device__ constexpr bool uses_table(int code) { return code == kCodeHYB || code == kCodeTable; }
+// Codes whose values come from a table in shared memory (2^Q words; the
+// table code's Q is L; the E8 code's 256 shapes take 2 words each, Q = 9).
+__host__ __device__ constexpr bool uses_table(int code) {
+    return code == kCodeHYB || code == kCodeTable || code == kCodeE8P;
+}
 constexpr int kMaxTableBits = 9;  // 2^9 entries x 32 lanes x 4 bytes = 64 KiB replicated
 
 constexpr uint32_t kA1MAD = 0x61616D4Bu, kB1MAD = 0xE29B5692u;
@@ -133,6 +136,49 @@ __device__ __forceinline__ uint32_t code_v2(uint32_t s, const uint32_t* lut_lane
     static_assert(CODE == kCodeHYB || CODE == kCodeTable, "V = 2 needs a table code");
     if (CODE == kCodeHYB) return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
     return lut_lane[s * 32u];
+}
+
+// E8 code (V = 8, one 16-bit state per 8 values): the fp16 pairs of the
+// state's codeword, coordinates 2p and 2p + 1 in pair p.  The state holds the
+// shape index a (bits 8..15), the signs of coordinates 0..6 (bits 1..7: set =
+// negative) and the shift (bit 0: +1/4, else -1/4).  Shape a is table words
+// 2a (coordinates 0..3) and 2a + 1 (4..7), one byte per coordinate: the high
+// byte of its magnitude in fp16 (the low byte is zero); bit 31 of word 2a + 1
+// is the shape's parity bit, (sum of 2|T_i|) / 2 mod 2.  The sign of
+// coordinate 7 is that bit xor the parity of the other seven signs, which
+// makes the signed shape's coordinate sum even: a point of E8.
+__device__ __forceinline__ void e8p_pairs(uint32_t s, const uint32_t* lut_lane, uint32_t (&pr)[4]) {
+    const uint32_t a = s >> 8;
+    const uint32_t w0 = lut_lane[(2u * a) * 32u], w1 = lut_lane[(2u * a + 1u) * 32u];
+    const uint32_t sb = (s >> 1) & 0x7Fu;
+    const uint32_t x = sb | ((__popc(sb) & 1u) << 7);  // sign bits of coordinates 0..7 (bit 7: the parity)
+    const uint32_t d = (s & 1u) ? 0x34003400u : 0xB400B400u;  // +1/4 or -1/4 in both halves
+    // bit 2p of x to bit 15, bit 2p + 1 to bit 31: one multiply by 2^15 + 2^30
+    pr[0] = hadd2_u32(__byte_perm(w0, 0u, 0x1404) ^ ((x * 0x40008000u) & 0x80008000u), d);
+    pr[1] = hadd2_u32(__byte_perm(w0, 0u, 0x3424) ^ (((x >> 2) * 0x40008000u) & 0x80008000u), d);
+    pr[2] = hadd2_u32(__byte_perm(w1, 0u, 0x1404) ^ (((x >> 4) * 0x40008000u) & 0x80008000u), d);
+    pr[3] = hadd2_u32(__byte_perm(w1, 0u, 0x3424) ^ (((x >> 6) * 0x40008000u) & 0x80008000u), d);
+}
+
+// Fill the per-lane replicated table (HYB, the table code's codebook, the E8
+// code's shapes) in shared memory: word 32 i + l holds entry i for lane l.
+// Thread k reads entries k and k + blockDim (both loads first) and writes each
+// one's 32 copies (128 contiguous bytes) as eight 16-byte stores, starting at
+// chunk i % 8 so that eight consecutive threads cover all 32 banks.
+__device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lut, int entries) {
+    const int bd = blockDim.x;
+    for (int i = threadIdx.x; i < entries; i += 2 * bd) {
+        const bool two = i + bd < entries;
+        const uint32_t v0 = __ldg(lut + i), v1 = two ? __ldg(lut + i + bd) : 0u;
+        uint4* d0 = reinterpret_cast<uint4*>(smem + 32 * i);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d0[(q + i) & 7] = make_uint4(v0, v0, v0, v0);
+        if (two) {
+            uint4* d1 = reinterpret_cast<uint4*>(smem + 32 * (i + bd));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) d1[(q + i + bd) & 7] = make_uint4(v1, v1, v1, v1);
+        }
+    }
 }
 
 // Bits [a, a + 32) of a thread-row's bit string (most significant bit first):

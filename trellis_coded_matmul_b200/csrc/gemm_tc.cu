@@ -177,9 +177,30 @@ __device__ __forceinline__ int tc_tiles16(const TcPart& pt, int tile) {  // row 
 // (K2 = 2k; with a half-integer k a run starts inside a word).  Output: 16
 // half2 words, columns 2i and 2i + 1 of the run in word i.
 template <int CODE, int K2, int V, bool L16, int HQ>
+__device__ __forceinline__ void decode_run32_trellis(const uint32_t (&w)[K2 + 1], uint32_t lmask,
+                                                     const uint32_t* lut_lane, int qshift, uint32_t (&out)[16]);
+
+template <int CODE, int K2, int V, bool L16, int HQ>
 __device__ __forceinline__ void decode_run32(const uint32_t (&w)[K2 + 1], uint32_t lmask, const uint32_t* lut_lane,
                                              int qshift, uint32_t (&out)[16]) {
     static_assert((K2 * V) % 2 == 0, "a step carries a whole number of bits");
+    if constexpr (CODE == kCodeE8P) {  // four 16-bit steps of 8 weights: words 1 + 2 HQ and 2 + 2 HQ
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            uint32_t pr[4];
+            const uint32_t wd = w[1 + 2 * HQ + t / 2];
+            e8p_pairs((t & 1) ? (wd & 0xFFFFu) : (wd >> 16), lut_lane, pr);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) out[4 * t + q] = pr[q];
+        }
+    } else {
+        decode_run32_trellis<CODE, K2, V, L16, HQ>(w, lmask, lut_lane, qshift, out);
+    }
+}
+
+template <int CODE, int K2, int V, bool L16, int HQ>
+__device__ __forceinline__ void decode_run32_trellis(const uint32_t (&w)[K2 + 1], uint32_t lmask,
+                                                     const uint32_t* lut_lane, int qshift, uint32_t (&out)[16]) {
     constexpr int kV = K2 * V / 2;
     constexpr int NS = 32 / V;
     constexpr int T0 = HQ * NS;
@@ -256,6 +277,10 @@ __device__ __forceinline__ void decode_stage_tmem(uint32_t code, uint32_t a_tadd
 template <int CODE, int V, bool L16>
 __device__ __forceinline__ void decode_stage_k2(int k2, uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
                                                 uint32_t lmask, const uint32_t* lut_lane, int qshift) {
+    if constexpr (V == 8) {  // the E8 code: 16 bits per 8 weights
+        decode_stage_tmem<CODE, 4, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift);
+        return;
+    }
     switch (k2) {
         case 2: decode_stage_tmem<CODE, 2, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
         case 3: if constexpr (V == 2) decode_stage_tmem<CODE, 3, V, L16>(code, a_taddr, qtr, q, lane, lmask, lut_lane, qshift); break;
@@ -309,8 +334,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
         mbar_fence_init();
     }
     uint32_t* lut_smem = reinterpret_cast<uint32_t*>(smem + L.lut);
-    if (uses_table(CODE))
-        for (int i = threadIdx.x; i < p.lut_entries * 32; i += blockDim.x) lut_smem[i] = p.lut[i >> 5];
+    if (uses_table(CODE)) fill_lut_smem(lut_smem, p.lut, p.lut_entries);
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_base_smem), kTcTmemCols);
         tmem_relinquish();
@@ -552,6 +576,7 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
         return L.V == 1 ? launch_gemm_t<kCodeTable, 1, false>(a, grid, smem, st)
                         : launch_gemm_t<kCodeTable, 2, false>(a, grid, smem, st);
     }
+    if (L.code == kCodeE8P) return l16 ? launch_gemm_t<kCodeE8P, 8, true>(a, grid, smem, st) : cudaErrorInvalidValue;
     if (L.V == 1) return l16 ? launch_gemm_t<kCodeHYB, 1, true>(a, grid, smem, st)
                              : launch_gemm_t<kCodeHYB, 1, false>(a, grid, smem, st);
     return l16 ? launch_gemm_t<kCodeHYB, 2, true>(a, grid, smem, st) : launch_gemm_t<kCodeHYB, 2, false>(a, grid, smem, st);
@@ -566,6 +591,7 @@ cudaError_t prepare_gemm_kernels(const Layer& L) {
         if (l16) return cudaErrorInvalidValue;
         return L.V == 1 ? QLK_PREP(kCodeTable, 1, false) : QLK_PREP(kCodeTable, 2, false);
     }
+    if (L.code == kCodeE8P) return l16 ? QLK_PREP(kCodeE8P, 8, true) : cudaErrorInvalidValue;
     if (L.V == 1) return l16 ? QLK_PREP(kCodeHYB, 1, true) : QLK_PREP(kCodeHYB, 1, false);
     return l16 ? QLK_PREP(kCodeHYB, 2, true) : QLK_PREP(kCodeHYB, 2, false);
 #undef QLK_PREP

@@ -110,11 +110,6 @@ __device__ __forceinline__ void load_unit(uint32_t (&w)[2][K2], const uint32_t* 
 }
 
 
-// Fill the per-lane replicated table (HYB, or the table code's codebook) in shared memory.
-__device__ __forceinline__ void fill_lut_smem(uint32_t* smem, const uint32_t* lut, int entries) {
-    for (int i = threadIdx.x; i < entries * 32; i += blockDim.x) smem[i] = lut[i >> 5];
-}
-
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -163,7 +158,7 @@ struct StepMMAs {
     template <bool XSMEM>
     static __device__ __forceinline__ void run(const uint32_t (&cw)[2][NW], uint32_t lmask, const uint32_t* lut_lane,
                                                int qshift, const uint4* xsrc, int xstride, bool use_x,
-                                               float (&acc)[4]) {
+                                               float (&acc)[2][4]) {
 #pragma unroll
         for (int u = 0; u < NM; u += 2) {
             if (kQuad && ((u / (kQuad ? MP : 1)) & 1)) continue;  // produced together with MMAs u - MP, u - MP + 1
@@ -196,12 +191,40 @@ struct StepMMAs {
                 b0 = XSMEM ? xsrc[(u >> 1) * xstride] : __ldg(xsrc + (u >> 1) * xstride);
                 if (kQuad) b1 = XSMEM ? xsrc[((u + MP) >> 1) * xstride] : __ldg(xsrc + ((u + MP) >> 1) * xstride);
             }
-            mma_16816(acc, a[0], b0.x, b0.y);
-            mma_16816(acc, a[1], b0.z, b0.w);
+            // two accumulators: two dependent MMA chains of half the length
+            mma_16816(acc[0], a[0], b0.x, b0.y);
+            mma_16816(acc[1], a[1], b0.z, b0.w);
             if (kQuad) {
-                mma_16816(acc, a[2], b1.x, b1.y);
-                mma_16816(acc, a[3], b1.z, b1.w);
+                mma_16816(acc[0], a[2], b1.x, b1.y);
+                mma_16816(acc[1], a[3], b1.z, b1.w);
             }
+        }
+    }
+};
+
+// The E8 code (V = 8): each 16-bit step gives 8 weights, four fp16 pairs;
+// step t of the lane's run (the high half of word 1 + t/2 when t is even, the
+// low half when odd) feeds MMAs 2t (pairs 0, 1) and 2t + 1 (pairs 2, 3), whose
+// B words are the 16-byte group t.
+template <int K2, bool L16>
+struct StepMMAs<kCodeE8P, K2, 8, L16> {
+    static constexpr int NW = K2 + 1;
+    template <bool XSMEM>
+    static __device__ __forceinline__ void run(const uint32_t (&cw)[2][NW], uint32_t, const uint32_t* lut_lane, int,
+                                               const uint4* xsrc, int xstride, bool use_x, float (&acc)[2][4]) {
+        static_assert(K2 == 4, "the E8 code stores 16 bits per 8 weights");
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            uint32_t p0[4], p1[4];  // rows g and g + 8
+            const uint32_t w0 = cw[0][1 + t / 2], w1 = cw[1][1 + t / 2];
+            e8p_pairs((t & 1) ? (w0 & 0xFFFFu) : (w0 >> 16), lut_lane, p0);
+            e8p_pairs((t & 1) ? (w1 & 0xFFFFu) : (w1 >> 16), lut_lane, p1);
+            uint4 b = make_uint4(0u, 0u, 0u, 0u);
+            if (use_x) b = XSMEM ? xsrc[t * xstride] : __ldg(xsrc + t * xstride);
+            const uint32_t a0[4] = {p0[0], p1[0], p0[1], p1[1]};
+            const uint32_t a1[4] = {p0[2], p1[2], p0[3], p1[3]};
+            mma_16816(acc[0], a0, b.x, b.y);
+            mma_16816(acc[1], a1, b.z, b.w);
         }
     }
 };
@@ -235,6 +258,7 @@ struct GemvArgs {
     float out_scale;        // alpha (times C1 for 1MAD) / sqrt(B_m)
     void* y;                // [batch][m]
     int y_f16;
+    int fuse_out;           // the output transform runs in this kernel (else a separate kernel after it)
     int smem_floats;        // dynamic shared memory of the launch, in 4-byte words
 };
 
@@ -266,7 +290,7 @@ __device__ __forceinline__ void load_unit_k2(uint32_t (&w)[2][8], const uint32_t
 template <int CODE, int K2, int V, bool L16, bool XSMEM, int NXW>
 __device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][NXW], const uint32_t* next_base, int next_k2, int lane,
                                           int src_lane, const GemvArgs& p, const uint32_t* lut_lane, const uint4* xsrc,
-                                          int xstride, bool use_x, float (&acc)[4]) {
+                                          int xstride, bool use_x, float (&acc)[2][4]) {
     uint32_t cw[2][K2 + 1];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -283,11 +307,35 @@ __device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][NXW], const uint32_
     StepMMAs<CODE, K2, V, L16>::template run<XSMEM>(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
 }
 
+// One unit of a one-part layer whose code words are in buf[0]: the buffered
+// units move down one slot, the unit PD ahead of this one starts loading into
+// buf[PD-1] (pf: its address, or null), then decode and multiply.
+template <int CODE, int K2, int V, bool L16, bool XSMEM, int PD>
+__device__ __forceinline__ void gemv_unit_pd(uint32_t (&buf)[PD][2][K2], const uint32_t* pf, int lane, int src_lane,
+                                             const GemvArgs& p, const uint32_t* lut_lane, const uint4* xsrc,
+                                             int xstride, bool use_x, float (&acc)[2][4]) {
+    uint32_t cw[2][K2 + 1];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < K2; ++i) cw[h][i + 1] = buf[0][h][i];
+#pragma unroll
+    for (int d = 0; d + 1 < PD; ++d)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < K2; ++i) buf[d][h][i] = buf[d + 1][h][i];
+    if (pf) load_unit<K2>(buf[PD - 1], pf, lane);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
+    StepMMAs<CODE, K2, V, L16>::template run<XSMEM>(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
+}
+
 // The unit's bitwidth picks the decoder (V = 1 has whole bitwidths only).
 template <int CODE, int V, bool L16, bool XSMEM>
 __device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2,
                                              int lane, int src_lane, const GemvArgs& p, const uint32_t* lut_lane,
-                                             const uint4* xsrc, int xstride, bool use_x, float (&acc)[4]) {
+                                             const uint4* xsrc, int xstride, bool use_x, float (&acc)[2][4]) {
 #define QLK_UNIT(K) gemv_unit<CODE, K, V, L16, XSMEM, 8>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xsrc, \
                                                          xstride, use_x, acc)
     switch (k2) {
@@ -331,13 +379,18 @@ __device__ __forceinline__ void input_transform_smem(const GemvArgs& p, uint32_t
 
 // The output transform of Hadamard block hb for every batch row (as many rows
 // at once as `buf` holds): y = out_scale * s_out (H z); z returns to zero.
+// The block's B/32 sign words are staged in shared memory after the rows.
 __device__ __forceinline__ void output_transform_block(const GemvArgs& p, int hb, float* buf) {
     const int B = p.B_m, m = p.m;
-    int rows = p.smem_floats / (B + B / 16);
+    const int w0 = (hb * B) >> 5, nw = ((hb * B + B - 1) >> 5) - w0 + 1;  // sign words of the block's rows
+    int rows = (p.smem_floats - nw) / (B + B / 16);
     rows = rows < 1 ? 1 : (rows > p.batch ? p.batch : rows);
+    uint32_t* sgn = reinterpret_cast<uint32_t*>(buf + rows * (B + B / 16));
+    for (int i = threadIdx.x; i < nw; i += blockDim.x) sgn[i] = p.sout_bits[w0 + i];
+    // (the barrier after the first load phase makes the sign words visible)
     for (int b0 = 0; b0 < p.batch; b0 += rows) {
         const int nr = p.batch - b0 < rows ? p.batch - b0 : rows;
-        fwht_blocks_smem(
+        fwht_blocks_smem<2>(
             buf, nr * B, B,
             [&](int i, float (&v)[8]) {
                 const int bb = b0 + i / B, r = hb * B + (i % B);
@@ -350,7 +403,7 @@ __device__ __forceinline__ void output_transform_block(const GemvArgs& p, int hb
             },
             [&](int i, const float (&v)[4]) {
                 const int bb = b0 + i / B, r = hb * B + (i % B);
-                const uint32_t sw = p.sout_bits[r >> 5] >> (r & 31);  // r % 4 == 0
+                const uint32_t sw = sgn[(r >> 5) - w0] >> (r & 31);  // r % 4 == 0: bits r .. r+3 in one word
                 float o[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) o[q] = ((sw >> q) & 1u) ? -v[q] * p.out_scale : v[q] * p.out_scale;
@@ -409,8 +462,9 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     constexpr int NXW = K2F ? K2F : 8;
     const int lane = threadIdx.x & 31;
     const int lut_words = uses_table(CODE) ? p.lut_entries * 32 : 0;
+    constexpr int VX = V == 1 ? 1 : 2;  // x' layout: one column per B word (V = 1) or two
     uint32_t* xs_words = smem + lut_words;
-    float* work = reinterpret_cast<float*>(smem + lut_words + (XSMEM ? p.batch * p.n / V : 0));
+    float* work = reinterpret_cast<float*>(smem + lut_words + (XSMEM ? p.batch * p.n / VX : 0));
     if (uses_table(CODE)) fill_lut_smem(smem, p.lut, p.lut_entries);
     const uint32_t* lut_lane = smem + lane;
 
@@ -435,16 +489,22 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     // bits are written once at create time, so the first unit's words are
     // fetched before waiting for the previous kernel (the producer of x or x',
     // the previous forward that used z).
+    // A one-part layer keeps PD units in flight per warp (two at up to 2 bits
+    // per weight, where a unit's decode is shortest), a multi-part layer one.
+    constexpr int PD = (K2F != 0 && K2F <= 4) ? 2 : 1;
+    constexpr int UWF = 64 * (K2F ? K2F : 1);  // words per unit of a one-part layer
     uint32_t nxt[2][NXW];
-    if (u0 < u1) {
-        if constexpr (K2F != 0)
-            load_unit<K2F>(nxt, unit_base(pt, t, j), lane);
-        else
-            load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
+    uint32_t buf[PD][2][K2F ? K2F : 1];
+    if constexpr (K2F != 0) {
+#pragma unroll
+        for (int d = 0; d < PD; ++d)
+            if (u0 + d < u1) load_unit<K2F>(buf[d], p.part[0].words + (size_t)(u0 + d) * UWF, lane);
+    } else if (u0 < u1) {
+        load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
     }
     grid_dependency_wait();
     if constexpr (XSMEM)
-        input_transform_smem<V>(p, xs_words, work);  // ends with a CTA barrier (the table is filled too)
+        input_transform_smem<VX>(p, xs_words, work);  // ends with a CTA barrier (the table is filled too)
     else if (uses_table(CODE))
         __syncthreads();
     grid_launch_dependents();
@@ -452,18 +512,18 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     const uint4* xbase = XSMEM ? reinterpret_cast<const uint4*>(xs_words) : p.xstep;
     const int xstride = batch * 4;  // uint4 groups between consecutive u2
     const bool use_x = g < batch;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     int cur_pt = pt, cur_t = t;
     auto flush = [&](int part, int tile) {
         const int row = p.part[part].row0 + tile * kRowTile + g;
         const int b0 = 2 * c, b1 = 2 * c + 1;
         if (b0 < batch) {
-            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0]);
-            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[2]);
+            atomicAdd(p.z + (size_t)b0 * p.m + row, acc[0][0] + acc[1][0]);
+            atomicAdd(p.z + (size_t)b0 * p.m + row + 8, acc[0][2] + acc[1][2]);
         }
         if (b1 < batch) {
-            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[1]);
-            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[3]);
+            atomicAdd(p.z + (size_t)b1 * p.m + row, acc[0][1] + acc[1][1]);
+            atomicAdd(p.z + (size_t)b1 * p.m + row + 8, acc[0][3] + acc[1][3]);
         }
     };
     for (long long unit = u0; unit < u1; ++unit) {
@@ -478,14 +538,16 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
         const uint32_t* next_base = unit + 1 < u1 ? unit_base(npt, nt, nj) : nullptr;
         if (pt != cur_pt || t != cur_t) {
             flush(cur_pt, cur_t);
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[0][i] = acc[1][i] = 0.f;
             cur_pt = pt;
             cur_t = t;
         }
-        const uint4* xsrc = xbase + ((size_t)j * (16 / V) * batch + g) * 4 + c;
+        const uint4* xsrc = xbase + ((size_t)j * (16 / VX) * batch + g) * 4 + c;
         if constexpr (K2F != 0)
-            gemv_unit<CODE, K2F, V, L16, XSMEM, NXW>(nxt, next_base, K2F, lane, src_lane, p, lut_lane, xsrc, xstride,
-                                                     use_x, acc);
+            gemv_unit_pd<CODE, K2F, V, L16, XSMEM, PD>(
+                buf, unit + PD < u1 ? p.part[0].words + (size_t)(unit + PD) * UWF : nullptr, lane, src_lane, p,
+                lut_lane, xsrc, xstride, use_x, acc);
         else
             gemv_unit_k2<CODE, V, L16, XSMEM>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p,
                                               lut_lane, xsrc, xstride, use_x, acc);
@@ -494,7 +556,7 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
         j = nj;
     }
     if (u0 < u1) flush(cur_pt, cur_t);
-    output_epilogue(p, reinterpret_cast<float*>(smem), c0, c1);
+    if (p.fuse_out) output_epilogue(p, reinterpret_cast<float*>(smem), c0, c1);
 }
 
 // ---- the forward's launch plan and dispatch ----
@@ -509,22 +571,27 @@ GemvPlan plan_gemv(const Layer& L, int batch) {
     pl.threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
     const long long lut_words = uses_table(L.code) ? (32ll << L.Q) : 0;
     const long long elems = (long long)batch * L.n;
-    const long long xs_words = elems / L.V;
+    const long long xs_words = elems / (L.V == 1 ? 1 : 2);
     const long long work_words = elems + elems / 16;
     const long long budget = kGemvMaxSmem / 4;
     pl.xsmem = elems <= kFuseInElems && lut_words + xs_words + work_words <= budget;
     long long main_words = lut_words + (pl.xsmem ? xs_words + work_words : 0);
-    // the output transform: as many batch rows of one Hadamard block as fit
+    // the output transform in-kernel when one CTA's share of it is small, as
+    // many batch rows of one Hadamard block at once as fit (plus its sign words)
+    pl.fuse_out = (long long)batch * L.B_m <= kFuseOutElems;
     const long long row_words = L.B_m + L.B_m / 16;
-    long long rows = budget / row_words;
+    const long long sign_words = L.B_m / 32 + 2;
+    long long rows = (budget - sign_words) / row_words;
     if (rows > batch) rows = batch;
     if (rows < 1) rows = 1;
-    const long long epi_words = rows * row_words;
+    const long long epi_words = pl.fuse_out ? rows * row_words + sign_words : 0;
     pl.smem_bytes = (int)((main_words > epi_words ? main_words : epi_words) * 4);
     return pl;
 }
 
-size_t gemv_xstep_bytes(const Layer& L, int batch) { return (size_t)batch * L.n / L.V * 4; }
+float gemv_z_scale(const Layer& L) { return L.code == kCode1MAD ? kC1 : 1.0f; }
+
+size_t gemv_xstep_bytes(const Layer& L, int batch) { return (size_t)batch * L.n / (L.V == 1 ? 1 : 2) * 4; }
 
 template <int CODE, int K2, int V, bool L16>
 struct GemvLaunch {
@@ -659,7 +726,7 @@ __device__ __forceinline__ void for_each_mma(const uint32_t (&cw)[2][K2 + 1], ui
 // ---- qlinear_decode: one warp per unit, fp16 W_hat row-major ----
 template <int CODE, int K2, int V, bool L16>
 __global__ void __launch_bounds__(256) trellis_decode_kernel(DecodeArgs p, __half* __restrict__ w_hat, int n, int row0) {
-    extern __shared__ uint32_t lut_smem[];
+    extern __shared__ __align__(16) uint32_t lut_smem[];
     using UL = UnitLayout<K2>;
     const int lane = threadIdx.x & 31;
     if (uses_table(CODE)) {
@@ -683,14 +750,29 @@ __global__ void __launch_bounds__(256) trellis_decode_kernel(DecodeArgs p, __hal
             cw[h][0] = __shfl_sync(0xffffffffu, w[h][K2 - 1], src_lane);
         }
         const int R = (int)(unit / p.nb), j = (int)(unit % p.nb);
-        for_each_mma<CODE, K2, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
+        if constexpr (CODE == kCodeE8P) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const size_t row = (size_t)row0 + R * kRowTile + 8 * h + g;
-                uint2* dst = (uint2*)(w_hat + row * n + (size_t)j * kT + 64 * c + 4 * u);
-                *dst = make_uint2(a[h], a[2 + h]);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    uint32_t pr[4];
+                    const uint32_t wd = cw[h][1 + t / 2];
+                    e8p_pairs((t & 1) ? (wd & 0xFFFFu) : (wd >> 16), lut_lane, pr);
+                    *reinterpret_cast<uint4*>(w_hat + row * n + (size_t)j * kT + 64 * c + 8 * t) =
+                        make_uint4(pr[0], pr[1], pr[2], pr[3]);
+                }
             }
-        });
+        } else {
+            for_each_mma<CODE, K2, V, L16>(cw, p.lmask, lut_lane, p.qshift, [&](int u, const uint32_t(&a)[4]) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const size_t row = (size_t)row0 + R * kRowTile + 8 * h + g;
+                    uint2* dst = (uint2*)(w_hat + row * n + (size_t)j * kT + 64 * c + 4 * u);
+                    *dst = make_uint2(a[h], a[2 + h]);
+                }
+            });
+        }
     }
 }
 
@@ -698,7 +780,7 @@ __global__ void __launch_bounds__(256) trellis_decode_kernel(DecodeArgs p, __hal
 template <int CODE, int V>
 __global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count, uint32_t lmask, int qshift,
                                  const uint32_t* __restrict__ lut, int lut_entries, __half* __restrict__ out) {
-    extern __shared__ uint32_t lut_smem[];
+    extern __shared__ __align__(16) uint32_t lut_smem[];
     const int lane = threadIdx.x & 31;
     if (uses_table(CODE)) {
         fill_lut_smem(lut_smem, lut, lut_entries);
@@ -706,7 +788,13 @@ __global__ void eval_code_kernel(const uint32_t* __restrict__ states, int count,
     }
     const uint32_t* lut_lane = lut_smem + lane;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if constexpr (V == 2) {
+    if constexpr (CODE == kCodeE8P) {
+        if (t < count) {
+            uint32_t pr[4];
+            e8p_pairs(states[t] & 0xFFFFu, lut_lane, pr);
+            reinterpret_cast<uint4*>(out)[t] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        }
+    } else if constexpr (V == 2) {
         if (t < count) ((uint32_t*)out)[t] = code_v2<CODE>(states[t] & lmask, lut_lane, qshift);
     } else {
         const int i0 = 2 * t;
@@ -759,6 +847,8 @@ static cudaError_t dispatch_l(int code, int k2, int V, Args&&... args) {
     if constexpr (!L16) {
         if (code == kCodeTable && V == 1) return dispatch_k2<F, kCodeTable, 1, false>(k2, args...);
         if (code == kCodeTable && V == 2) return dispatch_k2<F, kCodeTable, 2, false>(k2, args...);
+    } else {
+        if (code == kCodeE8P && V == 8 && k2 == 4) return F<kCodeE8P, 4, 8, true>::run(args...);
     }
     return cudaErrorInvalidValue;
 }
@@ -810,14 +900,14 @@ struct EvalLaunch {
     static cudaError_t run(const uint32_t* states, int count, uint32_t lmask, int qshift, const uint32_t* lut,
                            int entries, __half* out, cudaStream_t st) {
         // one instance per (code, V) suffices: the code ignores k and L
-        if (K2 != 2 || L16 == (CODE == kCodeTable)) return cudaErrorInvalidValue;
+        if (CODE != kCodeE8P && (K2 != 2 || L16 == (CODE == kCodeTable))) return cudaErrorInvalidValue;
         const size_t smem = (size_t)entries * 32 * 4;
         auto kern = eval_code_kernel<CODE, V>;
         if (smem > 48 * 1024) {
             cudaError_t e = ensure_smem_limit<eval_code_kernel<CODE, V>>(32 * 512 * 4);
             if (e != cudaSuccess) return e;
         }
-        const int items = V == 2 ? count : (count + 1) / 2;
+        const int items = V >= 2 ? count : (count + 1) / 2;
         kern<<<(items + 255) / 256, 256, smem, st>>>(states, count, lmask, qshift, lut, entries, out);
         return cudaGetLastError();
     }
@@ -827,6 +917,8 @@ cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_
                              int count, void* out, cudaStream_t st) {
     const uint32_t lmask = (1u << L) - 1u;
     const int entries = uses_table(code) ? (1 << Q) : 0;
+    if (code == kCodeE8P)
+        return EvalLaunch<kCodeE8P, 4, 8, true>::run(states, count, lmask, 32 - Q, lut_words, entries, (__half*)out, st);
     return dispatch<EvalLaunch>(code, 2, V, code != kCodeTable, states, count, lmask, 32 - Q, lut_words, entries,
                                 (__half*)out, st);
 }
@@ -861,9 +953,10 @@ cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const
     a.tickets = tickets;
     a.B_m = L.B_m;
     a.sout_bits = L.sout_bits;
-    a.out_scale = L.alpha * (L.code == kCode1MAD ? kC1 : 1.0f) / sqrtf((float)L.B_m);
+    a.out_scale = L.alpha * gemv_z_scale(L) / sqrtf((float)L.B_m);
     a.y = y;
     a.y_f16 = y_dtype == QL_F16;
+    a.fuse_out = pl.fuse_out;
     a.smem_floats = pl.smem_bytes / 4;
     const bool l16 = L.L == 16;
     if (L.nparts > 1) return l16 ? gemv_multi_l<true>(L.code, L.V, a, pl, st) : gemv_multi_l<false>(L.code, L.V, a, pl, st);

@@ -20,6 +20,7 @@ constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory l
 #define QL_FUSE_IN_ELEMS 16384
 #endif
 constexpr int kFuseInElems = QL_FUSE_IN_ELEMS;  // batch * n up to which the GEMV computes x' itself
+constexpr int kFuseOutElems = 8192;  // batch * B_m up to which the GEMV's last CTA per block does the output transform
 constexpr int kMaxParts = 8;          // row parts of one layer (layers fused along m, own bitwidth each)
 constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
 constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
@@ -144,8 +145,9 @@ cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* 
 // x (fp16 [batch][n]) -> x' as tensor-core operand tiles: [n/64][npad][128 B],
 // the 16-byte chunk c of row b at chunk c ^ (b % 8) (rows >= batch untouched).
 cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st);
-// z (fp32 [batch][m]) -> y = alpha s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
-cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st);
+// z (fp32 [batch][m]) -> y = alpha zscale s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
+cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st,
+                           float zscale = 1.0f);
 
 // How one decode-GEMV launch is shaped: grid and CTA size, whether the input
 // transform runs inside it (xsmem: x' computed by every CTA into its shared
@@ -153,12 +155,15 @@ cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_d
 struct GemvPlan {
     int grid, threads;
     bool xsmem;
+    bool fuse_out;  // output transform in the GEMV's epilogue (else launch_rht_out after it)
     int smem_bytes;
 };
 GemvPlan plan_gemv(const Layer& L, int batch);
 // Bytes of x' step words for `batch` rows (the input-transform kernel's output
 // when the plan does not compute x' in-kernel).
 size_t gemv_xstep_bytes(const Layer& L, int batch);
+// The factor between the decode-GEMV's z and W_hat x' (the 1MAD code's C1, else 1).
+float gemv_z_scale(const Layer& L);
 // The whole forward for batch <= 8 after the input transform: decode-GEMV over
 // all row parts, z accumulation, and the output transform into y (fp32 or
 // fp16) by the CTA that completes each output Hadamard block.  z ([batch][m]

@@ -1,7 +1,11 @@
 // qlinear_abi.cu -- the C ABI declared in include/qlinear.h (host side).
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <array>
 #include <cmath>
+#include <vector>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -81,6 +85,7 @@ void free_layer(Layer& L) {
 
 int check_code(const ql_code_t& code, int V, int L) {
     if (code.kind == QL_CODE_1MAD || code.kind == QL_CODE_3INST) return V == 1 ? QL_OK : QL_E_UNSUPPORTED;
+    if (code.kind == QL_CODE_E8P) return V == 8 && L == 16 ? QL_OK : QL_E_UNSUPPORTED;
     if (code.kind != QL_CODE_HYB && code.kind != QL_CODE_TABLE) return QL_E_ARG;
     if (V != 1 && V != 2) return QL_E_ARG;
     if (code.kind == QL_CODE_HYB && (code.Q < 1 || code.Q > kMaxTableBits)) return QL_E_UNSUPPORTED;
@@ -89,9 +94,51 @@ int check_code(const ql_code_t& code, int V, int L) {
     return QL_OK;
 }
 
-// Index bits of the code's table (the table code's codebook has 2^L entries).
+// Index bits of the code's table in words (the table code's codebook has 2^L
+// entries; the E8 code's 256 shapes take 2 words each).
 int table_bits(const ql_code_t& code, int L) {
-    return code.kind == QL_CODE_HYB ? code.Q : code.kind == QL_CODE_TABLE ? L : 0;
+    return code.kind == QL_CODE_HYB ? code.Q : code.kind == QL_CODE_TABLE ? L : code.kind == QL_CODE_E8P ? 9 : 0;
+}
+
+// The E8 code's shape table (include/qlinear.h): the 256 vectors of
+// nonnegative half-odd coordinates T = n/2 (n odd) with the smallest norm,
+// ties broken by n in lexicographic order.  Shape a takes words 2a and 2a+1:
+// byte i of the pair is the high byte of fp16(n_i / 2) (its low byte is
+// zero), and bit 31 of word 2a+1 holds (sum of n_i) / 2 mod 2.
+const std::array<uint32_t, 512>& e8p_shape_words() {
+    static const std::array<uint32_t, 512> words = [] {
+        std::vector<std::array<int, 9>> all;  // [sum of n_i^2, n_0 .. n_7]
+        all.reserve(1 << 16);
+        for (int code = 0; code < (1 << 16); ++code) {
+            std::array<int, 9> v{};
+            for (int i = 0; i < 8; ++i) {
+                v[1 + i] = 2 * ((code >> (2 * (7 - i))) & 3) + 1;  // 1, 3, 5, 7
+                v[0] += v[1 + i] * v[1 + i];
+            }
+            all.push_back(v);
+        }
+        std::sort(all.begin(), all.end());
+        std::array<uint32_t, 512> w{};
+        for (int a = 0; a < 256; ++a) {
+            int sum = 0;
+            for (int i = 0; i < 8; ++i) {
+                const int nv = all[a][1 + i];
+                sum += nv;
+                const uint32_t hi = __half_as_ushort(__float2half_rn(0.5f * (float)nv)) >> 8;
+                w[2 * a + i / 4] |= hi << (8 * (i % 4));
+            }
+            w[2 * a + 1] |= (uint32_t)((sum % 4) / 2) << 31;
+        }
+        return w;
+    }();
+    return words;
+}
+
+// Copies the code's table into `dst` (2^Q words) on stream st.
+cudaError_t copy_code_table(const ql_code_t& code, int Q, int V, uint32_t* dst, cudaStream_t st) {
+    if (code.kind == QL_CODE_E8P)
+        return cudaMemcpyAsync(dst, e8p_shape_words().data(), 512 * 4, cudaMemcpyHostToDevice, st);
+    return launch_copy_lut(code.lut, Q, V, dst, st);
 }
 
 // Shared by the create calls. parts: [(rows, kv)], host arrays; kv = bits per
@@ -103,7 +150,8 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (!out) return QL_E_ARG;
     *out = nullptr;
     if (m <= 0 || n <= 0 || !std::isfinite(alpha)) return QL_E_ARG;
-    if (V != 1 && V != 2) return QL_E_ARG;
+    if (V != 1 && V != 2 && !(V == 8 && code.kind == QL_CODE_E8P)) return QL_E_ARG;
+    if (code.kind == QL_CODE_E8P && (nparts != 1 || !part_kv || part_kv[0] != 16)) return QL_E_UNSUPPORTED;
     if (n % kT != 0 || m % kRowTile != 0) return QL_E_UNSUPPORTED;
     if (pow2_block(n) > kMaxHadamard || pow2_block(m) > kMaxHadamard) return QL_E_UNSUPPORTED;
     if (nparts < 1 || nparts > kMaxParts || !part_rows || !part_kv) return QL_E_ARG;
@@ -168,7 +216,7 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
         e = launch_relayout(packed_codes + Ly.parts[i].word_off, Ly.words, Ly.parts[i], n, st);
     if (e == cudaSuccess) e = launch_pack_signs(s_in, n, Ly.sin_bits, Ly.status, st);
     if (e == cudaSuccess) e = launch_pack_signs(s_out, m, Ly.sout_bits, Ly.status, st);
-    if (e == cudaSuccess && uses_table(Ly.code)) e = launch_copy_lut(code.lut, Ly.Q, V, Ly.lut, st);
+    if (e == cudaSuccess && uses_table(Ly.code)) e = copy_code_table(code, Ly.Q, V, Ly.lut, st);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     int status = 0;
     if (e == cudaSuccess) e = cudaMemcpy(&status, Ly.status, sizeof(int), cudaMemcpyDeviceToHost);
@@ -253,7 +301,7 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
     if (rc == QL_OK) rc = prepare_acc(L, (size_t)batch * L.m * 4, st);
     if (rc != QL_OK) return rc;
     cudaError_t e = cudaSuccess;
-    L.last_launches = pl.xsmem ? 1 : 2;
+    L.last_launches = 1 + (pl.xsmem ? 0 : 1) + (pl.fuse_out ? 0 : 1);
     if (!pl.xsmem) e = launch_rht_in_xstep(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
@@ -264,6 +312,7 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
         L.prof_next = (L.prof_next + 1) % L.prof_cap;
         if (L.prof_count < L.prof_cap) ++L.prof_count;
     }
+    if (e == cudaSuccess && !pl.fuse_out) e = launch_rht_out(L, z_of(L, L.acc), batch, y, y_dtype, st, gemv_z_scale(L));
     if (e != cudaSuccess) {
         cudaGetLastError();
         L.acc_dirty = 1;  // a partial forward may have left sums in z or counts in the tickets
@@ -320,7 +369,7 @@ int qlinear_create(qlinear_t* out, int m, int n, int k, int L, int V, ql_code_t 
     if (!out) return QL_E_ARG;
     *out = nullptr;
     if (k < 1 || k > 4) return QL_E_UNSUPPORTED;
-    if (V != 1 && V != 2) return QL_E_ARG;
+    if (V != 1 && V != 2 && !(V == 8 && code.kind == QL_CODE_E8P)) return QL_E_ARG;
     const int rows[1] = {m};
     const int kvs[1] = {k * V};
     return create_common(out, m, n, 1, rows, kvs, L, V, code, packed_codes, n_words, s_in, s_out, alpha);
@@ -426,7 +475,7 @@ int qlinear_eval_code(ql_code_t code, int L, int V, const uint32_t* states, int 
             cudaGetLastError();
             return QL_E_OOM;
         }
-        if (launch_copy_lut(code.lut, Q, V, lut_words, st) != cudaSuccess) {
+        if (copy_code_table(code, Q, V, lut_words, st) != cudaSuccess) {
             cudaGetLastError();
             cudaFreeAsync(lut_words, st);
             return QL_E_CUDA;
@@ -692,10 +741,11 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     cudaError_t e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
     if (e == cudaSuccess && !pl.xsmem) e = launch_rht_in_xstep(L, x, batch, xp, st);
     if (e == cudaSuccess) e = launch_gemv(L, pl, x, xp, batch, z, tickets, y, y_dtype, st);
+    if (e == cudaSuccess && !pl.fuse_out) e = launch_rht_out(L, z, batch, y, y_dtype, st, gemv_z_scale(L));
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.last_launches = pl.xsmem ? 1 : 2;
+    L.last_launches = 1 + (pl.xsmem ? 0 : 1) + (pl.fuse_out ? 0 : 1);
     return QL_OK;
 }

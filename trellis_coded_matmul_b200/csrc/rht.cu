@@ -48,11 +48,11 @@ static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
     return g;
 }
 
-// Output layouts of x': the decode-GEMV's step words for V = 1 or V = 2
-// (xstep.cuh), row-major [batch][n], or the tensor-core operand tiles
-// (64-column K stages of npad rows of 128 bytes, 16-byte chunk c of row b
-// stored at chunk c ^ (b % 8)).
-enum { kXpStep1 = 0, kXpRowMajor = 1, kXpUmma = 2, kXpStep2 = 3 };
+// Output layouts of x': row-major [batch][n], or the tensor-core operand
+// tiles (64-column K stages of npad rows of 128 bytes, 16-byte chunk c of row
+// b stored at chunk c ^ (b % 8)).  (The decode-GEMV's step words come from
+// rht_in_block_kernel below.)
+enum { kXpRowMajor = 1, kXpUmma = 2 };
 
 __device__ __forceinline__ size_t umma_tile_index4(int col, int b, int npad) {
     const int s = col >> 6, kin = col & 63;
@@ -100,11 +100,6 @@ __global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_in_kernel(const __hal
     const float scale = rsqrtf((float)B);
 #pragma unroll
     for (int q = 0; q < E; q += 4) {
-        if (MODE == kXpStep1 || MODE == kXpStep2) {
-            const float w4[4] = {v[q] * scale, v[q + 1] * scale, v[q + 2] * scale, v[q + 3] * scale};
-            store_xstep4<MODE == kXpStep1 ? 1 : 2>(reinterpret_cast<uint32_t*>(out), col + q, b, batch, w4);
-            continue;
-        }
         const __half2 lo = __floats2half2_rn(v[q] * scale, v[q + 1] * scale);
         const __half2 hi = __floats2half2_rn(v[q + 2] * scale, v[q + 3] * scale);
         uint2 w;
@@ -135,8 +130,53 @@ static cudaError_t launch_rht_in(const Layer& L, const void* x, int batch, void*
                          : launch_rht_in_e<MODE, 16>(L, x, batch, xp, npad, st);
 }
 
+// x' for the decode-GEMV, one CTA per (256-column block j, batch row b).
+// With B = B_n = 256 R, H_B = H_R (x) H_256 (Sylvester order: the high index
+// bits go to H_R), so the block's 256 outputs are
+//     x'[256 j + i] = H_256 w / sqrt(B),  w[t] = sum_a H_R[j mod R][a] u[B hb + 256 a + t]
+// (u = s_in * x, hb = the Hadamard block of column 256 j): R signed sums per
+// entry and one 256-point transform, so every block is computed by its own
+// CTA in parallel instead of one CTA per Hadamard block.
+template <int VX>
+__global__ void __launch_bounds__(256) rht_in_block_kernel(const __half* __restrict__ x, int n, int B,
+                                                          const uint32_t* __restrict__ sin_bits, int batch,
+                                                          uint32_t* __restrict__ xstep) {
+    __shared__ float w[256];
+    __shared__ float buf[256 + 16];
+    const int j = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+    const int R = B / 256, jr = j % R;
+    const int base = (j / R) * B;  // first column of the Hadamard block
+    grid_dependency_wait();
+    const __half* xr = x + (size_t)b * n + base + t;
+    float acc = 0.f;
+    for (int a = 0; a < R; ++a) {
+        const int col = base + 256 * a + t;
+        float v = __half2float(xr[256 * a]);
+        if ((sin_bits[col >> 5] >> (col & 31)) & 1u) v = -v;
+        acc += (__popc(jr & a) & 1) ? -v : v;
+    }
+    w[t] = acc;
+    __syncthreads();
+    grid_launch_dependents();
+    const float scale = rsqrtf((float)B);
+    fwht_blocks_smem(
+        buf, 256, 256,
+        [&](int i, float (&v)[8]) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = w[i + e];
+        },
+        [&](int i, const float (&v)[4]) {
+            const float o[4] = {v[0] * scale, v[1] * scale, v[2] * scale, v[3] * scale};
+            store_xstep4<VX>(xstep, 256 * j + i, b, batch, o);
+        });
+}
+
 cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* xp, cudaStream_t st) {
-    return L.V == 1 ? launch_rht_in<kXpStep1>(L, x, batch, xp, 0, st) : launch_rht_in<kXpStep2>(L, x, batch, xp, 0, st);
+    const dim3 grid(L.n / 256, batch);
+    return L.V == 1 ? launch_pdl(rht_in_block_kernel<1>, grid, dim3(256), 0, st, (const __half*)x, L.n, L.B_n,
+                                 (const uint32_t*)L.sin_bits, batch, (uint32_t*)xp)
+                    : launch_pdl(rht_in_block_kernel<2>, grid, dim3(256), 0, st, (const __half*)x, L.n, L.B_n,
+                                 (const uint32_t*)L.sin_bits, batch, (uint32_t*)xp);
 }
 
 cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st) {
@@ -199,7 +239,7 @@ __global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_out_kernel(float* __r
 }
 
 template <bool F16, int E>
-static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y, cudaStream_t st) {
+static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y, cudaStream_t st, float zscale) {
     const RhtGeometry geo = rht_geometry(L.m, L.B_m, batch, E);
     const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
     auto kern = rht_out_kernel<F16, E>;
@@ -207,18 +247,22 @@ static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y
     if (e != cudaSuccess) return e;
     const int grid = (geo.total + geo.groups - 1) / geo.groups;
     return launch_pdl(kern, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, z, batch, L.m, geo,
-                      (const uint32_t*)L.sout_bits, L.alpha, y);
+                      (const uint32_t*)L.sout_bits, L.alpha * zscale, y);
 }
 
-cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st) {
+cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st, float zscale) {
     const bool f16 = y_dtype == QL_F16;
     // Small batches (a few CTAs, latency-bound): 8 entries per thread up to blocks
     // of 4096 (512 threads), shorter chains per thread.  Large batches (many
     // CTAs, bandwidth-bound): 16, fewer and fuller CTAs.
-    if (L.B_m > 16384) return f16 ? launch_rht_out_e<true, 32>(L, z, batch, y, st) : launch_rht_out_e<false, 32>(L, z, batch, y, st);
+    if (L.B_m > 16384)
+        return f16 ? launch_rht_out_e<true, 32>(L, z, batch, y, st, zscale)
+                   : launch_rht_out_e<false, 32>(L, z, batch, y, st, zscale);
     if (L.B_m > 4096 || batch > kGemvMaxBatch)
-        return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st) : launch_rht_out_e<false, 16>(L, z, batch, y, st);
-    return f16 ? launch_rht_out_e<true, 8>(L, z, batch, y, st) : launch_rht_out_e<false, 8>(L, z, batch, y, st);
+        return f16 ? launch_rht_out_e<true, 16>(L, z, batch, y, st, zscale)
+                   : launch_rht_out_e<false, 16>(L, z, batch, y, st, zscale);
+    return f16 ? launch_rht_out_e<true, 8>(L, z, batch, y, st, zscale)
+               : launch_rht_out_e<false, 8>(L, z, batch, y, st, zscale);
 }
 
 template <int MODE>
@@ -239,7 +283,7 @@ static cudaError_t prepare_rht_out(const Layer& L) {
 // The transform kernels launch_rht_in_xstep, launch_rht_in_umma and
 // launch_rht_out can pick for this layer.
 cudaError_t prepare_rht_kernels(const Layer& L) {
-    cudaError_t e = L.V == 1 ? prepare_rht_in<kXpStep1>(L) : prepare_rht_in<kXpStep2>(L);
+    cudaError_t e = L.V == 1 ? preload_kernel<rht_in_block_kernel<1>>(0) : preload_kernel<rht_in_block_kernel<2>>(0);
     if (e == cudaSuccess) e = prepare_rht_in<kXpUmma>(L);
     if (e == cudaSuccess) e = prepare_rht_out<true>(L);
     if (e == cudaSuccess) e = prepare_rht_out<false>(L);

@@ -75,15 +75,24 @@ __device__ __forceinline__ void fwht_regs(float (&v)[E]) {
 // transformed entries i .. i+3.  Strides 1..4 run in registers, the rest in
 // radix-16 passes over the buffer with a CTA barrier after each.  Every thread
 // of the CTA must call this; the caller synchronises before reusing `buf`.
-template <typename Load8, typename Store4>
+// U > 1: each thread issues the loads of U chunks before transforming any of
+// them (more loads in flight when the source is global memory).
+template <int U = 1, typename Load8, typename Store4>
 __device__ __forceinline__ void fwht_blocks_smem(float* buf, int count, int B, Load8&& load8, Store4&& store4) {
     const int tid = threadIdx.x, nt = blockDim.x;
-    for (int i = tid * 8; i < count; i += nt * 8) {
-        float v[8];
-        load8(i, v);
-        fwht_regs<8>(v);
+    for (int i0 = tid * 8; i0 < count; i0 += nt * 8 * U) {
+        float v[U][8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) buf[pad16(i + q)] = v[q];
+        for (int u = 0; u < U; ++u)
+            if (i0 + u * nt * 8 < count) load8(i0 + u * nt * 8, v[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * nt * 8;
+            if (i >= count) break;
+            fwht_regs<8>(v[u]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) buf[pad16(i + q)] = v[u][q];
+        }
     }
     __syncthreads();
     int logh = 3;
