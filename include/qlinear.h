@@ -194,10 +194,10 @@ int qlinear_create_kv(qlinear_t* out, int m, int n, int nparts, const int* part_
  *   x: device pointer, fp16 [batch][n] row-major.
  *   y: device pointer, [batch][m] row-major, fp32 (y_dtype = QL_F32) or fp16 (QL_F16).
  *   batch >= 0 (0 is a no-op).  batch <= 8 runs the fused decode-GEMV kernel
- *   (the whole forward in one launch when batch*n <= 16384, else after an
- *   input-transform kernel); larger batches run the decode-to-tensor-memory
- *   tcgen05 GEMM between the two transform kernels.  x and y must be 16-byte
- *   aligned.
+ *   after an input-transform kernel, with the output transform inside it
+ *   when batch * B(m) <= 256, else before an output-transform kernel; larger
+ *   batches run the decode-to-tensor-memory tcgen05 GEMM between the two
+ *   transform kernels.  x and y must be 16-byte aligned.
  * The first call with a batch larger than any before it allocates scratch;
  * make such a call before capturing forward into a CUDA graph.
  * Errors: QL_E_ARG, QL_E_OOM, QL_E_CUDA (launch failure). */
@@ -219,8 +219,7 @@ int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_hos
  *   input transform runs as its own kernel) x' live in one fixed array of
  *   QL_NOALLOC_SCRATCH_BYTES in the library's static device memory, per
  *   device: round_up(4*m/B(m), 256) + round_up(4*batch*m, 256) bytes, plus
- *   x' when batch*n > 16384 (4*batch*n bytes at V = 1, 2*batch*n at V = 2
- *   or 8), must fit, else
+ *   x' (4*batch*n bytes at V = 1, 2*batch*n at V = 2 or 8), must fit, else
  *   QL_E_SCRATCH (before any device work).  Every call clears its tickets
  *   and z on `stream` first.
  *   Sharing: all handles on a device share the array, so calls that overlap

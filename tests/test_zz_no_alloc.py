@@ -44,9 +44,9 @@ def _same(y, y_ref):
 
 
 CASES = [
-    # name, batch, out dtype: the in-kernel input transform (batch * n <= 16K),
-    # the separate input-transform kernel, HYB V = 2, half-TCQ (two launches),
-    # and fp16 output.
+    # name, batch, out dtype: the output transform in the GEMV's epilogue
+    # (tiny) and in its own kernel, HYB V = 2, half-TCQ (two row parts), and
+    # fp16 output.
     ("tiny", 1, torch.float32),
     ("attn4096", 1, torch.float32),
     ("attn4096", 8, torch.float32),
@@ -93,15 +93,15 @@ def test_noalloc_against_the_oracle():
 
 def _noalloc_bytes(m, n, V, B_m, batch):
     """Scratch of one call as the header states it: the output-block tickets,
-    z, and x' when the input transform runs as its own kernel."""
+    z and x'."""
     up = lambda b: (b + 255) // 256 * 256  # noqa: E731
-    return up(4 * (m // B_m)) + up(4 * batch * m) + (0 if batch * n <= 16384 else 4 * batch * n // V)
+    return up(4 * (m // B_m)) + up(4 * batch * m) + 4 * batch * n // (1 if V == 1 else 2)
 
 
 def test_noalloc_scratch_limit_and_batch_limit():
     # m = 81920 (Hadamard blocks of 16384), n = 256: batch 6 needs
-    # 256 + 6*81920*4 = 1966336 bytes of scratch (fits in 2 MiB), batch 7
-    # needs 2294016 (does not).
+    # 256 + 6*81920*4 + 6*256*4 = 1972480 bytes of scratch (fits in 2 MiB),
+    # batch 7 needs 2301184 (does not).
     m, n = 81920, 256
     li = wl.random_layer(m, n, 2, 16, 1, wl.CODE_3INST, seed=11, alpha=0.5)
     h = make_handle(li)

@@ -118,25 +118,66 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// The A operand paired with decode (qlinear_decode uses code_pair / code_v2 of
-// codes.cuh, which round each value to fp16; the forward uses these words).
+// (qlinear_decode uses code_pair / code_v2 of codes.cuh, which round each
+// value to fp16; the forward's MMAs take the split words below.)
+
+// The forward's decode ends with one instruction per step word that turns a
+// "pre" word into the MMA's A word: 3INST (pre & MASK) ^ XOR; 1MAD one dp4a
+// giving {1536 + d, -1536}; HYB the table word xor the hashed state's bit 15;
+// the table code none.  That instruction runs inside the MMA's asm block, so
+// the finished words are allocated as the MMA's operand registers (computed
+// into arbitrary registers they would be copied into an aligned quad).
+template <int CODE, int V>
+__device__ __forceinline__ void step_pre(uint32_t s, const uint32_t* lut_lane, int qshift, uint32_t& pre,
+                                         uint32_t& aux) {
+    if constexpr (CODE == kCode1MAD) {
+        pre = kA1MAD * s + kB1MAD;
+    } else if constexpr (CODE == kCode3INST) {
+        pre = kA3INST * s + kB3INST;
+    } else if constexpr (CODE == kCodeHYB) {
+        aux = kAHYB * s + kBHYB;
+        pre = lut_lane[(aux >> qshift) * 32u];
+    } else {
+        pre = lut_lane[s * 32u];
+    }
+}
+
 // 1MAD: {1536 + d, -1536} as two halves (0x6600 is 1536.0; 0xE600 is -1536.0).
 constexpr uint32_t kDp4aSplitAcc = 0xE6006600u - 510u;
 constexpr float kC1 = 443.0f / 65536.0f;  // the 1MAD scale
 
-template <int CODE, int V>
-__device__ __forceinline__ uint32_t step_word(uint32_t s, const uint32_t* lut_lane, int qshift) {
-    if constexpr (V == 2) {
-        return code_v2<CODE>(s, lut_lane, qshift);
+template <int CODE>
+__device__ __forceinline__ void mma_step(float (&d)[4], const uint32_t (&pre)[4], const uint32_t (&aux)[4], uint32_t b0,
+                                         uint32_t b1) {
+#define QLK_MMA_TAIL \
+    "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {a0,a1,a2,a3}, {%8,%9}, {%0,%1,%2,%3};\n\t}"
+    if constexpr (CODE == kCode3INST) {
+        asm volatile(
+            "{\n\t.reg .b32 a0, a1, a2, a3;\n\t"
+            "lop3.b32 a0, %4, %10, %11, 0x6a;\n\tlop3.b32 a1, %5, %10, %11, 0x6a;\n\t"
+            "lop3.b32 a2, %6, %10, %11, 0x6a;\n\tlop3.b32 a3, %7, %10, %11, 0x6a;\n\t" QLK_MMA_TAIL
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(pre[0]), "r"(pre[1]), "r"(pre[2]), "r"(pre[3]), "r"(b0), "r"(b1), "n"(kMask3INST), "n"(kXor3INST));
     } else if constexpr (CODE == kCode1MAD) {
-        return __dp4a(kA1MAD * s + kB1MAD, 0x01010101u, kDp4aSplitAcc);
-    } else if constexpr (CODE == kCode3INST) {
-        return ((kA3INST * s + kB3INST) & kMask3INST) ^ kXor3INST;
+        asm volatile(
+            "{\n\t.reg .b32 a0, a1, a2, a3;\n\t"
+            "dp4a.u32.u32 a0, %4, %10, %11;\n\tdp4a.u32.u32 a1, %5, %10, %11;\n\t"
+            "dp4a.u32.u32 a2, %6, %10, %11;\n\tdp4a.u32.u32 a3, %7, %10, %11;\n\t" QLK_MMA_TAIL
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(pre[0]), "r"(pre[1]), "r"(pre[2]), "r"(pre[3]), "r"(b0), "r"(b1), "n"(0x01010101u),
+              "n"(kDp4aSplitAcc));
     } else if constexpr (CODE == kCodeHYB) {
-        return hyb_word(kAHYB * s + kBHYB, lut_lane, qshift);
+        asm volatile(
+            "{\n\t.reg .b32 a0, a1, a2, a3;\n\t"
+            "lop3.b32 a0, %4, %10, %14, 0x78;\n\tlop3.b32 a1, %5, %11, %14, 0x78;\n\t"
+            "lop3.b32 a2, %6, %12, %14, 0x78;\n\tlop3.b32 a3, %7, %13, %14, 0x78;\n\t" QLK_MMA_TAIL
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(pre[0]), "r"(pre[1]), "r"(pre[2]), "r"(pre[3]), "r"(b0), "r"(b1), "r"(aux[0]), "r"(aux[1]),
+              "r"(aux[2]), "r"(aux[3]), "n"(0x8000u));
     } else {
-        return lut_lane[s * 32u];
+        mma_16816(d, pre, b0, b1);
     }
+#undef QLK_MMA_TAIL
 }
 
 // Decode + MMA of one unit: lane (g, c) holds, for thread-row h (row g + 8h),
@@ -155,14 +196,13 @@ struct StepMMAs {
     static constexpr int NM = 32 / V;                // MMAs per unit
     static constexpr int NW = K2 + 1;
 
-    template <bool XSMEM>
     static __device__ __forceinline__ void run(const uint32_t (&cw)[2][NW], uint32_t lmask, const uint32_t* lut_lane,
                                                int qshift, const uint4* xsrc, int xstride, bool use_x,
                                                float (&acc)[2][4]) {
 #pragma unroll
         for (int u = 0; u < NM; u += 2) {
             if (kQuad && ((u / (kQuad ? MP : 1)) & 1)) continue;  // produced together with MMAs u - MP, u - MP + 1
-            uint32_t a[4][4];
+            uint32_t pre[4][4], aux[4][4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -172,31 +212,31 @@ struct StepMMAs {
                     if constexpr (kQuad) {
                         uint32_t s, s2;
                         state_pair<kV, L16>(cw[h], t, lmask, s, s2);
-                        a[q][r] = step_word<CODE, V>(s, lut_lane, qshift);
-                        a[2 + q][r] = step_word<CODE, V>(s2, lut_lane, qshift);
+                        step_pre<CODE, V>(s, lut_lane, qshift, pre[q][r], aux[q][r]);
+                        step_pre<CODE, V>(s2, lut_lane, qshift, pre[2 + q][r], aux[2 + q][r]);
                     } else if constexpr (kPair) {  // MP == 1: step t pairs with step t + 2, of MMA u + 1
                         if (e < 2) {
                             uint32_t s, s2;
                             state_pair<kV, L16>(cw[h], t, lmask, s, s2);
-                            a[0][r] = step_word<CODE, V>(s, lut_lane, qshift);
-                            a[1][r] = step_word<CODE, V>(s2, lut_lane, qshift);
+                            step_pre<CODE, V>(s, lut_lane, qshift, pre[0][r], aux[0][r]);
+                            step_pre<CODE, V>(s2, lut_lane, qshift, pre[1][r], aux[1][r]);
                         }
                     } else {
-                        a[q][r] = step_word<CODE, V>(state_one<kV, L16>(cw[h], t, lmask), lut_lane, qshift);
+                        step_pre<CODE, V>(state_one<kV, L16>(cw[h], t, lmask), lut_lane, qshift, pre[q][r], aux[q][r]);
                     }
                 }
             }
             uint4 b0 = make_uint4(0u, 0u, 0u, 0u), b1 = b0;
             if (use_x) {
-                b0 = XSMEM ? xsrc[(u >> 1) * xstride] : __ldg(xsrc + (u >> 1) * xstride);
-                if (kQuad) b1 = XSMEM ? xsrc[((u + MP) >> 1) * xstride] : __ldg(xsrc + ((u + MP) >> 1) * xstride);
+                b0 = __ldg(xsrc + (u >> 1) * xstride);
+                if (kQuad) b1 = __ldg(xsrc + ((u + MP) >> 1) * xstride);
             }
             // two accumulators: two dependent MMA chains of half the length
-            mma_16816(acc[0], a[0], b0.x, b0.y);
-            mma_16816(acc[1], a[1], b0.z, b0.w);
+            mma_step<CODE>(acc[0], pre[0], aux[0], b0.x, b0.y);
+            mma_step<CODE>(acc[1], pre[1], aux[1], b0.z, b0.w);
             if (kQuad) {
-                mma_16816(acc[0], a[2], b1.x, b1.y);
-                mma_16816(acc[1], a[3], b1.z, b1.w);
+                mma_step<CODE>(acc[0], pre[2], aux[2], b1.x, b1.y);
+                mma_step<CODE>(acc[1], pre[3], aux[3], b1.z, b1.w);
             }
         }
     }
@@ -209,7 +249,6 @@ struct StepMMAs {
 template <int K2, bool L16>
 struct StepMMAs<kCodeE8P, K2, 8, L16> {
     static constexpr int NW = K2 + 1;
-    template <bool XSMEM>
     static __device__ __forceinline__ void run(const uint32_t (&cw)[2][NW], uint32_t, const uint32_t* lut_lane, int,
                                                const uint4* xsrc, int xstride, bool use_x, float (&acc)[2][4]) {
         static_assert(K2 == 4, "the E8 code stores 16 bits per 8 weights");
@@ -220,7 +259,7 @@ struct StepMMAs<kCodeE8P, K2, 8, L16> {
             e8p_pairs((t & 1) ? (w0 & 0xFFFFu) : (w0 >> 16), lut_lane, p0);
             e8p_pairs((t & 1) ? (w1 & 0xFFFFu) : (w1 >> 16), lut_lane, p1);
             uint4 b = make_uint4(0u, 0u, 0u, 0u);
-            if (use_x) b = XSMEM ? xsrc[t * xstride] : __ldg(xsrc + t * xstride);
+            if (use_x) b = __ldg(xsrc + t * xstride);
             const uint32_t a0[4] = {p0[0], p1[0], p0[1], p1[1]};
             const uint32_t a1[4] = {p0[2], p1[2], p0[3], p1[3]};
             mma_16816(acc[0], a0, b.x, b.y);
@@ -243,14 +282,11 @@ struct GemvArgs {
     long long units;        // (row tile, block) units over all parts
     uint32_t lmask;         // (1 << L) - 1
     int qshift;             // HYB: 32 - Q
-    const uint32_t* lut;    // HYB / table code: 2^Q words
+    const uint32_t* lut;    // HYB / table code / E8 shapes: 2^Q words
     int lut_entries;
     int batch;              // 1..8
     int m, n;
-    const __half* x;        // [batch][n] (in-kernel input transform)
-    const uint32_t* sin_bits;
-    int B_n;
-    const uint4* xstep;     // x' step words from the input-transform kernel (else unused)
+    const uint4* xstep;     // x' step words from the input-transform kernel
     float* z;               // [batch][m], all-zero on entry and on exit
     int* tickets;           // [m / B_m], all-zero on entry and on exit
     int B_m;
@@ -287,7 +323,7 @@ __device__ __forceinline__ void load_unit_k2(uint32_t (&w)[2][8], const uint32_t
 // One unit at K2 = 2k: take its words from nxt, start the next unit's load
 // into nxt (NXW = K2: a one-part layer; NXW = 8: the next unit's own K2),
 // then decode and multiply.
-template <int CODE, int K2, int V, bool L16, bool XSMEM, int NXW>
+template <int CODE, int K2, int V, bool L16, int NXW>
 __device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][NXW], const uint32_t* next_base, int next_k2, int lane,
                                           int src_lane, const GemvArgs& p, const uint32_t* lut_lane, const uint4* xsrc,
                                           int xstride, bool use_x, float (&acc)[2][4]) {
@@ -297,46 +333,24 @@ __device__ __forceinline__ void gemv_unit(uint32_t (&nxt)[2][NXW], const uint32_
 #pragma unroll
         for (int i = 0; i < K2; ++i) cw[h][i + 1] = nxt[h][i];
     if (next_base) {
-        if constexpr (NXW == K2)
-            load_unit<K2>(nxt, next_base, lane);
-        else
+        // NXW = 8 holds any bitwidth: the next unit may belong to a part of
+        // another bitwidth (it follows its own next_k2); else a one-part layer
+        if constexpr (NXW == 8)
             load_unit_k2(nxt, next_base, next_k2, lane);
+        else
+            load_unit<K2>(nxt, next_base, lane);
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
-    StepMMAs<CODE, K2, V, L16>::template run<XSMEM>(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
-}
-
-// One unit of a one-part layer whose code words are in buf[0]: the buffered
-// units move down one slot, the unit PD ahead of this one starts loading into
-// buf[PD-1] (pf: its address, or null), then decode and multiply.
-template <int CODE, int K2, int V, bool L16, bool XSMEM, int PD>
-__device__ __forceinline__ void gemv_unit_pd(uint32_t (&buf)[PD][2][K2], const uint32_t* pf, int lane, int src_lane,
-                                             const GemvArgs& p, const uint32_t* lut_lane, const uint4* xsrc,
-                                             int xstride, bool use_x, float (&acc)[2][4]) {
-    uint32_t cw[2][K2 + 1];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int i = 0; i < K2; ++i) cw[h][i + 1] = buf[0][h][i];
-#pragma unroll
-    for (int d = 0; d + 1 < PD; ++d)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int i = 0; i < K2; ++i) buf[d][h][i] = buf[d + 1][h][i];
-    if (pf) load_unit<K2>(buf[PD - 1], pf, lane);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) cw[h][0] = __shfl_sync(0xffffffffu, cw[h][K2], src_lane);
-    StepMMAs<CODE, K2, V, L16>::template run<XSMEM>(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
+    StepMMAs<CODE, K2, V, L16>::run(cw, p.lmask, lut_lane, p.qshift, xsrc, xstride, use_x, acc);
 }
 
 // The unit's bitwidth picks the decoder (V = 1 has whole bitwidths only).
-template <int CODE, int V, bool L16, bool XSMEM>
+template <int CODE, int V, bool L16>
 __device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], const uint32_t* next_base, int next_k2,
                                              int lane, int src_lane, const GemvArgs& p, const uint32_t* lut_lane,
                                              const uint4* xsrc, int xstride, bool use_x, float (&acc)[2][4]) {
-#define QLK_UNIT(K) gemv_unit<CODE, K, V, L16, XSMEM, 8>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xsrc, \
+#define QLK_UNIT(K) gemv_unit<CODE, K, V, L16, 8>(nxt, next_base, next_k2, lane, src_lane, p, lut_lane, xsrc, \
                                                          xstride, use_x, acc)
     switch (k2) {
         case 2: QLK_UNIT(2); break;
@@ -348,33 +362,6 @@ __device__ __forceinline__ void gemv_unit_k2(int k2, uint32_t (&nxt)[2][8], cons
         default: QLK_UNIT(8); break;
     }
 #undef QLK_UNIT
-}
-
-// x' = H_n diag(s_in) x for every batch row, as step words in shared memory
-// (fp32 transform in `work`, then one rounding to fp16).
-template <int V>
-__device__ __forceinline__ void input_transform_smem(const GemvArgs& p, uint32_t* xs_words, float* work) {
-    const int n = p.n, batch = p.batch;
-    const float scale = rsqrtf((float)p.B_n);
-    fwht_blocks_smem(
-        work, batch * n, p.B_n,
-        [&](int i, float (&v)[8]) {
-            const int b = i / n, col = i - b * n;
-            const uint4 raw = *reinterpret_cast<const uint4*>(p.x + (size_t)b * n + col);
-            const uint32_t sw = p.sin_bits[col >> 5] >> (col & 31);  // 8 consecutive sign bits (col % 8 == 0)
-            const __half* hv = reinterpret_cast<const __half*>(&raw);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float f = __half2float(hv[e]);
-                v[e] = ((sw >> e) & 1u) ? -f : f;
-            }
-        },
-        [&](int i, const float (&v)[4]) {
-            const int b = i / n, col = i - b * n;
-            const float w[4] = {v[0] * scale, v[1] * scale, v[2] * scale, v[3] * scale};
-            store_xstep4<V>(xs_words, col, b, batch, w);
-        });
-    __syncthreads();
 }
 
 // The output transform of Hadamard block hb for every batch row (as many rows
@@ -419,7 +406,9 @@ __device__ __forceinline__ void output_transform_block(const GemvArgs& p, int hb
 }
 
 // After the CTA's last atomics into z: count its units into the tickets of the
-// Hadamard blocks they touch and transform the blocks it completes.
+// Hadamard blocks they touch and transform the blocks it completes.  The
+// CTA's units are [c0, c1) of the row-tile-major walk (unit = T nb + j, T the
+// global row tile).
 constexpr int kEpiOwnedMax = 32;
 __device__ __forceinline__ void output_epilogue(const GemvArgs& p, float* buf, long long c0, long long c1) {
     __shared__ int owned[kEpiOwnedMax];
@@ -452,19 +441,19 @@ __device__ __forceinline__ void output_epilogue(const GemvArgs& p, float* buf, l
     }
 }
 
-// One CTA per SM (at most).  CTA i takes units [U*i/G, U*(i+1)/G) and splits
-// them evenly over its warps.  K2F: the bitwidth of a one-part layer (decoder
-// fixed at compile time), 0 for several parts (decoder per unit).  Every
-// thread runs every phase, since the transforms use CTA barriers.
-template <int CODE, int V, bool L16, bool XSMEM, int K2F>
+// One CTA per SM (at most).  CTA i takes units [U*i/G, U*(i+1)/G) of the
+// row-tile-major walk (unit = T nb + j over the global row tile T; partial
+// sums accumulate over the blocks of a tile) and splits them evenly over its
+// warps; x' comes from the input-transform kernel.  K2F: the bitwidth of a
+// one-part layer (decoder fixed at compile time), 0 for several parts
+// (decoder per unit).  Every thread runs the epilogue, which uses CTA
+// barriers.
+template <int CODE, int V, bool L16, int K2F>
 __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(GemvArgs p) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int NXW = K2F ? K2F : 8;
-    const int lane = threadIdx.x & 31;
-    const int lut_words = uses_table(CODE) ? p.lut_entries * 32 : 0;
     constexpr int VX = V == 1 ? 1 : 2;  // x' layout: one column per B word (V = 1) or two
-    uint32_t* xs_words = smem + lut_words;
-    float* work = reinterpret_cast<float*>(smem + lut_words + (XSMEM ? p.batch * p.n / VX : 0));
+    const int lane = threadIdx.x & 31;
     if (uses_table(CODE)) fill_lut_smem(smem, p.lut, p.lut_entries);
     const uint32_t* lut_lane = smem + lane;
 
@@ -477,11 +466,12 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     const int src_lane = (lane & ~3) | ((c + 3) & 3);
     const int batch = p.batch;
 
-    // walker over (part, row tile, block)
+    // walker over (part, row tile in the part, block)
+    long long Tg = u0 / nb;
+    int j = (int)(u0 % nb);
     int pt = 0;
-    long long rest = u0;
-    while (pt + 1 < p.nparts && rest >= (long long)p.part[pt].rt * nb) rest -= (long long)p.part[pt++].rt * nb;
-    int t = (int)(rest / nb), j = (int)(rest % nb);
+    while (pt + 1 < p.nparts && Tg >= p.part[pt].rt) Tg -= p.part[pt++].rt;
+    int t = (int)Tg;
     auto unit_base = [&](int part, int tile, int blk) {
         return p.part[part].words + ((size_t)tile * nb + blk) * 64 * p.part[part].k2;
     };
@@ -489,27 +479,18 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     // bits are written once at create time, so the first unit's words are
     // fetched before waiting for the previous kernel (the producer of x or x',
     // the previous forward that used z).
-    // A one-part layer keeps PD units in flight per warp (two at up to 2 bits
-    // per weight, where a unit's decode is shortest), a multi-part layer one.
-    constexpr int PD = (K2F != 0 && K2F <= 4) ? 2 : 1;
-    constexpr int UWF = 64 * (K2F ? K2F : 1);  // words per unit of a one-part layer
     uint32_t nxt[2][NXW];
-    uint32_t buf[PD][2][K2F ? K2F : 1];
-    if constexpr (K2F != 0) {
-#pragma unroll
-        for (int d = 0; d < PD; ++d)
-            if (u0 + d < u1) load_unit<K2F>(buf[d], p.part[0].words + (size_t)(u0 + d) * UWF, lane);
-    } else if (u0 < u1) {
-        load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
+    if (u0 < u1) {
+        if constexpr (K2F != 0)
+            load_unit<K2F>(nxt, unit_base(pt, t, j), lane);
+        else
+            load_unit_k2(nxt, unit_base(pt, t, j), p.part[pt].k2, lane);
     }
     grid_dependency_wait();
-    if constexpr (XSMEM)
-        input_transform_smem<VX>(p, xs_words, work);  // ends with a CTA barrier (the table is filled too)
-    else if (uses_table(CODE))
-        __syncthreads();
+    if (uses_table(CODE)) __syncthreads();
     grid_launch_dependents();
 
-    const uint4* xbase = XSMEM ? reinterpret_cast<const uint4*>(xs_words) : p.xstep;
+    const uint4* xbase = p.xstep;
     const int xstride = batch * 4;  // uint4 groups between consecutive u2
     const bool use_x = g < batch;
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -545,11 +526,10 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
         }
         const uint4* xsrc = xbase + ((size_t)j * (16 / VX) * batch + g) * 4 + c;
         if constexpr (K2F != 0)
-            gemv_unit_pd<CODE, K2F, V, L16, XSMEM, PD>(
-                buf, unit + PD < u1 ? p.part[0].words + (size_t)(unit + PD) * UWF : nullptr, lane, src_lane, p,
-                lut_lane, xsrc, xstride, use_x, acc);
+            gemv_unit<CODE, K2F, V, L16, NXW>(nxt, next_base, K2F, lane, src_lane, p, lut_lane, xsrc, xstride,
+                                                     use_x, acc);
         else
-            gemv_unit_k2<CODE, V, L16, XSMEM>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p,
+            gemv_unit_k2<CODE, V, L16>(p.part[pt].k2, nxt, next_base, p.part[npt].k2, lane, src_lane, p,
                                               lut_lane, xsrc, xstride, use_x, acc);
         pt = npt;
         t = nt;
@@ -563,19 +543,15 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
 
 GemvPlan plan_gemv(const Layer& L, int batch) {
     GemvPlan pl;
-    long long units = 0;
-    for (int i = 0; i < L.nparts; ++i) units += (long long)(L.parts[i].rows / kRowTile) * (L.n / kT);
+    long long rt_total = 0;
+    for (int i = 0; i < L.nparts; ++i) rt_total += L.parts[i].rows / kRowTile;
+    const long long units = rt_total * (L.n / kT);
     pl.grid = (int)(units < L.num_sms ? units : L.num_sms);
     const long long per_cta = (units + pl.grid - 1) / pl.grid;
     const long long per_warp = (per_cta + kGemvMaxWarps - 1) / kGemvMaxWarps;
     pl.threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
     const long long lut_words = uses_table(L.code) ? (32ll << L.Q) : 0;
-    const long long elems = (long long)batch * L.n;
-    const long long xs_words = elems / (L.V == 1 ? 1 : 2);
-    const long long work_words = elems + elems / 16;
     const long long budget = kGemvMaxSmem / 4;
-    pl.xsmem = elems <= kFuseInElems && lut_words + xs_words + work_words <= budget;
-    long long main_words = lut_words + (pl.xsmem ? xs_words + work_words : 0);
     // the output transform in-kernel when one CTA's share of it is small, as
     // many batch rows of one Hadamard block at once as fit (plus its sign words)
     pl.fuse_out = (long long)batch * L.B_m <= kFuseOutElems;
@@ -585,7 +561,7 @@ GemvPlan plan_gemv(const Layer& L, int batch) {
     if (rows > batch) rows = batch;
     if (rows < 1) rows = 1;
     const long long epi_words = pl.fuse_out ? rows * row_words + sign_words : 0;
-    pl.smem_bytes = (int)((main_words > epi_words ? main_words : epi_words) * 4);
+    pl.smem_bytes = (int)((lut_words > epi_words ? lut_words : epi_words) * 4);
     return pl;
 }
 
@@ -595,16 +571,12 @@ size_t gemv_xstep_bytes(const Layer& L, int batch) { return (size_t)batch * L.n 
 
 template <int CODE, int K2, int V, bool L16>
 struct GemvLaunch {
-    template <bool XSMEM>
-    static cudaError_t go(const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
-        constexpr int K2F = K2 == 99 ? 0 : K2;
-        cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, V, L16, XSMEM, K2F>>(kGemvMaxSmem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(trellis_gemv_kernel<CODE, V, L16, XSMEM, K2F>, dim3(pl.grid), dim3(pl.threads),
-                          (size_t)pl.smem_bytes, st, a);
-    }
     static cudaError_t run(const GemvArgs& a, const GemvPlan& pl, cudaStream_t st) {
-        return pl.xsmem ? go<true>(a, pl, st) : go<false>(a, pl, st);
+        constexpr int K2F = K2 == 99 ? 0 : K2;
+        cudaError_t e = ensure_smem_limit<trellis_gemv_kernel<CODE, V, L16, K2F>>(kGemvMaxSmem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(trellis_gemv_kernel<CODE, V, L16, K2F>, dim3(pl.grid), dim3(pl.threads),
+                          (size_t)pl.smem_bytes, st, a);
     }
 };
 
@@ -612,9 +584,7 @@ template <int CODE, int K2, int V, bool L16>
 struct GemvPrepare {
     static cudaError_t run() {
         constexpr int K2F = K2 == 99 ? 0 : K2;
-        cudaError_t e = preload_kernel<trellis_gemv_kernel<CODE, V, L16, true, K2F>>(kGemvMaxSmem);
-        if (e == cudaSuccess) e = preload_kernel<trellis_gemv_kernel<CODE, V, L16, false, K2F>>(kGemvMaxSmem);
-        return e;
+        return preload_kernel<trellis_gemv_kernel<CODE, V, L16, K2F>>(kGemvMaxSmem);
     }
 };
 
@@ -924,8 +894,8 @@ cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_
 }
 
 
-cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
-                        int* tickets, void* y, int y_dtype, cudaStream_t st) {
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, int batch, float* z, int* tickets,
+                        void* y, int y_dtype, cudaStream_t st) {
     GemvArgs a;
     a.nparts = L.nparts;
     a.nb = L.n / kT;
@@ -945,9 +915,6 @@ cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const
     a.batch = batch;
     a.m = L.m;
     a.n = L.n;
-    a.x = (const __half*)x;
-    a.sin_bits = L.sin_bits;
-    a.B_n = L.B_n;
     a.xstep = (const uint4*)xstep;
     a.z = z;
     a.tickets = tickets;

@@ -16,11 +16,7 @@ constexpr int kMaxHadamard = 32768;
 
 constexpr int kGemvMaxWarps = 16;        // decode-GEMV: warps of its one CTA per SM (<= 128 registers/thread)
 constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
-#ifndef QL_FUSE_IN_ELEMS
-#define QL_FUSE_IN_ELEMS 16384
-#endif
-constexpr int kFuseInElems = QL_FUSE_IN_ELEMS;  // batch * n up to which the GEMV computes x' itself
-constexpr int kFuseOutElems = 8192;  // batch * B_m up to which the GEMV's last CTA per block does the output transform
+constexpr int kFuseOutElems = 256;  // batch * B_m up to which the GEMV's last CTA per block does the output transform
 constexpr int kMaxParts = 8;          // row parts of one layer (layers fused along m, own bitwidth each)
 constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
 constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
@@ -149,12 +145,10 @@ cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npa
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st,
                            float zscale = 1.0f);
 
-// How one decode-GEMV launch is shaped: grid and CTA size, whether the input
-// transform runs inside it (xsmem: x' computed by every CTA into its shared
-// memory), and its dynamic shared memory.
+// How one decode-GEMV launch is shaped: grid and CTA size, whether the
+// output transform runs in its epilogue, and its dynamic shared memory.
 struct GemvPlan {
     int grid, threads;
-    bool xsmem;
     bool fuse_out;  // output transform in the GEMV's epilogue (else launch_rht_out after it)
     int smem_bytes;
 };
@@ -164,14 +158,13 @@ GemvPlan plan_gemv(const Layer& L, int batch);
 size_t gemv_xstep_bytes(const Layer& L, int batch);
 // The factor between the decode-GEMV's z and W_hat x' (the 1MAD code's C1, else 1).
 float gemv_z_scale(const Layer& L);
-// The whole forward for batch <= 8 after the input transform: decode-GEMV over
-// all row parts, z accumulation, and the output transform into y (fp32 or
-// fp16) by the CTA that completes each output Hadamard block.  z ([batch][m]
-// fp32) and tickets ([m / B_m] int) must be all-zero on entry and are all-zero
-// again when the kernel completes.  With pl.xsmem x' is computed from x
-// in-kernel, else read from xstep.
-cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
-                        int* tickets, void* y, int y_dtype, cudaStream_t st);
+// The forward for batch <= 8 after the input-transform kernel: decode-GEMV
+// over all row parts into z, and (pl.fuse_out) the output transform into y
+// (fp32 or fp16) by the CTA that completes each output Hadamard block; else
+// launch_rht_out follows.  z ([batch][m] fp32) and tickets ([m / B_m] int)
+// must be all-zero on entry and are all-zero again when the forward is done.
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, int batch, float* z, int* tickets,
+                        void* y, int y_dtype, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
 // z[b][row] += W_hat x' for all parts (z all-zero on entry), x' in tensor-core
 // tiles with npad (multiple of 16, <= 256) rows, b < batch; the (128-row tile,

@@ -297,16 +297,14 @@ int prepare_acc(Layer& L, size_t z_bytes, cudaStream_t st) {
 // kernel; the output transform in its epilogue).
 int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
     const GemvPlan pl = plan_gemv(L, batch);
-    int rc = pl.xsmem ? QL_OK : ensure(&L.xp, &L.xp_bytes, gemv_xstep_bytes(L, batch));
+    int rc = ensure(&L.xp, &L.xp_bytes, gemv_xstep_bytes(L, batch));
     if (rc == QL_OK) rc = prepare_acc(L, (size_t)batch * L.m * 4, st);
     if (rc != QL_OK) return rc;
-    cudaError_t e = cudaSuccess;
-    L.last_launches = 1 + (pl.xsmem ? 0 : 1) + (pl.fuse_out ? 0 : 1);
-    if (!pl.xsmem) e = launch_rht_in_xstep(L, x, batch, L.xp, st);
+    L.last_launches = 2 + (pl.fuse_out ? 0 : 1);
+    cudaError_t e = launch_rht_in_xstep(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-    if (e == cudaSuccess)
-        e = launch_gemv(L, pl, x, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
+    if (e == cudaSuccess) e = launch_gemv(L, pl, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
     if (e == cudaSuccess && slot >= 0) {
         e = record_event(L.prof_ev[2 * slot + 1], st);
         L.prof_next = (L.prof_next + 1) % L.prof_cap;
@@ -721,12 +719,11 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     if (!x || !y) return QL_E_ARG;
     if (batch > kGemvMaxBatch) return QL_E_UNSUPPORTED;
     Layer& L = h->L;
-    // array layout: output-block tickets, z, then x' when the input transform
-    // runs as its own kernel
+    // array layout: output-block tickets, z, x'
     const GemvPlan pl = plan_gemv(L, batch);
     const size_t t_bytes = ticket_bytes(L);
     const size_t z_bytes = ((size_t)batch * L.m * 4 + 255) / 256 * 256;
-    const size_t xp_bytes = pl.xsmem ? 0 : gemv_xstep_bytes(L, batch);
+    const size_t xp_bytes = gemv_xstep_bytes(L, batch);
     if (t_bytes + z_bytes + xp_bytes > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_E_SCRATCH;
     DeviceGuard g(L.device);
     if (!g.ok) return QL_E_CUDA;
@@ -739,13 +736,13 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     cudaStream_t st = (cudaStream_t)stream;
     // tickets and z must start at zero; another handle's failed call may have left sums there
     cudaError_t e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
-    if (e == cudaSuccess && !pl.xsmem) e = launch_rht_in_xstep(L, x, batch, xp, st);
-    if (e == cudaSuccess) e = launch_gemv(L, pl, x, xp, batch, z, tickets, y, y_dtype, st);
+    if (e == cudaSuccess) e = launch_rht_in_xstep(L, x, batch, xp, st);
+    if (e == cudaSuccess) e = launch_gemv(L, pl, xp, batch, z, tickets, y, y_dtype, st);
     if (e == cudaSuccess && !pl.fuse_out) e = launch_rht_out(L, z, batch, y, y_dtype, st, gemv_z_scale(L));
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.last_launches = 1 + (pl.xsmem ? 0 : 1) + (pl.fuse_out ? 0 : 1);
+    L.last_launches = 2 + (pl.fuse_out ? 0 : 1);
     return QL_OK;
 }

@@ -148,12 +148,26 @@ __global__ void __launch_bounds__(256) rht_in_block_kernel(const __half* __restr
     const int base = (j / R) * B;  // first column of the Hadamard block
     grid_dependency_wait();
     const __half* xr = x + (size_t)b * n + base + t;
+    const uint32_t* sr = sin_bits + ((base + t) >> 5);  // + 8 a: the sign word of column base + 256 a + t
     float acc = 0.f;
-    for (int a = 0; a < R; ++a) {
-        const int col = base + 256 * a + t;
-        float v = __half2float(xr[256 * a]);
-        if ((sin_bits[col >> 5] >> (col & 31)) & 1u) v = -v;
-        acc += (__popc(jr & a) & 1) ? -v : v;
+    for (int a0 = 0; a0 < R; a0 += 16) {  // R is a power of two: sixteen (or R) loads in flight
+        const int na = R - a0 < 16 ? R - a0 : 16;
+        float v[16];
+        uint32_t sw[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (q < na) {
+                v[q] = __half2float(__ldg(xr + 256 * (a0 + q)));
+                sw[q] = __ldg(sr + 8 * (a0 + q));
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (q < na) {
+                const uint32_t neg = ((sw[q] >> (t & 31)) ^ (uint32_t)__popc(jr & (a0 + q))) & 1u;
+                acc += neg ? -v[q] : v[q];
+            }
+        }
     }
     w[t] = acc;
     __syncthreads();
