@@ -239,7 +239,7 @@ def job_tokens_per_s(world, steps, batch, secs):
 # the sources each profiled kernel is built from (its DRAM-traffic capture is
 # valid while these are unchanged)
 KERNEL_SOURCES = {
-    "gemv": ("gemv.cu", "codes.cuh", "layout.cuh", "fwht.cuh", "internal.h"),
+    "gemv": ("gemv.cu", "codes.cuh", "layout.cuh", "fwht.cuh", "xstep.cuh", "internal.h"),
     "gemm": ("gemm_tc.cu", "codes.cuh", "layout.cuh", "tc_ptx.cuh", "internal.h"),
 }
 
@@ -253,7 +253,8 @@ def _source_hash(kind):
     return h.hexdigest()[:16]
 
 
-_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "inst": 1, "": 1, "nsecond": 1e-9,
+_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "inst": 1, "": 1, "nsecond": 1e-9, "ns": 1e-9,
+          "us": 1e-6, "ms": 1e-3,
           "usecond": 1e-6, "msecond": 1e-3}
 _COUNTER_METRICS = {"dram__bytes_read.sum": "dram_read", "dram__bytes_write.sum": "dram_write",
                     "smsp__inst_executed.sum": "warp_inst", "smsp__thread_inst_executed.sum": "thread_inst",

@@ -14,8 +14,11 @@
 // layer are cut into one contiguous run per CTA, one CTA per SM, so every SM
 // decodes the same number of weights whatever the tile count.  A CTA's run
 // falls into segments of consecutive blocks of one tile; each segment is
-// accumulated in tensor memory and added into z with fp32 reductions (z is
-// all-zero when the kernel starts, so tiles split between CTAs sum up).
+// accumulated in tensor memory and written with plain stores to its own slot
+// of a partial-sum workspace (slot = the segment's rank in unit order, so the
+// one to three segments of a tile have consecutive slots); the output
+// transform sums a tile's slots as it reads them.  No atomics, and nothing to
+// re-zero between forwards.
 //
 // Warp roles (a warp runs on SM sub-partition warp % 4, and may only touch
 // tensor-memory lanes 32 * (warp % 4) .. + 31):
@@ -25,8 +28,10 @@
 //                  per lane, 64 consecutive trellis steps per lane, and writes
 //                  the decoded fp16 pairs straight into the stage's A slot in
 //                  tensor memory (tcgen05.st): decoded weights never touch
-//                  shared memory.  At the end of a segment the decoders read
-//                  the accumulator back and reduce it into z;
+//                  shared memory;
+//   4 epilogue     at the end of each segment, read the accumulator back (one
+//     warps        lane quarter each) and store it to the segment's slot, while
+//                  the decoders go on filling the A slots of the next segment;
 //   MMA warp       allocates tensor memory (accumulator in columns [0, 256),
 //                  A slots of 32 columns from 256 on); one lane issues the 4
 //                  MMAs (K = 16 each, A from tensor memory, x' from shared
@@ -42,6 +47,8 @@
 // and still frees its tensor memory.
 #include <cuda_fp16.h>
 
+#include <vector>
+
 #include "codes.cuh"
 #include "internal.h"
 #include "layout.cuh"
@@ -53,9 +60,10 @@ constexpr int kTcRows = 128;         // M of one tile
 constexpr int kTcK = 64;             // K of one stage (one 128-byte swizzled row of fp16)
 constexpr int kTcDecoders = 16;      // decoder warps: four groups of 4, group g decodes quarter g of each block
 constexpr int kTcGroup = 4;          // decoder warps per group (one per 32-row lane quarter)
-constexpr int kTcWarps = 20;
+constexpr int kTcWarps = 23;
 constexpr int kTcThreads = kTcWarps * 32;
-constexpr int kWarpMma = 16, kWarpXProd = 17, kWarpCodeProd = 18;  // warp 19 only joins set-up and teardown
+constexpr int kWarpMma = 16, kWarpXProd = 17, kWarpCodeProd = 18;
+constexpr int kWarpEpi0 = 19, kTcEpiWarps = 4;  // warps 19..22: lane quarters 3, 0, 1, 2
 constexpr int kTcMaxStages = 8;      // stage slots (A in tensor memory, x' tile in shared memory)
 constexpr uint32_t kTcTmemCols = 512;  // accumulator [0, 256) and up to 8 A slots of 32 columns
 constexpr uint32_t kTcTmemA = 256;     // first A-slot column
@@ -81,7 +89,6 @@ __device__ __forceinline__ bool decoder_role(int w, int& grp, int& qtr) {
 struct TcPart {
     const uint32_t* words;  // kernel layout
     int rt;                 // row tiles of 16 rows
-    int row0;               // first layer row
     int k2;                 // 2k: bits per two weights
     int tiles;              // 128-row tiles
 };
@@ -98,8 +105,8 @@ struct GemmArgs {
     const uint8_t* xt;      // x' tiles: [n / 64][npad][128 B, swizzled]
     int npad;               // MMA N: batch padded to a multiple of 16 (<= 256)
     int batch;              // valid columns
-    float* z;               // [batch][m], all-zero on entry
-    int m;
+    float* ws;              // partial sums: [segment slot][npad][128 rows], columns < batch written
+    const int* cta_seg;     // slot of each CTA's first segment
     int* status;
     int wait_tries;         // try_wait calls of up to kTcSuspendNs before a wait is declared expired
     int withhold;           // test hook: the x' producer withholds its first stage (its waits then expire)
@@ -329,7 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             mbar_init(empty(i), 1);            // MMA commit
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kTcDecoders);
+        mbar_init(acc_empty, kTcEpiWarps);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -433,13 +440,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             if (last) ++seg;
         }
     } else if (decoder_role(warp, grp, qtr)) {
-        // ---------------- decoders, and the epilogue of every segment ----------------
+        // ---------------- decoders ----------------
         const uint32_t* lut_lane = lut_smem + lane;
-        const int share = warp >> 2;   // 4 warps per lane quarter split the accumulator columns
-        const int chunks = p.npad / 16;
         const uint32_t lane_base = (uint32_t)(qtr * 32) << 16;
-        int seg = 0;
-        bool z_ready = false;
         TcRing rc(0, C), rs(grp, S);  // code block i, stage 4 i + grp
         for (TcWalk w(p, u0); w.u < u1; w.next(p), rc.advance(1, C), rs.advance(4, S)) {
             const int slot = rc.slot;
@@ -465,28 +468,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             }
             if (!ok) break;
             if (lane == 0) mbar_arrive(code_empty(slot));
-            if (w.u + 1 < u1 && w.j + 1 < p.nb) continue;
-            // ---- end of a segment: accumulator -> z (fp32 reductions) ----
-            if (!z_ready) {
-                grid_dependency_wait();  // z was last touched by the previous kernels
-                z_ready = true;
+        }
+    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kTcEpiWarps) {
+        // ---------------- epilogue: accumulator -> the segment's workspace slot ----------------
+        const int qtr = warp & 3;
+        const int rloc = qtr * 32 + lane;  // row within the tile
+        const uint32_t tbase = tmem + ((uint32_t)(qtr * 32) << 16);
+        int seg = 0;
+        float* ws = nullptr;
+        for (TcWalk w(p, u0); w.u < u1; w.next(p)) {
+            if (w.u + 1 < u1 && w.j + 1 < p.nb) continue;  // not the last unit of a segment
+            if (!ws) {
+                grid_dependency_wait();  // the previous kernels may still read the workspace
+                ws = p.ws + (size_t)p.cta_seg[blockIdx.x] * p.npad * kTcRows + rloc;
             }
             if (!wait_bar(acc_full, seg & 1, abort_flag, p.status, p.wait_tries)) break;
             tc_fence_after();
-            const int rloc = qtr * 32 + lane;  // row within the tile
-            const int tile = w.tile(p);
-            const int row = pt.row0 + tile * kTcRows + rloc;
-            const bool row_ok = tile * kTcRows + rloc < pt.rt * kRowTile;
-            for (int ci = share * chunks / 4; ci < (share + 1) * chunks / 4; ++ci) {
-                const int c0 = ci * 16;
-                uint32_t v[16];
-                tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
-                tmem_ld_wait();
-                if (row_ok) {
+            float* dst = ws + (size_t)seg * p.npad * kTcRows;
+            auto store16 = [&](const uint32_t (&v)[16], int c0) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c0 + e < p.batch) red_add_f32(p.z + (size_t)(c0 + e) * p.m + row, __uint_as_float(v[e]));
-                }
+                for (int e = 0; e < 16; ++e)
+                    if (c0 + e < p.batch) dst[(size_t)(c0 + e) * kTcRows] = __uint_as_float(v[e]);
+            };
+            // two register sets: the next chunk's load is in flight while this one is stored
+            uint32_t va[16], vb[16];
+            tmem_ld16(tbase, va);
+            for (int c0 = 0; c0 < p.npad; c0 += 32) {
+                tmem_ld_wait(va);
+                const bool more = c0 + 16 < p.npad;
+                if (more) tmem_ld16(tbase + (uint32_t)(c0 + 16), vb);
+                store16(va, c0);
+                if (!more) break;
+                tmem_ld_wait(vb);
+                if (c0 + 32 < p.npad) tmem_ld16(tbase + (uint32_t)(c0 + 32), va);
+                store16(vb, c0 + 16);
             }
             tc_fence_before();
             __syncwarp();
@@ -532,7 +547,43 @@ size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
     return 0;
 }
 
-cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st) {
+int tc_units(const Layer& L) {
+    int tiles = 0;
+    for (int i = 0; i < L.nparts; ++i) tiles += (L.parts[i].rows + kTcRows - 1) / kTcRows;
+    return tiles * (L.n / kT);
+}
+
+int tc_grid(const Layer& L) {
+    const int units = tc_units(L);
+    return units < L.num_sms ? units : L.num_sms;
+}
+
+// The stream-K segments in unit order: CTA c runs units [c U / G, (c+1) U / G)
+// and starts a new segment at its first unit and at every tile's first block.
+// cta_seg[c] = slot of CTA c's first segment (c <= G, cta_seg[G] = all
+// segments); tile_seg[t] = slot of tile t's first segment (t <= tiles).  The
+// segments of tile t are the slots tile_seg[t] .. tile_seg[t + 1] - 1.
+void tc_segments(const Layer& L, std::vector<int>& cta_seg, std::vector<int>& tile_seg) {
+    const int nb = L.n / kT, units = tc_units(L), G = tc_grid(L);
+    const int tiles = units / nb;
+    cta_seg.assign(G + 1, 0);
+    tile_seg.assign(tiles + 1, 0);
+    int slot = 0;
+    for (int c = 0; c < G; ++c) {
+        const int u0 = (int)((long long)c * units / G), u1 = (int)((long long)(c + 1) * units / G);
+        cta_seg[c] = slot;
+        for (int u = u0; u < u1; ++u) {
+            if (u == u0 || u % nb == 0) {
+                if (u % nb == 0) tile_seg[u / nb] = slot;
+                ++slot;
+            }
+        }
+    }
+    cta_seg[G] = slot;
+    tile_seg[tiles] = slot;
+}
+
+cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* ws, cudaStream_t st) {
     GemmArgs a;
     int k2max = 0;
     a.nparts = L.nparts;
@@ -542,7 +593,6 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
         const Part& pt = L.parts[i];
         a.part[i].words = L.words + pt.word_off;
         a.part[i].rt = pt.rows / kRowTile;
-        a.part[i].row0 = pt.row0;
         a.part[i].k2 = pt.k2;
         a.part[i].tiles = (pt.rows + kTcRows - 1) / kTcRows;
         tiles += a.part[i].tiles;
@@ -557,15 +607,15 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     a.xt = (const uint8_t*)xt;
     a.npad = npad;
     a.batch = batch;
-    a.z = z;
-    a.m = L.m;
+    a.ws = ws;
+    a.cta_seg = L.tc_seg;
     a.status = L.status;
     a.wait_tries = L.test_wait_tries > 0 ? L.test_wait_tries : kTcWaitTries;
     a.withhold = L.test_withhold;
     a.code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
     const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots);
     if (smem == 0) return cudaErrorInvalidValue;
-    const int grid = a.units < L.num_sms ? a.units : L.num_sms;
+    const int grid = tc_grid(L);
     const bool l16 = L.L == 16;
     if (L.code == kCode1MAD) return l16 ? launch_gemm_t<kCode1MAD, 1, true>(a, grid, smem, st)
                                         : launch_gemm_t<kCode1MAD, 1, false>(a, grid, smem, st);

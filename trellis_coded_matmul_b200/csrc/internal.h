@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <vector>
 
 #include "../../include/qlinear.h"
 
@@ -65,6 +66,15 @@ struct Layer {
     int last_launches;    // kernels launched by the most recent forward
     void* host_stage;     // device staging for qlinear_forward_host (x then y)
     size_t host_stage_bytes;
+    // tensor-core GEMM (batch > 8): its stream-K segment table (device, written at
+    // create: the slot of each CTA's first segment [grid + 1], then the slot of
+    // each 128-row tile's first segment [tiles + 1]) and the partial-sum workspace
+    // ([segment slot][npad][128] fp32, grown on demand)
+    int* tc_seg;
+    const int* tc_tile_seg;
+    int tc_slots;
+    void* tcws;
+    size_t tcws_bytes;
     int num_sms;
     // test hooks of the tensor-core GEMM (qlinear_test_stall): a shorter
     // limit on its bounded waits and a stage that never arrives
@@ -144,6 +154,11 @@ cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npa
 // z (fp32 [batch][m]) -> y = alpha zscale s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st,
                            float zscale = 1.0f);
+// The tensor-core GEMM's partial sums (launch_gemm_tc's workspace, npad
+// columns per slot) -> y = alpha s_out (H_m z), z = the sum of each tile's
+// segment slots; the workspace is only read.
+cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int npad, void* y, int y_dtype,
+                              cudaStream_t st);
 
 // How one decode-GEMV launch is shaped: grid and CTA size, whether the
 // output transform runs in its epilogue, and its dynamic shared memory.
@@ -166,10 +181,19 @@ float gemv_z_scale(const Layer& L);
 cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, int batch, float* z, int* tickets,
                         void* y, int y_dtype, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
-// z[b][row] += W_hat x' for all parts (z all-zero on entry), x' in tensor-core
-// tiles with npad (multiple of 16, <= 256) rows, b < batch; the (128-row tile,
-// 256-column block) units are split evenly over one CTA per SM.
-cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* z, cudaStream_t st);
+// W_hat x' for all parts, x' in tensor-core tiles with npad (multiple of 16,
+// <= 256) rows, b < batch; the (128-row tile, 256-column block) units are
+// split evenly over one CTA per SM (stream-K), and each CTA's segment (its
+// units within one tile) is stored to workspace slot L.tc_seg[cta] + k:
+// ws[slot][b][r] for the tile's row r < 128 (L.tc_slots slots of npad * 128
+// floats).
+cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, float* ws, cudaStream_t st);
+// The GEMM's (128-row tile, 256-column block) units, its grid, and its
+// segment table (slot of each CTA's first segment, grid + 1 entries; slot of
+// each tile's first segment, tiles + 1 entries).
+int tc_units(const Layer& L);
+int tc_grid(const Layer& L);
+void tc_segments(const Layer& L, std::vector<int>& cta_seg, std::vector<int>& tile_seg);
 // Preload (preload_kernel) every kernel a handle can launch: decode-GEMV
 // (both input-transform variants) and qlinear_decode (gemv.cu), the transform
 // kernels (rht.cu), the tensor-core GEMM (gemm_tc.cu).

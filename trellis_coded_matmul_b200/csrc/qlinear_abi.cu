@@ -5,11 +5,11 @@
 #include <algorithm>
 #include <array>
 #include <cmath>
-#include <vector>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "codes.cuh"
 #include "encode.h"
@@ -80,6 +80,8 @@ void free_layer(Layer& L) {
     cudaFree(L.xp);
     cudaFree(L.acc);
     cudaFree(L.host_stage);
+    cudaFree(L.tc_seg);
+    cudaFree(L.tcws);
     std::memset(&L, 0, sizeof(L));
 }
 
@@ -205,6 +207,9 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (rc == QL_OK) rc = dev_alloc(&Ly.sout_bits, (size_t)((m + 31) / 32) * 4);
     if (rc == QL_OK) rc = dev_alloc(&Ly.status, sizeof(int));
     if (rc == QL_OK && uses_table(Ly.code)) rc = dev_alloc(&Ly.lut, ((size_t)1 << Ly.Q) * 4);
+    std::vector<int> cta_seg, tile_seg;
+    tc_segments(Ly, cta_seg, tile_seg);
+    if (rc == QL_OK) rc = dev_alloc(&Ly.tc_seg, (cta_seg.size() + tile_seg.size()) * sizeof(int));
     if (rc != QL_OK) {
         free_layer(Ly);
         delete h;
@@ -217,6 +222,13 @@ int create_common(qlinear_t* out, int m, int n, int nparts, const int* part_rows
     if (e == cudaSuccess) e = launch_pack_signs(s_in, n, Ly.sin_bits, Ly.status, st);
     if (e == cudaSuccess) e = launch_pack_signs(s_out, m, Ly.sout_bits, Ly.status, st);
     if (e == cudaSuccess && uses_table(Ly.code)) e = copy_code_table(code, Ly.Q, V, Ly.lut, st);
+    Ly.tc_tile_seg = Ly.tc_seg + cta_seg.size();
+    Ly.tc_slots = cta_seg.back();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(Ly.tc_seg, cta_seg.data(), cta_seg.size() * sizeof(int), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(Ly.tc_seg + cta_seg.size(), tile_seg.data(), tile_seg.size() * sizeof(int),
+                       cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     int status = 0;
     if (e == cudaSuccess) e = cudaMemcpy(&status, Ly.status, sizeof(int), cudaMemcpyDeviceToHost);
@@ -275,10 +287,10 @@ size_t ticket_bytes(const Layer& L) { return ((size_t)(L.m / L.B_m) * 4 + 255) /
 int* tickets_of(void* acc) { return (int*)acc; }
 float* z_of(const Layer& L, void* acc) { return (float*)((char*)acc + ticket_bytes(L)); }
 
-// The accumulator (tickets and z) is all-zero between forwards: it is zeroed
-// when allocated, and the kernel that consumes z re-zeroes it (the
-// decode-GEMV's output transform, or the output-transform kernel after the
-// tensor-core GEMM, which adds into z and needs the same invariant).
+// The decode-GEMV's accumulator (tickets and z) is all-zero between forwards:
+// it is zeroed when allocated, and the kernel that consumes z re-zeroes it
+// (the decode-GEMV's output-transform epilogue or the output-transform
+// kernel after it).
 int prepare_acc(Layer& L, size_t z_bytes, cudaStream_t st) {
     const size_t bytes = ticket_bytes(L) + z_bytes;
     if (L.acc_bytes >= bytes && !L.acc_dirty) return QL_OK;
@@ -319,15 +331,16 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
     return QL_OK;
 }
 
-// batch > 8: input transform into tensor-core operand tiles, tcgen05 GEMM,
-// output transform; batches above 256 run in passes of 256.
+// batch > 8: input transform into tensor-core operand tiles, tcgen05 GEMM
+// into the partial-sum workspace, output transform summing a tile's partials;
+// batches above 256 run in passes of 256.
 int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
     const int chunk = batch < kTcMaxN ? batch : kTcMaxN;
     const int npad_max = (chunk + 15) / 16 * 16;
     int rc = ensure(&L.xp, &L.xp_bytes, (size_t)npad_max * L.n * 2);
-    if (rc == QL_OK) rc = prepare_acc(L, (size_t)chunk * L.m * 4, st);
+    if (rc == QL_OK) rc = ensure(&L.tcws, &L.tcws_bytes, (size_t)L.tc_slots * npad_max * 128 * 4);
     if (rc != QL_OK) return rc;
-    float* z = z_of(L, L.acc);
+    float* ws = (float*)L.tcws;
     const size_t ysz = y_dtype == QL_F16 ? 2 : 4;
     L.last_launches = 3 * ((batch + kTcMaxN - 1) / kTcMaxN);
     for (int b0 = 0; b0 < batch; b0 += kTcMaxN) {
@@ -338,16 +351,15 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
         cudaError_t e = launch_rht_in_umma(L, xb, nb, npad, L.xp, st);
         const int slot = L.prof_cap ? L.prof_next : -1;
         if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-        if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, z, st);
+        if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, ws, st);
         if (e == cudaSuccess && slot >= 0) {
             e = record_event(L.prof_ev[2 * slot + 1], st);
             L.prof_next = (L.prof_next + 1) % L.prof_cap;
             if (L.prof_count < L.prof_cap) ++L.prof_count;
         }
-        if (e == cudaSuccess) e = launch_rht_out(L, z, nb, yb, y_dtype, st);
+        if (e == cudaSuccess) e = launch_rht_out_tc(L, ws, nb, npad, yb, y_dtype, st);
         if (e != cudaSuccess) {
             cudaGetLastError();
-            L.acc_dirty = 1;
             return QL_E_CUDA;
         }
     }
@@ -589,7 +601,7 @@ int qlinear_info(qlinear_t h, ql_info_t* info) {
     info->stream_bytes = words * 4;
     info->sign_bytes = (size_t)((L.n + 31) / 32 + (L.m + 31) / 32) * 4;
     info->lut_bytes = uses_table(L.code) ? ((size_t)1 << L.Q) * L.V * 2 : 0;
-    info->scratch_bytes = L.xp_bytes + L.acc_bytes + L.host_stage_bytes;
+    info->scratch_bytes = L.xp_bytes + L.acc_bytes + L.host_stage_bytes + L.tcws_bytes;
     info->last_launches = L.last_launches;
     info->nparts = L.nparts;
     for (int i = 0; i < L.nparts; ++i) {

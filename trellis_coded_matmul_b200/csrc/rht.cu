@@ -279,6 +279,146 @@ cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_d
                : launch_rht_out_e<false, 8>(L, z, batch, y, st, zscale);
 }
 
+// Where the tensor-core GEMM's partial sums of a layer row live: row r of
+// part p (rows row0[p] ..) is row (r - row0[p]) % 128 of the part's tile
+// (r - row0[p]) / 128, which is global tile tile0[p] + that.
+struct TcRowMap {
+    int nparts;
+    int row0[kMaxParts];
+    int tile0[kMaxParts];
+};
+
+// y = alpha s_out (H_m z) with z read as the sum of each tile's segment slots
+// of the GEMM's workspace (ws[slot][b][row in tile], npad columns per slot).
+// The same groups and butterflies as rht_out_kernel; four rows (one float4 of
+// every slot) are looked up at a time: a part's rows come in multiples of 16,
+// so four aligned rows never straddle a tile.
+template <bool F16, int E>
+__global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_out_tc_kernel(const float* __restrict__ ws, int npad,
+                                                                          int m, RhtGeometry geo, TcRowMap map,
+                                                                          const int* __restrict__ tile_seg,
+                                                                          const uint32_t* __restrict__ sout_bits,
+                                                                          float alpha, void* __restrict__ y) {
+    extern __shared__ float smem[];
+    const int B = geo.B;
+    const int grp = threadIdx.x / geo.tpg, tid = threadIdx.x % geo.tpg;
+    const int item = blockIdx.x * geo.groups + grp;
+    const bool active = item < geo.total;
+    float* buf = smem + (size_t)grp * (B + B / 16);
+    const int b = active ? item / geo.per_row : 0;
+    const int row = (active ? (item % geo.per_row) * B : 0) + tid * E;
+    // the sign bits and the segment table are written once at create time: read before the wait
+    const uint32_t sw = active ? sout_bits[row >> 5] >> (row & 31) : 0u;
+    int off[E / 4], s0[E / 4], s1[E / 4];
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+        const int r = row + 4 * q;
+        int pi = 0;
+        while (pi + 1 < map.nparts && r >= map.row0[pi + 1]) ++pi;
+        const int rr = r - map.row0[pi];
+        const int gt = map.tile0[pi] + (rr >> 7);
+        off[q] = b * 128 + (rr & 127);
+        s0[q] = active ? tile_seg[gt] : 0;
+        s1[q] = active ? tile_seg[gt + 1] : 0;
+    }
+    const float scale = alpha * rsqrtf((float)B);
+    grid_dependency_wait();
+    // A tile has one to three segments unless the layer has fewer units than
+    // the GEMM has CTAs.  E = 8: the first three slots of every float4 are
+    // loaded at once (all loads in flight), further slots one by one; larger E
+    // (64 registers a thread) take one slot of every float4 at a time.
+    constexpr int kFirst = E == 8 ? 3 : 1;
+    const size_t slot_stride = (size_t)npad * 128;
+    float v[E];
+    float4 t[E / 4][kFirst];
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+#pragma unroll
+        for (int k = 0; k < kFirst; ++k)
+            t[q][k] = s0[q] + k < s1[q] ? __ldcs(reinterpret_cast<const float4*>(ws + (s0[q] + k) * slot_stride + off[q]))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+        float4 acc = t[q][0];
+#pragma unroll
+        for (int k = 1; k < kFirst; ++k) {
+            acc.x += t[q][k].x;
+            acc.y += t[q][k].y;
+            acc.z += t[q][k].z;
+            acc.w += t[q][k].w;
+        }
+        for (int sl = s0[q] + kFirst; sl < s1[q]; ++sl) {
+            const float4 u = __ldcs(reinterpret_cast<const float4*>(ws + sl * slot_stride + off[q]));
+            acc.x += u.x;
+            acc.y += u.y;
+            acc.z += u.z;
+            acc.w += u.w;
+        }
+        v[4 * q] = acc.x;
+        v[4 * q + 1] = acc.y;
+        v[4 * q + 2] = acc.z;
+        v[4 * q + 3] = acc.w;
+    }
+    fwht_block<E>(v, B, tid, geo.tpg, buf);
+    grid_launch_dependents();
+    if (!active) return;
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = ((sw >> q) & 1u) ? -v[q] * scale : v[q] * scale;
+    if (F16) {
+        __half* ys = (__half*)y + (size_t)b * m + row;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) {
+            const __half2 lo = __floats2half2_rn(v[q], v[q + 1]);
+            const __half2 hi = __floats2half2_rn(v[q + 2], v[q + 3]);
+            uint2 w;
+            w.x = *reinterpret_cast<const uint32_t*>(&lo);
+            w.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(ys + q) = w;
+        }
+    } else {
+        float* ys = (float*)y + (size_t)b * m + row;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) *reinterpret_cast<float4*>(ys + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+    }
+}
+
+static TcRowMap tc_row_map(const Layer& L) {
+    TcRowMap map = {};
+    map.nparts = L.nparts;
+    int tiles = 0;
+    for (int i = 0; i < L.nparts; ++i) {
+        map.row0[i] = L.parts[i].row0;
+        map.tile0[i] = tiles;
+        tiles += (L.parts[i].rows + 127) / 128;
+    }
+    return map;
+}
+
+template <bool F16, int E>
+static cudaError_t launch_rht_out_tc_e(const Layer& L, const float* ws, int batch, int npad, void* y, cudaStream_t st) {
+    const RhtGeometry geo = rht_geometry(L.m, L.B_m, batch, E);
+    const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
+    cudaError_t e = ensure_smem_limit<rht_out_tc_kernel<F16, E>>((kMaxHadamard + kMaxHadamard / 16) * 4);
+    if (e != cudaSuccess) return e;
+    const int grid = (geo.total + geo.groups - 1) / geo.groups;
+    return launch_pdl(rht_out_tc_kernel<F16, E>, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, ws, npad, L.m, geo,
+                      tc_row_map(L), L.tc_tile_seg, (const uint32_t*)L.sout_bits, L.alpha, y);
+}
+
+cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int npad, void* y, int y_dtype,
+                              cudaStream_t st) {
+    const bool f16 = y_dtype == QL_F16;
+    if (L.B_m > 16384)
+        return f16 ? launch_rht_out_tc_e<true, 32>(L, ws, batch, npad, y, st)
+                   : launch_rht_out_tc_e<false, 32>(L, ws, batch, npad, y, st);
+    if (L.B_m > 4096)
+        return f16 ? launch_rht_out_tc_e<true, 16>(L, ws, batch, npad, y, st)
+                   : launch_rht_out_tc_e<false, 16>(L, ws, batch, npad, y, st);
+    return f16 ? launch_rht_out_tc_e<true, 8>(L, ws, batch, npad, y, st)
+               : launch_rht_out_tc_e<false, 8>(L, ws, batch, npad, y, st);
+}
+
 template <int MODE>
 static cudaError_t prepare_rht_in(const Layer& L) {
     const int limit = (kMaxHadamard + kMaxHadamard / 16) * 4;
@@ -288,9 +428,14 @@ static cudaError_t prepare_rht_in(const Layer& L) {
 template <bool F16>
 static cudaError_t prepare_rht_out(const Layer& L) {
     const int limit = (kMaxHadamard + kMaxHadamard / 16) * 4;
-    if (L.B_m > 16384) return preload_kernel<rht_out_kernel<F16, 32>>(limit);
+    if (L.B_m > 16384) {
+        cudaError_t e = preload_kernel<rht_out_kernel<F16, 32>>(limit);
+        return e == cudaSuccess ? preload_kernel<rht_out_tc_kernel<F16, 32>>(limit) : e;
+    }
     cudaError_t e = preload_kernel<rht_out_kernel<F16, 16>>(limit);
     if (e == cudaSuccess && L.B_m <= 4096) e = preload_kernel<rht_out_kernel<F16, 8>>(limit);
+    if (e == cudaSuccess) e = L.B_m > 4096 ? preload_kernel<rht_out_tc_kernel<F16, 16>>(limit)
+                                           : preload_kernel<rht_out_tc_kernel<F16, 8>>(limit);
     return e;
 }
 
