@@ -313,6 +313,21 @@ int qlinear_info(qlinear_t h, ql_info_t* info);
  * Errors: QL_E_ARG (capacity < 0 or > 65536), QL_E_CUDA. */
 int qlinear_profile_enable(qlinear_t h, int capacity);
 
+/* Timing: launch the forward's dominant kernel alone (the decode-GEMV for
+ * batch <= 8, the tensor-core GEMM for the first 256 rows of a larger batch)
+ * on `stream`, on the operands the handle's most recent forward left in its
+ * scratch: that forward must have had this batch.  The kernel does exactly
+ * the work it does inside a forward (same launch configuration, same code
+ * words and x'), so back-to-back launches time it apart from the transforms
+ * around it.  Its output is not a result: the decode-GEMV's fp32 sums stay in
+ * the handle's accumulator (the next forward re-zeroes it first), and where
+ * the decode-GEMV transforms its own output (batch * B_m <= 256) it writes y
+ * (fp32 or fp16 [batch][m], y_dtype as in qlinear_forward); y is not used
+ * otherwise and may then be null.  Works inside CUDA graph capture.
+ * Errors: QL_E_ARG (batch < 1, a different batch than the last forward, no
+ * forward yet, bad y_dtype, y null when written), QL_E_CUDA. */
+int qlinear_launch_main_kernel(qlinear_t h, int batch, void* y, int y_dtype, void* stream);
+
 /* Synchronise the device and report the summed elapsed time of the recorded
  * slots (each slot counted once, with its most recent record) and how many
  * slots hold a record.  Slots keep their records; graph replays overwrite

@@ -485,10 +485,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
             if (!wait_bar(acc_full, seg & 1, abort_flag, p.status, p.wait_tries)) break;
             tc_fence_after();
             float* dst = ws + (size_t)seg * p.npad * kTcRows;
+            // (the epilogue warps share their sub-partitions with issue-bound
+            // decoders: a full chunk is 16 plain stores at immediate offsets)
             auto store16 = [&](const uint32_t (&v)[16], int c0) {
+                float* d = dst + (size_t)c0 * kTcRows;
+                if (c0 + 16 <= p.batch) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    if (c0 + e < p.batch) dst[(size_t)(c0 + e) * kTcRows] = __uint_as_float(v[e]);
+                    for (int e = 0; e < 16; ++e) d[e * kTcRows] = __uint_as_float(v[e]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e < p.batch) d[e * kTcRows] = __uint_as_float(v[e]);
+                }
             };
             // two register sets: the next chunk's load is in flight while this one is stored
             uint32_t va[16], vb[16];
@@ -526,13 +534,23 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaS
     return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, a);
 }
 
-// Ring depths: the most stage slots (up to kTcMaxStages), then the deepest
-// code ring (up to kTcMaxCodeSlots blocks) that fit in shared memory.
+// Ring depths: a code ring of kTcMaxCodeSlots blocks (the code words come
+// from HBM: a deep ring hides their latency) with as many stage slots as
+// fit, if that leaves at least 4; else the most stage slots, then the deepest
+// code ring that fit in shared memory.
 size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
     int k2max = 0;
     for (int i = 0; i < L.nparts; ++i) k2max = L.parts[i].k2 > k2max ? L.parts[i].k2 : k2max;
     const int code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
     const int lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
+    for (int s = kTcMaxStages; s >= 4; --s) {
+        const TcSmem lay = tc_smem_layout(s, kTcMaxCodeSlots, npad, code_slot_words, lut_entries);
+        if (lay.total + 1024 <= kTcMaxSmem) {
+            *stages = s;
+            *code_slots = kTcMaxCodeSlots;
+            return (size_t)lay.total + 1024;
+        }
+    }
     for (int s = kTcMaxStages; s >= 2; --s) {
         for (int c = kTcMaxCodeSlots; c >= 2; --c) {
             const TcSmem lay = tc_smem_layout(s, c, npad, code_slot_words, lut_entries);

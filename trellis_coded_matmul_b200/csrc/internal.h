@@ -64,6 +64,7 @@ struct Layer {
     size_t acc_bytes;
     int acc_dirty;        // z or a ticket may be non-zero (a forward failed part-way)
     int last_launches;    // kernels launched by the most recent forward
+    int last_batch;       // batch of the most recent successful forward (0: none)
     void* host_stage;     // device staging for qlinear_forward_host (x then y)
     size_t host_stage_bytes;
     // tensor-core GEMM (batch > 8): its stream-K segment table (device, written at

@@ -367,7 +367,32 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
 }
 
 int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
-    return batch <= kGemvMaxBatch ? forward_gemv(L, x, batch, y, y_dtype, st) : forward_tc(L, x, batch, y, y_dtype, st);
+    const int rc = batch <= kGemvMaxBatch ? forward_gemv(L, x, batch, y, y_dtype, st)
+                                          : forward_tc(L, x, batch, y, y_dtype, st);
+    L.last_batch = rc == QL_OK ? batch : 0;
+    return rc;
+}
+
+// The dominant kernel of a forward with this batch alone, on the scratch the
+// last forward (same batch) left: qlinear_launch_main_kernel.
+int launch_main(Layer& L, int batch, void* y, int y_dtype, cudaStream_t st) {
+    cudaError_t e;
+    if (batch <= kGemvMaxBatch) {
+        const GemvPlan pl = plan_gemv(L, batch);
+        if (pl.fuse_out && !y) return QL_E_ARG;
+        e = launch_gemv(L, pl, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
+        if (!pl.fuse_out) L.acc_dirty = 1;  // the sums stay in z
+    } else {
+        const int nb = batch < kTcMaxN ? batch : kTcMaxN;
+        e = launch_gemm_tc(L, L.xp, nb, (nb + 15) / 16 * 16, (float*)L.tcws, st);
+    }
+    L.last_launches = 1;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        L.acc_dirty = 1;
+        return QL_E_CUDA;
+    }
+    return QL_OK;
 }
 
 }  // namespace
@@ -428,6 +453,14 @@ int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype,
     DeviceGuard g(h->L.device);
     if (!g.ok) return QL_E_CUDA;
     return forward_device(h->L, x, batch, y, y_dtype, (cudaStream_t)stream);
+}
+
+int qlinear_launch_main_kernel(qlinear_t h, int batch, void* y, int y_dtype, void* stream) {
+    if (!h || batch < 1 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
+    if (h->L.last_batch != batch) return QL_E_ARG;
+    DeviceGuard g(h->L.device);
+    if (!g.ok) return QL_E_CUDA;
+    return launch_main(h->L, batch, y, y_dtype, (cudaStream_t)stream);
 }
 
 int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype, void* stream) {
