@@ -496,7 +496,7 @@ class Runner:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.stream):
             for i in range(self.n_inst):
-                tcm.qlinear_launch_main_kernel(self.handles[i], self.batch, self.ys[i], stream=self.stream)
+                tcm.qlinear_launch_main_kernel(self.handles[i], self.batch, self.xs[i], self.ys[i], stream=self.stream)
         self.graphs.append(g)
         reps = max(2, -(-steps // self.n_inst))
         with torch.cuda.stream(self.stream):

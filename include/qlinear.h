@@ -316,7 +316,9 @@ int qlinear_profile_enable(qlinear_t h, int capacity);
 /* Timing: launch the forward's dominant kernel alone (the decode-GEMV for
  * batch <= 8, the tensor-core GEMM for the first 256 rows of a larger batch)
  * on `stream`, on the operands the handle's most recent forward left in its
- * scratch: that forward must have had this batch.  The kernel does exactly
+ * scratch: that forward must have had this batch.  x (device, fp16
+ * [batch][n], as in qlinear_forward) is read where the decode-GEMV computes
+ * x' itself (batch <= 2 with x' of at most 48 KB); it may be null otherwise.  The kernel does exactly
  * the work it does inside a forward (same launch configuration, same code
  * words and x'), so back-to-back launches time it apart from the transforms
  * around it.  Its output is not a result: the decode-GEMV's fp32 sums stay in
@@ -326,7 +328,7 @@ int qlinear_profile_enable(qlinear_t h, int capacity);
  * otherwise and may then be null.  Works inside CUDA graph capture.
  * Errors: QL_E_ARG (batch < 1, a different batch than the last forward, no
  * forward yet, bad y_dtype, y null when written), QL_E_CUDA. */
-int qlinear_launch_main_kernel(qlinear_t h, int batch, void* y, int y_dtype, void* stream);
+int qlinear_launch_main_kernel(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream);
 
 /* Synchronise the device and report the summed elapsed time of the recorded
  * slots (each slot counted once, with its most recent record) and how many

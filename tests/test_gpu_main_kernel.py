@@ -19,10 +19,10 @@ def test_main_kernel_alone_then_forward_is_unchanged(name, batch):
     x = torch.from_numpy(wl.make_x(sp, batch)).cuda()
     y0 = tcm.qlinear_forward(h, x)
     with pytest.raises(tcm.QLinearError):
-        tcm.qlinear_launch_main_kernel(h, batch + 1)  # not the last forward's batch
+        tcm.qlinear_launch_main_kernel(h, batch + 1, None)  # not the last forward's batch
     y = torch.empty_like(y0)
     for _ in range(3):
-        tcm.qlinear_launch_main_kernel(h, batch, y)
+        tcm.qlinear_launch_main_kernel(h, batch, x, y)
     torch.cuda.synchronize()
     assert tcm.qlinear_info(h)["last_launches"] == 1
     y1 = tcm.qlinear_forward(h, x)
@@ -36,4 +36,4 @@ def test_main_kernel_needs_a_forward_first():
     sp = wl.WORKLOADS["tiny"]
     h = make_handle(wl.make_layer(sp))
     with pytest.raises(tcm.QLinearError):
-        tcm.qlinear_launch_main_kernel(h, 1)
+        tcm.qlinear_launch_main_kernel(h, 1, None)

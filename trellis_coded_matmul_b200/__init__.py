@@ -69,7 +69,7 @@ _lib.qlinear_create_kv.argtypes = [ctypes.POINTER(_vp), _i, _i, _i, ctypes.POINT
 _lib.qlinear_forward.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_host.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_forward_noalloc.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
-_lib.qlinear_launch_main_kernel.argtypes = [_vp, _i, _vp, _i, _vp]
+_lib.qlinear_launch_main_kernel.argtypes = [_vp, _vp, _i, _vp, _i, _vp]
 _lib.qlinear_encode.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp]
 _lib.qlinear_encode_kv.argtypes = [ql_code_t, _i, _i, _i, _vp, _i, _vp, _vp, _vp]
 _lib.qlinear_decode.argtypes = [_vp, _vp, _vp]
@@ -230,19 +230,26 @@ def qlinear_forward(h: QLinearHandle, x, y=None, out_dtype=None, stream=None):
     return y
 
 
-def qlinear_launch_main_kernel(h: QLinearHandle, batch: int, y=None, stream=None) -> None:
+def qlinear_launch_main_kernel(h: QLinearHandle, batch: int, x=None, y=None, stream=None) -> None:
     """Launch the dominant kernel of a forward with this batch alone, on the
     scratch the handle's last forward (same batch) left (for timing; see the
-    C header).  y: CUDA fp32/fp16 [batch, m], written only where the
-    decode-GEMV transforms its own output."""
+    C header).  x: the forward's CUDA fp16 [batch, n] input, read where the
+    decode-GEMV computes x' itself.  y: CUDA fp32/fp16 [batch, m], written
+    only where the decode-GEMV transforms its own output."""
     import torch
+    xp = None
+    if x is not None:
+        _cuda(x, "x", torch.float16)
+        if tuple(x.shape) != (batch, h.n):
+            raise ValueError("x must be [batch, n]")
+        xp = _ptr(x)
     yp, ydt = None, QL_F32
     if y is not None:
         _cuda(y, "y", (torch.float32, torch.float16))
         if tuple(y.shape) != (batch, h.m):
             raise ValueError("y must be [batch, m]")
         yp, ydt = _ptr(y), (QL_F16 if y.dtype == torch.float16 else QL_F32)
-    _check(_lib.qlinear_launch_main_kernel(h.ptr, batch, yp, ydt, _stream(stream)), "qlinear_launch_main_kernel")
+    _check(_lib.qlinear_launch_main_kernel(h.ptr, xp, batch, yp, ydt, _stream(stream)), "qlinear_launch_main_kernel")
 
 
 def qlinear_forward_host(h: QLinearHandle, x, y=None, out_dtype=None, stream=None):

@@ -228,8 +228,8 @@ struct StepMMAs {
             }
             uint4 b0 = make_uint4(0u, 0u, 0u, 0u), b1 = b0;
             if (use_x) {
-                b0 = __ldg(xsrc + (u >> 1) * xstride);
-                if (kQuad) b1 = __ldg(xsrc + ((u + MP) >> 1) * xstride);
+                b0 = xsrc[(u >> 1) * xstride];
+                if (kQuad) b1 = xsrc[((u + MP) >> 1) * xstride];
             }
             // two accumulators: two dependent MMA chains of half the length
             mma_step<CODE>(acc[0], pre[0], aux[0], b0.x, b0.y);
@@ -259,7 +259,7 @@ struct StepMMAs<kCodeE8P, K2, 8, L16> {
             e8p_pairs((t & 1) ? (w0 & 0xFFFFu) : (w0 >> 16), lut_lane, p0);
             e8p_pairs((t & 1) ? (w1 & 0xFFFFu) : (w1 >> 16), lut_lane, p1);
             uint4 b = make_uint4(0u, 0u, 0u, 0u);
-            if (use_x) b = __ldg(xsrc + t * xstride);
+            if (use_x) b = xsrc[t * xstride];
             const uint32_t a0[4] = {p0[0], p1[0], p0[1], p1[1]};
             const uint32_t a1[4] = {p0[2], p1[2], p0[3], p1[3]};
             mma_16816(acc[0], a0, b.x, b.y);
@@ -286,7 +286,12 @@ struct GemvArgs {
     int lut_entries;
     int batch;              // 1..8
     int m, n;
-    const uint4* xstep;     // x' step words from the input-transform kernel
+    const uint4* xstep;     // x' step words from the input-transform kernel (x_e == 0)
+    const __half* x;        // x_e > 0: the input, transformed by every CTA into shared memory
+    const uint32_t* sin_bits;
+    int B_n;
+    int x_e;                // entries per thread of that transform (8 or 16), 0: x' from xstep
+    int xs_word0;           // first shared-memory word of x' (after the code table)
     float* z;               // [batch][m], all-zero on entry and on exit
     int* tickets;           // [m / B_m], all-zero on entry and on exit
     int B_m;
@@ -491,6 +496,15 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) trellis_gemv_kernel(Gem
     grid_launch_dependents();
 
     const uint4* xbase = p.xstep;
+    if (p.x_e) {  // x' of the whole batch in shared memory, computed by this CTA (x was just written)
+        uint32_t* xs = smem + p.xs_word0;
+        float* scratch = reinterpret_cast<float*>(xs + (size_t)batch * p.n / VX);
+        if (p.x_e == 8)
+            xstep_transform_cta<VX, 8>(p.x, p.n, p.B_n, p.sin_bits, batch, xs, scratch);
+        else
+            xstep_transform_cta<VX, 16>(p.x, p.n, p.B_n, p.sin_bits, batch, xs, scratch);
+        xbase = reinterpret_cast<const uint4*>(xs);
+    }
     const int xstride = batch * 4;  // uint4 groups between consecutive u2
     const bool use_x = g < batch;
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -561,7 +575,30 @@ GemvPlan plan_gemv(const Layer& L, int batch) {
     if (rows > batch) rows = batch;
     if (rows < 1) rows = 1;
     const long long epi_words = pl.fuse_out ? rows * row_words + sign_words : 0;
-    pl.smem_bytes = (int)((lut_words > epi_words ? lut_words : epi_words) * 4);
+    // the input transform in-kernel for the smallest batches: every CTA computes
+    // all of x' into shared memory (groups of T = B_n / E threads, E = 8 or 16,
+    // T a power of two within the CTA), in place of a kernel and its boundary
+    pl.x_e = 0;
+    pl.xs_word0 = (int)lut_words;
+    long long main_words = lut_words;
+    int tmax = 32;
+    while (tmax * 2 <= pl.threads) tmax *= 2;
+    const int e = L.B_n / tmax < 8 ? 8 : L.B_n / tmax;
+    const int T = L.B_n / e;
+    const long long items = (long long)batch * (L.n / L.B_n);
+    // measured: a transform of more than one block per group (rounds of loads
+    // and barriers), or of blocks above 4096 entries, costs more in-kernel than
+    // the input-transform kernel and its launch boundary
+    const bool one_round = items <= pl.threads / T;
+    if (batch <= kXInKernelMaxBatch && (e == 8 || e == 16) && T <= pl.threads && L.B_n <= 4096 && one_round) {
+        const long long xs_words = (long long)batch * L.n / (L.V == 1 ? 1 : 2);
+        const long long scratch = T > 32 ? (long long)(pl.threads / T) * (L.B_n + L.B_n / 16) : 0;
+        if (xs_words * 4 <= kXInKernelMaxBytes && lut_words + xs_words + scratch <= budget) {
+            pl.x_e = e;
+            main_words = lut_words + xs_words + scratch;
+        }
+    }
+    pl.smem_bytes = (int)((main_words > epi_words ? main_words : epi_words) * 4);
     return pl;
 }
 
@@ -894,8 +931,8 @@ cudaError_t launch_eval_code(int code, int L, int V, int Q, const uint32_t* lut_
 }
 
 
-cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, int batch, float* z, int* tickets,
-                        void* y, int y_dtype, cudaStream_t st) {
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
+                        int* tickets, void* y, int y_dtype, cudaStream_t st) {
     GemvArgs a;
     a.nparts = L.nparts;
     a.nb = L.n / kT;
@@ -916,6 +953,11 @@ cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, i
     a.m = L.m;
     a.n = L.n;
     a.xstep = (const uint4*)xstep;
+    a.x = (const __half*)x;
+    a.sin_bits = L.sin_bits;
+    a.B_n = L.B_n;
+    a.x_e = pl.x_e;
+    a.xs_word0 = pl.xs_word0;
     a.z = z;
     a.tickets = tickets;
     a.B_m = L.B_m;

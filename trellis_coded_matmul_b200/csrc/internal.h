@@ -18,6 +18,8 @@ constexpr int kMaxHadamard = 32768;
 constexpr int kGemvMaxWarps = 16;        // decode-GEMV: warps of its one CTA per SM (<= 128 registers/thread)
 constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
 constexpr int kFuseOutElems = 256;  // batch * B_m up to which the GEMV's last CTA per block does the output transform
+constexpr int kXInKernelMaxBatch = 2;          // batches up to which every GEMV CTA computes x' itself
+constexpr int kXInKernelMaxBytes = 48 * 1024;  // and x' fits in this much shared memory
 constexpr int kMaxParts = 8;          // row parts of one layer (layers fused along m, own bitwidth each)
 constexpr int kGemvMaxBatch = 8;      // larger batches use the tensor-core GEMM
 constexpr int kTcMaxN = 256;          // tensor-core GEMM: batch columns per pass
@@ -166,6 +168,8 @@ cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int np
 struct GemvPlan {
     int grid, threads;
     bool fuse_out;  // output transform in the GEMV's epilogue (else launch_rht_out after it)
+    int x_e;        // > 0: every CTA computes x' from x into shared memory (E entries a thread), no input-transform kernel
+    int xs_word0;   // first shared-memory word of that x'
     int smem_bytes;
 };
 GemvPlan plan_gemv(const Layer& L, int batch);
@@ -174,13 +178,14 @@ GemvPlan plan_gemv(const Layer& L, int batch);
 size_t gemv_xstep_bytes(const Layer& L, int batch);
 // The factor between the decode-GEMV's z and W_hat x' (the 1MAD code's C1, else 1).
 float gemv_z_scale(const Layer& L);
-// The forward for batch <= 8 after the input-transform kernel: decode-GEMV
-// over all row parts into z, and (pl.fuse_out) the output transform into y
-// (fp32 or fp16) by the CTA that completes each output Hadamard block; else
+// The forward for batch <= 8: decode-GEMV over all row parts into z, x' from
+// x in the kernel itself (pl.x_e > 0) or from xstep (the input-transform
+// kernel's output), and (pl.fuse_out) the output transform into y (fp32 or
+// fp16) by the CTA that completes each output Hadamard block; else
 // launch_rht_out follows.  z ([batch][m] fp32) and tickets ([m / B_m] int)
 // must be all-zero on entry and are all-zero again when the forward is done.
-cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* xstep, int batch, float* z, int* tickets,
-                        void* y, int y_dtype, cudaStream_t st);
+cudaError_t launch_gemv(const Layer& L, const GemvPlan& pl, const void* x, const void* xstep, int batch, float* z,
+                        int* tickets, void* y, int y_dtype, cudaStream_t st);
 cudaError_t launch_decode(const Layer& L, const Part& part, void* w_hat, cudaStream_t st);
 // W_hat x' for all parts, x' in tensor-core tiles with npad (multiple of 16,
 // <= 256) rows, b < batch; the (128-row tile, 256-column block) units are

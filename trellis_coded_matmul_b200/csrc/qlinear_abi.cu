@@ -312,11 +312,11 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
     int rc = ensure(&L.xp, &L.xp_bytes, gemv_xstep_bytes(L, batch));
     if (rc == QL_OK) rc = prepare_acc(L, (size_t)batch * L.m * 4, st);
     if (rc != QL_OK) return rc;
-    L.last_launches = 2 + (pl.fuse_out ? 0 : 1);
-    cudaError_t e = launch_rht_in_xstep(L, x, batch, L.xp, st);
+    L.last_launches = (pl.x_e ? 1 : 2) + (pl.fuse_out ? 0 : 1);
+    cudaError_t e = pl.x_e ? cudaSuccess : launch_rht_in_xstep(L, x, batch, L.xp, st);
     const int slot = L.prof_cap ? L.prof_next : -1;
     if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
-    if (e == cudaSuccess) e = launch_gemv(L, pl, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
+    if (e == cudaSuccess) e = launch_gemv(L, pl, x, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
     if (e == cudaSuccess && slot >= 0) {
         e = record_event(L.prof_ev[2 * slot + 1], st);
         L.prof_next = (L.prof_next + 1) % L.prof_cap;
@@ -375,12 +375,12 @@ int forward_device(Layer& L, const void* x, int batch, void* y, int y_dtype, cud
 
 // The dominant kernel of a forward with this batch alone, on the scratch the
 // last forward (same batch) left: qlinear_launch_main_kernel.
-int launch_main(Layer& L, int batch, void* y, int y_dtype, cudaStream_t st) {
+int launch_main(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
     cudaError_t e;
     if (batch <= kGemvMaxBatch) {
         const GemvPlan pl = plan_gemv(L, batch);
-        if (pl.fuse_out && !y) return QL_E_ARG;
-        e = launch_gemv(L, pl, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
+        if ((pl.fuse_out && !y) || (pl.x_e && !x)) return QL_E_ARG;
+        e = launch_gemv(L, pl, x, L.xp, batch, z_of(L, L.acc), tickets_of(L.acc), y, y_dtype, st);
         if (!pl.fuse_out) L.acc_dirty = 1;  // the sums stay in z
     } else {
         const int nb = batch < kTcMaxN ? batch : kTcMaxN;
@@ -455,12 +455,12 @@ int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype,
     return forward_device(h->L, x, batch, y, y_dtype, (cudaStream_t)stream);
 }
 
-int qlinear_launch_main_kernel(qlinear_t h, int batch, void* y, int y_dtype, void* stream) {
+int qlinear_launch_main_kernel(qlinear_t h, const void* x, int batch, void* y, int y_dtype, void* stream) {
     if (!h || batch < 1 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
     if (h->L.last_batch != batch) return QL_E_ARG;
     DeviceGuard g(h->L.device);
     if (!g.ok) return QL_E_CUDA;
-    return launch_main(h->L, batch, y, y_dtype, (cudaStream_t)stream);
+    return launch_main(h->L, x, batch, y, y_dtype, (cudaStream_t)stream);
 }
 
 int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype, void* stream) {
@@ -781,13 +781,13 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     cudaStream_t st = (cudaStream_t)stream;
     // tickets and z must start at zero; another handle's failed call may have left sums there
     cudaError_t e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
-    if (e == cudaSuccess) e = launch_rht_in_xstep(L, x, batch, xp, st);
-    if (e == cudaSuccess) e = launch_gemv(L, pl, xp, batch, z, tickets, y, y_dtype, st);
+    if (e == cudaSuccess && !pl.x_e) e = launch_rht_in_xstep(L, x, batch, xp, st);
+    if (e == cudaSuccess) e = launch_gemv(L, pl, x, xp, batch, z, tickets, y, y_dtype, st);
     if (e == cudaSuccess && !pl.fuse_out) e = launch_rht_out(L, z, batch, y, y_dtype, st, gemv_z_scale(L));
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    L.last_launches = 2 + (pl.fuse_out ? 0 : 1);
+    L.last_launches = (pl.x_e ? 1 : 2) + (pl.fuse_out ? 0 : 1);
     return QL_OK;
 }

@@ -122,4 +122,62 @@ __device__ __forceinline__ void fwht_blocks_smem(float* buf, int count, int B, L
     }
 }
 
+// x' = H_B (s_in * x) / sqrt(B) of `batch` rows of x (fp16 [batch][n],
+// 16-byte aligned), per block of B consecutive entries, written as step words
+// to `xs` (shared memory, the layout above) by every thread of the CTA.
+// Groups of T = B / E threads (a power of two, at most blockDim.x) take one
+// block each, E consecutive entries a thread: strides below E in registers,
+// then warp shuffles, then `scratch` (floor(blockDim.x / T) * (B + B / 16)
+// floats of shared memory) when T > 32.  All threads of the CTA must call
+// this; it ends with a CTA barrier.
+template <int VX, int E>
+__device__ __forceinline__ void xstep_transform_cta(const __half* __restrict__ x, int n, int B,
+                                                    const uint32_t* __restrict__ sin_bits, int batch, uint32_t* xs,
+                                                    float* scratch) {
+    const int T = B / E;
+    const int G = blockDim.x / T;
+    const int grp = threadIdx.x / T, tid = threadIdx.x % T;
+    const bool member = grp < G;
+    const int per_row = n / B, items = batch * per_row;
+    const float scale = rsqrtf((float)B);
+    auto load = [&](int item, float (&v)[E]) {  // entries tid*E .. +E-1 of item, signs applied (0 past the end)
+        if (!member || item >= items) {
+#pragma unroll
+            for (int q = 0; q < E; ++q) v[q] = 0.f;
+            return;
+        }
+        const int b = item / per_row, col = (item % per_row) * B + tid * E;
+        const uint32_t sw = sin_bits[col >> 5] >> (col & 31);  // E <= 32 consecutive sign bits
+#pragma unroll
+        for (int q = 0; q < E; q += 8) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(x + (size_t)b * n + col + q);
+            const __half* hv = reinterpret_cast<const __half*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float f = __half2float(hv[e]);
+                v[q + e] = ((sw >> (q + e)) & 1u) ? -f : f;
+            }
+        }
+    };
+    auto store = [&](int item, float (&v)[E]) {
+        if (!member || item >= items) return;
+        const int b = item / per_row, col = (item % per_row) * B + tid * E;
+#pragma unroll
+        for (int q = 0; q < E; q += 4) {
+            const float o[4] = {v[q] * scale, v[q + 1] * scale, v[q + 2] * scale, v[q + 3] * scale};
+            store_xstep4<VX>(xs, col + q, b, batch, o);
+        }
+    };
+    float* buf = scratch + (size_t)(member ? grp : 0) * (B + B / 16);
+    for (int i0 = 0; i0 < items; i0 += G) {
+        const int item = i0 + grp;
+        float v[E];
+        load(item, v);
+        fwht_block<E>(v, B, tid, T, buf, member && item < items);
+        store(item, v);
+        if (T > 32) __syncthreads();  // buf is written again by the next round
+    }
+    __syncthreads();
+}
+
 }  // namespace qlk
