@@ -264,8 +264,129 @@ static cudaError_t launch_rht_out_e(const Layer& L, float* z, int batch, void* y
                       (const uint32_t*)L.sout_bits, L.alpha * zscale, y);
 }
 
+// The output transform with T = B / 16 threads per Hadamard block (256 <= B
+// <= 8192, so T <= 512), one CTA per (block, batch row), 16 entries a thread:
+//   1. thread t takes rows t + T q (q < 16) and transforms over q in registers
+//      (the strides T, 2T, 4T, 8T);
+//   2. one transpose through shared memory (one pad word per 16) gives it rows
+//      16 t .. 16 t + 15, transformed in registers (strides 1, 2, 4, 8);
+//   3. the strides 16 .. T / 2 pair threads t and t ^ (stride / 16): warp
+//      shuffles, as T <= 512 keeps them inside a warp (none for T <= 16).
+// SLOTS: z of a row is the sum of the row's tile's segment slots of the
+// tensor-core GEMM's workspace (src = ws, [slot][npad][128]; needs every part's
+// rows to be whole 128-row tiles, so that row r lies in global tile r / 128);
+// else src = z ([batch][m] fp32), re-zeroed after it is read.  All loads of
+// a thread are in flight at once (three slots of every entry; further slots,
+// for layers with fewer units than the GEMM has CTAs, one by one).
+template <bool F16, bool SLOTS>
+__global__ void __launch_bounds__(512) rht_out_lean_kernel(float* __restrict__ src, int npad, int m, int B,
+                                                           const int* __restrict__ tile_seg,
+                                                           const uint32_t* __restrict__ sout_bits, float scale,
+                                                           void* __restrict__ y) {
+    extern __shared__ float buf[];  // B + B / 16 floats
+    const int T = B >> 4, t = threadIdx.x;
+    const int b = blockIdx.y;
+    const int base = blockIdx.x * B;
+    // the sign bits and the segment table are written once at create time: read before the wait
+    const uint32_t sw = sout_bits[(base + 16 * t) >> 5] >> ((base + 16 * t) & 31);
+    grid_dependency_wait();
+    // every load of the 16 entries is issued before any of them is used
+    float v[16];
+    if constexpr (SLOTS) {
+        const size_t stride = (size_t)npad * 128;
+        int s0[16], ns[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int row = base + T * q + t;
+            s0[q] = tile_seg[row >> 7];
+            ns[q] = tile_seg[(row >> 7) + 1] - s0[q];
+        }
+        float a1[16], a2[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float* p = src + ((size_t)s0[q] * npad + b) * 128 + ((base + T * q + t) & 127);
+            v[q] = __ldcs(p);
+            a1[q] = ns[q] > 1 ? __ldcs(p + stride) : 0.f;
+            a2[q] = ns[q] > 2 ? __ldcs(p + 2 * stride) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            v[q] += a1[q] + a2[q];
+            for (int k = 3; k < ns[q]; ++k)  // tiles of more than three segments (layers with few units)
+                v[q] += __ldcs(src + ((size_t)(s0[q] + k) * npad + b) * 128 + ((base + T * q + t) & 127));
+        }
+    } else {
+        float* p = src + (size_t)b * m + base + t;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] = p[T * q];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) p[T * q] = 0.f;
+    }
+    fwht_regs<16>(v);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) buf[pad16(T * q + t)] = v[q];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = buf[pad16(16 * t + j)];
+    fwht_regs<16>(v);
+    const int lane = t & 31;
+    for (int h = 1; h < T / 16; h <<= 1) {  // row stride 16 h (the strides from T on were step 1)
+        const bool upper = lane & h;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[j], h);
+            v[j] = upper ? o - v[j] : v[j] + o;
+        }
+    }
+    grid_launch_dependents();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = ((sw >> j) & 1u) ? -v[j] * scale : v[j] * scale;
+    const size_t o = (size_t)b * m + base + 16 * t;
+    if (F16) {
+        __half* ys = (__half*)y + o;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const __half2 lo = __floats2half2_rn(v[j], v[j + 1]);
+            const __half2 hi = __floats2half2_rn(v[j + 2], v[j + 3]);
+            *reinterpret_cast<uint2*>(ys + j) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        }
+    } else {
+        float* ys = (float*)y + o;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(ys + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+}
+
+// The lean kernel covers 256 <= B_m <= 8192 (and, after the GEMM, layers whose
+// parts are whole 128-row tiles).
+static bool lean_out_ok(const Layer& L) { return L.B_m >= 256 && L.B_m <= 8192; }
+
+static bool tc_tiles_whole(const Layer& L) {
+    for (int i = 0; i < L.nparts; ++i)
+        if (L.parts[i].rows % 128) return false;
+    return true;
+}
+
+template <bool F16, bool SLOTS>
+static cudaError_t launch_rht_out_lean(const Layer& L, float* src, int npad, int batch, void* y, float scale,
+                                       cudaStream_t st) {
+    const dim3 grid(L.m / L.B_m, batch);
+    const size_t smem = (size_t)(L.B_m + L.B_m / 16) * sizeof(float);
+    return launch_pdl(rht_out_lean_kernel<F16, SLOTS>, grid, dim3(L.B_m / 16), smem, st, src, npad, L.m, L.B_m,
+                      L.tc_tile_seg, (const uint32_t*)L.sout_bits, scale, y);
+}
+
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st, float zscale) {
     const bool f16 = y_dtype == QL_F16;
+    // measured on a B200: the lean kernel wins when one or two CTAs do the whole
+    // transform (batch 1 of a layer with one Hadamard block of rows); with more
+    // blocks or batch rows the older kernel's shorter per-thread chains win
+    if (lean_out_ok(L) && (long long)batch * (L.m / L.B_m) <= 2) {
+        const float scale = L.alpha * zscale * rsqrtf((float)L.B_m);
+        return f16 ? launch_rht_out_lean<true, false>(L, z, 0, batch, y, scale, st)
+                   : launch_rht_out_lean<false, false>(L, z, 0, batch, y, scale, st);
+    }
     // Small batches (a few CTAs, latency-bound): 8 entries per thread up to blocks
     // of 4096 (512 threads), shorter chains per thread.  Large batches (many
     // CTAs, bandwidth-bound): 16, fewer and fuller CTAs.
@@ -409,6 +530,14 @@ static cudaError_t launch_rht_out_tc_e(const Layer& L, const float* ws, int batc
 cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int npad, void* y, int y_dtype,
                               cudaStream_t st) {
     const bool f16 = y_dtype == QL_F16;
+    // measured on a B200: the lean kernel wins at the large batches (many CTAs,
+    // throughput-bound: ~107 -> ~30 instructions per output), not at batch 16
+    if (lean_out_ok(L) && tc_tiles_whole(L) && batch >= 32) {
+        const float scale = L.alpha * rsqrtf((float)L.B_m);
+        float* w = const_cast<float*>(ws);  // only read (SLOTS)
+        return f16 ? launch_rht_out_lean<true, true>(L, w, npad, batch, y, scale, st)
+                   : launch_rht_out_lean<false, true>(L, w, npad, batch, y, scale, st);
+    }
     if (L.B_m > 16384)
         return f16 ? launch_rht_out_tc_e<true, 32>(L, ws, batch, npad, y, st)
                    : launch_rht_out_tc_e<false, 32>(L, ws, batch, npad, y, st);
@@ -428,6 +557,11 @@ static cudaError_t prepare_rht_in(const Layer& L) {
 template <bool F16>
 static cudaError_t prepare_rht_out(const Layer& L) {
     const int limit = (kMaxHadamard + kMaxHadamard / 16) * 4;
+    if (lean_out_ok(L)) {
+        cudaError_t e = preload_kernel<rht_out_lean_kernel<F16, false>>(0);
+        if (e == cudaSuccess) e = preload_kernel<rht_out_lean_kernel<F16, true>>(0);
+        if (e != cudaSuccess) return e;
+    }
     if (L.B_m > 16384) {
         cudaError_t e = preload_kernel<rht_out_kernel<F16, 32>>(limit);
         return e == cudaSuccess ? preload_kernel<rht_out_tc_kernel<F16, 32>>(limit) : e;
