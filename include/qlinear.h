@@ -218,10 +218,12 @@ int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_hos
  *   Scratch: the output-block tickets, the fp32 accumulator z and (when the
  *   input transform runs as its own kernel) x' live in one fixed array of
  *   QL_NOALLOC_SCRATCH_BYTES in the library's static device memory, per
- *   device: round_up(4*m/B(m), 256) + round_up(4*batch*m, 256) bytes, plus
- *   x' (4*batch*n bytes at V = 1, 2*batch*n at V = 2 or 8), must fit, else
- *   QL_E_SCRATCH (before any device work).  Every call clears its tickets
- *   and z on `stream` first.
+ *   device: round_up(4*m/B(m), 256) + round_up(4*batch*m, 256) bytes from its
+ *   start, plus x' (4*batch*n bytes at V = 1, 2*batch*n at V = 2 or 8) at its
+ *   end, must fit, else QL_E_SCRATCH (before any device work).  Tickets and z
+ *   are all-zero again after every successful call; a call clears them on
+ *   `stream` first only when an earlier call failed or wrote x' where they
+ *   now lie.
  *   Sharing: all handles on a device share the array, so calls that overlap
  *   in time (different streams or host threads) race and give wrong y; calls
  *   in order on one stream are safe.

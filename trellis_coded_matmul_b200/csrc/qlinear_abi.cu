@@ -737,6 +737,12 @@ namespace {
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_base[kNoAllocMaxDevices];
+// Bytes from the array's start known to be all-zero (tickets and z of every
+// call live there and are all-zero again after a successful call; x' is
+// written at the array's end).  Starts whole: a __device__ array is
+// zero-initialised.
+size_t g_noalloc_clean[kNoAllocMaxDevices];
+bool g_noalloc_clean_set[kNoAllocMaxDevices];
 
 // The array's address on `device` (current on entry).  Looked up once per
 // device, on that device's first call; the lookup may load the library's
@@ -752,8 +758,31 @@ int noalloc_scratch(int device, void** base) {
         }
         g_noalloc_base[device] = p;
     }
+    if (!g_noalloc_clean_set[device]) {
+        g_noalloc_clean[device] = QL_NOALLOC_SCRATCH_BYTES;
+        g_noalloc_clean_set[device] = true;
+    }
     *base = g_noalloc_base[device];
     return QL_OK;
+}
+
+// Before a call whose tickets and z take the first `need` bytes and whose x'
+// takes the last `xp` bytes: whether the first `need` bytes must be zeroed
+// first; records the call's effect on the clean prefix.
+bool noalloc_claim(int device, size_t need, size_t xp) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    size_t& clean = g_noalloc_clean[device];
+    const bool zero = need > clean;
+    if (zero) clean = need;
+    const size_t xp_start = (size_t)QL_NOALLOC_SCRATCH_BYTES - xp;
+    if (xp && xp_start < clean) clean = xp_start;  // not reached: need + xp fits
+    return zero;
+}
+
+// A call failed part-way: sums or counts may be left anywhere.
+void noalloc_taint(int device) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    g_noalloc_clean[device] = 0;
 }
 
 }  // namespace
@@ -764,11 +793,11 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     if (!x || !y) return QL_E_ARG;
     if (batch > kGemvMaxBatch) return QL_E_UNSUPPORTED;
     Layer& L = h->L;
-    // array layout: output-block tickets, z, x'
+    // array layout: output-block tickets and z from the start, x' at the end
     const GemvPlan pl = plan_gemv(L, batch);
     const size_t t_bytes = ticket_bytes(L);
     const size_t z_bytes = ((size_t)batch * L.m * 4 + 255) / 256 * 256;
-    const size_t xp_bytes = gemv_xstep_bytes(L, batch);
+    const size_t xp_bytes = (gemv_xstep_bytes(L, batch) + 255) / 256 * 256;
     if (t_bytes + z_bytes + xp_bytes > (size_t)QL_NOALLOC_SCRATCH_BYTES) return QL_E_SCRATCH;
     DeviceGuard g(L.device);
     if (!g.ok) return QL_E_CUDA;
@@ -777,15 +806,18 @@ extern "C" int qlinear_forward_noalloc(qlinear_t h, const void* x, int batch, vo
     if (rc != QL_OK) return rc;
     int* tickets = (int*)base;
     float* z = (float*)((char*)base + t_bytes);
-    void* xp = (char*)base + t_bytes + z_bytes;
+    void* xp = (char*)base + QL_NOALLOC_SCRATCH_BYTES - xp_bytes;
     cudaStream_t st = (cudaStream_t)stream;
-    // tickets and z must start at zero; another handle's failed call may have left sums there
-    cudaError_t e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
+    // tickets and z must start at zero: they are unless a failed call, or an
+    // earlier call's x', left something there (then they are zeroed first)
+    cudaError_t e = cudaSuccess;
+    if (noalloc_claim(L.device, t_bytes + z_bytes, pl.x_e ? 0 : xp_bytes)) e = cudaMemsetAsync(base, 0, t_bytes + z_bytes, st);
     if (e == cudaSuccess && !pl.x_e) e = launch_rht_in_xstep(L, x, batch, xp, st);
     if (e == cudaSuccess) e = launch_gemv(L, pl, x, xp, batch, z, tickets, y, y_dtype, st);
     if (e == cudaSuccess && !pl.fuse_out) e = launch_rht_out(L, z, batch, y, y_dtype, st, gemv_z_scale(L));
     if (e != cudaSuccess) {
         cudaGetLastError();
+        noalloc_taint(L.device);
         return QL_E_CUDA;
     }
     L.last_launches = (pl.x_e ? 1 : 2) + (pl.fuse_out ? 0 : 1);
