@@ -581,6 +581,12 @@ GemvPlan plan_gemv(const Layer& L, int batch) {
     pl.x_e = 0;
     pl.xs_word0 = (int)lut_words;
     long long main_words = lut_words;
+    // with the whole batch-1 transform in-kernel, as many threads as give it
+    // 8 entries each (shorter chains), when that does not raise the most
+    // units a warp takes
+    if (batch <= kXInKernelMaxBatch && L.B_n / 8 > pl.threads && L.B_n / 8 <= kGemvMaxWarps * 32 &&
+        (per_cta + L.B_n / 256 - 1) / (L.B_n / 256) == per_warp)
+        pl.threads = L.B_n / 8;
     int tmax = 32;
     while (tmax * 2 <= pl.threads) tmax *= 2;
     const int e = L.B_n / tmax < 8 ? 8 : L.B_n / tmax;
