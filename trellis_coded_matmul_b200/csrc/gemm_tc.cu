@@ -67,6 +67,14 @@ constexpr int kWarpEpi0 = 19, kTcEpiWarps = 4;  // warps 19..22: lane quarters 3
 constexpr int kTcMaxStages = 8;      // stage slots (A in tensor memory, x' tile in shared memory)
 constexpr uint32_t kTcTmemCols = 512;  // accumulator [0, 256) and up to 8 A slots of 32 columns
 constexpr uint32_t kTcTmemA = 256;     // first A-slot column
+// Split A words (computed codes at batch <= 128): each weight is one 32-bit
+// word whose two fp16 halves sum to it, and x' sits twice along K, so the MMA
+// does the sum (the decode-GEMV's form): a stage's A slot is 64 columns, from
+// column 128 (the accumulator then has at most 128), and its x' tile is two
+// 128-byte swizzled sub-tiles.
+constexpr uint32_t kTcTmemASplit = 128;
+constexpr int kTcMaxStagesSplit = 6;  // (512 - 128) / 64
+constexpr int kTcMaxSplitN = 128;
 constexpr int kTcMaxCodeSlots = 4;   // code-word blocks in flight
 #ifndef QL_TC_XSPLIT
 #define QL_TC_XSPLIT 1
@@ -280,6 +288,79 @@ __device__ __forceinline__ void decode_stage_tmem(uint32_t code, uint32_t a_tadd
     tmem_st16(a_taddr + 16, out);
 }
 
+// A split word of one state: two fp16 halves whose sum is the code value (for
+// 1MAD the value is 1536 + (byte sum - 510) - 1536, so the sum comes out in
+// units of the 1MAD scale, which the output transform applies).
+template <int CODE>
+__device__ __forceinline__ uint32_t split_word(uint32_t s) {
+    if constexpr (CODE == kCode3INST) {
+        return ((kA3INST * s + kB3INST) & kMask3INST) ^ kXor3INST;
+    } else {
+        static_assert(CODE == kCode1MAD, "split words exist for the computed codes");
+        return __dp4a(kA1MAD * s + kB1MAD, 0x01010101u, 0xE6000000u + kDp4aAcc);
+    }
+}
+
+// decode_stage_tmem with split words: the quarter's 64 weights become 64
+// words, tensor-memory columns a_col .. + 63 of the thread's lane (weight i of
+// the quarter in column i).
+template <int CODE, int K2, bool L16>
+__device__ __forceinline__ void decode_stage_tmem_split(uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
+                                                        uint32_t lmask) {
+    using UL = UnitLayout<K2>;
+    constexpr int kV = K2 / 2;  // V = 1
+    constexpr bool kPair = (16 % kV) == 0;
+    constexpr int P = kPair ? 16 / kV : 1;
+    const int r = 32 * qtr + lane;
+    const int h = (r >> 3) & 1, g = r & 7;
+    const uint32_t unit = code + (r >> 4) * UL::UW * 4;
+    const int own = 4 * g + q;
+    auto addr = [&](int slot_lane, int e) -> uint32_t {
+        return unit + 4 * (((h * UL::NV + e / UL::VW) * 32 + slot_lane) * UL::VW + (e % UL::VW));
+    };
+    uint32_t w[K2 + 1];
+    w[0] = lds32(addr(4 * g + ((q + 3) & 3), K2 - 1));
+#pragma unroll
+    for (int c = 0; c < K2 / UL::VW; ++c) {
+        if (UL::VW == 4)
+            lds128(addr(own, 4 * c), w[1 + 4 * c], w[2 + 4 * c], w[3 + 4 * c], w[4 + 4 * c]);
+        else if (UL::VW == 2)
+            lds64(addr(own, 2 * c), w[1 + 2 * c], w[2 + 2 * c]);
+        else
+            w[1 + c] = lds32(addr(own, c));
+    }
+#pragma unroll
+    for (int hq = 0; hq < 4; ++hq) {  // 16 steps (weights) per tensor-memory store
+        uint32_t out[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const int step = 16 * hq + t;
+            if (kPair) {
+                if (((t / P) & 1) == 0) {
+                    uint32_t s0, s1;
+                    state_pair<kV, L16>(w, step, lmask, s0, s1);
+                    out[t] = split_word<CODE>(s0);
+                    if (t + P < 16) out[t + P] = split_word<CODE>(s1);
+                }
+            } else {
+                out[t] = split_word<CODE>(state_one<kV, L16>(w, step, lmask));
+            }
+        }
+        tmem_st16(a_taddr + 16 * hq, out);
+    }
+}
+
+template <int CODE, bool L16>
+__device__ __forceinline__ void decode_stage_split_k2(int k2, uint32_t code, uint32_t a_taddr, int qtr, int q,
+                                                      int lane, uint32_t lmask) {
+    switch (k2) {
+        case 2: decode_stage_tmem_split<CODE, 2, L16>(code, a_taddr, qtr, q, lane, lmask); break;
+        case 4: decode_stage_tmem_split<CODE, 4, L16>(code, a_taddr, qtr, q, lane, lmask); break;
+        case 6: decode_stage_tmem_split<CODE, 6, L16>(code, a_taddr, qtr, q, lane, lmask); break;
+        default: decode_stage_tmem_split<CODE, 8, L16>(code, a_taddr, qtr, q, lane, lmask); break;
+    }
+}
+
 // The part's bitwidth picks the decoder (V = 1 has whole bitwidths only).
 template <int CODE, int V, bool L16>
 __device__ __forceinline__ void decode_stage_k2(int k2, uint32_t code, uint32_t a_taddr, int qtr, int q, int lane,
@@ -299,13 +380,17 @@ __device__ __forceinline__ void decode_stage_k2(int k2, uint32_t code, uint32_t 
     }
 }
 
-template <int CODE, int V, bool L16>
+template <int CODE, int V, bool L16, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p) {
+    constexpr uint32_t kAcol0 = SPLIT ? kTcTmemASplit : kTcTmemA;  // first A-slot column
+    constexpr uint32_t kAcols = SPLIT ? kTcK : kTcK / 2;            // columns of one A slot
+    constexpr int kMmas = SPLIT ? 2 * kTcK / 16 : kTcK / 16;        // MMAs (K = 16) per stage
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived by indexing the shared array so that
     // accesses through it stay shared-memory accesses
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const TcSmem L = tc_smem_layout(p.stages, p.code_slots, p.npad, p.code_slot_words, p.lut_entries);
+    const int xrows = SPLIT ? 2 * p.npad : p.npad;  // 128-byte x' rows of one stage
+    const TcSmem L = tc_smem_layout(p.stages, p.code_slots, xrows, p.code_slot_words, p.lut_entries);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
     const int S = p.stages, C = p.code_slots;
     const uint32_t bar0 = smem_u32(bars);
@@ -324,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
     const int u1 = (int)((long long)(blockIdx.x + 1) * p.units / gridDim.x);
     const uint32_t b_base = smem_u32(smem + L.b);
     const uint32_t code_base = smem_u32(smem + L.code);
-    const uint32_t b_bytes = (uint32_t)p.npad * 128;
+    const uint32_t b_bytes = (uint32_t)xrows * 128;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C; ++i) {
@@ -425,11 +510,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
                 }
                 tc_fence_after();
                 if (elect_one()) {
-                    const uint32_t a_t = tmem + kTcTmemA + (uint32_t)st * (kTcK / 2);
+                    const uint32_t a_t = tmem + kAcol0 + (uint32_t)st * kAcols;
                     const uint32_t b_lo = b_lo0 + (uint32_t)st * b_step;
+                    // K chunk kk: A columns 8 kk .. + 7; x' sub-tile kk / 4 (npad rows of 128
+                    // bytes, 8 p.npad 16-byte units), 32 bytes per chunk within it
 #pragma unroll
-                    for (int kk = 0; kk < kTcK / 16; ++kk)
-                        tc_mma_f16_ts(tmem, a_t + kk * 8, ((uint64_t)b_hi << 32) | (b_lo + kk * 2), idesc,
+                    for (int kk = 0; kk < kMmas; ++kk)
+                        tc_mma_f16_ts(tmem, a_t + kk * 8,
+                                      ((uint64_t)b_hi << 32) | (b_lo + (kk >> 2) * 8 * p.npad + (kk & 3) * 2), idesc,
                                       (first && q == 0 && kk == 0) ? 0u : 1u);
                     tc_commit(empty(st));
                     if (last && q == 3) tc_commit(acc_full);
@@ -458,8 +546,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
                     tc_fence_after();  // the MMAs that read this A slot have completed
                     // Rows of row tiles beyond a ragged last tile decode whatever the
                     // slot holds; their accumulator rows are never stored.
-                    const uint32_t a_taddr = tmem + lane_base + kTcTmemA + (uint32_t)st * (kTcK / 2);
-                    decode_stage_k2<CODE, V, L16>(pt.k2, code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift);
+                    const uint32_t a_taddr = tmem + lane_base + kAcol0 + (uint32_t)st * kAcols;
+                    if constexpr (SPLIT)
+                        decode_stage_split_k2<CODE, L16>(pt.k2, code, a_taddr, qtr, grp, lane, p.lmask);
+                    else
+                        decode_stage_k2<CODE, V, L16>(pt.k2, code, a_taddr, qtr, grp, lane, p.lmask, lut_lane, p.qshift);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
@@ -527,9 +618,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) trellis_gemm_kernel(GemmArgs p)
 }
 
 template <int CODE, int V, bool L16>
-static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaStream_t st) {
-    auto kern = trellis_gemm_kernel<CODE, V, L16>;
-    cudaError_t e = ensure_smem_limit<trellis_gemm_kernel<CODE, V, L16>>(kTcMaxSmem);
+static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaStream_t st, bool split = false) {
+    if constexpr (CODE == kCode1MAD || CODE == kCode3INST) {
+        if (split) {
+            cudaError_t e = ensure_smem_limit<trellis_gemm_kernel<CODE, V, L16, true>>(kTcMaxSmem);
+            if (e != cudaSuccess) return e;
+            return launch_pdl(trellis_gemm_kernel<CODE, V, L16, true>, dim3(grid), dim3(kTcThreads), smem, st, a);
+        }
+    }
+    auto kern = trellis_gemm_kernel<CODE, V, L16, false>;
+    cudaError_t e = ensure_smem_limit<trellis_gemm_kernel<CODE, V, L16, false>>(kTcMaxSmem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, a);
 }
@@ -538,22 +636,24 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, int grid, size_t smem, cudaS
 // from HBM: a deep ring hides their latency) with as many stage slots as
 // fit, if that leaves at least 4; else the most stage slots, then the deepest
 // code ring that fit in shared memory.
-size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots) {
+size_t tc_smem_bytes(const Layer& L, int npad, int* stages, int* code_slots, bool split) {
+    const int xrows = split ? 2 * npad : npad;  // 128-byte x' rows of one stage
+    const int max_stages = split ? kTcMaxStagesSplit : kTcMaxStages;
     int k2max = 0;
     for (int i = 0; i < L.nparts; ++i) k2max = L.parts[i].k2 > k2max ? L.parts[i].k2 : k2max;
     const int code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
     const int lut_entries = uses_table(L.code) ? (1 << L.Q) : 0;
-    for (int s = kTcMaxStages; s >= 4; --s) {
-        const TcSmem lay = tc_smem_layout(s, kTcMaxCodeSlots, npad, code_slot_words, lut_entries);
+    for (int s = max_stages; s >= 4; --s) {
+        const TcSmem lay = tc_smem_layout(s, kTcMaxCodeSlots, xrows, code_slot_words, lut_entries);
         if (lay.total + 1024 <= kTcMaxSmem) {
             *stages = s;
             *code_slots = kTcMaxCodeSlots;
             return (size_t)lay.total + 1024;
         }
     }
-    for (int s = kTcMaxStages; s >= 2; --s) {
+    for (int s = max_stages; s >= 2; --s) {
         for (int c = kTcMaxCodeSlots; c >= 2; --c) {
-            const TcSmem lay = tc_smem_layout(s, c, npad, code_slot_words, lut_entries);
+            const TcSmem lay = tc_smem_layout(s, c, xrows, code_slot_words, lut_entries);
             if (lay.total + 1024 <= kTcMaxSmem) {
                 *stages = s;
                 *code_slots = c;
@@ -569,6 +669,10 @@ int tc_units(const Layer& L) {
     int tiles = 0;
     for (int i = 0; i < L.nparts; ++i) tiles += (L.parts[i].rows + kTcRows - 1) / kTcRows;
     return tiles * (L.n / kT);
+}
+
+bool tc_split(const Layer& L, int npad) {
+    return (L.code == kCode1MAD || L.code == kCode3INST) && L.V == 1 && npad <= kTcMaxSplitN;
 }
 
 int tc_grid(const Layer& L) {
@@ -631,14 +735,15 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
     a.wait_tries = L.test_wait_tries > 0 ? L.test_wait_tries : kTcWaitTries;
     a.withhold = L.test_withhold;
     a.code_slot_words = (kTcRows / kRowTile) * 64 * k2max;
-    const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots);
+    const bool split = tc_split(L, npad);
+    const size_t smem = tc_smem_bytes(L, npad, &a.stages, &a.code_slots, split);
     if (smem == 0) return cudaErrorInvalidValue;
     const int grid = tc_grid(L);
     const bool l16 = L.L == 16;
-    if (L.code == kCode1MAD) return l16 ? launch_gemm_t<kCode1MAD, 1, true>(a, grid, smem, st)
-                                        : launch_gemm_t<kCode1MAD, 1, false>(a, grid, smem, st);
-    if (L.code == kCode3INST) return l16 ? launch_gemm_t<kCode3INST, 1, true>(a, grid, smem, st)
-                                         : launch_gemm_t<kCode3INST, 1, false>(a, grid, smem, st);
+    if (L.code == kCode1MAD) return l16 ? launch_gemm_t<kCode1MAD, 1, true>(a, grid, smem, st, split)
+                                        : launch_gemm_t<kCode1MAD, 1, false>(a, grid, smem, st, split);
+    if (L.code == kCode3INST) return l16 ? launch_gemm_t<kCode3INST, 1, true>(a, grid, smem, st, split)
+                                         : launch_gemm_t<kCode3INST, 1, false>(a, grid, smem, st, split);
     if (L.code == kCodeTable) {
         if (l16) return cudaErrorInvalidValue;  // codebooks hold at most 2^9 entries
         return L.V == 1 ? launch_gemm_t<kCodeTable, 1, false>(a, grid, smem, st)
@@ -652,9 +757,11 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
 
 cudaError_t prepare_gemm_kernels(const Layer& L) {
     const bool l16 = L.L == 16;
-#define QLK_PREP(C, V_, L_) preload_kernel<trellis_gemm_kernel<C, V_, L_>>(kTcMaxSmem)
-    if (L.code == kCode1MAD) return l16 ? QLK_PREP(kCode1MAD, 1, true) : QLK_PREP(kCode1MAD, 1, false);
-    if (L.code == kCode3INST) return l16 ? QLK_PREP(kCode3INST, 1, true) : QLK_PREP(kCode3INST, 1, false);
+#define QLK_PREP(C, V_, L_) preload_kernel<trellis_gemm_kernel<C, V_, L_, false>>(kTcMaxSmem)
+#define QLK_PREP2(C, L_) \
+    (QLK_PREP(C, 1, L_) == cudaSuccess ? preload_kernel<trellis_gemm_kernel<C, 1, L_, true>>(kTcMaxSmem) : cudaErrorUnknown)
+    if (L.code == kCode1MAD) return l16 ? QLK_PREP2(kCode1MAD, true) : QLK_PREP2(kCode1MAD, false);
+    if (L.code == kCode3INST) return l16 ? QLK_PREP2(kCode3INST, true) : QLK_PREP2(kCode3INST, false);
     if (L.code == kCodeTable) {
         if (l16) return cudaErrorInvalidValue;
         return L.V == 1 ? QLK_PREP(kCodeTable, 1, false) : QLK_PREP(kCodeTable, 2, false);
@@ -663,6 +770,7 @@ cudaError_t prepare_gemm_kernels(const Layer& L) {
     if (L.V == 1) return l16 ? QLK_PREP(kCodeHYB, 1, true) : QLK_PREP(kCodeHYB, 1, false);
     return l16 ? QLK_PREP(kCodeHYB, 2, true) : QLK_PREP(kCodeHYB, 2, false);
 #undef QLK_PREP
+#undef QLK_PREP2
 }
 
 }  // namespace qlk

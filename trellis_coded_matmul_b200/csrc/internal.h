@@ -152,8 +152,11 @@ cudaError_t launch_copy_lut(const void* lut_f16, int Q, int V, uint32_t* dst, cu
 // x (fp16 [batch][n]) -> x' as the decode-GEMV's step words (xstep.cuh).
 cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* xstep, cudaStream_t st);
 // x (fp16 [batch][n]) -> x' as tensor-core operand tiles: [n/64][npad][128 B],
-// the 16-byte chunk c of row b at chunk c ^ (b % 8) (rows >= batch untouched).
-cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st);
+// the 16-byte chunk c of row b at chunk c ^ (b % 8) (rows >= batch untouched);
+// with dup, every value twice along K ([2n/64][npad][128 B], K index 2c and
+// 2c + 1 for column c).
+cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st,
+                               bool dup = false);
 // z (fp32 [batch][m]) -> y = alpha zscale s_out (H_m z), fp32 or fp16; re-zeroes the consumed z.
 cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_dtype, cudaStream_t st,
                            float zscale = 1.0f);
@@ -161,7 +164,7 @@ cudaError_t launch_rht_out(const Layer& L, float* z, int batch, void* y, int y_d
 // columns per slot) -> y = alpha s_out (H_m z), z = the sum of each tile's
 // segment slots; the workspace is only read.
 cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int npad, void* y, int y_dtype,
-                              cudaStream_t st);
+                              cudaStream_t st, float zscale = 1.0f);
 
 // How one decode-GEMV launch is shaped: grid and CTA size, whether the
 // output transform runs in its epilogue, and its dynamic shared memory.
@@ -199,6 +202,11 @@ cudaError_t launch_gemm_tc(const Layer& L, const void* xt, int batch, int npad, 
 // each tile's first segment, tiles + 1 entries).
 int tc_units(const Layer& L);
 int tc_grid(const Layer& L);
+// Whether the GEMM takes split A words at this padded batch (computed codes,
+// V = 1, npad <= 128): x' tiles then hold every value twice along K
+// (launch_rht_in_umma with dup), and the 1MAD sums come out in units of its
+// scale (gemv_z_scale).
+bool tc_split(const Layer& L, int npad);
 void tc_segments(const Layer& L, std::vector<int>& cta_seg, std::vector<int>& tile_seg);
 // Preload (preload_kernel) every kernel a handle can launch: decode-GEMV
 // (both input-transform variants) and qlinear_decode (gemv.cu), the transform

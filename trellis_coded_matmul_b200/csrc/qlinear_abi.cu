@@ -337,7 +337,9 @@ int forward_gemv(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaS
 int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStream_t st) {
     const int chunk = batch < kTcMaxN ? batch : kTcMaxN;
     const int npad_max = (chunk + 15) / 16 * 16;
-    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)npad_max * L.n * 2);
+    // x' tiles hold every value twice along K where the GEMM takes split A words
+    const size_t xp_dup = tc_split(L, 16) ? 2 : 1;
+    int rc = ensure(&L.xp, &L.xp_bytes, (size_t)npad_max * L.n * 2 * xp_dup);
     if (rc == QL_OK) rc = ensure(&L.tcws, &L.tcws_bytes, (size_t)L.tc_slots * npad_max * 128 * 4);
     if (rc != QL_OK) return rc;
     float* ws = (float*)L.tcws;
@@ -348,7 +350,8 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
         const int npad = (nb + 15) / 16 * 16;
         const void* xb = (const char*)x + (size_t)b0 * L.n * 2;
         void* yb = (char*)y + (size_t)b0 * L.m * ysz;
-        cudaError_t e = launch_rht_in_umma(L, xb, nb, npad, L.xp, st);
+        const bool split = tc_split(L, npad);
+        cudaError_t e = launch_rht_in_umma(L, xb, nb, npad, L.xp, st, split);
         const int slot = L.prof_cap ? L.prof_next : -1;
         if (e == cudaSuccess && slot >= 0) e = record_event(L.prof_ev[2 * slot], st);
         if (e == cudaSuccess) e = launch_gemm_tc(L, L.xp, nb, npad, ws, st);
@@ -357,7 +360,7 @@ int forward_tc(Layer& L, const void* x, int batch, void* y, int y_dtype, cudaStr
             L.prof_next = (L.prof_next + 1) % L.prof_cap;
             if (L.prof_count < L.prof_cap) ++L.prof_count;
         }
-        if (e == cudaSuccess) e = launch_rht_out_tc(L, ws, nb, npad, yb, y_dtype, st);
+        if (e == cudaSuccess) e = launch_rht_out_tc(L, ws, nb, npad, yb, y_dtype, st, split ? gemv_z_scale(L) : 1.0f);
         if (e != cudaSuccess) {
             cudaGetLastError();
             return QL_E_CUDA;

@@ -52,12 +52,30 @@ static RhtGeometry rht_geometry(int d, int B, int batch, int E) {
 // tiles (64-column K stages of npad rows of 128 bytes, 16-byte chunk c of row
 // b stored at chunk c ^ (b % 8)).  (The decode-GEMV's step words come from
 // rht_in_block_kernel below.)
-enum { kXpRowMajor = 1, kXpUmma = 2 };
+enum { kXpRowMajor = 1, kXpUmma = 2, kXpUmmaDup = 3 };
 
 // batches from which the tensor-core operand tiles come from the lean input
 // transform (measured on a B200: 1.4 us faster at batch 256, 0.7-1.3 us slower
 // at batch 16-64, where the older kernel stays)
 constexpr int kLeanInMinBatch = 128;
+
+// The 16-byte chunk holding K indices kk .. kk + 7 (kk % 8 == 0) of row b, in halves.
+__device__ __forceinline__ size_t umma_chunk_index(int kk, int b, int npad) {
+    const int s = kk >> 6, chunk = ((kk & 63) >> 3) ^ (b & 7);
+    return (((size_t)s * npad + b) * 128 + chunk * 16) / 2;
+}
+
+// Columns col .. col + 3 (col % 4 == 0) of row b, each value twice along K,
+// as one 16-byte store.
+__device__ __forceinline__ void store_umma_dup4(__half* out, int col, int b, int npad, __half2 lo, __half2 hi) {
+    const __half2 d0 = __half2(__low2half(lo), __low2half(lo));
+    const __half2 d1 = __half2(__high2half(lo), __high2half(lo));
+    const __half2 d2 = __half2(__low2half(hi), __low2half(hi));
+    const __half2 d3 = __half2(__high2half(hi), __high2half(hi));
+    *reinterpret_cast<uint4*>(out + umma_chunk_index(2 * col, b, npad)) =
+        make_uint4(*reinterpret_cast<const uint32_t*>(&d0), *reinterpret_cast<const uint32_t*>(&d1),
+                   *reinterpret_cast<const uint32_t*>(&d2), *reinterpret_cast<const uint32_t*>(&d3));
+}
 
 __device__ __forceinline__ size_t umma_tile_index4(int col, int b, int npad) {
     const int s = col >> 6, kin = col & 63;
@@ -110,7 +128,9 @@ __global__ void __launch_bounds__(E == 8 ? 512 : 1024) rht_in_kernel(const __hal
         uint2 w;
         w.x = *reinterpret_cast<const uint32_t*>(&lo);
         w.y = *reinterpret_cast<const uint32_t*>(&hi);
-        if (MODE == kXpUmma)
+        if (MODE == kXpUmmaDup)
+            store_umma_dup4(out, col + q, b, npad, lo, hi);
+        else if (MODE == kXpUmma)
             *reinterpret_cast<uint2*>(out + umma_tile_index4(col + q, b, npad)) = w;
         else
             *reinterpret_cast<uint2*>(out + (size_t)b * n + col + q) = w;
@@ -205,6 +225,7 @@ cudaError_t launch_rht_in_xstep(const Layer& L, const void* x, int batch, void* 
 // it columns 16 t .. 16 t + 15, transformed in registers, then the strides 16
 // .. T / 2 by warp shuffles; it writes its 16 fp16 values as four 8-byte
 // pieces of the swizzled tiles.
+template <bool DUP>
 __global__ void __launch_bounds__(512) rht_in_umma_lean_kernel(const __half* __restrict__ x, int n, int B,
                                                               const uint32_t* __restrict__ sin_bits, int npad,
                                                               __half* __restrict__ out) {
@@ -246,21 +267,26 @@ __global__ void __launch_bounds__(512) rht_in_umma_lean_kernel(const __half* __r
     for (int j = 0; j < 16; j += 4) {
         const __half2 lo = __floats2half2_rn(v[j] * scale, v[j + 1] * scale);
         const __half2 hi = __floats2half2_rn(v[j + 2] * scale, v[j + 3] * scale);
-        *reinterpret_cast<uint2*>(out + umma_tile_index4(col0 + j, b, npad)) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        if constexpr (DUP)
+            store_umma_dup4(out, col0 + j, b, npad, lo, hi);
+        else
+            *reinterpret_cast<uint2*>(out + umma_tile_index4(col0 + j, b, npad)) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
     }
 }
 
 static bool lean_in_ok(const Layer& L, int batch) { return L.B_n >= 256 && L.B_n <= 8192 && batch >= kLeanInMinBatch; }
 
-cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st) {
+cudaError_t launch_rht_in_umma(const Layer& L, const void* x, int batch, int npad, void* xt, cudaStream_t st,
+                               bool dup) {
     if (lean_in_ok(L, batch)) {
         const dim3 grid(L.n / L.B_n, batch);
         const size_t smem = (size_t)(L.B_n + L.B_n / 16) * sizeof(float);
-        return launch_pdl(rht_in_umma_lean_kernel, grid, dim3(L.B_n / 16), smem, st, (const __half*)x, L.n, L.B_n,
+        auto kern = dup ? rht_in_umma_lean_kernel<true> : rht_in_umma_lean_kernel<false>;
+        return launch_pdl(kern, grid, dim3(L.B_n / 16), smem, st, (const __half*)x, L.n, L.B_n,
                           (const uint32_t*)L.sin_bits, npad, (__half*)xt);
     }
-    return launch_rht_in<kXpUmma>(L, x, batch, xt, npad, st);
+    return dup ? launch_rht_in<kXpUmmaDup>(L, x, batch, xt, npad, st) : launch_rht_in<kXpUmma>(L, x, batch, xt, npad, st);
 }
 
 // Entries per thread of the output transform: B_m may be as small as 16.
@@ -583,35 +609,36 @@ static TcRowMap tc_row_map(const Layer& L) {
 }
 
 template <bool F16, int E>
-static cudaError_t launch_rht_out_tc_e(const Layer& L, const float* ws, int batch, int npad, void* y, cudaStream_t st) {
+static cudaError_t launch_rht_out_tc_e(const Layer& L, const float* ws, int batch, int npad, void* y, cudaStream_t st,
+                                       float zscale) {
     const RhtGeometry geo = rht_geometry(L.m, L.B_m, batch, E);
     const size_t smem = geo.tpg > 32 ? (size_t)geo.groups * (geo.B + geo.B / 16) * sizeof(float) : 0;
     cudaError_t e = ensure_smem_limit<rht_out_tc_kernel<F16, E>>((kMaxHadamard + kMaxHadamard / 16) * 4);
     if (e != cudaSuccess) return e;
     const int grid = (geo.total + geo.groups - 1) / geo.groups;
     return launch_pdl(rht_out_tc_kernel<F16, E>, dim3(grid), dim3(geo.groups * geo.tpg), smem, st, ws, npad, L.m, geo,
-                      tc_row_map(L), L.tc_tile_seg, (const uint32_t*)L.sout_bits, L.alpha, y);
+                      tc_row_map(L), L.tc_tile_seg, (const uint32_t*)L.sout_bits, L.alpha * zscale, y);
 }
 
 cudaError_t launch_rht_out_tc(const Layer& L, const float* ws, int batch, int npad, void* y, int y_dtype,
-                              cudaStream_t st) {
+                              cudaStream_t st, float zscale) {
     const bool f16 = y_dtype == QL_F16;
     // measured on a B200: the lean kernel wins at the large batches (many CTAs,
     // throughput-bound: ~107 -> ~30 instructions per output), not at batch 16
     if (lean_out_ok(L) && tc_tiles_whole(L) && batch >= 32) {
-        const float scale = L.alpha * rsqrtf((float)L.B_m);
+        const float scale = L.alpha * zscale * rsqrtf((float)L.B_m);
         float* w = const_cast<float*>(ws);  // only read (SLOTS)
         return f16 ? launch_rht_out_lean<true, true>(L, w, npad, batch, y, scale, st)
                    : launch_rht_out_lean<false, true>(L, w, npad, batch, y, scale, st);
     }
     if (L.B_m > 16384)
-        return f16 ? launch_rht_out_tc_e<true, 32>(L, ws, batch, npad, y, st)
-                   : launch_rht_out_tc_e<false, 32>(L, ws, batch, npad, y, st);
+        return f16 ? launch_rht_out_tc_e<true, 32>(L, ws, batch, npad, y, st, zscale)
+                   : launch_rht_out_tc_e<false, 32>(L, ws, batch, npad, y, st, zscale);
     if (L.B_m > 4096)
-        return f16 ? launch_rht_out_tc_e<true, 16>(L, ws, batch, npad, y, st)
-                   : launch_rht_out_tc_e<false, 16>(L, ws, batch, npad, y, st);
-    return f16 ? launch_rht_out_tc_e<true, 8>(L, ws, batch, npad, y, st)
-               : launch_rht_out_tc_e<false, 8>(L, ws, batch, npad, y, st);
+        return f16 ? launch_rht_out_tc_e<true, 16>(L, ws, batch, npad, y, st, zscale)
+                   : launch_rht_out_tc_e<false, 16>(L, ws, batch, npad, y, st, zscale);
+    return f16 ? launch_rht_out_tc_e<true, 8>(L, ws, batch, npad, y, st, zscale)
+               : launch_rht_out_tc_e<false, 8>(L, ws, batch, npad, y, st, zscale);
 }
 
 template <int MODE>
@@ -644,7 +671,9 @@ static cudaError_t prepare_rht_out(const Layer& L) {
 cudaError_t prepare_rht_kernels(const Layer& L) {
     cudaError_t e = L.V == 1 ? preload_kernel<rht_in_block_kernel<1>>(0) : preload_kernel<rht_in_block_kernel<2>>(0);
     if (e == cudaSuccess) e = prepare_rht_in<kXpUmma>(L);
-    if (e == cudaSuccess && L.B_n >= 256 && L.B_n <= 8192) e = preload_kernel<rht_in_umma_lean_kernel>(0);
+    if (e == cudaSuccess && L.B_n >= 256 && L.B_n <= 8192) e = preload_kernel<rht_in_umma_lean_kernel<false>>(0);
+    if (e == cudaSuccess && L.B_n >= 256 && L.B_n <= 8192) e = preload_kernel<rht_in_umma_lean_kernel<true>>(0);
+    if (e == cudaSuccess) e = prepare_rht_in<kXpUmmaDup>(L);
     if (e == cudaSuccess) e = prepare_rht_out<true>(L);
     if (e == cudaSuccess) e = prepare_rht_out<false>(L);
     return e;
