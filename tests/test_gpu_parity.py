@@ -252,6 +252,21 @@ def test_forward_small_tensor_core_path(case, batch):
     assert rel_err(y.cpu().numpy(), y_ref) <= TOL_TC
 
 
+# The GEMM's operand forms around their switch points: split A words (computed
+# codes, padded batch <= 128) with x' twice along K, and the lean input
+# transform of the operand tiles (batch >= 128), alone and together.
+@pytest.mark.parametrize("case", [SMALL[0], SMALL[1], SMALL[2], SMALL[9]],
+                         ids=lambda c: f"{c[0]}x{c[1]}_k{c[2]}_L{c[3]}_c{c[5]}")
+@pytest.mark.parametrize("batch", [112, 120, 128, 129, 200])
+def test_forward_operand_form_boundaries(case, batch):
+    li = _small_layer(*case)
+    h = make_handle(li)
+    x = wl.make_x(li.spec, batch, instance=19)
+    y = tcm.qlinear_forward(h, torch.from_numpy(x).cuda())
+    y_ref = oq.Layer.from_inputs(li).forward(x)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_TC
+
+
 @pytest.mark.parametrize("batch", [2, 24])
 def test_parts_with_the_hyb_code(batch):
     split = ((16, 2), (32, 3), (16, 4))
