@@ -325,7 +325,7 @@ int qlinear_profile_enable(qlinear_t h, int capacity);
  * words and x'), so back-to-back launches time it apart from the transforms
  * around it.  Its output is not a result: the decode-GEMV's fp32 sums stay in
  * the handle's accumulator (the next forward re-zeroes it first), and where
- * the decode-GEMV transforms its own output (batch * B_m <= 256) it writes y
+ * the decode-GEMV transforms its own output (batch * m <= 256) it writes y
  * (fp32 or fp16 [batch][m], y_dtype as in qlinear_forward); y is not used
  * otherwise and may then be null.  Works inside CUDA graph capture.
  * Errors: QL_E_ARG (batch < 1, a different batch than the last forward, no

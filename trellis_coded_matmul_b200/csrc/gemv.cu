@@ -566,9 +566,12 @@ GemvPlan plan_gemv(const Layer& L, int batch) {
     pl.threads = (int)((per_cta + per_warp - 1) / per_warp) * 32;
     const long long lut_words = uses_table(L.code) ? (32ll << L.Q) : 0;
     const long long budget = kGemvMaxSmem / 4;
-    // the output transform in-kernel when one CTA's share of it is small, as
-    // many batch rows of one Hadamard block at once as fit (plus its sign words)
-    pl.fuse_out = (long long)batch * L.B_m <= kFuseOutElems;
+    // the output transform in-kernel when all of it is small (measured: with
+    // many output blocks, e.g. m = 11008 in blocks of 256, the drain before
+    // the tickets and the per-CTA transforms cost more than the separate
+    // kernel), as many batch rows of one Hadamard block at once as fit (plus
+    // its sign words)
+    pl.fuse_out = (long long)batch * L.m <= kFuseOutElems;
     const long long row_words = L.B_m + L.B_m / 16;
     const long long sign_words = L.B_m / 32 + 2;
     long long rows = (budget - sign_words) / row_words;

@@ -17,7 +17,7 @@ constexpr int kMaxHadamard = 32768;
 
 constexpr int kGemvMaxWarps = 16;        // decode-GEMV: warps of its one CTA per SM (<= 128 registers/thread)
 constexpr int kGemvMaxSmem = 200 * 1024;  // decode-GEMV dynamic shared memory limit
-constexpr int kFuseOutElems = 256;  // batch * B_m up to which the GEMV's last CTA per block does the output transform
+constexpr int kFuseOutElems = 256;  // batch * m up to which the GEMV's last CTA per block does the output transform
 constexpr int kXInKernelMaxBatch = 2;          // batches up to which every GEMV CTA computes x' itself
 constexpr int kXInKernelMaxBytes = 48 * 1024;  // and x' fits in this much shared memory
 constexpr int kMaxParts = 8;          // row parts of one layer (layers fused along m, own bitwidth each)
