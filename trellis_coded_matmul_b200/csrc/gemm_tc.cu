@@ -1,11 +1,13 @@
-// gemm_tc.cu -- decode-to-shared-memory + tcgen05 tensor-core GEMM for
-// batches above 8: z[b][row] += sum_c W_hat[row][c] x'[b][c].
+// gemm_tc.cu -- trellis decode into tensor memory + tcgen05 tensor-core GEMM
+// for batches above 8: z[b][row] = sum_c W_hat[row][c] x'[b][c], as partial
+// sums per stream-K segment (below).
 //
 // The contraction is dense (M = 128 rows of W_hat per tile, N = batch padded
-// to 16, K = n), so it runs on the 5th-generation tensor cores: fp16 A and B
-// operands in shared memory (K-major, 128-byte swizzle), fp32 accumulator in
-// tensor memory, one thread issuing tcgen05.mma.  The A operand is produced
-// on the fly by decoder warps from the trellis code words (QTIP discussion:
+// to 16, K = n), so it runs on the 5th-generation tensor cores: the fp16 A
+// operand in tensor memory, B = x' in shared memory (K-major, 128-byte
+// swizzle), fp32 accumulator in tensor memory, one thread issuing
+// tcgen05.mma.  The A operand is produced on the fly by decoder warps from
+// the trellis code words (QTIP discussion:
 // decode with computed codes or a small table; the bitshift trellis makes any
 // run of steps decodable from the bits around it), so decoded weights never
 // reach HBM.

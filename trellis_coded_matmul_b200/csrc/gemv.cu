@@ -35,16 +35,18 @@
 // Forward in one launch (batch <= 8):
 //   1. code words of the first unit in flight, then the wait for the previous
 //      kernel (programmatic dependent launch);
-//   2. x' = H_n diag(s_in) x into shared memory when batch * n is small (every
-//      CTA computes all of it), else read from the input-transform kernel's
-//      output;
+//   2. x' = H_n diag(s_in) x into shared memory at batch 1 when one thread
+//      group holds a Hadamard block (every CTA computes all of it), else read
+//      from the input-transform kernel's output;
 //   3. decode + MMA over the warp's units, atomics into z;
-//   4. the output transform (QuIP# page, Fig. 2; QTIP discussion,
-//      "Incoherence Processing (W2)"): a CTA adds the units it finished in
-//      each output Hadamard block to that block's ticket; the CTA that
-//      completes a ticket owns the block, reads its z, applies
-//      y = alpha diag(s_out) H_B z, writes y and returns z and the ticket to
-//      zero for the next forward.  No CTA waits for another.
+//   4. when the whole output is small (batch * m <= 256), the output
+//      transform (QuIP# page, Fig. 2; QTIP discussion, "Incoherence
+//      Processing (W2)"): a CTA adds the units it finished in each output
+//      Hadamard block to that block's ticket; the CTA that completes a ticket
+//      owns the block, reads its z, applies y = alpha diag(s_out) H_B z,
+//      writes y and returns z and the ticket to zero for the next forward.
+//      No CTA waits for another.  Otherwise the output-transform kernel
+//      follows.
 #include <cuda_fp16.h>
 
 #include "codes.cuh"

@@ -81,11 +81,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  : "memory");
 }
 
-// z[i] += v in global memory, result unused (fp32 reduction at L2).
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 // Generic-proxy shared-memory writes -> visible to the async proxy (tcgen05.mma).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
