@@ -42,3 +42,25 @@ def test_record_counters_reads_the_first_launch(tmp_path, monkeypatch):
     assert bench._counters("gemv_attn4096_b1")["warp_inst"] == 5.78e6
     monkeypatch.setattr(bench, "_source_hash", lambda kind: "changed")
     assert bench._counters("gemv_attn4096_b1") is None
+
+
+def test_nanosecond_durations_are_read():
+    bench = _bench()
+    assert bench._UNITS["ns"] == 1e-9 and bench._UNITS["us"] == 1e-6 and bench._UNITS["ms"] == 1e-3
+
+
+def test_roofline_takes_the_burst_peak_for_short_loops_only():
+    bench = _bench()
+    import workloads as wl
+    sp = wl.WORKLOADS["halftcq"]
+    pk = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    short = bench.roofline(sp, 256, 40e-6, pk, "measured", 1965.0, 148, "t", burst_gemm=True, chain_s=45e-6)
+    long_ = bench.roofline(sp, 256, 40e-6, pk, "measured", 1965.0, 148, "t", burst_gemm=False)
+    flops = 2.0 * sp.m * sp.n * 256
+    assert short["bound"] == "tensor" and abs(short["achieved"] - flops / 40e-6 / 1e12) < 1e-9
+    assert short["peak"] == 1600.0 and long_["peak"] == 1400.0
+    assert abs(short["frac"] * 1600.0 - long_["frac"] * 1400.0) < 1e-9
+    assert abs(short["kernel_us_in_forward"] - 45.0) < 1e-9 and "kernel_us_in_forward" not in long_
+    gemv = bench.roofline(wl.WORKLOADS["attn4096"], 1, 8e-6, pk, "measured", 1965.0, 148, "t", burst_gemm=True)
+    alg = wl.WORKLOADS["attn4096"].stream_bytes + 4096 * 2 + 4096 * 4
+    assert gemv["bound"] == "hbm" and abs(gemv["achieved"] - alg / 8e-6 / 1e9) < 1e-6
