@@ -206,7 +206,9 @@ int qlinear_forward(qlinear_t h, const void* x, int batch, void* y, int y_dtype,
 /* As qlinear_forward, with x and y in host memory: copies x to the device,
  * runs forward and copies y back, all on `stream`, and waits for the stream
  * before returning (y is ready on return).  Pinned host memory makes the
- * copies asynchronous DMA transfers; pageable memory also works. */
+ * copies asynchronous DMA transfers; pageable memory also works.  A y of at
+ * most 64 KB in pinned host memory that the device can address (16-byte
+ * aligned) is written there by the forward's last kernel instead of copied. */
 int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype,
                          void* stream);
 

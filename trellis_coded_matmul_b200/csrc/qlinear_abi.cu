@@ -466,6 +466,10 @@ int qlinear_launch_main_kernel(qlinear_t h, const void* x, int batch, void* y, i
     return launch_main(h->L, x, batch, y, y_dtype, (cudaStream_t)stream);
 }
 
+// outputs up to this size in pinned, device-addressable host memory are written
+// there directly by the forward's last kernel
+constexpr size_t kHostZeroCopyMaxBytes = 64 * 1024;
+
 int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_host, int y_dtype, void* stream) {
     if (!h || batch < 0 || (y_dtype != QL_F32 && y_dtype != QL_F16)) return QL_E_ARG;
     if (batch == 0) return QL_OK;
@@ -484,9 +488,19 @@ int qlinear_forward_host(qlinear_t h, const void* x_host, int batch, void* y_hos
         cudaGetLastError();
         return QL_E_CUDA;
     }
-    rc = forward_device(L, stage + xoff, batch, stage, y_dtype, st);
+    // A small y in pinned host memory that the device can address is written
+    // there by the forward's last kernel (no copy command after it).
+    void* y_mapped = nullptr;
+    if (ybytes <= kHostZeroCopyMaxBytes && ((uintptr_t)y_host & 15) == 0) {
+        cudaPointerAttributes pa;
+        if (cudaPointerGetAttributes(&pa, y_host) == cudaSuccess && pa.type == cudaMemoryTypeHost && pa.devicePointer)
+            y_mapped = pa.devicePointer;
+        else
+            cudaGetLastError();
+    }
+    rc = forward_device(L, stage + xoff, batch, y_mapped ? y_mapped : (void*)stage, y_dtype, st);
     if (rc != QL_OK) return rc;
-    if (cudaMemcpyAsync(y_host, stage, ybytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+    if ((!y_mapped && cudaMemcpyAsync(y_host, stage, ybytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
         cudaStreamSynchronize(st) != cudaSuccess) {
         cudaGetLastError();
         return QL_E_CUDA;
