@@ -32,6 +32,7 @@ CASES = [
     (15, 1, 1, wl.CODE_1MAD, 0),
     (16, 1, 2, wl.CODE_HYB, 9),
     (16, 3, 1, wl.CODE_HYB, 9),
+    (16, 4, 1, wl.CODE_1MAD, 0),
     # L = 16 at one bit per step: the dynamic programme shared by a cluster of 4 CTAs
     (16, 1, 1, wl.CODE_HYB, 9),
     (16, 1, 1, wl.CODE_3INST, 0),
@@ -162,16 +163,21 @@ def test_encoded_words_round_trip_through_a_layer():
     tcm.qlinear_destroy(h)
 
 
-def test_cluster_encoder_loops_over_more_blocks_than_clusters():
-    """80 blocks at L = 16: more than the clusters that run at once, so every
-    cluster encodes several blocks in turn; sampled blocks match the oracle."""
-    L, k, V, code = 16, 2, 1, wl.CODE_3INST
-    x = _source(80, seed=77)
+@pytest.mark.parametrize("k,blocks", [(2, 300), (1, 100)], ids=["one_cta", "cluster"])
+def test_encoder_loops_over_more_blocks_than_workers(k, blocks):
+    """More blocks at L = 16 than the CTAs (k = 2: one a block) or clusters
+    (k = 1: four CTAs a block) that run at once, so each encodes several blocks
+    in turn.  Block i repeats source block i % 3 (consecutive blocks of one
+    worker differ), so every block must give the oracle's words for its source."""
+    L, V, code = 16, 1, wl.CODE_3INST
+    base = _source(3, seed=77 + k)
+    pick = np.arange(blocks) % 3
+    x = np.ascontiguousarray(base[pick])
     words = tcm.qlinear_encode(code, L, k, V, torch.from_numpy(x).cuda())
     torch.cuda.synchronize()
     got = words.cpu().numpy().view(np.uint32)
-    for b in (0, 1, 36, 37, 38, 79):
-        assert np.array_equal(got[b], _oracle_words(x[b:b + 1], L, k, V, code, None)[0]), b
+    ref = _oracle_words(base, L, k, V, code, None)
+    assert np.array_equal(got, ref[pick])
 
 
 def test_gaussian_distortion_at_L16_beats_L14():

@@ -22,7 +22,9 @@
 // (every case but L = 16 with kV = 1): it stores only M_t(a) = min_h
 // cost_{t-1}(a + hG), 2^(L-kV) floats per buffer, and recomputes a state's
 // cost M_t(s >> kV) + d(t, s) when it reads it (the same float32 operations
-// as storing it), with the code values computed on the fly.  L = 16 with
+// as storing it), with the code values computed on the fly, or, at L = 16
+// with one value and 2-4 bits per step, held in registers for the whole
+// kernel (128 states a thread of 512).  L = 16 with
 // kV = 1 splits the 2^16 states over a thread-block cluster of 4 CTAs,
 // 16384 states each, which keep their costs and code values (fp16, which they
 // are exactly) in shared memory and read the predecessors' costs from the
@@ -396,6 +398,158 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
     }
 }
 
+// ---- L = 16, V = 1: the group-minima search with the code values in registers ----
+// The same search, the same float32 operations and the same tie rules as
+// encode_gm_kernel.  Each of the 512 threads owns the groups a = tid + 512 i
+// and keeps the fp16 values of their 2^kV predecessor states (128 states, 64
+// registers a thread) for the whole kernel, so a step costs each state one
+// shared-memory load, the distance, the addition and the comparison, instead
+// of recomputing its code value 2 x 255 times per block.
+constexpr int kEncRegThreads = 512;
+constexpr int kEncRegL = 16;
+
+template <int KV>
+struct RegVals {
+    static constexpr int G = (1 << kEncRegL) >> KV;
+    static constexpr int NG = G / kEncRegThreads;  // groups a thread
+    static constexpr int C = 1 << KV;
+    uint32_t w[NG][C / 2];  // states a + h G and a + (h + 1) G (h even): low and high half
+    __device__ __forceinline__ float at(int i, int h) const {
+        const uint32_t v = w[i][h >> 1];
+        return __half2float(__ushort_as_half((unsigned short)((h & 1) ? (v >> 16) : (v & 0xFFFFu))));
+    }
+};
+
+// One step for this thread's groups: Mn(a) = min_h cost_{t-1}(a + h G), the
+// first minimum in ascending h, recorded in ch[a] in pass 2.  Pass 1 needs only
+// the value, and fminf returns the same one: equal costs are the same float
+// (no cost is -0), and both forms skip a NaN cost.
+template <int KV, bool CHOICE>
+__device__ __forceinline__ void reg_step(const RegVals<KV>& rv, const float* __restrict__ Mp, float* __restrict__ Mn,
+                                         float xt, uint8_t* __restrict__ ch) {
+    using R = RegVals<KV>;
+    const int tid = threadIdx.x;
+    // (a + h G) >> kV with a = tid + 512 i: 512 and G are multiples of 2^kV
+    const float* Mt = Mp + (tid >> KV);
+#pragma unroll
+    for (int i = 0; i < R::NG; ++i) {
+        float m = INFINITY;
+        int hb = 0;
+#pragma unroll
+        for (int h = 0; h < R::C; ++h) {
+            const float d0 = __fsub_rn(xt, rv.at(i, h));
+            const float c = __fadd_rn(Mt[i * (kEncRegThreads >> KV) + h * (R::G >> KV)], __fmul_rn(d0, d0));
+            if constexpr (CHOICE) {
+                if (c < m) m = c, hb = h;
+            } else {
+                m = fminf(m, c);
+            }
+        }
+        const int a = tid + i * kEncRegThreads;
+        Mn[a] = m;
+        if constexpr (CHOICE) ch[a] = (uint8_t)hb;
+    }
+}
+
+template <int KV>
+__global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArgs p) {
+    extern __shared__ __align__(16) unsigned char sm[];
+    using R = RegVals<KV>;
+    constexpr int S = 1 << kEncRegL, G = R::G, T = 256;
+    float* Ma = reinterpret_cast<float*>(sm);
+    float* Mb = Ma + G;
+    float* xs = Mb + G;
+    float* red_v = xs + 256;
+    int* red_i = reinterpret_cast<int*>(red_v + 32);
+    const int tid = threadIdx.x;
+    R rv;
+#pragma unroll
+    for (int i = 0; i < R::NG; ++i)
+#pragma unroll
+        for (int h = 0; h < R::C; h += 2) {
+            const uint32_t q = (uint32_t)(tid + i * kEncRegThreads + h * G);
+            rv.w[i][h >> 1] = __byte_perm(code_word_global(p, q), code_word_global(p, q + G), 0x5410);
+        }
+    uint8_t* choice = p.choice + (size_t)blockIdx.x * T * G;
+    for (int blk = blockIdx.x; blk < p.blocks; blk += gridDim.x) {
+        for (int i = tid; i < 256; i += blockDim.x) xs[i] = p.x[(size_t)blk * 256 + i];
+        __syncthreads();
+        int prefix = 0, last = 0;
+        for (int pass = 0; pass < 2; ++pass) {
+            float* Mp = Ma;
+            float* Mn = Mb;
+            for (int a = tid; a < G; a += blockDim.x) Mp[a] = (pass == 0 || a == prefix) ? 0.f : INFINITY;
+            __syncthreads();
+            for (int t = 1; t < T; ++t) {
+                const float xt = xs[t - 1];
+                if (pass == 0) reg_step<KV, false>(rv, Mp, Mn, xt, nullptr);
+                else reg_step<KV, true>(rv, Mp, Mn, xt, choice + (size_t)t * G);
+                __syncthreads();
+                float* tmp = Mp;
+                Mp = Mn;
+                Mn = tmp;
+            }
+            // best final state (pass 2: only the states whose low bits, their group, are the prefix)
+            const float xl = xs[T - 1];
+            float bv = INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < R::NG; ++i) {
+                const int a = tid + i * kEncRegThreads;
+                if (pass == 1 && a != prefix) continue;
+#pragma unroll
+                for (int h = 0; h < R::C; ++h) {
+                    const int s = a + h * G;
+                    const float d0 = __fsub_rn(xl, rv.at(i, h));
+                    const float c = __fadd_rn(Mp[s >> KV], __fmul_rn(d0, d0));
+                    if (c < bv || (c == bv && s < bi)) bv = c, bi = s;
+                }
+            }
+            argmin_cta(bv, bi, red_v, red_i);
+            if (bi < 0 || bi >= S) {
+                if (tid == 0) atomicOr(p.status, kStatusBadInput);
+                bi = 0;
+            }
+            if (pass == 0) prefix = bi & (G - 1);
+            last = bi;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            constexpr int words_per_block = T * KV / 32;
+            uint32_t* out = p.words + (size_t)blk * words_per_block;
+            for (int i = 0; i < words_per_block; ++i) out[i] = 0u;
+            int s = last;
+            float err = 0.f;
+            for (int t = T - 1; t >= 0; --t) {
+                const uint32_t chunk = (uint32_t)(s & (R::C - 1));
+                for (int b = 0; b < KV; ++b) {
+                    const int pos = t * KV + b;
+                    out[pos >> 5] |= ((chunk >> (KV - 1 - b)) & 1u) << (31 - (pos & 31));
+                }
+                const float v = __half2float(__ushort_as_half((unsigned short)(code_word_global(p, (uint32_t)s) & 0xFFFFu)));
+                const float diff = xs[t] - v;
+                err += diff * diff;
+                if (t) {
+                    const int a = s >> KV;
+                    s = a + (int)choice[(size_t)t * G + a] * G;
+                }
+            }
+            if (p.err) p.err[blk] = err;
+        }
+        __syncthreads();
+    }
+}
+
+static size_t reg_smem_bytes(int kv) { return ((size_t)2 * ((size_t)1 << (kEncRegL - kv)) + 256 + 64) * 4; }
+
+template <int KV>
+static cudaError_t launch_reg(const EncodeArgs& a, int workers, cudaStream_t st) {
+    cudaError_t e = ensure_smem_limit<encode_reg_kernel<KV>>(kTcMaxSmem);
+    if (e != cudaSuccess) return e;
+    encode_reg_kernel<KV><<<workers, kEncRegThreads, reg_smem_bytes(KV), st>>>(a);
+    return cudaGetLastError();
+}
+
 static size_t gm_smem_bytes(int L, int kv, int code, int Q) {
     const size_t G = (size_t)1 << (L - kv);
     size_t b = (2 * G + 256 + 64) * 4;
@@ -404,6 +558,12 @@ static size_t gm_smem_bytes(int L, int kv, int code, int Q) {
 }
 
 static bool use_gm(int L, int kv, int code, int Q) { return gm_smem_bytes(L, kv, code, Q) <= (size_t)kTcMaxSmem; }
+
+// the register-cached search: L = 16, one value per step, 2..4 bits per step
+// (128 code values a thread), where the group minima fit one CTA
+static bool use_reg(int L, int kv, int V, int code, int Q) {
+    return L == kEncRegL && V == 1 && kv >= 2 && kv <= 4 && use_gm(L, kv, code, Q);
+}
 
 size_t encode_smem_bytes(int L, int kv, int V, int code, int Q) {
     if (use_gm(L, kv, code, Q)) return gm_smem_bytes(L, kv, code, Q);
@@ -524,6 +684,14 @@ cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t*
     a.choice = choice;
     a.status = status;
     a.nc = encode_cluster_size(L);
+    if (use_reg(L, kv, V, code, Q)) {
+        switch (kv) {
+            case 2: return launch_reg<2>(a, workers, st);
+            case 3: return launch_reg<3>(a, workers, st);
+            case 4: return launch_reg<4>(a, workers, st);
+        }
+        return cudaErrorInvalidValue;
+    }
     if (use_gm(L, kv, code, Q)) {
         const size_t smem = gm_smem_bytes(L, kv, code, Q);
         if (V == 1) {
