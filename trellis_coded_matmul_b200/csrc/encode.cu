@@ -400,24 +400,28 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
 
 // ---- L = 16, V = 1: the group-minima search with the code values in registers ----
 // The same search, the same float32 operations and the same tie rules as
-// encode_gm_kernel.  Each of the 512 threads owns the groups a = tid + 512 i
-// and keeps the fp16 values of their 2^kV predecessor states (128 states, 64
-// registers a thread) for the whole kernel, so a step costs each state one
-// shared-memory load, the distance, the addition and the comparison, instead
-// of recomputing its code value 2 x 255 times per block.
+// encode_gm_kernel.  Each of the 512 threads owns runs ("units") of R
+// consecutive groups a = base .. base + R - 1, R = min(2^kV, 8), base a
+// multiple of R: all of them have the predecessor minima M(base >> kV + h
+// G / 2^kV), so one shared-memory load per h serves R groups, and the unit's
+// R new minima (and, in pass 2, its R choices) go out as one vector store.
+// The fp16 values of the thread's 128 states stay in registers (64) for the
+// whole kernel instead of being recomputed 2 x 255 times per block.
 constexpr int kEncRegThreads = 512;
 constexpr int kEncRegL = 16;
 
 template <int KV>
 struct RegVals {
     static constexpr int G = (1 << kEncRegL) >> KV;
-    static constexpr int NG = G / kEncRegThreads;  // groups a thread
     static constexpr int C = 1 << KV;
-    uint32_t w[NG][C / 2];  // states a + h G and a + (h + 1) G (h even): low and high half
-    __device__ __forceinline__ float at(int i, int h) const {
-        const uint32_t v = w[i][h >> 1];
+    static constexpr int R = C < 8 ? C : 8;               // groups a unit
+    static constexpr int NU = G / (kEncRegThreads * R);  // units a thread: unit j starts at (tid + 512 j) R
+    uint32_t w[NU][R][C / 2];  // states base + r + h G and base + r + (h + 1) G (h even): low and high half
+    __device__ __forceinline__ float at(int j, int r, int h) const {
+        const uint32_t v = w[j][r][h >> 1];
         return __half2float(__ushort_as_half((unsigned short)((h & 1) ? (v >> 16) : (v & 0xFFFFu))));
     }
+    __device__ __forceinline__ static int base(int j) { return ((int)threadIdx.x + j * kEncRegThreads) * R; }
 };
 
 // One step for this thread's groups: Mn(a) = min_h cost_{t-1}(a + h G), the
@@ -427,49 +431,63 @@ struct RegVals {
 template <int KV, bool CHOICE>
 __device__ __forceinline__ void reg_step(const RegVals<KV>& rv, const float* __restrict__ Mp, float* __restrict__ Mn,
                                          float xt, uint8_t* __restrict__ ch) {
-    using R = RegVals<KV>;
-    const int tid = threadIdx.x;
-    // (a + h G) >> kV with a = tid + 512 i: 512 and G are multiples of 2^kV
-    const float* Mt = Mp + (tid >> KV);
+    using Rv = RegVals<KV>;
+    constexpr int R = Rv::R, C = Rv::C;
 #pragma unroll
-    for (int i = 0; i < R::NG; ++i) {
-        float m = INFINITY;
-        int hb = 0;
+    for (int j = 0; j < Rv::NU; ++j) {
+        const int b = Rv::base(j);
+        float mp[C];
 #pragma unroll
-        for (int h = 0; h < R::C; ++h) {
-            const float d0 = __fsub_rn(xt, rv.at(i, h));
-            const float c = __fadd_rn(Mt[i * (kEncRegThreads >> KV) + h * (R::G >> KV)], __fmul_rn(d0, d0));
-            if constexpr (CHOICE) {
-                if (c < m) m = c, hb = h;
-            } else {
-                m = fminf(m, c);
+        for (int h = 0; h < C; ++h) mp[h] = Mp[(b >> KV) + h * (Rv::G >> KV)];
+        float m[R];
+        uint32_t hw[R / 4] = {};
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            m[r] = INFINITY;
+            int hb = 0;
+#pragma unroll
+            for (int h = 0; h < C; ++h) {
+                const float d0 = __fsub_rn(xt, rv.at(j, r, h));
+                const float c = __fadd_rn(mp[h], __fmul_rn(d0, d0));
+                if constexpr (CHOICE) {
+                    if (c < m[r]) m[r] = c, hb = h;
+                } else {
+                    m[r] = fminf(m[r], c);
+                }
             }
+            if constexpr (CHOICE) hw[r >> 2] |= (uint32_t)hb << (8 * (r & 3));
         }
-        const int a = tid + i * kEncRegThreads;
-        Mn[a] = m;
-        if constexpr (CHOICE) ch[a] = (uint8_t)hb;
+#pragma unroll
+        for (int q = 0; q < R; q += 4)
+            *reinterpret_cast<float4*>(Mn + b + q) = make_float4(m[q], m[q + 1], m[q + 2], m[q + 3]);
+        if constexpr (CHOICE) {
+            if constexpr (R == 4) *reinterpret_cast<uint32_t*>(ch + b) = hw[0];
+            else *reinterpret_cast<uint2*>(ch + b) = make_uint2(hw[0], hw[1]);
+        }
     }
 }
 
 template <int KV>
 __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArgs p) {
     extern __shared__ __align__(16) unsigned char sm[];
-    using R = RegVals<KV>;
-    constexpr int S = 1 << kEncRegL, G = R::G, T = 256;
+    using Rv = RegVals<KV>;
+    constexpr int S = 1 << kEncRegL, G = Rv::G, T = 256, R = Rv::R, C = Rv::C;
     float* Ma = reinterpret_cast<float*>(sm);
     float* Mb = Ma + G;
     float* xs = Mb + G;
     float* red_v = xs + 256;
     int* red_i = reinterpret_cast<int*>(red_v + 32);
     const int tid = threadIdx.x;
-    R rv;
+    Rv rv;
 #pragma unroll
-    for (int i = 0; i < R::NG; ++i)
+    for (int j = 0; j < Rv::NU; ++j)
 #pragma unroll
-        for (int h = 0; h < R::C; h += 2) {
-            const uint32_t q = (uint32_t)(tid + i * kEncRegThreads + h * G);
-            rv.w[i][h >> 1] = __byte_perm(code_word_global(p, q), code_word_global(p, q + G), 0x5410);
-        }
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int h = 0; h < C; h += 2) {
+                const uint32_t q = (uint32_t)(Rv::base(j) + r + h * G);
+                rv.w[j][r][h >> 1] = __byte_perm(code_word_global(p, q), code_word_global(p, q + G), 0x5410);
+            }
     uint8_t* choice = p.choice + (size_t)blockIdx.x * T * G;
     for (int blk = blockIdx.x; blk < p.blocks; blk += gridDim.x) {
         for (int i = tid; i < 256; i += blockDim.x) xs[i] = p.x[(size_t)blk * 256 + i];
@@ -494,17 +512,19 @@ __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArg
             float bv = INFINITY;
             int bi = 0x7fffffff;
 #pragma unroll
-            for (int i = 0; i < R::NG; ++i) {
-                const int a = tid + i * kEncRegThreads;
-                if (pass == 1 && a != prefix) continue;
+            for (int j = 0; j < Rv::NU; ++j)
 #pragma unroll
-                for (int h = 0; h < R::C; ++h) {
-                    const int s = a + h * G;
-                    const float d0 = __fsub_rn(xl, rv.at(i, h));
-                    const float c = __fadd_rn(Mp[s >> KV], __fmul_rn(d0, d0));
-                    if (c < bv || (c == bv && s < bi)) bv = c, bi = s;
+                for (int r = 0; r < R; ++r) {
+                    const int a = Rv::base(j) + r;
+                    if (pass == 1 && a != prefix) continue;
+#pragma unroll
+                    for (int h = 0; h < C; ++h) {
+                        const int s = a + h * G;
+                        const float d0 = __fsub_rn(xl, rv.at(j, r, h));
+                        const float c = __fadd_rn(Mp[s >> KV], __fmul_rn(d0, d0));
+                        if (c < bv || (c == bv && s < bi)) bv = c, bi = s;
+                    }
                 }
-            }
             argmin_cta(bv, bi, red_v, red_i);
             if (bi < 0 || bi >= S) {
                 if (tid == 0) atomicOr(p.status, kStatusBadInput);
@@ -521,7 +541,7 @@ __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArg
             int s = last;
             float err = 0.f;
             for (int t = T - 1; t >= 0; --t) {
-                const uint32_t chunk = (uint32_t)(s & (R::C - 1));
+                const uint32_t chunk = (uint32_t)(s & (C - 1));
                 for (int b = 0; b < KV; ++b) {
                     const int pos = t * KV + b;
                     out[pos >> 5] |= ((chunk >> (KV - 1 - b)) & 1u) << (31 - (pos & 31));
