@@ -60,6 +60,8 @@ def parse_args():
                    help="time the trellis-coded quantizer (qlinear_encode, k = 2, 3INST) on an N(0,1) "
                         "source instead of the forward")
     p.add_argument("--encode-L", type=int, default=16, help="state bits of the --encode run (at most 16)")
+    p.add_argument("--encode-blocks", type=int, default=148 * 8,
+                   help="source blocks of 256 values per --encode step (a smaller count for profiler captures)")
     p.add_argument("--record-counters", nargs=3, metavar=("NCU_CSV", "KEY", "CAPTURE"),
                    help="store the counters of an ncu --csv log in profiles/counters.json under KEY (e.g. "
                         "gemv_attn4096_b1) and exit; CAPTURE names the profile that gives the command")
@@ -304,7 +306,7 @@ def run_encode(args):
     import torch
     import trellis_coded_matmul_b200 as tcm
     L, k, V, code = args.encode_L, 2, 1, wl.CODE_3INST
-    blocks = 148 * 8
+    blocks = args.encode_blocks
     x = torch.randn((blocks, 256), generator=torch.Generator().manual_seed(7)).cuda()
     for _ in range(args.warmup):
         tcm.qlinear_encode(code, L, k, V, x)

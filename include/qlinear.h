@@ -280,12 +280,15 @@ int qlinear_test_stall(qlinear_t h, int enable, int wait_tries);
  *           block's reconstruction.
  *   L <= 16, k*V <= 8; code as in qlinear_create (HYB and the table code: the
  *   fp16 table is read; the table code with L = kV is nearest-codeword VQ / NUQ).
- *   Up to L = 14 one CTA holds a block's whole dynamic programme in its shared
- *   memory; at L = 15 and 16 a thread-block cluster of 2 or 4 CTAs shares it
+ *   One CTA holds a block's whole dynamic programme (the group minima of its
+ *   2^L states) in its shared memory whenever they fit, i.e. everything but
+ *   L = 16 at one bit per step, where a thread-block cluster of 4 CTAs shares it
  *   (16384 states per CTA, predecessors' costs read from the other CTAs'
  *   shared memory).
- * Allocates scratch (256/V * 2^(L-kV) bytes per CTA or cluster that runs at
- * once) and returns when the result is ready (synchronises the stream).
+ * Scratch (256/V * 2^(L-kV) bytes per CTA or cluster that runs at once, at
+ * most about 620 MB) comes from a memory pool of the library on the current
+ * device, which keeps it mapped for later calls until the process exits.
+ * Returns when the result is ready (synchronises the stream).
  * Errors: QL_E_ARG, QL_E_UNSUPPORTED (L > 16, or too large for shared memory),
  * QL_E_OOM, QL_E_CUDA, QL_E_DEVICE (non-finite source values). */
 int qlinear_encode(ql_code_t code, int L, int k, int V, const float* x, int blocks, uint32_t* words, float* err,

@@ -180,6 +180,18 @@ def test_encoder_loops_over_more_blocks_than_workers(k, blocks):
     assert np.array_equal(got, ref[pick])
 
 
+def test_encoder_scratch_reuse_leaves_results_unchanged():
+    """The search's scratch comes from a memory pool that the library keeps
+    between calls: a call after a smaller one (other sizes, dirty scratch)
+    gives the same words and errors as the first call on the same source."""
+    x = torch.from_numpy(_source(200, seed=91)).cuda()
+    w1, e1 = tcm.qlinear_encode(wl.CODE_3INST, 16, 2, 1, x, with_error=True)
+    tcm.qlinear_encode(wl.CODE_1MAD, 14, 1, 1, x[:7])
+    w2, e2 = tcm.qlinear_encode(wl.CODE_3INST, 16, 2, 1, x, with_error=True)
+    torch.cuda.synchronize()
+    assert torch.equal(w1, w2) and torch.equal(e1, e2)
+
+
 def test_gaussian_distortion_at_L16_beats_L14():
     """The discussion's setting (L = 16, k = 2): distortion between the Gaussian
     rate-distortion bound and the 2-bit Lloyd-Max quantizer, and below L = 14's

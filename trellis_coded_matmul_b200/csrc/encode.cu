@@ -421,8 +421,32 @@ struct RegVals {
         const uint32_t v = w[j][r][h >> 1];
         return __half2float(__ushort_as_half((unsigned short)((h & 1) ? (v >> 16) : (v & 0xFFFFu))));
     }
+    // v(state) - x, see sub_f16_f32
+    __device__ __forceinline__ float sub_at(int j, int r, int h, float x) const;
     __device__ __forceinline__ static int base(int j) { return ((int)threadIdx.x + j * kEncRegThreads) * R; }
 };
+
+// v - x for the fp16 v in the low (HI = false) or high half of a word and a
+// float32 x, rounded to nearest once: the mixed-precision subtraction of
+// sm_100, which widens v exactly.  Its square is the square of x - v bit for
+// bit (rounding to nearest is symmetric in sign).  The word is split inside the
+// asm so that the halves are not kept as separate registers.
+template <bool HI>
+__device__ __forceinline__ float sub_f16_f32(uint32_t w, float x) {
+    float d;
+    if constexpr (HI)
+        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, hi, %2;\n\t}"
+            : "=f"(d) : "r"(w), "f"(x));
+    else
+        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, lo, %2;\n\t}"
+            : "=f"(d) : "r"(w), "f"(x));
+    return d;
+}
+
+template <int KV>
+__device__ __forceinline__ float RegVals<KV>::sub_at(int j, int r, int h, float x) const {
+    return (h & 1) ? sub_f16_f32<true>(w[j][r][h >> 1], x) : sub_f16_f32<false>(w[j][r][h >> 1], x);
+}
 
 // One step for this thread's groups: Mn(a) = min_h cost_{t-1}(a + h G), the
 // first minimum in ascending h, recorded in ch[a] in pass 2.  Pass 1 needs only
@@ -447,7 +471,7 @@ __device__ __forceinline__ void reg_step(const RegVals<KV>& rv, const float* __r
             int hb = 0;
 #pragma unroll
             for (int h = 0; h < C; ++h) {
-                const float d0 = __fsub_rn(xt, rv.at(j, r, h));
+                const float d0 = rv.sub_at(j, r, h, xt);
                 const float c = __fadd_rn(mp[h], __fmul_rn(d0, d0));
                 if constexpr (CHOICE) {
                     if (c < m[r]) m[r] = c, hb = h;
