@@ -33,6 +33,8 @@ CASES = [
     (16, 1, 2, wl.CODE_HYB, 9),
     (16, 3, 1, wl.CODE_HYB, 9),
     (16, 4, 1, wl.CODE_1MAD, 0),
+    (15, 2, 1, wl.CODE_HYB, 9),
+    (15, 3, 1, wl.CODE_3INST, 0),
     # L = 16 at one bit per step: the dynamic programme shared by a cluster of 4 CTAs
     (16, 1, 1, wl.CODE_HYB, 9),
     (16, 1, 1, wl.CODE_3INST, 0),

@@ -22,9 +22,9 @@
 // (every case but L = 16 with kV = 1): it stores only M_t(a) = min_h
 // cost_{t-1}(a + hG), 2^(L-kV) floats per buffer, and recomputes a state's
 // cost M_t(s >> kV) + d(t, s) when it reads it (the same float32 operations
-// as storing it), with the code values computed on the fly, or, at L = 16
+// as storing it), with the code values computed on the fly, or, at L = 14-16
 // with one value and 2-4 bits per step, held in registers for the whole
-// kernel (128 states a thread of 512).  L = 16 with
+// kernel (2^L / 512 states a thread).  L = 16 with
 // kV = 1 splits the 2^16 states over a thread-block cluster of 4 CTAs,
 // 16384 states each, which keep their costs and code values (fp16, which they
 // are exactly) in shared memory and read the predecessors' costs from the
@@ -398,24 +398,25 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
     }
 }
 
-// ---- L = 16, V = 1: the group-minima search with the code values in registers ----
+// ---- L = 14..16, V = 1: the group-minima search with the code values in registers ----
 // The same search, the same float32 operations and the same tie rules as
 // encode_gm_kernel.  Each of the 512 threads owns runs ("units") of R
 // consecutive groups a = base .. base + R - 1, R = min(2^kV, 8), base a
 // multiple of R: all of them have the predecessor minima M(base >> kV + h
 // G / 2^kV), so one shared-memory load per h serves R groups, and the unit's
 // R new minima (and, in pass 2, its R choices) go out as one vector store.
-// The fp16 values of the thread's 128 states stay in registers (64) for the
-// whole kernel instead of being recomputed 2 x 255 times per block.
+// The fp16 values of the thread's 2^L / 512 states (128 at L = 16) stay in
+// registers for the whole kernel instead of being recomputed 2 x 255 times
+// per block.  Needs G >= 512 R (L = 16: kV <= 4; 15: kV <= 3; 14: kV = 2).
 constexpr int kEncRegThreads = 512;
-constexpr int kEncRegL = 16;
 
-template <int KV>
+template <int LL, int KV>
 struct RegVals {
-    static constexpr int G = (1 << kEncRegL) >> KV;
+    static constexpr int G = (1 << LL) >> KV;
     static constexpr int C = 1 << KV;
     static constexpr int R = C < 8 ? C : 8;               // groups a unit
     static constexpr int NU = G / (kEncRegThreads * R);  // units a thread: unit j starts at (tid + 512 j) R
+    static_assert(NU >= 1, "fewer groups than 512 units");
     uint32_t w[NU][R][C / 2];  // states base + r + h G and base + r + (h + 1) G (h even): low and high half
     __device__ __forceinline__ float at(int j, int r, int h) const {
         const uint32_t v = w[j][r][h >> 1];
@@ -443,8 +444,8 @@ __device__ __forceinline__ float sub_f16_f32(uint32_t w, float x) {
     return d;
 }
 
-template <int KV>
-__device__ __forceinline__ float RegVals<KV>::sub_at(int j, int r, int h, float x) const {
+template <int LL, int KV>
+__device__ __forceinline__ float RegVals<LL, KV>::sub_at(int j, int r, int h, float x) const {
     return (h & 1) ? sub_f16_f32<true>(w[j][r][h >> 1], x) : sub_f16_f32<false>(w[j][r][h >> 1], x);
 }
 
@@ -452,10 +453,10 @@ __device__ __forceinline__ float RegVals<KV>::sub_at(int j, int r, int h, float 
 // first minimum in ascending h, recorded in ch[a] in pass 2.  Pass 1 needs only
 // the value, and fminf returns the same one: equal costs are the same float
 // (no cost is -0), and both forms skip a NaN cost.
-template <int KV, bool CHOICE>
-__device__ __forceinline__ void reg_step(const RegVals<KV>& rv, const float* __restrict__ Mp, float* __restrict__ Mn,
-                                         float xt, uint8_t* __restrict__ ch) {
-    using Rv = RegVals<KV>;
+template <int LL, int KV, bool CHOICE>
+__device__ __forceinline__ void reg_step(const RegVals<LL, KV>& rv, const float* __restrict__ Mp,
+                                         float* __restrict__ Mn, float xt, uint8_t* __restrict__ ch) {
+    using Rv = RegVals<LL, KV>;
     constexpr int R = Rv::R, C = Rv::C;
 #pragma unroll
     for (int j = 0; j < Rv::NU; ++j) {
@@ -491,11 +492,11 @@ __device__ __forceinline__ void reg_step(const RegVals<KV>& rv, const float* __r
     }
 }
 
-template <int KV>
+template <int LL, int KV>
 __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArgs p) {
     extern __shared__ __align__(16) unsigned char sm[];
-    using Rv = RegVals<KV>;
-    constexpr int S = 1 << kEncRegL, G = Rv::G, T = 256, R = Rv::R, C = Rv::C;
+    using Rv = RegVals<LL, KV>;
+    constexpr int S = 1 << LL, G = Rv::G, T = 256, R = Rv::R, C = Rv::C;
     float* Ma = reinterpret_cast<float*>(sm);
     float* Mb = Ma + G;
     float* xs = Mb + G;
@@ -524,8 +525,8 @@ __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArg
             __syncthreads();
             for (int t = 1; t < T; ++t) {
                 const float xt = xs[t - 1];
-                if (pass == 0) reg_step<KV, false>(rv, Mp, Mn, xt, nullptr);
-                else reg_step<KV, true>(rv, Mp, Mn, xt, choice + (size_t)t * G);
+                if (pass == 0) reg_step<LL, KV, false>(rv, Mp, Mn, xt, nullptr);
+                else reg_step<LL, KV, true>(rv, Mp, Mn, xt, choice + (size_t)t * G);
                 __syncthreads();
                 float* tmp = Mp;
                 Mp = Mn;
@@ -584,13 +585,13 @@ __global__ void __launch_bounds__(kEncRegThreads, 1) encode_reg_kernel(EncodeArg
     }
 }
 
-static size_t reg_smem_bytes(int kv) { return ((size_t)2 * ((size_t)1 << (kEncRegL - kv)) + 256 + 64) * 4; }
+static size_t reg_smem_bytes(int L, int kv) { return ((size_t)2 * ((size_t)1 << (L - kv)) + 256 + 64) * 4; }
 
-template <int KV>
+template <int LL, int KV>
 static cudaError_t launch_reg(const EncodeArgs& a, int workers, cudaStream_t st) {
-    cudaError_t e = ensure_smem_limit<encode_reg_kernel<KV>>(kTcMaxSmem);
+    cudaError_t e = ensure_smem_limit<encode_reg_kernel<LL, KV>>(kTcMaxSmem);
     if (e != cudaSuccess) return e;
-    encode_reg_kernel<KV><<<workers, kEncRegThreads, reg_smem_bytes(KV), st>>>(a);
+    encode_reg_kernel<LL, KV><<<workers, kEncRegThreads, reg_smem_bytes(LL, KV), st>>>(a);
     return cudaGetLastError();
 }
 
@@ -603,10 +604,13 @@ static size_t gm_smem_bytes(int L, int kv, int code, int Q) {
 
 static bool use_gm(int L, int kv, int code, int Q) { return gm_smem_bytes(L, kv, code, Q) <= (size_t)kTcMaxSmem; }
 
-// the register-cached search: L = 16, one value per step, 2..4 bits per step
-// (128 code values a thread), where the group minima fit one CTA
+// the register-cached search: one value per step, at least 2 bits per step
+// and 512 units of groups (L = 16: kV 2..4, L = 15: 2..3, L = 14: 2), where
+// the group minima fit one CTA
 static bool use_reg(int L, int kv, int V, int code, int Q) {
-    return L == kEncRegL && V == 1 && kv >= 2 && kv <= 4 && use_gm(L, kv, code, Q);
+    const int R = kv >= 3 ? 8 : 4;
+    return L >= 14 && L <= 16 && V == 1 && kv >= 2 && kv <= 4 && ((1 << (L - kv)) >= kEncRegThreads * R) &&
+           use_gm(L, kv, code, Q);
 }
 
 size_t encode_smem_bytes(int L, int kv, int V, int code, int Q) {
@@ -729,10 +733,13 @@ cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t*
     a.status = status;
     a.nc = encode_cluster_size(L);
     if (use_reg(L, kv, V, code, Q)) {
-        switch (kv) {
-            case 2: return launch_reg<2>(a, workers, st);
-            case 3: return launch_reg<3>(a, workers, st);
-            case 4: return launch_reg<4>(a, workers, st);
+        switch (L * 8 + kv) {
+            case 16 * 8 + 2: return launch_reg<16, 2>(a, workers, st);
+            case 16 * 8 + 3: return launch_reg<16, 3>(a, workers, st);
+            case 16 * 8 + 4: return launch_reg<16, 4>(a, workers, st);
+            case 15 * 8 + 2: return launch_reg<15, 2>(a, workers, st);
+            case 15 * 8 + 3: return launch_reg<15, 3>(a, workers, st);
+            case 14 * 8 + 2: return launch_reg<14, 2>(a, workers, st);
         }
         return cudaErrorInvalidValue;
     }
