@@ -137,6 +137,22 @@ def test_forward_host_buffers():
     assert rel_err(y.numpy(), y_ref) <= TOL_GEMV
 
 
+@pytest.mark.parametrize("case,batch,pinned", [(0, 1, True), (2, 2, False), (4, 72, True), (1, 6, True)],
+                         ids=["1mad_b1_pinned", "1mad_b2_pageable", "hyb_b72_large_x", "3inst_b6_pinned"])
+def test_forward_host_input_paths(case, batch, pinned):
+    """qlinear_forward_host with pinned and pageable host buffers, x from 512 B
+    to 72 KB (72 x 512 fp16), on the GEMV and tensor-core paths, against the
+    oracle."""
+    li = _small_layer(*SMALL[case])
+    h = make_handle(li)
+    x = torch.from_numpy(wl.make_x(li.spec, batch, instance=8))
+    if pinned:
+        x = x.pin_memory()
+    y = tcm.qlinear_forward_host(h, x)
+    tol = TOL_GEMV if batch <= 8 else TOL_TC
+    assert rel_err(y.numpy(), oq.Layer.from_inputs(li).forward(x.numpy())) <= tol
+
+
 def test_forward_mixed_small():
     li = wl.random_layer(64, 512, 0, 16, 1, wl.CODE_3INST, 5, m_top=32, k_top=2, k_bot=3)
     h = make_handle(li)
