@@ -26,6 +26,7 @@ CASES = [
     (12, 2, 2, wl.CODE_HYB, 6),
     (14, 2, 1, wl.CODE_3INST, 0),
     (13, 3, 1, wl.CODE_HYB, 9),
+    (13, 2, 1, wl.CODE_1MAD, 0),
     (14, 2, 2, wl.CODE_HYB, 9),
     # L = 15, 16: one CTA holds the group minima of the search whenever they fit
     (16, 2, 1, wl.CODE_3INST, 0),

@@ -22,7 +22,7 @@
 // (every case but L = 16 with kV = 1): it stores only M_t(a) = min_h
 // cost_{t-1}(a + hG), 2^(L-kV) floats per buffer, and recomputes a state's
 // cost M_t(s >> kV) + d(t, s) when it reads it (the same float32 operations
-// as storing it), with the code values computed on the fly, or, at L = 14-16
+// as storing it), with the code values computed on the fly, or, at L = 13-16
 // with one value and 2-4 bits per step, held in registers for the whole
 // kernel (2^L / 512 states a thread).  L = 16 with
 // kV = 1 splits the 2^16 states over a thread-block cluster of 4 CTAs,
@@ -115,6 +115,23 @@ __device__ __forceinline__ void values_of(uint32_t s, const uint32_t* lut_lane, 
     if constexpr (V == 2) v[1] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
 }
 
+// v - x for the fp16 v in the low (HI = false) or high half of a word and a
+// float32 x, rounded to nearest once: the mixed-precision subtraction of
+// sm_100, which widens v exactly.  Its square is the square of x - v bit for
+// bit (rounding to nearest is symmetric in sign).  The word is split inside the
+// asm so that the halves are not kept as separate registers.
+template <bool HI>
+__device__ __forceinline__ float sub_f16_f32(uint32_t w, float x) {
+    float d;
+    if constexpr (HI)
+        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, hi, %2;\n\t}"
+            : "=f"(d) : "r"(w), "f"(x));
+    else
+        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, lo, %2;\n\t}"
+            : "=f"(d) : "r"(w), "f"(x));
+    return d;
+}
+
 template <int V>
 __device__ __forceinline__ float dist_of(const float* xt, const float (&v)[V]) {
     const float d0 = __fsub_rn(xt[0], v[0]);
@@ -125,6 +142,24 @@ __device__ __forceinline__ float dist_of(const float* xt, const float (&v)[V]) {
     }
     return d;
 }
+
+// Squared distance of state s's values (computed from the code) to xt[0..V),
+// with the float32 rule of dist_of, each difference one mixed-precision
+// subtraction on the fp16 value.
+template <int CODE, int V>
+__device__ __forceinline__ float dist_of_state(uint32_t s, const uint32_t* lut_lane, int qshift, const float* xt) {
+    uint32_t w;
+    if constexpr (V == 2) w = code_v2<CODE>(s, lut_lane, qshift);
+    else w = code_pair<CODE>(s, s, lut_lane, qshift);
+    const float d0 = sub_f16_f32<false>(w, xt[0]);
+    float d = __fmul_rn(d0, d0);
+    if constexpr (V == 2) {
+        const float d1 = sub_f16_f32<true>(w, xt[1]);
+        d = __fadd_rn(d, __fmul_rn(d1, d1));
+    }
+    return d;
+}
+
 
 template <int CODE, int KV, int V>
 __global__ void __launch_bounds__(1024, 1) encode_gm_kernel(EncodeArgs p) {
@@ -163,9 +198,7 @@ __global__ void __launch_bounds__(1024, 1) encode_gm_kernel(EncodeArgs p) {
 #pragma unroll (C <= 16 ? C : 4)
                     for (int h = 0; h < C; ++h) {
                         const uint32_t q = (uint32_t)(a + h * G);
-                        float v[V];
-                        values_of<CODE, V>(q, lut_lane, qshift, v);
-                        const float c = __fadd_rn(Mp[q >> KV], dist_of<V>(xt, v));
+                        const float c = __fadd_rn(Mp[q >> KV], dist_of_state<CODE, V>(q, lut_lane, qshift, xt));
                         if (c < m) m = c, hb = h;
                     }
                     Mn[a] = m;
@@ -398,7 +431,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
     }
 }
 
-// ---- L = 14..16, V = 1: the group-minima search with the code values in registers ----
+// ---- L = 13..16, V = 1: the group-minima search with the code values in registers ----
 // The same search, the same float32 operations and the same tie rules as
 // encode_gm_kernel.  Each of the 512 threads owns runs ("units") of R
 // consecutive groups a = base .. base + R - 1, R = min(2^kV, 8), base a
@@ -407,7 +440,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) encode_cluster_kernel(EncodeAr
 // R new minima (and, in pass 2, its R choices) go out as one vector store.
 // The fp16 values of the thread's 2^L / 512 states (128 at L = 16) stay in
 // registers for the whole kernel instead of being recomputed 2 x 255 times
-// per block.  Needs G >= 512 R (L = 16: kV <= 4; 15: kV <= 3; 14: kV = 2).
+// per block.  Needs G >= 512 R (L = 16: kV <= 4; 15: kV <= 3; 13, 14: kV = 2).
 constexpr int kEncRegThreads = 512;
 
 template <int LL, int KV>
@@ -426,23 +459,6 @@ struct RegVals {
     __device__ __forceinline__ float sub_at(int j, int r, int h, float x) const;
     __device__ __forceinline__ static int base(int j) { return ((int)threadIdx.x + j * kEncRegThreads) * R; }
 };
-
-// v - x for the fp16 v in the low (HI = false) or high half of a word and a
-// float32 x, rounded to nearest once: the mixed-precision subtraction of
-// sm_100, which widens v exactly.  Its square is the square of x - v bit for
-// bit (rounding to nearest is symmetric in sign).  The word is split inside the
-// asm so that the halves are not kept as separate registers.
-template <bool HI>
-__device__ __forceinline__ float sub_f16_f32(uint32_t w, float x) {
-    float d;
-    if constexpr (HI)
-        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, hi, %2;\n\t}"
-            : "=f"(d) : "r"(w), "f"(x));
-    else
-        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tsub.rn.f32.f16 %0, lo, %2;\n\t}"
-            : "=f"(d) : "r"(w), "f"(x));
-    return d;
-}
 
 template <int LL, int KV>
 __device__ __forceinline__ float RegVals<LL, KV>::sub_at(int j, int r, int h, float x) const {
@@ -605,11 +621,11 @@ static size_t gm_smem_bytes(int L, int kv, int code, int Q) {
 static bool use_gm(int L, int kv, int code, int Q) { return gm_smem_bytes(L, kv, code, Q) <= (size_t)kTcMaxSmem; }
 
 // the register-cached search: one value per step, at least 2 bits per step
-// and 512 units of groups (L = 16: kV 2..4, L = 15: 2..3, L = 14: 2), where
+// and 512 units of groups (L = 16: kV 2..4, L = 15: 2..3, L = 13, 14: 2), where
 // the group minima fit one CTA
 static bool use_reg(int L, int kv, int V, int code, int Q) {
     const int R = kv >= 3 ? 8 : 4;
-    return L >= 14 && L <= 16 && V == 1 && kv >= 2 && kv <= 4 && ((1 << (L - kv)) >= kEncRegThreads * R) &&
+    return L >= 13 && L <= 16 && V == 1 && kv >= 2 && kv <= 4 && ((1 << (L - kv)) >= kEncRegThreads * R) &&
            use_gm(L, kv, code, Q);
 }
 
@@ -740,6 +756,7 @@ cudaError_t launch_encode(int code, int L, int kv, int V, int Q, const uint32_t*
             case 15 * 8 + 2: return launch_reg<15, 2>(a, workers, st);
             case 15 * 8 + 3: return launch_reg<15, 3>(a, workers, st);
             case 14 * 8 + 2: return launch_reg<14, 2>(a, workers, st);
+            case 13 * 8 + 2: return launch_reg<13, 2>(a, workers, st);
         }
         return cudaErrorInvalidValue;
     }
